@@ -1,0 +1,380 @@
+"""Benchmark: weight GB/s and % of HBM peak of the M-row FP8 LM-head GEMV on B200.
+
+Workload (one "step"): the synthetic FP8 E4M3 LM head W [248320, 5120] (1.27 GB) with
+per-row float32 scales, run W8A16 through `lm_head_fp8_w8a16` once for each row count
+M in {1, 2, 4, 8, 16, 17, 32, 128} (16-row chunks above 16 rows: 17 weight passes per
+step).  Inputs are resident in HBM before timing; the 1.27 GB weight is 10x the L2, so no
+flush is needed between passes.
+
+Output: one JSON line (rank 0).  `value` = algorithmic weight+scale bytes of all passes of
+all ranks / max-over-ranks device time.  `roofline` covers the W8A16 kernel (the only kernel
+in the timed region), `e2e` the same metric with the per-step host->device copy of x and
+device->host copy of the logits inside the timed region, `cpu_baseline` the CPU oracle on a
+bounded sample of the same workload.
+
+`--impl reference` times the CPU oracle (the only reference this method has) on the same
+workload, metric and units, one bounded sample per step.
+"""
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "weight GB/s and % of HBM peak for M-row quantized LM-head GEMV (M=1..128)"
+VOCAB, HIDDEN = 248320, 5120
+ROWS = (1, 2, 4, 8, 16, 17, 32, 128)
+CHUNK = 16
+SPEC_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def passes(m):
+    return (m + CHUNK - 1) // CHUNK
+
+
+def weight_bytes():
+    return VOCAB * HIDDEN + VOCAB * 4
+
+
+def algo_bytes(m):
+    """Algorithmic bytes of one call at m rows: weight+scales per pass, x once, logits once."""
+    return passes(m) * weight_bytes() + m * HIDDEN * 2 + m * VOCAB * 2
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in ("rowtile_gemv.cuh", "gemv_kernels.cu", "dlmh_common.cuh"):
+        with open(os.path.join(ROOT, "decode_lm_head_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic():
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on this kernel source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get("fp8_w8a16_head")
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return None
+        sms, maxs, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sms.append(float(parts[1]))
+                    maxs.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for name, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(name)
+        if not sms:
+            return None
+        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxs), "samples": len(sms),
+                "reasons": sorted(reasons)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(v, world):
+    if world == 1:
+        return v
+    import torch.distributed as dist
+
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------------------
+# CPU oracle leg
+# ---------------------------------------------------------------------------------------
+
+
+def oracle_sample(rows_sample=32768, seed=1):
+    """Time the CPU oracle on a bounded sample: `rows_sample` vocab rows of the head at every
+    M of the step.  Returns (weight GB/s in the metric's units, seconds, description)."""
+    from decode_lm_head_b200 import synth
+    from oracle import gemv as og
+
+    w = synth.to_numpy_bits(synth.fp8_weight(rows_sample, HIDDEN, seed, "cpu"))
+    s = synth.to_numpy_bits(synth.row_scales(rows_sample, seed, "cpu"))
+    x = synth.to_numpy_bits(synth.bf16_rows(max(ROWS), HIDDEN, seed, "cpu", std=0.5))
+    t0 = time.perf_counter()
+    nbytes = 0
+    for m in ROWS:
+        og.w8a16_gemv(w, s, x[:m])
+        nbytes += passes(m) * rows_sample * (HIDDEN + 4)
+    dt = time.perf_counter() - t0
+    desc = f"{rows_sample} of {VOCAB} vocab rows x {HIDDEN}, M in {list(ROWS)}, float64 numpy oracle"
+    return nbytes / dt / 1e9, dt, desc
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n and n[0]:
+            return int(n[0])
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def run_reference(args):
+    world, rank, _ = int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0
+    if rank != 0:
+        return
+    sample_rows = 4096
+    times = []
+    for i in range(args.warmup + args.steps):
+        gbs, dt, desc = oracle_sample(sample_rows)
+        if i >= args.warmup:
+            times.append((gbs, dt))
+    value = statistics.median(g for g, _ in times)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * statistics.median(d for _, d in times), 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"FP8 E4M3 LM head W8A16 {VOCAB}x{HIDDEN}, M in {list(ROWS)}",
+                   "rows_per_step": list(ROWS), "sample_vocab_rows": sample_rows},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cpu_threads(), "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------------------
+# GPU leg
+# ---------------------------------------------------------------------------------------
+
+
+def run_ours(args):
+    world, rank, local = dist_setup(args)
+    import decode_lm_head_b200 as dl
+    from decode_lm_head_b200 import synth
+
+    dl.lib()
+    dev = torch.device("cuda", local)
+    seed = 1 + rank
+    w = synth.fp8_weight(VOCAB, HIDDEN, seed, dev)
+    s = synth.row_scales(VOCAB, seed, dev)
+    x = synth.bf16_rows(max(ROWS), HIDDEN, seed, dev, std=0.5)
+    outs = {m: torch.empty(m, VOCAB, dtype=torch.bfloat16, device=dev) for m in ROWS}
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        for m in ROWS:
+            dl.lm_head_fp8_w8a16(w, s, x[:m], out=outs[m], stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # ---- device-timed region (inputs resident)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    per_m_events = {m: [] for m in ROWS}
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            for m in ROWS:
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                dl.lm_head_fp8_w8a16(w, s, x[:m], out=outs[m], stream=stream)
+                b.record(stream)
+                per_m_events[m].append((a, b))
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    elapsed_ms = max_over_ranks(ev0.elapsed_time(ev1), world)
+    clocks = clk.summary()
+
+    step_bytes = sum(passes(m) * weight_bytes() for m in ROWS)
+    value = world * args.steps * step_bytes / (elapsed_ms * 1e-3) / 1e9
+    launches_per_step = sum(passes(m) for m in ROWS)
+    per_m = {}
+    for m in ROWS:
+        us = statistics.median(a.elapsed_time(b) for a, b in per_m_events[m]) * 1e3
+        per_m[str(m)] = {"us": round(us, 2), "weight_gbs": round(passes(m) * weight_bytes() / (us * 1e-6) / 1e9, 1),
+                         "passes": passes(m)}
+
+    peak, peak_kind = measured_peaks()
+    algo = sum(algo_bytes(m) for m in ROWS)
+    achieved = args.steps * algo / (elapsed_ms * 1e-3) / 1e9  # per rank: this rank's kernels only
+    traffic = ncu_traffic()
+
+    # ---- end to end through the public API, host buffers, copies inside the region
+    xh = x.cpu().pin_memory()
+    outh = {m: torch.empty(m, VOCAB, dtype=torch.bfloat16).pin_memory() for m in ROWS}
+    xd = torch.empty_like(x)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(max(1, args.warmup // 2)):
+        for m in ROWS:
+            xd[:m].copy_(xh[:m], non_blocking=True)
+            dl.lm_head_fp8_w8a16(w, s, xd[:m], out=outs[m], stream=stream)
+            outh[m].copy_(outs[m], non_blocking=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0.record(stream)
+    for _ in range(args.steps):
+        for m in ROWS:
+            xd[:m].copy_(xh[:m], non_blocking=True)
+            dl.lm_head_fp8_w8a16(w, s, xd[:m], out=outs[m], stream=stream)
+            outh[m].copy_(outs[m], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    e2e_value = world * args.steps * step_bytes / (e2e_ms * 1e-3) / 1e9
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        gbs, dt, desc = oracle_sample()
+        cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": cpu_threads(), "kind": "oracle",
+               "sample": f"{desc}; {dt:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(elapsed_ms / args.steps, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f16-mma/f32-acc (e4m3 weights, bf16 rows)",
+            "data": "synthetic (seeded; E4M3 of clamp(N(0,1)*64), scales U[1e-3,4e-3], x bf16 N(0,1)*0.5)",
+            "config": {"workload": f"FP8 E4M3 LM head W8A16 {VOCAB}x{HIDDEN} (1.27 GB), one call per M",
+                       "rows_per_step": list(ROWS), "weight_passes_per_step": launches_per_step,
+                       "chunk_rows": CHUNK, "l2": "weight 1.27 GB > 126 MB L2: no flush needed",
+                       "parallelism": f"replica per GPU (vocab-shard layout), {world} rank(s)"},
+            "hbm_fraction": {"of_measured_copy": round(value / world / peak, 4),
+                             "of_spec_8tbs": round(value / world / SPEC_HBM_GBS, 4)},
+            "per_m": per_m,
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
+                         "traffic": traffic["dram_bytes_per_launch"] if traffic else None,
+                         "kernel": "rowtile_gemv_kernel<FmtW8A16>",
+                         "algorithmic_bytes_per_step": algo},
+            "e2e": {"value": round(e2e_value, 1), "unit": "GB/s",
+                    "h2d_bytes_per_step": sum(m * HIDDEN * 2 for m in ROWS),
+                    "d2h_bytes_per_step": sum(m * VOCAB * 2 for m in ROWS)},
+            "gpu_launches": args.steps * launches_per_step,
+            "clocks": clocks,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--vocab", type=int, default=VOCAB,
+                    help="head rows; smaller values only for profiling captures (the workload is 248320)")
+    args = ap.parse_args()
+    global VOCAB
+    VOCAB = args.vocab
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

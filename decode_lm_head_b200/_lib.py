@@ -1,0 +1,293 @@
+"""ctypes binding of libdlmh.so: argument marshalling only.
+
+Every function here takes torch CUDA tensors, checks that they are on the GPU with the
+layout the C ABI wants, and passes raw pointers, sizes, leading dimensions and the current
+CUDA stream to the library.  There is no fallback: without the built library, or with CPU
+tensors, every call raises.
+"""
+
+import ctypes
+import os
+import re
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdlmh.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "dlmh.h")
+
+# op ids of dlmh_plan_chunks (dlmh_op in dlmh.h)
+OP_W8A16, OP_W8A8, OP_W4A16, OP_Q6K = 0, 1, 2, 3
+
+W8A8_MAX_ROWS = 128
+W8A16_CHUNK_ROWS = 16
+W4A16_MAX_ROWS = 32
+Q6K_CHUNK_ROWS = 8
+Q8_1_BLOCK_BYTES = 36
+Q6K_BLOCK_BYTES = 210
+
+
+class DlmhError(RuntimeError):
+    def __init__(self, code, what):
+        self.code = code
+        super().__init__(f"{what}: {error_string(code)} (status {code})")
+
+
+_lib = None
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_L = ctypes.c_int64
+_F = ctypes.c_float
+
+_SIGNATURES = {
+    "lm_head_fp8_w8a16": [_P, _P, _I, _I, _P, _L, _I, _P, _L, _P],
+    "w8a8_quantize_rows": [_P, _L, _I, _I, _P, _L, _P, _P],
+    "w8a8_silu_quantize_rows": [_P, _P, _L, _I, _I, _P, _L, _P, _P],
+    "w8a8_gemv": [_P, _P, _I, _I, _P, _L, _P, _I, _P, _L, _P],
+    "w8a8_proj": [_P, _P, _I, _I, _P, _L, _I, _P, _L, _P, _P, _P],
+    "w8a8_silu_proj": [_P, _P, _I, _I, _P, _P, _L, _I, _P, _L, _P, _P, _P],
+    "w4a16_gemv": [_P, _P, _F, _I, _I, _P, _L, _I, _P, _L, _P],
+    "q8_1_quantize_rows": [_P, _L, _I, _I, _P, _P],
+    "q6k_mmvq": [_P, _I, _I, _P, _I, _P, _L, _P],
+    "q6k_lm_head": [_P, _I, _I, _P, _L, _I, _P, _L, _P, _P],
+    "dlmh_plan_chunks": [_I, _I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I), _I],
+    "dlmh_version": [],
+}
+
+
+def lib():
+    """Load libdlmh.so (built in-tree by ``python -m decode_lm_head_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m decode_lm_head_b200.build`")
+        h = ctypes.CDLL(LIB_PATH)
+        for name, args in _SIGNATURES.items():
+            fn = getattr(h, name)
+            fn.argtypes = args
+            fn.restype = _I
+        h.dlmh_error_string.argtypes = [_I]
+        h.dlmh_error_string.restype = ctypes.c_char_p
+        _lib = h
+    return _lib
+
+
+def header_functions():
+    """Names of the functions declared in include/dlmh.h."""
+    with open(HEADER_PATH) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b([a-z_0-9]+)\s*\(", text, flags=re.M)))
+
+
+def error_string(code):
+    return lib().dlmh_error_string(int(code)).decode()
+
+
+def version():
+    return lib().dlmh_version()
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise DlmhError(rc, what)
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _cuda(t, dtype, name, ndim):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (libdlmh has no CPU path)")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {t.dim()}")
+    if ndim >= 1 and t.shape[-1] > 1 and t.stride(-1) != 1:
+        raise ValueError(f"{name} must be contiguous in its last dim")
+    return t
+
+
+def _ld(t):
+    return t.stride(0) if t.shape[0] > 1 else max(t.shape[1], t.stride(0))
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def plan_chunks(op, rows, k):
+    """Host-only: list of (offset, count, tier) passes for op/rows/k (no GPU needed)."""
+    n = lib().dlmh_plan_chunks(op, rows, k, None, None, None, 0)
+    if n < 0:
+        raise DlmhError(n, "dlmh_plan_chunks")
+    if n == 0:
+        return []
+    arr = (_I * n)
+    o, c, t = arr(), arr(), arr()
+    rc = lib().dlmh_plan_chunks(op, rows, k, o, c, t, n)
+    if rc != n:
+        raise DlmhError(rc, "dlmh_plan_chunks")
+    return list(zip(o, c, t))
+
+
+# ---------------------------------------------------------------------------
+# entry points
+# ---------------------------------------------------------------------------
+
+
+def lm_head_fp8_w8a16(w, w_scale, x, out=None, stream=None):
+    """FP8 E4M3 W8A16 GEMV: out[m, n] = bf16(s[n] * sum_k e4m3(w[n,k]) x[m,k])."""
+    _cuda(w, torch.uint8, "w", 2)
+    _cuda(w_scale, torch.float32, "w_scale", 1)
+    _cuda(x, torch.bfloat16, "x", 2)
+    n, k = w.shape
+    rows = x.shape[0]
+    if out is None:
+        out = torch.empty(rows, n, dtype=torch.bfloat16, device=x.device)
+    _cuda(out, torch.bfloat16, "out", 2)
+    _check(lib().lm_head_fp8_w8a16(_ptr(w), _ptr(w_scale), n, k, _ptr(x), _ld(x), rows, _ptr(out), _ld(out),
+                                   _stream(stream)), "lm_head_fp8_w8a16")
+    return out
+
+
+def w8a8_quantize_rows(x, xq=None, x_scale=None, stream=None):
+    _cuda(x, torch.bfloat16, "x", 2)
+    rows, k = x.shape
+    if xq is None:
+        xq = torch.empty(rows, k, dtype=torch.uint8, device=x.device)
+    if x_scale is None:
+        x_scale = torch.empty(rows, dtype=torch.float32, device=x.device)
+    _check(lib().w8a8_quantize_rows(_ptr(x), _ld(x), rows, k, _ptr(xq), _ld(xq), _ptr(x_scale), _stream(stream)),
+           "w8a8_quantize_rows")
+    return xq, x_scale
+
+
+def w8a8_silu_quantize_rows(gate, up, xq=None, x_scale=None, stream=None):
+    _cuda(gate, torch.bfloat16, "gate", 2)
+    _cuda(up, torch.bfloat16, "up", 2)
+    if gate.shape != up.shape or _ld(gate) != _ld(up):
+        raise ValueError("gate and up must have the same shape and row stride")
+    rows, k = gate.shape
+    if xq is None:
+        xq = torch.empty(rows, k, dtype=torch.uint8, device=gate.device)
+    if x_scale is None:
+        x_scale = torch.empty(rows, dtype=torch.float32, device=gate.device)
+    _check(lib().w8a8_silu_quantize_rows(_ptr(gate), _ptr(up), _ld(gate), rows, k, _ptr(xq), _ld(xq),
+                                         _ptr(x_scale), _stream(stream)), "w8a8_silu_quantize_rows")
+    return xq, x_scale
+
+
+def w8a8_gemv(w, w_scale, xq, x_scale, out=None, stream=None):
+    _cuda(w, torch.uint8, "w", 2)
+    _cuda(w_scale, torch.float32, "w_scale", 1)
+    _cuda(xq, torch.uint8, "xq", 2)
+    _cuda(x_scale, torch.float32, "x_scale", 1)
+    n, k = w.shape
+    rows = xq.shape[0]
+    if out is None:
+        out = torch.empty(rows, n, dtype=torch.bfloat16, device=w.device)
+    _check(lib().w8a8_gemv(_ptr(w), _ptr(w_scale), n, k, _ptr(xq), _ld(xq), _ptr(x_scale), rows, _ptr(out),
+                           _ld(out), _stream(stream)), "w8a8_gemv")
+    return out
+
+
+def _w8a8_scratch(k, device, xq_scratch, xscale_scratch):
+    if xq_scratch is None:
+        xq_scratch = torch.empty(W8A8_MAX_ROWS * k, dtype=torch.uint8, device=device)
+    if xscale_scratch is None:
+        xscale_scratch = torch.empty(W8A8_MAX_ROWS, dtype=torch.float32, device=device)
+    return xq_scratch, xscale_scratch
+
+
+def w8a8_proj(w, w_scale, x, out=None, xq_scratch=None, xscale_scratch=None, stream=None):
+    _cuda(w, torch.uint8, "w", 2)
+    _cuda(w_scale, torch.float32, "w_scale", 1)
+    _cuda(x, torch.bfloat16, "x", 2)
+    n, k = w.shape
+    rows = x.shape[0]
+    if out is None:
+        out = torch.empty(rows, n, dtype=torch.bfloat16, device=x.device)
+    xq_scratch, xscale_scratch = _w8a8_scratch(k, x.device, xq_scratch, xscale_scratch)
+    _check(lib().w8a8_proj(_ptr(w), _ptr(w_scale), n, k, _ptr(x), _ld(x), rows, _ptr(out), _ld(out),
+                           _ptr(xq_scratch), _ptr(xscale_scratch), _stream(stream)), "w8a8_proj")
+    return out
+
+
+def w8a8_silu_proj(w, w_scale, gate, up, out=None, xq_scratch=None, xscale_scratch=None, stream=None):
+    _cuda(w, torch.uint8, "w", 2)
+    _cuda(w_scale, torch.float32, "w_scale", 1)
+    _cuda(gate, torch.bfloat16, "gate", 2)
+    _cuda(up, torch.bfloat16, "up", 2)
+    if gate.shape != up.shape or _ld(gate) != _ld(up):
+        raise ValueError("gate and up must have the same shape and row stride")
+    n, k = w.shape
+    rows = gate.shape[0]
+    if out is None:
+        out = torch.empty(rows, n, dtype=torch.bfloat16, device=gate.device)
+    xq_scratch, xscale_scratch = _w8a8_scratch(k, gate.device, xq_scratch, xscale_scratch)
+    _check(lib().w8a8_silu_proj(_ptr(w), _ptr(w_scale), n, k, _ptr(gate), _ptr(up), _ld(gate), rows, _ptr(out),
+                                _ld(out), _ptr(xq_scratch), _ptr(xscale_scratch), _stream(stream)), "w8a8_silu_proj")
+    return out
+
+
+def w4a16_gemv(w_packed, w_block_scale, global_scale, x, out=None, stream=None):
+    _cuda(w_packed, torch.uint8, "w_packed", 2)
+    _cuda(w_block_scale, torch.uint8, "w_block_scale", 2)
+    _cuda(x, torch.bfloat16, "x", 2)
+    n, k2 = w_packed.shape
+    k = 2 * k2
+    if tuple(w_block_scale.shape) != (n, k // 16):
+        raise ValueError("w_block_scale must be [n, k/16]")
+    rows = x.shape[0]
+    if out is None:
+        out = torch.empty(rows, n, dtype=torch.bfloat16, device=x.device)
+    _check(lib().w4a16_gemv(_ptr(w_packed), _ptr(w_block_scale), float(global_scale), n, k, _ptr(x), _ld(x), rows,
+                            _ptr(out), _ld(out), _stream(stream)), "w4a16_gemv")
+    return out
+
+
+def q8_1_quantize_rows(x, q8=None, stream=None):
+    _cuda(x, torch.bfloat16, "x", 2)
+    rows, k = x.shape
+    if q8 is None:
+        q8 = torch.empty(rows, k // 32, Q8_1_BLOCK_BYTES, dtype=torch.uint8, device=x.device)
+    _check(lib().q8_1_quantize_rows(_ptr(x), _ld(x), rows, k, _ptr(q8), _stream(stream)), "q8_1_quantize_rows")
+    return q8
+
+
+def q6k_mmvq(blocks, q8, out=None, stream=None):
+    _cuda(blocks, torch.uint8, "blocks", 3)
+    _cuda(q8, torch.uint8, "q8", 3)
+    if not blocks.is_contiguous() or not q8.is_contiguous():
+        raise ValueError("blocks and q8 must be contiguous")
+    n, nsb, _ = blocks.shape
+    k = nsb * 256
+    rows = q8.shape[0]
+    if out is None:
+        out = torch.empty(rows, n, dtype=torch.bfloat16, device=blocks.device)
+    _check(lib().q6k_mmvq(_ptr(blocks), n, k, _ptr(q8), rows, _ptr(out), _ld(out), _stream(stream)), "q6k_mmvq")
+    return out
+
+
+def q6k_lm_head(blocks, x, out=None, q8_scratch=None, stream=None):
+    _cuda(blocks, torch.uint8, "blocks", 3)
+    _cuda(x, torch.bfloat16, "x", 2)
+    if not blocks.is_contiguous():
+        raise ValueError("blocks must be contiguous")
+    n, nsb, _ = blocks.shape
+    k = nsb * 256
+    rows = x.shape[0]
+    if out is None:
+        out = torch.empty(rows, n, dtype=torch.bfloat16, device=x.device)
+    if q8_scratch is None:
+        q8_scratch = torch.empty(Q6K_CHUNK_ROWS * (k // 32) * Q8_1_BLOCK_BYTES, dtype=torch.uint8, device=x.device)
+    _check(lib().q6k_lm_head(_ptr(blocks), n, k, _ptr(x), _ld(x), rows, _ptr(out), _ld(out), _ptr(q8_scratch),
+                             _stream(stream)), "q6k_lm_head")
+    return out

@@ -1,0 +1,295 @@
+// The C ABI of libdlmh: argument checks, row chunking and tier choice, then launches.
+// Host code only; every check runs before any launch, so a rejected call touches nothing.
+#include <stdint.h>
+
+#include "dlmh_common.cuh"
+#include "gemv_launch.h"
+
+using dlmh::aligned16;
+
+namespace {
+
+constexpr int kMaxK = 1 << 20;
+
+inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+int check_rows(int rows, int cap) {
+  if (rows < 0) return DLMH_ERR_ROWS;
+  if (cap > 0 && rows > cap) return DLMH_ERR_ROWS;
+  return DLMH_OK;
+}
+
+int check_nk(int n, int k, int kmult) {
+  if (n <= 0 || k <= 0 || k > kMaxK || k % kmult != 0) return DLMH_ERR_SHAPE;
+  return DLMH_OK;
+}
+
+// x-like BF16 input: 16-byte aligned base, ld a multiple of 8 elements, ld >= k.
+int check_bf16_in(const void* x, int64_t ld, int k) {
+  if (!x) return DLMH_ERR_NULL;
+  if (ld < k) return DLMH_ERR_LD;
+  if (!aligned16(x) || ld % 8 != 0) return DLMH_ERR_ALIGN;
+  return DLMH_OK;
+}
+
+int check_out(const void* out, int64_t ldc, int n) {
+  if (!out) return DLMH_ERR_NULL;
+  if (ldc < n) return DLMH_ERR_LD;
+  if ((reinterpret_cast<uintptr_t>(out) & 1u) != 0) return DLMH_ERR_ALIGN;
+  return DLMH_OK;
+}
+
+#define DLMH_TRY(expr)            \
+  do {                            \
+    const int rc_ = (expr);       \
+    if (rc_ != DLMH_OK) return rc_; \
+  } while (0)
+
+// Rows per weight pass of each op at reduction length k (0 = not servable).
+int pass_rows(int op, int k) {
+  switch (op) {
+    case DLMH_OP_W8A16: {
+      const int t = dlmh::max_tier_rows(DLMH_OP_W8A16, k);
+      return t >= DLMH_W8A16_CHUNK_ROWS ? DLMH_W8A16_CHUNK_ROWS : 0;
+    }
+    case DLMH_OP_W8A8: return dlmh::max_tier_rows(DLMH_OP_W8A8, k);
+    case DLMH_OP_W4A16: return dlmh::max_tier_rows(DLMH_OP_W4A16, k);
+    case DLMH_OP_Q6K: return DLMH_Q6K_CHUNK_ROWS;
+    default: return 0;
+  }
+}
+
+int op_row_cap(int op) {
+  switch (op) {
+    case DLMH_OP_W4A16: return DLMH_W4A16_MAX_ROWS;
+    default: return 0;  // any rows
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+int dlmh_version(void) { return 100; }
+
+const char* dlmh_error_string(int code) {
+  switch (code) {
+    case DLMH_OK: return "ok";
+    case DLMH_ERR_NULL: return "a required pointer is NULL";
+    case DLMH_ERR_SHAPE: return "invalid shape (n, k or the format's k multiple)";
+    case DLMH_ERR_ALIGN: return "a pointer or leading dimension breaks the required alignment";
+    case DLMH_ERR_ROWS: return "rows is negative or above the entry point's cap";
+    case DLMH_ERR_LD: return "a leading dimension is smaller than the row it holds";
+    case DLMH_ERR_CUDA: return "a CUDA runtime call or kernel launch failed";
+    case DLMH_ERR_UNSUPPORTED: return "shape beyond this build's on-chip limits";
+    case DLMH_ERR_CAPACITY: return "output array too small";
+    default: return "unknown status";
+  }
+}
+
+int dlmh_plan_chunks(int op, int rows, int k, int* offsets, int* counts, int* tiers, int cap) {
+  if (op < DLMH_OP_W8A16 || op > DLMH_OP_Q6K) return DLMH_ERR_SHAPE;
+  if (k <= 0) return DLMH_ERR_SHAPE;
+  DLMH_TRY(check_rows(rows, op_row_cap(op)));
+  const int width = pass_rows(op, k);
+  if (width <= 0) return DLMH_ERR_UNSUPPORTED;
+  int nchunks = 0;
+  for (int done = 0; done < rows;) {
+    const int m = rows - done < width ? rows - done : width;
+    if (nchunks < cap) {
+      if (!offsets || !counts || !tiers) return DLMH_ERR_NULL;
+      offsets[nchunks] = done;
+      counts[nchunks] = m;
+      tiers[nchunks] = op == DLMH_OP_Q6K ? DLMH_Q6K_CHUNK_ROWS : dlmh::tier_width(m);
+    }
+    ++nchunks;
+    done += m;
+  }
+  if (cap > 0 && nchunks > cap) return DLMH_ERR_CAPACITY;
+  return nchunks;
+}
+
+int lm_head_fp8_w8a16(const uint8_t* w, const float* w_scale, int n, int k, const dlmh_bf16* x, int64_t ldx, int rows,
+                      dlmh_bf16* out, int64_t ldc, void* stream) {
+  DLMH_TRY(check_rows(rows, 0));
+  DLMH_TRY(check_nk(n, k, 16));
+  if (rows == 0) return DLMH_OK;
+  if (!w || !w_scale) return DLMH_ERR_NULL;
+  if (!aligned16(w)) return DLMH_ERR_ALIGN;
+  DLMH_TRY(check_bf16_in(x, ldx, k));
+  DLMH_TRY(check_out(out, ldc, n));
+  const int width = pass_rows(DLMH_OP_W8A16, k);
+  if (width <= 0) return DLMH_ERR_UNSUPPORTED;
+  for (int done = 0; done < rows;) {
+    const int m = rows - done < width ? rows - done : width;
+    DLMH_TRY(dlmh::w8a16_pass(w, w_scale, n, k, x + (int64_t)done * ldx, ldx, m, out + (int64_t)done * ldc, ldc,
+                              as_stream(stream)));
+    done += m;
+  }
+  return DLMH_OK;
+}
+
+static int check_quant_out(const uint8_t* xq, int64_t ldq, const float* xs, int k) {
+  if (!xq || !xs) return DLMH_ERR_NULL;
+  if (ldq < k) return DLMH_ERR_LD;
+  if (!aligned16(xq) || ldq % 16 != 0) return DLMH_ERR_ALIGN;
+  return DLMH_OK;
+}
+
+int w8a8_quantize_rows(const dlmh_bf16* x, int64_t ldx, int rows, int k, uint8_t* xq, int64_t ldq, float* x_scale,
+                       void* stream) {
+  DLMH_TRY(check_rows(rows, DLMH_W8A8_MAX_ROWS));
+  if (k <= 0 || k > kMaxK || k % 16) return DLMH_ERR_SHAPE;
+  if (rows == 0) return DLMH_OK;
+  DLMH_TRY(check_bf16_in(x, ldx, k));
+  DLMH_TRY(check_quant_out(xq, ldq, x_scale, k));
+  return dlmh::w8a8_quantize_launch(x, ldx, rows, k, xq, ldq, x_scale, as_stream(stream));
+}
+
+int w8a8_silu_quantize_rows(const dlmh_bf16* gate, const dlmh_bf16* up, int64_t ld, int rows, int k, uint8_t* xq,
+                            int64_t ldq, float* x_scale, void* stream) {
+  DLMH_TRY(check_rows(rows, DLMH_W8A8_MAX_ROWS));
+  if (k <= 0 || k > kMaxK || k % 16) return DLMH_ERR_SHAPE;
+  if (rows == 0) return DLMH_OK;
+  DLMH_TRY(check_bf16_in(gate, ld, k));
+  DLMH_TRY(check_bf16_in(up, ld, k));
+  DLMH_TRY(check_quant_out(xq, ldq, x_scale, k));
+  return dlmh::w8a8_silu_quantize_launch(gate, up, ld, rows, k, xq, ldq, x_scale, as_stream(stream));
+}
+
+int w8a8_gemv(const uint8_t* w, const float* w_scale, int n, int k, const uint8_t* xq, int64_t ldq,
+              const float* x_scale, int rows, dlmh_bf16* out, int64_t ldc, void* stream) {
+  DLMH_TRY(check_rows(rows, DLMH_W8A8_MAX_ROWS));
+  DLMH_TRY(check_nk(n, k, 16));
+  if (rows == 0) return DLMH_OK;
+  if (!w || !w_scale) return DLMH_ERR_NULL;
+  if (!aligned16(w)) return DLMH_ERR_ALIGN;
+  if (!xq || !x_scale) return DLMH_ERR_NULL;
+  if (ldq < k) return DLMH_ERR_LD;
+  if (!aligned16(xq) || ldq % 16 != 0) return DLMH_ERR_ALIGN;
+  DLMH_TRY(check_out(out, ldc, n));
+  const int width = pass_rows(DLMH_OP_W8A8, k);
+  if (width <= 0) return DLMH_ERR_UNSUPPORTED;
+  for (int done = 0; done < rows;) {
+    const int m = rows - done < width ? rows - done : width;
+    DLMH_TRY(dlmh::w8a8_gemv_pass(w, w_scale, n, k, xq + (int64_t)done * ldq, ldq, x_scale + done, m,
+                                  out + (int64_t)done * ldc, ldc, as_stream(stream)));
+    done += m;
+  }
+  return DLMH_OK;
+}
+
+static int w8a8_proj_impl(const uint8_t* w, const float* w_scale, int n, int k, const dlmh_bf16* x,
+                          const dlmh_bf16* up, int64_t ldx, int rows, dlmh_bf16* out, int64_t ldc, uint8_t* xq,
+                          float* xs, void* stream) {
+  DLMH_TRY(check_rows(rows, 0));
+  DLMH_TRY(check_nk(n, k, 16));
+  if (rows == 0) return DLMH_OK;
+  if (!w || !w_scale) return DLMH_ERR_NULL;
+  if (!aligned16(w)) return DLMH_ERR_ALIGN;
+  DLMH_TRY(check_bf16_in(x, ldx, k));
+  if (up) DLMH_TRY(check_bf16_in(up, ldx, k));
+  DLMH_TRY(check_out(out, ldc, n));
+  if (!xq || !xs) return DLMH_ERR_NULL;
+  if (!aligned16(xq) || k % 16 != 0) return DLMH_ERR_ALIGN;
+  if (pass_rows(DLMH_OP_W8A8, k) <= 0) return DLMH_ERR_UNSUPPORTED;
+  if (up && (size_t)k * sizeof(float) > 200 * 1024) return DLMH_ERR_UNSUPPORTED;
+  cudaStream_t s = as_stream(stream);
+  for (int done = 0; done < rows;) {
+    const int m = rows - done < DLMH_W8A8_MAX_ROWS ? rows - done : DLMH_W8A8_MAX_ROWS;
+    const dlmh_bf16* xc = x + (int64_t)done * ldx;
+    if (up)
+      DLMH_TRY(dlmh::w8a8_silu_quantize_launch(xc, up + (int64_t)done * ldx, ldx, m, k, xq, k, xs, s));
+    else
+      DLMH_TRY(dlmh::w8a8_quantize_launch(xc, ldx, m, k, xq, k, xs, s));
+    DLMH_TRY(w8a8_gemv(w, w_scale, n, k, xq, k, xs, m, out + (int64_t)done * ldc, ldc, stream));
+    done += m;
+  }
+  return DLMH_OK;
+}
+
+int w8a8_proj(const uint8_t* w, const float* w_scale, int n, int k, const dlmh_bf16* x, int64_t ldx, int rows,
+              dlmh_bf16* out, int64_t ldc, uint8_t* xq_scratch, float* xscale_scratch, void* stream) {
+  return w8a8_proj_impl(w, w_scale, n, k, x, nullptr, ldx, rows, out, ldc, xq_scratch, xscale_scratch, stream);
+}
+
+int w8a8_silu_proj(const uint8_t* w, const float* w_scale, int n, int k, const dlmh_bf16* gate, const dlmh_bf16* up,
+                   int64_t ld, int rows, dlmh_bf16* out, int64_t ldc, uint8_t* xq_scratch, float* xscale_scratch,
+                   void* stream) {
+  if (!up && rows != 0) return DLMH_ERR_NULL;
+  if (!up) return w8a8_proj_impl(w, w_scale, n, k, gate, nullptr, ld, rows, out, ldc, xq_scratch, xscale_scratch,
+                                 stream);
+  return w8a8_proj_impl(w, w_scale, n, k, gate, up, ld, rows, out, ldc, xq_scratch, xscale_scratch, stream);
+}
+
+int w4a16_gemv(const uint8_t* w_packed, const uint8_t* w_block_scale, float global_scale, int n, int k,
+               const dlmh_bf16* x, int64_t ldx, int rows, dlmh_bf16* out, int64_t ldc, void* stream) {
+  DLMH_TRY(check_rows(rows, DLMH_W4A16_MAX_ROWS));
+  DLMH_TRY(check_nk(n, k, 128));
+  if (rows == 0) return DLMH_OK;
+  if (!w_packed || !w_block_scale) return DLMH_ERR_NULL;
+  if (!aligned16(w_packed) || !aligned16(w_block_scale)) return DLMH_ERR_ALIGN;
+  DLMH_TRY(check_bf16_in(x, ldx, k));
+  DLMH_TRY(check_out(out, ldc, n));
+  const int width = pass_rows(DLMH_OP_W4A16, k);
+  if (width <= 0) return DLMH_ERR_UNSUPPORTED;
+  for (int done = 0; done < rows;) {
+    const int m = rows - done < width ? rows - done : width;
+    DLMH_TRY(dlmh::w4a16_pass(w_packed, w_block_scale, global_scale, n, k, x + (int64_t)done * ldx, ldx, m,
+                              out + (int64_t)done * ldc, ldc, as_stream(stream)));
+    done += m;
+  }
+  return DLMH_OK;
+}
+
+int q8_1_quantize_rows(const dlmh_bf16* x, int64_t ldx, int rows, int k, void* q8_out, void* stream) {
+  DLMH_TRY(check_rows(rows, 0));
+  if (k <= 0 || k > kMaxK || k % 32) return DLMH_ERR_SHAPE;
+  if (rows == 0) return DLMH_OK;
+  if (!x || !q8_out) return DLMH_ERR_NULL;
+  if (ldx < k) return DLMH_ERR_LD;
+  if ((reinterpret_cast<uintptr_t>(x) & 1u) || (reinterpret_cast<uintptr_t>(q8_out) & 3u)) return DLMH_ERR_ALIGN;
+  return dlmh::q8_1_quantize_launch(x, ldx, rows, k, static_cast<uint8_t*>(q8_out), as_stream(stream));
+}
+
+int q6k_mmvq(const void* blocks, int n, int k, const void* q8, int rows, dlmh_bf16* out, int64_t ldc, void* stream) {
+  DLMH_TRY(check_rows(rows, 0));
+  DLMH_TRY(check_nk(n, k, 256));
+  if (rows == 0) return DLMH_OK;
+  if (!blocks || !q8) return DLMH_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(blocks) & 1u) || (reinterpret_cast<uintptr_t>(q8) & 3u)) return DLMH_ERR_ALIGN;
+  DLMH_TRY(check_out(out, ldc, n));
+  const int64_t q8_row = (int64_t)(k / 32) * DLMH_Q8_1_BLOCK_BYTES;
+  for (int done = 0; done < rows;) {
+    const int m = rows - done < DLMH_Q6K_CHUNK_ROWS ? rows - done : DLMH_Q6K_CHUNK_ROWS;
+    DLMH_TRY(dlmh::q6k_mmvq_launch(static_cast<const uint8_t*>(blocks), n, k,
+                                   static_cast<const uint8_t*>(q8) + done * q8_row, m, out + (int64_t)done * ldc, ldc,
+                                   as_stream(stream)));
+    done += m;
+  }
+  return DLMH_OK;
+}
+
+int q6k_lm_head(const void* blocks, int n, int k, const dlmh_bf16* x, int64_t ldx, int rows, dlmh_bf16* out,
+                int64_t ldc, void* q8_scratch, void* stream) {
+  DLMH_TRY(check_rows(rows, 0));
+  DLMH_TRY(check_nk(n, k, 256));
+  if (rows == 0) return DLMH_OK;
+  if (!blocks || !x || !q8_scratch) return DLMH_ERR_NULL;
+  if (ldx < k) return DLMH_ERR_LD;
+  if ((reinterpret_cast<uintptr_t>(blocks) & 1u) || (reinterpret_cast<uintptr_t>(q8_scratch) & 3u) ||
+      (reinterpret_cast<uintptr_t>(x) & 1u))
+    return DLMH_ERR_ALIGN;
+  DLMH_TRY(check_out(out, ldc, n));
+  cudaStream_t s = as_stream(stream);
+  for (int done = 0; done < rows;) {
+    const int m = rows - done < DLMH_Q6K_CHUNK_ROWS ? rows - done : DLMH_Q6K_CHUNK_ROWS;
+    DLMH_TRY(dlmh::q8_1_quantize_launch(x + (int64_t)done * ldx, ldx, m, k, static_cast<uint8_t*>(q8_scratch), s));
+    DLMH_TRY(dlmh::q6k_mmvq_launch(static_cast<const uint8_t*>(blocks), n, k,
+                                   static_cast<const uint8_t*>(q8_scratch), m, out + (int64_t)done * ldc, ldc, s));
+    done += m;
+  }
+  return DLMH_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,31 @@
+// Internal launch entry points of libdlmh (host side).  Every function launches
+// asynchronously on `s` and returns a dlmh_status.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace dlmh {
+
+// Widest row count one weight pass of `op` (a dlmh_op) serves at reduction length k, or 0
+// when even the 8-row tier does not fit on chip.  Pure function of (op, k).
+int max_tier_rows(int op, int k);
+// Width (8, 16 or 32) of the narrowest compiled tier that covers `rows` (1..32).
+inline int tier_width(int rows) { return rows <= 8 ? 8 : (rows <= 16 ? 16 : 32); }
+
+int w8a16_pass(const uint8_t* w, const float* w_scale, int n, int k, const uint16_t* x, int64_t ldx, int rows,
+               uint16_t* out, int64_t ldc, cudaStream_t s);
+int w8a8_gemv_pass(const uint8_t* w, const float* w_scale, int n, int k, const uint8_t* xq, int64_t ldq,
+                   const float* x_scale, int rows, uint16_t* out, int64_t ldc, cudaStream_t s);
+int w4a16_pass(const uint8_t* wp, const uint8_t* wbs, float g, int n, int k, const uint16_t* x, int64_t ldx, int rows,
+               uint16_t* out, int64_t ldc, cudaStream_t s);
+
+int w8a8_quantize_launch(const uint16_t* x, int64_t ldx, int rows, int k, uint8_t* xq, int64_t ldq, float* sx,
+                         cudaStream_t s);
+int w8a8_silu_quantize_launch(const uint16_t* gate, const uint16_t* up, int64_t ld, int rows, int k, uint8_t* xq,
+                              int64_t ldq, float* sx, cudaStream_t s);
+int q8_1_quantize_launch(const uint16_t* x, int64_t ldx, int rows, int k, uint8_t* q8, cudaStream_t s);
+int q6k_mmvq_launch(const uint8_t* blocks, int n, int k, const uint8_t* q8, int rows, uint16_t* out, int64_t ldc,
+                    cudaStream_t s);
+
+}  // namespace dlmh

@@ -1,0 +1,228 @@
+/*
+ * dlmh.h -- C ABI of the B200 (sm_100a) decode LM-head / projection GEMV library.
+ *
+ * One library, libdlmh.so, turns M = 1..128 BF16 decode rows into BF16 logits or
+ * projection outputs against a quantized weight, reading the weight as few times as
+ * possible (one pass per row chunk).  Formats:
+ *   - FP8 E4M3 weights with one float32 scale per output row, run W8A16
+ *     ("metrale_model_engine/model/lm_head_fp8_rows.rs", module doc and lm_head_fp8_run);
+ *   - the same weights run W8A8 after a per-row dynamic E4M3 activation quantize, also
+ *     from bf16(silu(gate) * up) for an FFN down projection
+ *     ("metrale_model_layers/layers/w8a8_layer.rs", W8a8Ctx::proj and W8a8Ctx::silu_proj);
+ *   - NVFP4 W4A16: E2M1 codes two per byte, one E4M3 scale per 16 K-elements, one folded
+ *     float32 global ("metrale_model_layers/layers/w4a16_gemv_tiers.rs";
+ *     "metrale_model_layers/weight_map/fp8_lut.rs", dequant_nvfp4_to_bf16);
+ *   - Q6_K 210-byte super-blocks against block_q8_1-quantized rows
+ *     ("metrale_model_engine/model/lm_head_q6k.rs", lm_head_q6k_run).
+ *
+ * Conventions shared by every entry point
+ * ----------------------------------------
+ *   - Every pointer argument named w*, x*, gate, up, out*, xq*, *scale*, q8*, blocks or
+ *     *scratch is a DEVICE pointer on the current CUDA device.  The caller owns all of
+ *     them; the library allocates no device memory and keeps no pointer after return.
+ *   - BF16 values are passed as raw 16-bit patterns (dlmh_bf16).
+ *   - Matrices are row-major.  Leading dimensions (ld*) count ELEMENTS of the pointed-to
+ *     type, so row r of x starts at x + r * ldx.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ *     Every launch is asynchronous on that stream; no call synchronizes.
+ *   - rows == 0 is valid: after the shape checks (n, k) the call returns DLMH_OK without
+ *     looking at any pointer and launches nothing.
+ *   - Return value: DLMH_OK (0) or a negative dlmh_status.  On any argument error the
+ *     call returns before launching anything, so outputs are left untouched.
+ *     DLMH_ERR_CUDA reports a failed launch (cudaGetLastError after the launch).
+ *   - Output rows are independent of how many rows share a call: the same input row
+ *     gives the same output bits at any `rows` (row invariance, w8a8_layer.rs module
+ *     doc; lm_head_fp8_rows.rs, the W8A8 branch of lm_head_fp8_run).
+ *   - Alignment: weight, scale-block and x pointers must be 16-byte aligned, and ldx
+ *     (and ld of gate/up) must be a multiple of 8 elements, else DLMH_ERR_ALIGN.
+ *
+ * Thread safety: entry points are reentrant.  Calls that share a scratch buffer must be
+ * ordered on one stream (w8a8_layer.rs module doc: quantize -> GEMV pairs of one
+ * scratch never interleave).
+ */
+#ifndef DLMH_H_
+#define DLMH_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Exported symbols (the library is built with hidden visibility by default). */
+#if defined(__GNUC__)
+#define DLMH_API __attribute__((visibility("default")))
+#else
+#define DLMH_API
+#endif
+
+typedef uint16_t dlmh_bf16; /* raw BF16 bit pattern */
+
+typedef enum dlmh_status {
+  DLMH_OK = 0,
+  DLMH_ERR_NULL = -1,        /* a required pointer is NULL */
+  DLMH_ERR_SHAPE = -2,       /* n <= 0, k <= 0, k not a multiple of the format's block */
+  DLMH_ERR_ALIGN = -3,       /* a pointer or leading dimension breaks 16-byte alignment */
+  DLMH_ERR_ROWS = -4,        /* rows < 0, or rows above the entry point's cap */
+  DLMH_ERR_LD = -5,          /* a leading dimension is smaller than the row it holds */
+  DLMH_ERR_CUDA = -6,        /* a CUDA runtime call or launch failed */
+  DLMH_ERR_UNSUPPORTED = -7, /* the shape is valid but beyond this build's limits (k too large) */
+  DLMH_ERR_CAPACITY = -8     /* an output array passed to a host helper is too small */
+} dlmh_status;
+
+/* Largest row count of one W8A8 quantize / GEMV call (ops::W8A8_MAX_ROWS in
+ * lm_head_fp8_rows.rs and w8a8_layer.rs: one weight pass per 128 rows). */
+#define DLMH_W8A8_MAX_ROWS 128
+/* Rows per weight pass of the FP8 W8A16 head (16-row chunks above 16 rows,
+ * lm_head_fp8_rows.rs module doc). */
+#define DLMH_W8A16_CHUNK_ROWS 16
+/* Largest row count of one NVFP4 W4A16 call (w4a16_gemv_tiers.rs, kernel_within:
+ * more than 32 rows is refused). */
+#define DLMH_W4A16_MAX_ROWS 32
+/* Rows per Q6_K launch (MAX_M / KQ_MAX_M in lm_head_q6k.rs). */
+#define DLMH_Q6K_CHUNK_ROWS 8
+/* Bytes of one block_q8_1 (32 values) and one Q6_K super-block (256 values). */
+#define DLMH_Q8_1_BLOCK_BYTES 36
+#define DLMH_Q6K_BLOCK_BYTES 210
+
+/* ---------------------------------------------------------------------------------------
+ * FP8 E4M3 W8A16 GEMV (the FP8 LM head)
+ *   out[m, n] = bf16( s[n] * sum_k e4m3(w[n, k]) * x[m, k] )   for m < rows, n < n
+ * lm_head_fp8_rows.rs, module doc and lm_head_fp8_run (the W8A16 branch).
+ *   w       [n, k] E4M3 bytes, row stride k bytes, 16-byte aligned.
+ *   w_scale [n] float32, one per output row.
+ *   x       [rows, ldx] BF16, ldx >= k, ldx % 8 == 0, 16-byte aligned.
+ *   out     [rows, ldc] BF16, ldc >= n.
+ *   k % 16 == 0.  Any rows >= 0: one weight pass per 16 rows (rows above 16 run as
+ *   consecutive 16-row chunks, the last one ragged).
+ *   Numerics: E4M3 weights are exact in f16; each x row is scaled by a power of two into
+ *   f16 (exact for every |x| >= 2^-31 * max|x| of the row), products are exact and summed
+ *   in f32; the row scale and the power of two are applied to the f32 sum, then rounded
+ *   to BF16 (round-to-nearest-even).
+ *   k above the shared-memory limit of a 16-row chunk (k > 6144) returns
+ *   DLMH_ERR_UNSUPPORTED.
+ * ------------------------------------------------------------------------------------- */
+DLMH_API int lm_head_fp8_w8a16(const uint8_t* w, const float* w_scale, int n, int k, const dlmh_bf16* x,
+                      int64_t ldx, int rows, dlmh_bf16* out, int64_t ldc, void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * W8A8 per-row dynamic E4M3 activation quantize
+ *   per row m:  amax = max_k |x[m, k]|,  sx[m] = amax / 448  (float32 IEEE division),
+ *               xq[m, k] = e4m3_rn_sat( x[m, k] / sx[m] )    (float32 IEEE division,
+ *               round-to-nearest-even, magnitudes above 448 saturate to 448);
+ *               a row with sx == 0 gets all-zero codes.
+ * w8a8_layer.rs, W8a8Ctx::proj (the quantized rows live in the shared W8A8 scratch).
+ *   x       [rows, ldx] BF16;  xq [rows, ldq] E4M3 bytes (ldq >= k, ldq % 16 == 0,
+ *   16-byte aligned);  x_scale [rows] float32.  k % 16 == 0.  rows <= 128.
+ * ------------------------------------------------------------------------------------- */
+DLMH_API int w8a8_quantize_rows(const dlmh_bf16* x, int64_t ldx, int rows, int k, uint8_t* xq, int64_t ldq,
+                       float* x_scale, void* stream);
+
+/* Fused SiLU quantize: h[m, k] = bf16( silu(gate[m, k]) * up[m, k] ), silu(g) = g / (1 + e^-g),
+ * computed in f32 and rounded once to BF16, then quantized per row exactly as
+ * w8a8_quantize_rows; h is never written to memory.  w8a8_layer.rs, W8a8Ctx::silu_proj
+ * (ops::w8a8_act_quant_silu).  gate and up [rows, ld] BF16; rows <= 128. */
+DLMH_API int w8a8_silu_quantize_rows(const dlmh_bf16* gate, const dlmh_bf16* up, int64_t ld, int rows, int k,
+                            uint8_t* xq, int64_t ldq, float* x_scale, void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * W8A8 GEMV on already-quantized rows
+ *   out[m, n] = bf16( s[n] * sx[m] * sum_k e4m3(w[n, k]) * e4m3(xq[m, k]) )
+ * lm_head_fp8_rows.rs (W8A8 branch), w8a8_layer.rs (ops::w8a8_gemv).
+ *   rows <= 128; one weight pass per call.  xq [rows, ldq] as written by the quantize
+ *   entry points; x_scale [rows].  k % 16 == 0 and k <= 16384.
+ * ------------------------------------------------------------------------------------- */
+DLMH_API int w8a8_gemv(const uint8_t* w, const float* w_scale, int n, int k, const uint8_t* xq, int64_t ldq,
+              const float* x_scale, int rows, dlmh_bf16* out, int64_t ldc, void* stream);
+
+/* W8A8 projection of BF16 rows: quantize into the caller's scratch, then GEMV, on one
+ * stream, in 128-row chunks (lm_head_fp8_rows.rs, W8A8 branch of lm_head_fp8_run).
+ *   xq_scratch      device buffer of at least 128 * k bytes, 16-byte aligned (row stride k).
+ *   xscale_scratch  device buffer of at least 128 float32.
+ * After the call the scratch holds the last chunk's codes and scales. */
+DLMH_API int w8a8_proj(const uint8_t* w, const float* w_scale, int n, int k, const dlmh_bf16* x, int64_t ldx,
+              int rows, dlmh_bf16* out, int64_t ldc, uint8_t* xq_scratch, float* xscale_scratch,
+              void* stream);
+
+/* The down projection of a SiLU FFN: w8a8_silu_quantize_rows then w8a8_gemv per 128-row
+ * chunk (w8a8_layer.rs, W8a8Ctx::silu_proj).  Scratch as for w8a8_proj. */
+DLMH_API int w8a8_silu_proj(const uint8_t* w, const float* w_scale, int n, int k, const dlmh_bf16* gate,
+                   const dlmh_bf16* up, int64_t ld, int rows, dlmh_bf16* out, int64_t ldc,
+                   uint8_t* xq_scratch, float* xscale_scratch, void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * NVFP4 W4A16 GEMV
+ *   out[m, n] = bf16( g * sum_b e4m3(S[n, b]) * sum_{k in b} e2m1(W[n, k]) * x[m, k] )
+ * w4a16_gemv_tiers.rs (the W4A16 tiers; more than 32 rows refused);
+ * fp8_lut.rs, dequant_nvfp4_to_bf16 (layout and the folded global g).
+ *   w_packed      [n, k/2] bytes, element 2i in the low nibble of byte i.
+ *   w_block_scale [n, k/16] E4M3 bytes, one per 16 consecutive k of a row.
+ *   global_scale  the folded float32 multiplier g.
+ *   k % 128 == 0, k <= 8192.  rows <= 32 (else DLMH_ERR_ROWS); one weight pass per call.
+ * ------------------------------------------------------------------------------------- */
+DLMH_API int w4a16_gemv(const uint8_t* w_packed, const uint8_t* w_block_scale, float global_scale, int n, int k,
+               const dlmh_bf16* x, int64_t ldx, int rows, dlmh_bf16* out, int64_t ldc, void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * block_q8_1 row quantize (lm_head_q6k.rs, lm_head_q6k_run: kquant_q8_1_rows_bf16)
+ *   Block layout (36 bytes per 32 values): { f16 d; f16 s; int8 qs[32] }.
+ *   d = amax / 127 (f32 division), qs = round-half-away( x / d ) (f32 division; 0 when
+ *   d == 0), stored d = f16(d), s = f16( d * (float)sum(qs) ).
+ *   q8_out: [rows][k/32] blocks, row stride k/32 * 36 bytes, 4-byte aligned.  k % 32 == 0.
+ * ------------------------------------------------------------------------------------- */
+DLMH_API int q8_1_quantize_rows(const dlmh_bf16* x, int64_t ldx, int rows, int k, void* q8_out, void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * Q6_K x block_q8_1 GEMV
+ *   out[m, n] = bf16( sum_sb sum_j d(sb) * sc_j(sb) * d8(m, blk(j)) * sum_{i in j} (q_i - 32) * qs_i )
+ * lm_head_q6k.rs, lm_head_q6k_run (kquant_mmvq_q6_k_w).  Super-block byte map: ql[128] at 0,
+ * qh[64] at 128, int8 scales[16] at 192, f16 d at 208; element 128h + 32t + l takes its low
+ * 4 bits from ql[64h + 32(t&1) + l] (low nibble for t < 2, high for t >= 2) and its top
+ * 2 bits from bits 2t..2t+1 of qh[32h + l]; element i uses scales[i/16].
+ *   blocks [n][k/256] super-blocks, row stride k/256 * 210 bytes (the raw store layout).
+ *   q8     [rows][k/32] block_q8_1 as written by q8_1_quantize_rows.
+ *   k % 256 == 0 (set_lm_head_q6k requires hidden % 256 == 0).  Any rows (8-row launches).
+ * ------------------------------------------------------------------------------------- */
+DLMH_API int q6k_mmvq(const void* blocks, int n, int k, const void* q8, int rows, dlmh_bf16* out, int64_t ldc,
+             void* stream);
+
+/* The Q6_K head for BF16 rows (lm_head_q6k.rs, lm_head_q6k_run): for each chunk of up to
+ * 8 rows, q8_1_quantize_rows into q8_scratch, then q6k_mmvq.  q8_scratch holds at least
+ * 8 * k/32 * 36 bytes. */
+DLMH_API int q6k_lm_head(const void* blocks, int n, int k, const dlmh_bf16* x, int64_t ldx, int rows,
+                dlmh_bf16* out, int64_t ldc, void* q8_scratch, void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * Host helpers (no device work; callable without a GPU)
+ * ------------------------------------------------------------------------------------- */
+
+/* Operation ids for dlmh_plan_chunks. */
+typedef enum dlmh_op {
+  DLMH_OP_W8A16 = 0, /* lm_head_fp8_w8a16 */
+  DLMH_OP_W8A8 = 1,  /* w8a8_proj / w8a8_silu_proj */
+  DLMH_OP_W4A16 = 2, /* w4a16_gemv */
+  DLMH_OP_Q6K = 3    /* q6k_mmvq / q6k_lm_head */
+} dlmh_op;
+
+/* The weight passes an entry point runs for `rows` at reduction length k: pass i covers rows
+ * [offsets[i], offsets[i] + counts[i]) and runs the kernel tier of width tiers[i] (the
+ * narrowest compiled tier that covers counts[i], w4a16_gemv_tiers.rs select_tier).
+ * The pass width is a pure function of (op, k) (which activation tile fits on chip), so
+ * this needs no GPU.  Returns the number of passes (0 for rows == 0), DLMH_ERR_ROWS for
+ * rows < 0 or above the op's cap, DLMH_ERR_SHAPE for an unknown op or k <= 0,
+ * DLMH_ERR_UNSUPPORTED when no tier fits k, DLMH_ERR_CAPACITY when more than `cap`
+ * passes are needed.  Arrays may be NULL when cap == 0 (count only). */
+DLMH_API int dlmh_plan_chunks(int op, int rows, int k, int* offsets, int* counts, int* tiers, int cap);
+
+/* Static description of a status code (never NULL). */
+DLMH_API const char* dlmh_error_string(int code);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+DLMH_API int dlmh_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DLMH_H_ */

@@ -1,0 +1,110 @@
+"""CPU checks of the C ABI: the library loads, exports what include/dlmh.h declares, plans
+row chunks as the oracle's reading of the pages does, and rejects bad arguments before
+launching anything (no GPU is needed for any of this)."""
+
+import ctypes
+
+import pytest
+
+import decode_lm_head_b200 as dl
+from decode_lm_head_b200 import _lib
+from oracle import plan as op
+
+L = None
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _load():
+    global L
+    L = dl.lib()
+
+
+def test_library_exports_every_declared_function():
+    names = _lib.header_functions()
+    assert len(names) >= 13
+    for name in names:
+        assert hasattr(L, name), name
+
+
+def test_error_strings_and_version():
+    assert dl.version() >= 100
+    for code in range(-8, 1):
+        assert dl.error_string(code)
+    assert dl.error_string(-99) == "unknown status"
+
+
+@pytest.mark.parametrize("opid,k,width", [(dl.OP_W8A16, 5120, 16), (dl.OP_W8A16, 1024, 16), (dl.OP_W8A8, 5120, 32),
+                                           (dl.OP_W8A8, 14336, 8), (dl.OP_W4A16, 4096, 16), (dl.OP_Q6K, 7168, 8)])
+def test_plan_matches_oracle_rules(opid, k, width):
+    cap = 32 if opid == dl.OP_W4A16 else 300
+    for rows in range(0, cap + 1):
+        plan = dl.plan_chunks(opid, rows, k)
+        ref = op.chunk_plan(rows, width)
+        assert [(o, c) for o, c, _ in plan] == ref
+        widths = [8] if opid == dl.OP_Q6K else [8, 16, 32]
+        for _, c, tier in plan:
+            i = op.select_tier(c, widths, [True] * len(widths))
+            assert tier == widths[i]
+
+
+def test_plan_rejects():
+    assert L.dlmh_plan_chunks(dl.OP_W4A16, 33, 4096, None, None, None, 0) == -4
+    assert L.dlmh_plan_chunks(dl.OP_W8A16, -1, 5120, None, None, None, 0) == -4
+    assert L.dlmh_plan_chunks(9, 1, 5120, None, None, None, 0) == -2
+    assert L.dlmh_plan_chunks(dl.OP_W8A16, 1, 65536, None, None, None, 0) == -7
+    arr = (ctypes.c_int * 1)()
+    assert L.dlmh_plan_chunks(dl.OP_W8A16, 40, 5120, arr, arr, arr, 1) == -8
+
+
+# Fake device addresses: the argument checks must reject these calls before any CUDA call
+# (on this GPU-less host a call that got past them would return DLMH_ERR_CUDA instead).
+A = 1 << 20          # 16-byte aligned
+U = A + 2            # 2-byte aligned only
+
+
+def test_w8a16_argument_errors():
+    f = L.lm_head_fp8_w8a16
+    assert f(None, A, 16, 64, A, 64, 1, A, 16, None) == -1
+    assert f(A, A, 16, 64, None, 64, 1, A, 16, None) == -1
+    assert f(A, A, 0, 64, A, 64, 1, A, 16, None) == -2
+    assert f(A, A, 16, 63, A, 64, 1, A, 16, None) == -2
+    assert f(A, A, 16, 64, A, 32, 1, A, 16, None) == -5
+    assert f(A, A, 16, 64, A, 64, 1, A, 8, None) == -5
+    assert f(U, A, 16, 64, A, 64, 1, A, 16, None) == -3
+    assert f(A, A, 16, 64, U, 64, 1, A, 16, None) == -3
+    assert f(A, A, 16, 64, A, 68, 1, A, 16, None) == -3
+    assert f(A, A, 16, 64, A, 64, -1, A, 16, None) == -4
+    assert f(A, A, 16, 8192, A, 8192, 1, A, 16, None) == -7
+
+
+def test_w8a8_argument_errors():
+    assert L.w8a8_quantize_rows(A, 64, 129, 64, A, 64, A, None) == -4
+    assert L.w8a8_quantize_rows(A, 64, 1, 64, U, 64, A, None) == -3
+    assert L.w8a8_quantize_rows(A, 64, 1, 64, A, 48, A, None) == -5
+    assert L.w8a8_silu_quantize_rows(A, None, 64, 1, 64, A, 64, A, None) == -1
+    assert L.w8a8_gemv(A, A, 16, 64, A, 64, A, 129, A, 16, None) == -4
+    assert L.w8a8_proj(A, A, 16, 64, A, 64, 1, A, 16, None, A, None) == -1
+    assert L.w8a8_silu_proj(A, A, 16, 64, A, None, 64, 1, A, 16, A, A, None) == -1
+
+
+def test_w4a16_argument_errors():
+    f = L.w4a16_gemv
+    assert f(A, A, ctypes.c_float(1.0), 16, 128, A, 128, 33, A, 16, None) == -4
+    assert f(A, A, ctypes.c_float(1.0), 16, 64, A, 128, 1, A, 16, None) == -2
+    assert f(A, U, ctypes.c_float(1.0), 16, 128, A, 128, 1, A, 16, None) == -3
+    assert f(A, None, ctypes.c_float(1.0), 16, 128, A, 128, 1, A, 16, None) == -1
+
+
+def test_q6k_argument_errors():
+    assert L.q8_1_quantize_rows(A, 64, 1, 48, A, None) == -2
+    assert L.q8_1_quantize_rows(A, 16, 1, 64, A, None) == -5
+    assert L.q6k_mmvq(A, 16, 255, A, 1, A, 16, None) == -2
+    assert L.q6k_mmvq(A + 1, 16, 256, A, 1, A, 16, None) == -3
+    assert L.q6k_lm_head(A, 16, 256, A, 256, 1, A, 16, None, None) == -1
+    assert L.q6k_lm_head(A, 16, 256, A, 256, -3, A, 16, A, None) == -4
+
+
+def test_zero_rows_launch_nothing():
+    # valid arguments with rows == 0 return OK without touching CUDA
+    assert L.w8a8_quantize_rows(A, 64, 0, 64, A, 64, A, None) == 0
+    assert L.q8_1_quantize_rows(A, 64, 0, 64, A, None) == 0

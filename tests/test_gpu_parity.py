@@ -1,0 +1,287 @@
+"""GPU parity: every entry point of libdlmh against the CPU oracle on the same seeded inputs.
+
+Floating outputs must be within |err| <= 2^-7 |ref| + 1e-3 rms(ref); quantized bytes and
+scales must be bit-exact; a row's output bits must not depend on how many rows share the
+call (checked GPU against GPU).
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import decode_lm_head_b200 as dl
+from decode_lm_head_b200 import synth
+from oracle import gemv as og
+from oracle import numerics as nx
+from parity_util import assert_bf16_close
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def bits(t):
+    return synth.to_numpy_bits(t)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    dl.lib()
+
+
+# ---------------------------------------------------------------------------
+# FP8 W8A16
+# ---------------------------------------------------------------------------
+
+
+def test_w8a16_tiny_config_all_rows():
+    """N=8192, K=1024, M=1..4, seed 0 (the tiny FP8 config)."""
+    n, k = 8192, 1024
+    w = synth.fp8_weight(n, k, 0, DEV)
+    s = synth.row_scales(n, 0, DEV)
+    x = synth.bf16_rows(4, k, 0, DEV)
+    ref = og.w8a16_gemv(bits(w), bits(s), bits(x))
+    outs = {}
+    for m in (1, 2, 3, 4):
+        out = dl.lm_head_fp8_w8a16(w, s, x[:m])
+        torch.cuda.synchronize()
+        outs[m] = bits(out)
+        assert_bf16_close(outs[m], ref[:m], f"w8a16 tiny M={m}")
+    for m in (1, 2, 3):
+        assert np.array_equal(outs[m], outs[4][:m]), f"row invariance M={m} vs 4"
+
+
+@pytest.mark.parametrize("n,k", [(1000, 1040), (37, 5120), (4099, 2048)])
+def test_w8a16_ragged_shapes_and_tiers(n, k):
+    w = synth.fp8_weight(n, k, 5, DEV)
+    s = synth.row_scales(n, 5, DEV)
+    x = synth.bf16_rows(40, k, 5, DEV, std=0.5)
+    ref = og.w8a16_gemv(bits(w), bits(s), bits(x))
+    full = bits(dl.lm_head_fp8_w8a16(w, s, x))
+    assert_bf16_close(full, ref, f"w8a16 n={n} k={k} M=40")
+    for m in (1, 5, 8, 9, 16, 17, 33):
+        part = bits(dl.lm_head_fp8_w8a16(w, s, x[:m]))
+        assert np.array_equal(part, full[:m]), f"row invariance M={m}"
+    # the same row placed at every position of a 16-row chunk gives the same bits
+    xr = x[3:4].repeat(16, 1)
+    rep = bits(dl.lm_head_fp8_w8a16(w, s, xr))
+    assert (rep == full[3][None, :]).all()
+
+
+def test_w8a16_strided_io_and_zero_rows():
+    n, k = 515, 1024
+    w = synth.fp8_weight(n, k, 6, DEV)
+    s = synth.row_scales(n, 6, DEV)
+    xb = synth.bf16_rows(7, k + 64, 6, DEV)
+    x = xb[:, :k]                           # ldx = k + 64
+    outb = torch.full((7, n + 9), 7.0, dtype=torch.bfloat16, device=DEV)
+    out = outb[:, :n]                       # ldc = n + 9
+    dl.lm_head_fp8_w8a16(w, s, x, out=out)
+    ref = og.w8a16_gemv(bits(w), bits(s), bits(x))
+    assert_bf16_close(bits(out), ref, "w8a16 strided")
+    assert (outb[:, n:] == 7.0).all(), "padding columns of out were written"
+    empty = torch.empty(0, k, dtype=torch.bfloat16, device=DEV)
+    canary = torch.full((1, n), 3.0, dtype=torch.bfloat16, device=DEV)
+    dl.lm_head_fp8_w8a16(w, s, empty, out=canary[:0])
+    assert (canary == 3.0).all()
+
+
+def test_w8a16_extreme_codes_and_row_magnitudes():
+    n, k = 64, 1024
+    g = torch.Generator(device="cpu").manual_seed(7)
+    codes = torch.randint(0, 256, (n, k), generator=g, dtype=torch.int32).to(torch.uint8)
+    codes[(codes & 0x7F) == 0x7F] = 0x7E          # no NaN codes; keep +-448
+    codes[:8] = codes[:8] & 0x87                   # rows of subnormal codes only
+    w = codes.to(DEV)
+    s = synth.row_scales(n, 7, DEV)
+    x = synth.bf16_rows(6, k, 7, DEV)
+    x[1] *= 1e-25                                  # tiny row
+    x[2] *= 1e25                                   # huge row
+    x[3, ::3] = 0                                  # zeros
+    x[4] = 0                                       # all-zero row
+    x[5, 5] = 3.0e38                               # one huge value beside ordinary ones
+    out = bits(dl.lm_head_fp8_w8a16(w, s, x))
+    ref = og.w8a16_gemv(bits(w), bits(s), bits(x))
+    for m in range(6):
+        if m == 5:
+            continue  # |x| < 2^-31 amax for the ordinary values: outside the exactness range
+        assert_bf16_close(out[m:m + 1], ref[m:m + 1], f"w8a16 extreme row {m}")
+    assert not nx.bf16_decode(out[4]).any()
+
+
+# ---------------------------------------------------------------------------
+# W8A8
+# ---------------------------------------------------------------------------
+
+
+def test_w8a8_quantize_rows_bit_exact():
+    k = 5120
+    x = synth.bf16_rows(128, k, 2, DEV, std=0.5)
+    x[5] = 0
+    x[6] = 0
+    x[6, 17] = -2.5
+    x[7] *= 1e-30
+    x[8, :7] = torch.tensor([448.0, -448.0, 1e-4, -1e-4, 3.0, 0.0, -0.0], dtype=torch.bfloat16)
+    xq, sx = dl.w8a8_quantize_rows(x)
+    q_ref, sx_ref = og.w8a8_quantize_rows(bits(x))
+    assert np.array_equal(bits(sx).view(np.uint32), sx_ref.view(np.uint32))
+    assert np.array_equal(bits(xq), q_ref)
+    for rows in (0, 1, 3):
+        xq2, sx2 = dl.w8a8_quantize_rows(x[:rows])
+        assert np.array_equal(bits(xq2), q_ref[:rows])
+
+
+def _silu_flags(gate_bits, up_bits):
+    """Elements whose float64 silu(g)*up lies within 2^-18 (relative) of a BF16 midpoint."""
+    g = nx.bf16_decode(gate_bits)
+    u = nx.bf16_decode(up_bits)
+    with np.errstate(over="ignore"):
+        p = g / (1.0 + np.exp(-g)) * u
+    a = np.abs(p)
+    _, e = np.frexp(a)
+    quantum = np.ldexp(1.0, np.maximum(e - 1, -126) - 7)
+    frac = a / quantum - np.floor(a / quantum)
+    return (np.abs(frac - 0.5) * quantum <= a * 2.0 ** -18) & (a > 0)
+
+
+def test_w8a8_silu_quantize_bit_exact_off_midpoints():
+    k = 14336
+    gate = synth.bf16_rows(16, k, 3, DEV, tensor_id=4)
+    up = synth.bf16_rows(16, k, 3, DEV, tensor_id=5)
+    xq, sx = dl.w8a8_silu_quantize_rows(gate, up)
+    q_ref, sx_ref = og.silu_quantize_rows(bits(gate), bits(up))
+    flags = _silu_flags(bits(gate), bits(up))
+    assert flags.mean() < 1e-3
+    q = bits(xq)
+    sxg = bits(sx)
+    h_ref = nx.bf16_decode(og.silu_mul_bf16(bits(gate), bits(up)))
+    for m in range(16):
+        amax_i = int(np.argmax(np.abs(h_ref[m])))
+        if flags[m, amax_i]:
+            continue  # the row scale itself may legitimately differ; skip the row
+        assert sxg[m] == sx_ref[m], f"row {m} scale"
+        ok = ~flags[m]
+        assert np.array_equal(q[m][ok], q_ref[m][ok]), f"row {m} codes"
+
+
+@pytest.mark.parametrize("n,k", [(1000, 1024), (4096, 14336)])
+def test_w8a8_gemv_and_proj(n, k):
+    w = synth.fp8_weight(n, k, 8, DEV)
+    s = synth.row_scales(n, 8, DEV)
+    x = synth.bf16_rows(130, k, 8, DEV)
+    full = bits(dl.w8a8_proj(w, s, x))
+    q_ref, sx_ref = og.w8a8_quantize_rows(bits(x))
+    sub = slice(None) if n <= 1000 else slice(0, n, 5)
+    ref = og.w8a8_gemv(bits(w)[sub], bits(s)[sub], q_ref, sx_ref)
+    assert_bf16_close(full[:, sub], ref, f"w8a8 proj n={n} k={k} M=130")
+    for m in (1, 31, 32, 33, 128):
+        part = bits(dl.w8a8_proj(w, s, x[:m]))
+        assert np.array_equal(part, full[:m]), f"row invariance M={m}"
+    xq, sx = dl.w8a8_quantize_rows(x[:128])
+    direct = bits(dl.w8a8_gemv(w, s, xq, sx))
+    assert np.array_equal(direct, full[:128])
+
+
+def test_w8a8_silu_proj_down_projection():
+    n, k = 4096, 14336
+    w = synth.fp8_weight(n, k, 9, DEV)
+    s = synth.row_scales(n, 9, DEV)
+    gate = synth.bf16_rows(24, k, 9, DEV, tensor_id=4)
+    up = synth.bf16_rows(24, k, 9, DEV, tensor_id=5)
+    out = bits(dl.w8a8_silu_proj(w, s, gate, up))
+    xq, sx = dl.w8a8_silu_quantize_rows(gate, up)
+    sub = slice(0, n, 7)
+    ref = og.w8a8_gemv(bits(w)[sub], bits(s)[sub], bits(xq), bits(sx))   # GEMV checked on the GPU's codes
+    assert_bf16_close(out[:, sub], ref, "w8a8 silu proj")
+    ref2 = og.w8a8_silu_proj(bits(w)[sub], bits(s)[sub], bits(gate), bits(up))
+    assert_bf16_close(out[:, sub], ref2, "w8a8 silu proj vs oracle codes")
+
+
+# ---------------------------------------------------------------------------
+# NVFP4 W4A16
+# ---------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("n,k", [(2000, 4096), (77, 1024)])
+def test_w4a16_tiers(n, k):
+    wp, ws, gl = synth.nvfp4_weight(n, k, 10, DEV)
+    x = synth.bf16_rows(32, k, 10, DEV)
+    full = bits(dl.w4a16_gemv(wp, ws, gl, x))
+    ref = og.w4a16_gemv(bits(wp), bits(ws), np.float32(gl), bits(x))
+    assert_bf16_close(full, ref, f"w4a16 n={n} k={k} M=32")
+    for m in (1, 4, 5, 6, 7, 8, 16, 17):
+        part = bits(dl.w4a16_gemv(wp, ws, gl, x[:m]))
+        assert np.array_equal(part, full[:m]), f"row invariance M={m}"
+    with pytest.raises(dl.DlmhError):
+        dl.w4a16_gemv(wp, ws, gl, synth.bf16_rows(33, k, 10, DEV))
+
+
+# ---------------------------------------------------------------------------
+# q8_1 and Q6_K
+# ---------------------------------------------------------------------------
+
+
+def test_q8_1_quantize_bit_exact():
+    k = 7168
+    x = synth.bf16_rows(9, k, 4, DEV)
+    x[2, :64] = 0
+    x[3, :32] = torch.arange(32, dtype=torch.float32).to(torch.bfloat16) - 16.5
+    q8 = bits(dl.q8_1_quantize_rows(x))
+    ref = og.q8_1_quantize_rows(bits(x))
+    assert np.array_equal(q8, ref)
+
+
+@pytest.mark.parametrize("n,k", [(1000, 7168), (33, 512)])
+def test_q6k_mmvq_and_head(n, k):
+    blocks = synth.q6k_blocks(n, k, 4, DEV)
+    x = synth.bf16_rows(20, k, 4, DEV)
+    full = bits(dl.q6k_lm_head(blocks, x))
+    ref = og.q6k_mmvq(bits(blocks), og.q8_1_quantize_rows(bits(x)))
+    assert_bf16_close(full, ref, f"q6k n={n} k={k} M=20")
+    q8 = dl.q8_1_quantize_rows(x)
+    direct = bits(dl.q6k_mmvq(blocks, q8))
+    assert np.array_equal(direct, full)
+    for m in (1, 7, 8, 9):
+        part = bits(dl.q6k_lm_head(blocks, x[:m]))
+        assert np.array_equal(part, full[:m]), f"row invariance M={m}"
+
+
+# ---------------------------------------------------------------------------
+# full-size heads, sampled outputs
+# ---------------------------------------------------------------------------
+
+
+def _sample_rows(n):
+    idx = np.concatenate([np.arange(0, 1024), np.arange(1024, n - 1024, 97), np.arange(n - 1024, n)])
+    return np.unique(idx)
+
+
+def test_fp8_head_full_size_sampled():
+    n, k = 248320, 5120
+    w = synth.fp8_weight(n, k, 1, DEV)
+    s = synth.row_scales(n, 1, DEV)
+    x = synth.bf16_rows(128, k, 1, DEV, std=0.5)
+    idx = _sample_rows(n)
+    wi, si = bits(w[torch.from_numpy(idx).to(DEV)]), bits(s[torch.from_numpy(idx).to(DEV)])
+    full = bits(dl.lm_head_fp8_w8a16(w, s, x))
+    ref = og.w8a16_gemv(wi, si, bits(x))
+    assert_bf16_close(full[:, idx], ref, "fp8 head W8A16 M=128 sampled")
+    for m in (1, 2, 4, 8, 16, 17, 32):
+        part = bits(dl.lm_head_fp8_w8a16(w, s, x[:m]))
+        assert np.array_equal(part, full[:m]), f"row invariance M={m}"
+    # W8A8 on the same head, one 128-row call
+    out8 = bits(dl.w8a8_proj(w, s, x))
+    ref8 = og.w8a8_proj(wi, si, bits(x))
+    assert_bf16_close(out8[:, idx], ref8, "fp8 head W8A8 M=128 sampled")
+
+
+def test_q6k_head_full_size_sampled():
+    n, k = 129280, 7168
+    blocks = synth.q6k_blocks(n, k, 4, DEV)
+    x = synth.bf16_rows(16, k, 4, DEV)
+    idx = _sample_rows(n)
+    out = bits(dl.q6k_lm_head(blocks, x))
+    ref = og.q6k_mmvq(bits(blocks[torch.from_numpy(idx).to(DEV)]), og.q8_1_quantize_rows(bits(x)))
+    assert_bf16_close(out[:, idx], ref, "q6k head M=16 sampled")
