@@ -363,11 +363,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--vocab", type=int, default=VOCAB,
+    ap.add_argument("--vocab", type=int, default=248320,
                     help="head rows; smaller values only for profiling captures (the workload is 248320)")
     args = ap.parse_args()
-    global VOCAB
-    VOCAB = args.vocab
+    globals()["VOCAB"] = args.vocab
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":

@@ -153,7 +153,8 @@ def test_w8a8_silu_quantize_bit_exact_off_midpoints():
     xq, sx = dl.w8a8_silu_quantize_rows(gate, up)
     q_ref, sx_ref = og.silu_quantize_rows(bits(gate), bits(up))
     flags = _silu_flags(bits(gate), bits(up))
-    assert flags.mean() < 1e-3
+    # a 2^-18 band around midpoints spaced 2^-8 apart flags about 2^-9 of the elements
+    assert flags.mean() < 5e-3
     q = bits(xq)
     sxg = bits(sx)
     h_ref = nx.bf16_decode(og.silu_mul_bf16(bits(gate), bits(up)))
