@@ -22,6 +22,7 @@ from ._lib import (  # noqa: F401
     w4a16_gemv,
     w8a8_gemv,
     w8a8_proj,
+    w8a8_proj_noalloc,
     w8a8_quantize_rows,
     w8a8_silu_proj,
     w8a8_silu_quantize_rows,

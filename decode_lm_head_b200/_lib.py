@@ -47,6 +47,7 @@ _SIGNATURES = {
     "w8a8_gemv": [_P, _P, _I, _I, _P, _L, _P, _I, _P, _L, _P],
     "w8a8_proj": [_P, _P, _I, _I, _P, _L, _I, _P, _L, _P, _P, _P],
     "w8a8_silu_proj": [_P, _P, _I, _I, _P, _P, _L, _I, _P, _L, _P, _P, _P],
+    "w8a8_proj_noalloc": [_P, _P, _I, _I, _P, _L, _I, _P, _L, _P],
     "w4a16_gemv": [_P, _P, _F, _I, _I, _P, _L, _I, _P, _L, _P],
     "q8_1_quantize_rows": [_P, _L, _I, _I, _P, _P],
     "q6k_mmvq": [_P, _I, _I, _P, _I, _P, _L, _P],
@@ -217,6 +218,21 @@ def w8a8_proj(w, w_scale, x, out=None, xq_scratch=None, xscale_scratch=None, str
     xq_scratch, xscale_scratch = _w8a8_scratch(k, x.device, xq_scratch, xscale_scratch)
     _check(lib().w8a8_proj(_ptr(w), _ptr(w_scale), n, k, _ptr(x), _ld(x), rows, _ptr(out), _ld(out),
                            _ptr(xq_scratch), _ptr(xscale_scratch), _stream(stream)), "w8a8_proj")
+    return out
+
+
+def w8a8_proj_noalloc(w, w_scale, x, out=None, stream=None):
+    """w8a8_proj with the library's own fixed device scratch (no caller scratch, no allocation
+    inside the library)."""
+    _cuda(w, torch.uint8, "w", 2)
+    _cuda(w_scale, torch.float32, "w_scale", 1)
+    _cuda(x, torch.bfloat16, "x", 2)
+    n, k = w.shape
+    rows = x.shape[0]
+    if out is None:
+        out = torch.empty(rows, n, dtype=torch.bfloat16, device=x.device)
+    _check(lib().w8a8_proj_noalloc(_ptr(w), _ptr(w_scale), n, k, _ptr(x), _ld(x), rows, _ptr(out), _ld(out),
+                                   _stream(stream)), "w8a8_proj_noalloc")
     return out
 
 

@@ -152,6 +152,34 @@ DLMH_API int w8a8_silu_proj(const uint8_t* w, const float* w_scale, int n, int k
                    uint8_t* xq_scratch, float* xscale_scratch, void* stream);
 
 /* ---------------------------------------------------------------------------------------
+ * W8A8 projection that allocates nothing, not even caller scratch
+ *   Same operation, rows and results as w8a8_proj.  The quantized-activation scratch is a
+ *   fixed device array inside this library instead of a caller buffer.  The pages have no
+ *   counterpart: this entry point is this library's own addition.
+ *
+ *   Who it is for: callers that cannot call cudaMalloc.  Examples are engines whose device
+ *   memory belongs to a pre-reserved pool or to another framework's allocator, and decode
+ *   loops that cannot afford cudaMalloc's implicit device synchronization.  They still pass
+ *   w, w_scale, x and out.
+ *
+ *   Limit: k <= DLMH_NOALLOC_MAX_K (16384), else DLMH_ERR_UNSUPPORTED.  Every GPU that loads
+ *   the library holds the 2 MiB + 512 B array until the process exits.
+ *
+ *   Set-up: a device's first call looks the array's device address up
+ *   (cudaGetSymbolAddress, with that device current).  Make that first call before any
+ *   stream capture.
+ *
+ *   Sharing: all calls on a device share the one array, and it keeps the last call's codes
+ *   and scales.  Each call overwrites, before reading, every byte it uses, so nothing needs
+ *   clearing.  Calls that overlap on the GPU (concurrent streams, or several host threads)
+ *   race on the array: order them on one stream.
+ *   No cudaMalloc, cudaFree or allocating library routine is called.
+ * ------------------------------------------------------------------------------------- */
+#define DLMH_NOALLOC_MAX_K 16384
+DLMH_API int w8a8_proj_noalloc(const uint8_t* w, const float* w_scale, int n, int k, const dlmh_bf16* x,
+                               int64_t ldx, int rows, dlmh_bf16* out, int64_t ldc, void* stream);
+
+/* ---------------------------------------------------------------------------------------
  * NVFP4 W4A16 GEMV
  *   out[m, n] = bf16( g * sum_b e4m3(S[n, b]) * sum_{k in b} e2m1(W[n, k]) * x[m, k] )
  * w4a16_gemv_tiers.rs (the W4A16 tiers; more than 32 rows refused);
