@@ -13,7 +13,8 @@ import re
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libdlmh.so")
+# DLMH_LIBRARY may point at another build of the same library (for example a tuning build).
+LIB_PATH = os.environ.get("DLMH_LIBRARY") or os.path.join(_HERE, "libdlmh.so")
 HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "dlmh.h")
 
 # op ids of dlmh_plan_chunks (dlmh_op in dlmh.h)

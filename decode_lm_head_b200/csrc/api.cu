@@ -72,6 +72,8 @@ extern "C" {
 
 int dlmh_version(void) { return 100; }
 
+int dlmh_device_fault(int reset) { return dlmh::device_fault(reset); }
+
 const char* dlmh_error_string(int code) {
   switch (code) {
     case DLMH_OK: return "ok";

@@ -5,7 +5,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/dlmh.h"
+#include "dlmh.h"
 
 #if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
 #error "libdlmh is built for sm_100a only"
@@ -27,6 +27,13 @@ __device__ __forceinline__ uint4 ldg_nc(const void* p) {
   uint4 r;
   asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
   return r;
+}
+
+// 16-bit read-only load.
+__device__ __forceinline__ uint32_t ldg_u16(const void* p) {
+  uint16_t v;
+  asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
+  return v;
 }
 
 __device__ __forceinline__ uint4 lds128(uint32_t saddr) {

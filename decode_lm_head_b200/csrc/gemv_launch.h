@@ -10,6 +10,9 @@ namespace dlmh {
 // Widest row count one weight pass of `op` (a dlmh_op) serves at reduction length k, or 0
 // when even the 8-row tier does not fit on chip.  Pure function of (op, k).
 int max_tier_rows(int op, int k);
+// Fault bits recorded by bounded device waits since the last reset (0 in a healthy run);
+// reads synchronously.
+int device_fault(int reset);
 // Width (8, 16 or 32) of the narrowest compiled tier that covers `rows` (1..32).
 inline int tier_width(int rows) { return rows <= 8 ? 8 : (rows <= 16 ? 16 : 32); }
 

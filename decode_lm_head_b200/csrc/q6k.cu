@@ -26,11 +26,6 @@ constexpr int kQ6Threads = kQ6Warps * 32;
 constexpr int kQ6TileRows = 16;
 constexpr int kQ6MaxRows = 8;  // q8_1 rows per launch (one 8-column MMA tile)
 
-__device__ __forceinline__ uint32_t ldg_u16(const uint8_t* p) {
-  uint16_t v;
-  asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
-  return v;
-}
 __device__ __forceinline__ uint32_t ldg_u32_a2(const uint8_t* p) {  // 2-byte aligned 32-bit load
   return ldg_u16(p) | (ldg_u16(p + 2) << 16);
 }

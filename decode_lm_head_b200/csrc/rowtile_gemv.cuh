@@ -5,8 +5,7 @@
 //     contiguous tile range [c*T/G, (c+1)*T/G), so the per-SM load differs by at most
 //     one tile;
 //   * a tile's K is split into 64-byte "k-blocks" of every row (64 FP8 or 128 FP4 values);
-//     warp w of 16 owns k-blocks [w*nkb, (w+1)*nkb), so the CTA reads each tile as one
-//     contiguous 16-row region;
+//     warp w of 16 owns k-blocks w, w+16, w+32, ... (summed in that order);
 //   * inside a warp, lane (g = lane/4, t = lane%4) loads bytes [16t, 16t+16) of rows g and
 //     g+8 of every k-block with one 128-bit streaming load each, through a register ring
 //     that runs PF k-blocks ahead (across tile boundaries);
@@ -121,6 +120,7 @@ __device__ void stage_x_a16(const RowTileParams& p, uint8_t* xs, int rs, float* 
     float amax = 0.f;
     if (m < p.rows) {
       const uint16_t* xr = x + (int64_t)m * p.ldx;
+#pragma unroll 4
       for (int k8 = lane * 8; k8 < p.k; k8 += 32 * 8) {
         uint4 v = ldg_nc(xr + k8);
         uint32_t wv[4] = {v.x, v.y, v.z, v.w};
@@ -142,6 +142,7 @@ __device__ void stage_x_a16(const RowTileParams& p, uint8_t* xs, int rs, float* 
   // 2. convert 8-element groups
   constexpr int EL = F::kElemsPerKB / 4;   // elements owned by one lane per k-block
   const int groups_per_row = kb_total * (F::kElemsPerKB / 8);
+#pragma unroll 4
   for (int it = threadIdx.x; it < MT * groups_per_row; it += kThreads) {
     const int m = it / groups_per_row;
     const int g8 = it - m * groups_per_row;
@@ -176,6 +177,7 @@ __device__ void stage_x_a8(const RowTileParams& p, uint8_t* xs, int rs, float* r
   const uint8_t* x = static_cast<const uint8_t*>(p.x);
   if (threadIdx.x < MT) rowmul[threadIdx.x] = threadIdx.x < p.rows ? p.x_scale[threadIdx.x] : 0.f;
   const int groups_per_row = kb_total * 4;   // 16-byte groups
+#pragma unroll 4
   for (int it = threadIdx.x; it < MT * groups_per_row; it += kThreads) {
     const int m = it / groups_per_row;
     const int g16 = it - m * groups_per_row;
@@ -281,12 +283,6 @@ __global__ void __launch_bounds__(kThreads, 1) rowtile_gemv_kernel(const RowTile
   float* red = reinterpret_cast<float*>(smem + (size_t)MT * rs);
   float* rowmul = red + red_buffers<NT>() * kWarps * kTileRows * MT;
 
-  if constexpr (F::kXBytes == 2)
-    stage_x_a16<F, NT>(p, xs, rs, rowmul, kb_total);
-  else
-    stage_x_a8<F, NT>(p, xs, rs, rowmul, kb_total);
-  __syncthreads();
-
   const int ntiles = (p.n + kTileRows - 1) / kTileRows;
   const int T0 = (int)((int64_t)blockIdx.x * ntiles / gridDim.x);
   const int T1 = (int)((int64_t)(blockIdx.x + 1) * ntiles / gridDim.x);
@@ -294,32 +290,53 @@ __global__ void __launch_bounds__(kThreads, 1) rowtile_gemv_kernel(const RowTile
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
-  const int nkb = (kb_total + kWarps - 1) / kWarps;  // k-blocks per warp (uniform)
-  const int kb_first = warp * nkb;
+  const int nkb = (kb_total + kWarps - 1) / kWarps;          // k-blocks per warp (uniform)
+  // Warp w owns k-blocks w, w + 16, w + 32, ... in that order: the same split, and so the
+  // same summation order, as the streamed kernel (rowtile_tma.cuh), so that every tier of
+  // every kernel gives a row the same bits.
+  const int nvalid = max(0, min(nkb, (kb_total - warp + kWarps - 1) / kWarps));
   const int64_t wrb = p.w_row_bytes;
+  const int lane_col = warp * kKBlockBytes + 16 * t;          // byte column of the lane's first slot
+  constexpr int kSlotBytes = kWarps * kKBlockBytes;           // column step between a warp's slots
+  // bit j: slot j is inside K for this warp and the lane's 16 bytes lie inside the row
+  uint32_t colmask = 0;
+  for (int j = 0; j < nvalid; ++j)
+    if (lane_col + j * kSlotBytes < wrb) colmask |= 1u << j;
+  const int nfull = p.n / kTileRows;  // tiles whose 16 rows all exist
 
-  // ---- load side of the ring
+  // ---- load side of the ring: running pointers, no per-load index arithmetic
+  const int64_t row8 = 8 * wrb;
+  const int64_t tile_jump = kTileRows * wrb - (int64_t)nkb * kSlotBytes;
+  const uint8_t* lp = p.w + ((int64_t)T0 * kTileRows + g) * wrb + lane_col;
+  const int64_t srb = p.k / 16;  // FP4: block-scale bytes per row; a lane takes 2 per k-block
+  const int64_t s_row8 = 8 * srb;
+  const int64_t s_tile_jump = kTileRows * srb - (int64_t)nkb * kWarps * 8;
+  const uint8_t* sp = nullptr;
+  if constexpr (F::kBlockScale) sp = p.w_bscale + ((int64_t)T0 * kTileRows + g) * srb + warp * 8 + 2 * t;
   int ltile = T0, lkb = 0;
   auto issue = [&](uint4& ra, uint4& rb, uint32_t& sa, uint32_t& sb) {
     ra = make_uint4(0, 0, 0, 0);
     rb = ra;
     sa = sb = 0;
-    const int kb = kb_first + lkb;
-    const int64_t col = (int64_t)kb * kKBlockBytes + 16 * t;
-    if (ltile < T1 && col < wrb) {
+    if (ltile < T1 && ((colmask >> lkb) & 1u)) {
+      const bool full = ltile < nfull;
       const int r = ltile * kTileRows + g;
-      if (r < p.n) ra = ldg_stream(p.w + (int64_t)r * wrb + col);
-      if (r + 8 < p.n) rb = ldg_stream(p.w + (int64_t)(r + 8) * wrb + col);
-      if constexpr (F::kBlockScale) {
-        const int64_t srow = p.k / 16;
-        const int64_t sc = (int64_t)kb * 8 + 2 * t;
-        if (r < p.n) sa = *reinterpret_cast<const uint16_t*>(p.w_bscale + (int64_t)r * srow + sc);
-        if (r + 8 < p.n) sb = *reinterpret_cast<const uint16_t*>(p.w_bscale + (int64_t)(r + 8) * srow + sc);
+      if (full || r < p.n) {
+        ra = ldg_stream(lp);
+        if constexpr (F::kBlockScale) sa = ldg_u16(sp);
+      }
+      if (full || r + 8 < p.n) {
+        rb = ldg_stream(lp + row8);
+        if constexpr (F::kBlockScale) sb = ldg_u16(sp + s_row8);
       }
     }
+    lp += kSlotBytes;
+    if constexpr (F::kBlockScale) sp += kWarps * 8;
     if (++lkb == nkb) {
       lkb = 0;
       ++ltile;
+      lp += tile_jump;
+      if constexpr (F::kBlockScale) sp += s_tile_jump;
     }
   };
 
@@ -328,13 +345,31 @@ __global__ void __launch_bounds__(kThreads, 1) rowtile_gemv_kernel(const RowTile
 #pragma unroll
   for (int s = 0; s < PF; ++s) issue(bufa[s], bufb[s], bsa[s], bsb[s]);
 
+  // Stage the activation rows while the first PF k-blocks of weight are in flight.
+  if constexpr (F::kXBytes == 2)
+    stage_x_a16<F, NT>(p, xs, rs, rowmul, kb_total);
+  else
+    stage_x_a8<F, NT>(p, xs, rs, rowmul, kb_total);
+  __syncthreads();
+
+  // The reducing threads (one output each per tile) hold the row scale of their output
+  // for the current tile and fetch the next tile's one tile ahead, off the critical path.
+  const int red_rr = threadIdx.x % kTileRows, red_cc = threadIdx.x / kTileRows;
+  const bool reducer = threadIdx.x < kTileRows * MT;
+  float wscale_cur = 0.f;
+  if constexpr (!F::kBlockScale) {
+    const int row = T0 * kTileRows + red_rr;
+    if (reducer && row < p.n) wscale_cur = p.w_scale[row];
+  }
+
   float acc[NT][4];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
     for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
 
-  const uint32_t xs_lane = smem_u32(xs) + g * rs + t * 16;
+  const uint32_t xs_lane = smem_u32(xs) + g * rs + t * 16 + warp * XLayout<F>::kKBBytes;
+  uint32_t xa = xs_lane;
   int tile = T0, kb = 0, parity = 0;
 
   while (tile < T1) {
@@ -344,9 +379,7 @@ __global__ void __launch_bounds__(kThreads, 1) rowtile_gemv_kernel(const RowTile
         const uint4 ra = bufa[s], rb = bufb[s];
         const uint32_t sa = bsa[s], sb = bsb[s];
         issue(bufa[s], bufb[s], bsa[s], bsb[s]);
-        const int kbg = kb_first + kb;
-        if (kbg < kb_total) {
-          const uint32_t xa = xs_lane + kbg * XLayout<F>::kKBBytes;
+        if (kb < nvalid) {
           if constexpr (F::kBlockScale)
             kblock_w4a16<NT>(acc, ra, rb, sa, sb, xa, rs);
           else if constexpr (F::kXBytes == 1)
@@ -354,6 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1) rowtile_gemv_kernel(const RowTile
           else
             kblock_w8a16<NT>(acc, ra, rb, xa, rs);
         }
+        xa += kWarps * XLayout<F>::kKBBytes;
         if (++kb == nkb) {
           // ---- end of tile: fixed-order cross-warp reduction
           float* rb_ = red + parity * (kWarps * kTileRows * MT);
@@ -364,9 +398,15 @@ __global__ void __launch_bounds__(kThreads, 1) rowtile_gemv_kernel(const RowTile
             acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
           }
           __syncthreads();
-          for (int j = threadIdx.x; j < kTileRows * MT; j += kThreads) {
-            const int rr = j % kTileRows, cc = j / kTileRows;
+          if (reducer) {
+            const int rr = red_rr, cc = red_cc;
             const int row = tile * kTileRows + rr;
+            float wsc = 0.f;
+            if constexpr (!F::kBlockScale) {
+              wsc = wscale_cur;
+              const int nrow = row + kTileRows;
+              if (tile + 1 < T1 && nrow < p.n) wscale_cur = p.w_scale[nrow];
+            }
             if (cc < p.rows && row < p.n) {
               const int gg = rr & 7, up = rr >> 3;
               const int nt = cc >> 3, cl = cc & 7;
@@ -380,13 +420,14 @@ __global__ void __launch_bounds__(kThreads, 1) rowtile_gemv_kernel(const RowTile
               if constexpr (F::kBlockScale)
                 y = (sum * p.gscale) * rowmul[cc];
               else
-                y = (sum * p.w_scale[row]) * rowmul[cc];
+                y = (sum * wsc) * rowmul[cc];
               p.out[(int64_t)cc * p.ldc + row] = f32_to_bf16_bits(y);
             }
           }
           if constexpr (red_buffers<NT>() == 1) __syncthreads();
           else parity ^= 1;
           kb = 0;
+          xa = xs_lane;
           ++tile;
         }
       }

@@ -243,6 +243,13 @@ typedef enum dlmh_op {
  * passes are needed.  Arrays may be NULL when cap == 0 (count only). */
 DLMH_API int dlmh_plan_chunks(int op, int rows, int k, int* offsets, int* counts, int* tiers, int cap);
 
+/* Fault bits recorded on the current device by the kernels' bounded waits (a wait for a
+ * shared-memory stage that did not complete in time; the kernel then finishes without
+ * hanging and its output is not valid).  0 in a healthy run.  Synchronizes the device;
+ * reset != 0 clears the bits.  Returns DLMH_ERR_CUDA if the device cannot be read.
+ * (Library diagnostic, no counterpart on the pages.) */
+DLMH_API int dlmh_device_fault(int reset);
+
 /* Static description of a status code (never NULL). */
 DLMH_API const char* dlmh_error_string(int code);
 

@@ -53,7 +53,7 @@ def test_w8a16_tiny_config_all_rows():
         assert np.array_equal(outs[m], outs[4][:m]), f"row invariance M={m} vs 4"
 
 
-@pytest.mark.parametrize("n,k", [(1000, 1040), (37, 5120), (4099, 2048)])
+@pytest.mark.parametrize("n,k", [(1000, 1040), (37, 5120), (4099, 2048), (1000, 6144)])
 def test_w8a16_ragged_shapes_and_tiers(n, k):
     w = synth.fp8_weight(n, k, 5, DEV)
     s = synth.row_scales(n, 5, DEV)
@@ -167,7 +167,7 @@ def test_w8a8_silu_quantize_bit_exact_off_midpoints():
         assert np.array_equal(q[m][ok], q_ref[m][ok]), f"row {m} codes"
 
 
-@pytest.mark.parametrize("n,k", [(1000, 1024), (4096, 14336)])
+@pytest.mark.parametrize("n,k", [(1000, 1024), (1000, 5120), (4096, 14336)])
 def test_w8a8_gemv_and_proj(n, k):
     w = synth.fp8_weight(n, k, 8, DEV)
     s = synth.row_scales(n, 8, DEV)
@@ -205,7 +205,7 @@ def test_w8a8_silu_proj_down_projection():
 # ---------------------------------------------------------------------------
 
 
-@pytest.mark.parametrize("n,k", [(2000, 4096), (77, 1024)])
+@pytest.mark.parametrize("n,k", [(2000, 4096), (77, 1024), (300, 1152)])
 def test_w4a16_tiers(n, k):
     wp, ws, gl = synth.nvfp4_weight(n, k, 10, DEV)
     x = synth.bf16_rows(32, k, 10, DEV)
