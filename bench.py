@@ -63,7 +63,7 @@ def measured_peaks():
 
 def kernel_source_hash():
     h = hashlib.sha256()
-    for f in ("rowtile_gemv.cuh", "gemv_kernels.cu", "dlmh_common.cuh"):
+    for f in ("rowtile_gemv.cuh", "rowtile_tma.cuh", "gemv_kernels.cu", "dlmh_common.cuh"):
         with open(os.path.join(ROOT, "decode_lm_head_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -238,6 +238,106 @@ def run_reference(args):
 # ---------------------------------------------------------------------------------------
 
 
+def time_calls(fns, reps, stream):
+    """Median device time (us) of each callable, by CUDA events on `stream`; each callable is
+    replayed `reps` times back to back (its inputs rotate inside the callable)."""
+    out = []
+    for fn in fns:
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        out.append(a.elapsed_time(b) * 1e3 / reps)
+    return out
+
+
+def other_formats(dev, stream, peak):
+    """Weight GB/s of the other hot-path formats (secondary measurements, same protocol:
+    inputs resident, weights rotated through enough copies to exceed the 126 MB L2)."""
+    import decode_lm_head_b200 as dl
+    from decode_lm_head_b200 import synth
+
+    res = {}
+
+    def rotating(make, nbytes):
+        copies = max(1, -(-400_000_000 // nbytes))  # >= 400 MB of distinct weights
+        return [make(i) for i in range(copies)]
+
+    def entry(name, shape, wbytes, calls, rows_list):
+        per = {}
+        for m, fn in zip(rows_list, calls):
+            us = time_calls([fn], 20, stream)[0]
+            gbs = wbytes / (us * 1e-6) / 1e9
+            per[str(m)] = {"us": round(us, 2), "weight_gbs": round(gbs, 1), "frac_of_copy_peak": round(gbs / peak, 3)}
+        res[name] = {"shape": shape, "weight_bytes": wbytes, "per_m": per}
+
+    # W8A8 on the FP8 head (one pass per <= 32-row tier in this build)
+    n, k = VOCAB, HIDDEN
+    w = synth.fp8_weight(n, k, 2, dev)
+    s_ = synth.row_scales(n, 2, dev)
+    x = synth.bf16_rows(128, k, 2, dev, std=0.5)
+    xq = torch.empty(128 * k, dtype=torch.uint8, device=dev)
+    xs = torch.empty(128, dtype=torch.float32, device=dev)
+    outs = torch.empty(128, n, dtype=torch.bfloat16, device=dev)
+    rows_list = [1, 16, 32, 128]
+    calls = [(lambda m=m: dl.w8a8_proj(w, s_, x[:m], out=outs[:m], xq_scratch=xq, xscale_scratch=xs, stream=stream))
+             for m in rows_list]
+    entry("w8a8_head", f"{n}x{k}", n * k + 4 * n, calls, rows_list)
+    del w
+
+    # W8A8 FFN down projection from bf16(silu(gate)*up)
+    n, k = 4096, 14336
+    ws = rotating(lambda i: (synth.fp8_weight(n, k, 10 + i, dev), synth.row_scales(n, 10 + i, dev)), n * k)
+    gate = synth.bf16_rows(128, k, 3, dev, tensor_id=4)
+    up = synth.bf16_rows(128, k, 3, dev, tensor_id=5)
+    xq = torch.empty(128 * k, dtype=torch.uint8, device=dev)
+    outd = torch.empty(128, n, dtype=torch.bfloat16, device=dev)
+    ctr = [0]
+
+    def down(m):
+        w_, s2 = ws[ctr[0] % len(ws)]
+        ctr[0] += 1
+        dl.w8a8_silu_proj(w_, s2, gate[:m], up[:m], out=outd[:m], xq_scratch=xq, xscale_scratch=xs, stream=stream)
+
+    rows_list = [1, 16, 128]
+    entry("w8a8_silu_down", f"{n}x{k}", n * k + 4 * n, [(lambda m=m: down(m)) for m in rows_list], rows_list)
+    del ws
+
+    # NVFP4 W4A16
+    n, k = 14336, 4096
+    wf = rotating(lambda i: synth.nvfp4_weight(n, k, 20 + i, dev), n * k // 2)
+    xf = synth.bf16_rows(32, k, 4, dev)
+    outf = torch.empty(32, n, dtype=torch.bfloat16, device=dev)
+
+    def fp4(m):
+        wp, sc, gl = wf[ctr[0] % len(wf)]
+        ctr[0] += 1
+        dl.w4a16_gemv(wp, sc, gl, xf[:m], out=outf[:m], stream=stream)
+
+    rows_list = [1, 4, 8, 16, 32]
+    entry("nvfp4_w4a16", f"{n}x{k}", n * k // 2 + n * k // 16, [(lambda m=m: fp4(m)) for m in rows_list], rows_list)
+    del wf
+
+    # Q6_K head
+    n, k = 129280, 7168
+    blocks = synth.q6k_blocks(n, k, 4, dev)
+    xk = synth.bf16_rows(64, k, 4, dev)
+    q8s = torch.empty(8 * (k // 32) * 36, dtype=torch.uint8, device=dev)
+    outk = torch.empty(64, n, dtype=torch.bfloat16, device=dev)
+    rows_list = [1, 8, 16, 64]
+    calls = [(lambda m=m: dl.q6k_lm_head(blocks, xk[:m], out=outk[:m], q8_scratch=q8s, stream=stream))
+             for m in rows_list]
+    entry("q6k_head", f"{n}x{k}", n * (k // 256) * 210, calls, rows_list)
+    del blocks
+    torch.cuda.synchronize()
+    return res
+
+
 def run_ours(args):
     world, rank, local = dist_setup(args)
     import decode_lm_head_b200 as dl
@@ -318,6 +418,10 @@ def run_ours(args):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
     e2e_value = world * args.steps * step_bytes / (e2e_ms * 1e-3) / 1e9
 
+    formats = None
+    if args.all_formats:
+        formats = other_formats(dev, stream, measured_peaks()[0])
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         gbs, dt, desc = oracle_sample()
@@ -349,6 +453,8 @@ def run_ours(args):
             "clocks": clocks,
             "cpu_baseline": cpu,
         }
+        if formats is not None:
+            line["formats"] = formats
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
@@ -363,6 +469,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--all-formats", action="store_true",
+                    help="also time W8A8 (head, SiLU down), NVFP4 and Q6_K (extra 'formats' key)")
     ap.add_argument("--vocab", type=int, default=248320,
                     help="head rows; smaller values only for profiling captures (the workload is 248320)")
     args = ap.parse_args()
