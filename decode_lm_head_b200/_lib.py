@@ -54,6 +54,7 @@ _SIGNATURES = {
     "q6k_mmvq": [_P, _I, _I, _P, _I, _P, _L, _P],
     "q6k_lm_head": [_P, _I, _I, _P, _L, _I, _P, _L, _P, _P],
     "dlmh_plan_chunks": [_I, _I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I), _I],
+    "dlmh_device_fault": [_I],
     "dlmh_version": [],
 }
 
@@ -89,6 +90,14 @@ def error_string(code):
 
 def version():
     return lib().dlmh_version()
+
+
+def device_fault(reset=False):
+    """Fault bits of the kernels' bounded waits on the current device (0 when healthy)."""
+    rc = lib().dlmh_device_fault(1 if reset else 0)
+    if rc < 0:
+        raise DlmhError(rc, "dlmh_device_fault")
+    return rc
 
 
 def _check(rc, what):

@@ -52,7 +52,8 @@ int pass_rows(int op, int k) {
       const int t = dlmh::max_tier_rows(DLMH_OP_W8A16, k);
       return t >= DLMH_W8A16_CHUNK_ROWS ? DLMH_W8A16_CHUNK_ROWS : 0;
     }
-    case DLMH_OP_W8A8: return dlmh::max_tier_rows(DLMH_OP_W8A8, k);
+    case DLMH_OP_W8A8:
+      return dlmh::w8a8_umma_supported(k) ? DLMH_W8A8_MAX_ROWS : dlmh::max_tier_rows(DLMH_OP_W8A8, k);
     case DLMH_OP_W4A16: return dlmh::max_tier_rows(DLMH_OP_W4A16, k);
     case DLMH_OP_Q6K: return DLMH_Q6K_CHUNK_ROWS;
     default: return 0;
@@ -102,7 +103,12 @@ int dlmh_plan_chunks(int op, int rows, int k, int* offsets, int* counts, int* ti
       if (!offsets || !counts || !tiers) return DLMH_ERR_NULL;
       offsets[nchunks] = done;
       counts[nchunks] = m;
-      tiers[nchunks] = op == DLMH_OP_Q6K ? DLMH_Q6K_CHUNK_ROWS : dlmh::tier_width(m);
+      if (op == DLMH_OP_Q6K)
+        tiers[nchunks] = DLMH_Q6K_CHUNK_ROWS;
+      else if (op == DLMH_OP_W8A8 && dlmh::w8a8_umma_supported(k))
+        tiers[nchunks] = (m + 15) / 16 * 16;  // tensor-core tier: MMA N = rows rounded up to 16
+      else
+        tiers[nchunks] = dlmh::tier_width(m);
     }
     ++nchunks;
     done += m;
@@ -174,8 +180,12 @@ int w8a8_gemv(const uint8_t* w, const float* w_scale, int n, int k, const uint8_
   if (width <= 0) return DLMH_ERR_UNSUPPORTED;
   for (int done = 0; done < rows;) {
     const int m = rows - done < width ? rows - done : width;
-    DLMH_TRY(dlmh::w8a8_gemv_pass(w, w_scale, n, k, xq + (int64_t)done * ldq, ldq, x_scale + done, m,
-                                  out + (int64_t)done * ldc, ldc, as_stream(stream)));
+    if (dlmh::w8a8_umma_supported(k))
+      DLMH_TRY(dlmh::w8a8_umma_pass(w, w_scale, n, k, xq + (int64_t)done * ldq, ldq, x_scale + done, m,
+                                    out + (int64_t)done * ldc, ldc, as_stream(stream)));
+    else
+      DLMH_TRY(dlmh::w8a8_gemv_pass(w, w_scale, n, k, xq + (int64_t)done * ldq, ldq, x_scale + done, m,
+                                    out + (int64_t)done * ldc, ldc, as_stream(stream)));
     done += m;
   }
   return DLMH_OK;

@@ -242,7 +242,9 @@ int device_fault(int reset) {
     const int zero = 0;
     if (cudaMemcpyToSymbol(dlmh_fault_word, &zero, sizeof(int)) != cudaSuccess) return DLMH_ERR_CUDA;
   }
-  return v;
+  const int u = umma_fault(reset);
+  if (u < 0) return u;
+  return v | (u << 8);
 }
 
 int max_tier_rows(int op, int k) {

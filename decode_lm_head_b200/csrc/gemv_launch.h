@@ -20,6 +20,14 @@ int w8a16_pass(const uint8_t* w, const float* w_scale, int n, int k, const uint1
                uint16_t* out, int64_t ldc, cudaStream_t s);
 int w8a8_gemv_pass(const uint8_t* w, const float* w_scale, int n, int k, const uint8_t* xq, int64_t ldq,
                    const float* x_scale, int rows, uint16_t* out, int64_t ldc, cudaStream_t s);
+// Tensor-core W8A8 pass (tcgen05, TMA-fed): one weight pass for 1..128 rows.  Taken for every
+// row count whenever w8a8_umma_supported(k) holds (a pure function of k).
+bool w8a8_umma_supported(int k);
+int w8a8_umma_pass(const uint8_t* w, const float* w_scale, int n, int k, const uint8_t* xq, int64_t ldq,
+                   const float* x_scale, int rows, uint16_t* out, int64_t ldc, cudaStream_t s);
+// Fault bits of the tensor-core kernel's bounded waits (read synchronously).
+int umma_fault(int reset);
+
 int w4a16_pass(const uint8_t* wp, const uint8_t* wbs, float g, int n, int k, const uint16_t* x, int64_t ldx, int rows,
                uint16_t* out, int64_t ldc, cudaStream_t s);
 

@@ -33,15 +33,21 @@ def test_error_strings_and_version():
     assert dl.error_string(-99) == "unknown status"
 
 
-@pytest.mark.parametrize("opid,k,width", [(dl.OP_W8A16, 5120, 16), (dl.OP_W8A16, 1024, 16), (dl.OP_W8A8, 5120, 32),
-                                           (dl.OP_W8A8, 14336, 8), (dl.OP_W4A16, 4096, 16), (dl.OP_Q6K, 7168, 8)])
+@pytest.mark.parametrize("opid,k,width", [(dl.OP_W8A16, 5120, 16), (dl.OP_W8A16, 1024, 16), (dl.OP_W8A8, 5120, 128),
+                                           (dl.OP_W8A8, 14336, 128), (dl.OP_W8A8, 1040, 32), (dl.OP_W4A16, 4096, 16),
+                                           (dl.OP_Q6K, 7168, 8)])
 def test_plan_matches_oracle_rules(opid, k, width):
     cap = 32 if opid == dl.OP_W4A16 else 300
     for rows in range(0, cap + 1):
         plan = dl.plan_chunks(opid, rows, k)
         ref = op.chunk_plan(rows, width)
         assert [(o, c) for o, c, _ in plan] == ref
-        widths = [8] if opid == dl.OP_Q6K else [8, 16, 32]
+        if opid == dl.OP_Q6K:
+            widths = [8]
+        elif opid == dl.OP_W8A8 and k % 128 == 0:
+            widths = list(range(16, 129, 16))  # tensor-core tier: MMA N in steps of 16
+        else:
+            widths = [8, 16, 32]
         for _, c, tier in plan:
             i = op.select_tier(c, widths, [True] * len(widths))
             assert tier == widths[i]

@@ -185,6 +185,28 @@ def test_w8a8_gemv_and_proj(n, k):
     assert np.array_equal(direct, full[:128])
 
 
+@pytest.mark.parametrize("n,k", [(300, 1152), (130, 128), (9000, 384)])
+def test_w8a8_tensor_core_tier_ragged(n, k):
+    # k % 128 == 0 takes the tensor-core tier for every row count: ragged last 128-row tile,
+    # an odd number of 128-byte chunks (a half-empty last stage), strided rows and outputs
+    w = synth.fp8_weight(n, k, 11, DEV)
+    s = synth.row_scales(n, 11, DEV)
+    x = synth.bf16_rows(128, k, 11, DEV)
+    xq_full = torch.zeros(128, k + 48, dtype=torch.uint8, device=DEV)
+    xq, sx = dl.w8a8_quantize_rows(x)
+    xq_full[:, :k] = xq
+    out_full = torch.full((128, n + 24), 0x7FC0, dtype=torch.int16, device=DEV).view(torch.bfloat16)
+    dl.w8a8_gemv(w, s, xq_full[:, :k], sx, out=out_full[:, :n])
+    got = bits(out_full[:, :n])
+    ref = og.w8a8_gemv(bits(w), bits(s), bits(xq), bits(sx))
+    assert_bf16_close(got, ref, f"w8a8 tensor-core tier n={n} k={k}")
+    assert np.all(bits(out_full[:, n:]) == 0x7FC0), "wrote past n"
+    for m in (1, 15, 16, 17, 48, 100, 127):
+        part = bits(dl.w8a8_gemv(w, s, xq[:m], sx[:m]))
+        assert np.array_equal(part, got[:m]), f"row invariance M={m}"
+    assert dl.device_fault(reset=True) == 0
+
+
 def test_w8a8_silu_proj_down_projection():
     n, k = 4096, 14336
     w = synth.fp8_weight(n, k, 9, DEV)
