@@ -49,6 +49,7 @@ int check_out(const void* out, int64_t ldc, int n) {
 int pass_rows(int op, int k) {
   switch (op) {
     case DLMH_OP_W8A16: {
+      if (dlmh::w8a16_umma_supported(k)) return 128;
       const int t = dlmh::max_tier_rows(DLMH_OP_W8A16, k);
       return t >= DLMH_W8A16_CHUNK_ROWS ? DLMH_W8A16_CHUNK_ROWS : 0;
     }
@@ -105,7 +106,8 @@ int dlmh_plan_chunks(int op, int rows, int k, int* offsets, int* counts, int* ti
       counts[nchunks] = m;
       if (op == DLMH_OP_Q6K)
         tiers[nchunks] = DLMH_Q6K_CHUNK_ROWS;
-      else if (op == DLMH_OP_W8A8 && dlmh::w8a8_umma_supported(k))
+      else if ((op == DLMH_OP_W8A8 && dlmh::w8a8_umma_supported(k)) ||
+               (op == DLMH_OP_W8A16 && dlmh::w8a16_umma_supported(k)))
         tiers[nchunks] = (m + 15) / 16 * 16;  // tensor-core tier: MMA N = rows rounded up to 16
       else
         tiers[nchunks] = dlmh::tier_width(m);
@@ -126,6 +128,8 @@ int lm_head_fp8_w8a16(const uint8_t* w, const float* w_scale, int n, int k, cons
   if (!aligned16(w)) return DLMH_ERR_ALIGN;
   DLMH_TRY(check_bf16_in(x, ldx, k));
   DLMH_TRY(check_out(out, ldc, n));
+  if (dlmh::w8a16_umma_supported(k))
+    return dlmh::w8a16_umma_run(w, w_scale, n, k, x, ldx, rows, out, ldc, as_stream(stream));
   const int width = pass_rows(DLMH_OP_W8A16, k);
   if (width <= 0) return DLMH_ERR_UNSUPPORTED;
   for (int done = 0; done < rows;) {

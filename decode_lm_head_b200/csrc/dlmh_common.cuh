@@ -57,6 +57,14 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t v) {
   return r;
 }
 
+// Two f32 values -> two E4M3 codes (round-to-nearest-even, saturating to +-448);
+// `lo` lands in the low byte.
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
 // Two E2M1 codes in one byte (low nibble = element 0) -> f16x2 (exact).
 __device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte_in_low8) {
   uint32_t r;

@@ -28,6 +28,14 @@ int w8a8_umma_pass(const uint8_t* w, const float* w_scale, int n, int k, const u
 // Fault bits of the tensor-core kernel's bounded waits (read synchronously).
 int umma_fault(int reset);
 
+// Tensor-core W8A16 (the same kernel; activations split into two exact E4M3 terms): one
+// weight pass per 128 rows, taken for every row count whenever w8a16_umma_supported(k)
+// holds.  Runs its own row loop; the activation codes live in a library-owned stream-ordered
+// pool.
+bool w8a16_umma_supported(int k);
+int w8a16_umma_run(const uint8_t* w, const float* w_scale, int n, int k, const uint16_t* x, int64_t ldx, int rows,
+                   uint16_t* out, int64_t ldc, cudaStream_t s);
+
 int w4a16_pass(const uint8_t* wp, const uint8_t* wbs, float g, int n, int k, const uint16_t* x, int64_t ldx, int rows,
                uint16_t* out, int64_t ldc, cudaStream_t s);
 

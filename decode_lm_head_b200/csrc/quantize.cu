@@ -9,14 +9,6 @@ namespace {
 
 constexpr int kQThreads = 256;
 
-// Two f32 values -> two E4M3 codes (round-to-nearest-even, saturating to +-448);
-// `lo` lands in the low byte.
-__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
-  uint16_t r;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-
 __device__ __forceinline__ float block_max(float v, float* red) {
   v = warp_max(v);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;

@@ -1,0 +1,401 @@
+// E4M3-weight GEMV on the 5th-generation tensor cores: TMA -> shared memory -> tcgen05.mma
+// -> TMEM -> registers.  One weight pass serves up to 128 activation rows, for both
+//
+//   W8A8:   out[m, n] = bf16( s[n] * sx[m] * sum_k e4m3(W[n, k]) * e4m3(xq[m, k]) )
+//   W8A16:  out[m, n] = bf16( s[n] * 2^-e[m] * sum_k e4m3(W[n, k]) * (hi[m, k] + lo[m, k] / 16) )
+//
+// where, for W8A16, x'[m, :] = x[m, :] * 2^e[m] (max|x'| in [2^7, 2^8)) is split into two
+// E4M3 terms hi = e4m3(x'), lo = e4m3(16 (x' - hi)).  A BF16 value has 8 significant bits;
+// rounding it to E4M3's 4 leaves a residual of at most 4 bits, so hi + lo/16 == x' exactly
+// whenever |x'| >= 2^-6 (every element within 2^-13 of the row maximum); below that the
+// error is at most 2^-14 in x' units.  The two terms are the B operand's first and second
+// npad columns, so the weights stay E4M3 in the A operand: the tensor core takes an M=128,
+// K=32-byte instruction in the same ~142 clocks whatever N <= 256, i.e. it consumes A at
+// ~29 bytes/clock/SM, above the HBM share of an SM (~24); a 16-bit A operand would halve
+// the weight rate and make the kernel MMA-bound.
+//
+// Swap-AB: the weight is the MMA's A operand (M = 128 weight rows per tile) and the
+// activation codes are its B operand (N = rows rounded up to 16, twice that for W8A16).
+// Both operands are E4M3 bytes used as stored (kind::f8f6f4, f32 accumulation in TMEM).
+//
+// Operand staging: both matrices are read through 3-D tensor maps over [rows][K] bytes,
+// dims {128 (k within a chunk), rows, K/128 (chunk)}: one TMA load brings BM rows x KC
+// chunks, i.e. KC*128 contiguous bytes of every row, and writes shared memory as
+// [chunk][row][128 B] with the 128-byte swizzle, which is exactly the K-major SWIZZLE_128B
+// operand layout the MMA reads (8-row groups 1024 bytes apart).
+//
+// Roles (192 threads, one CTA per SM, persistent over a contiguous range of 128-row tiles):
+//   warp 0: producer (one thread issues the A and B tensor loads of every stage);
+//   warp 1: allocates tensor memory, then one thread issues the MMAs (4 per 128-byte
+//           chunk, K = 32 each) and commits each stage back to the producer and each
+//           finished tile to the epilogue;
+//   warps 2-5: epilogue -- tcgen05.ld the accumulator (warp w reads TMEM lanes 32*(w%4)...),
+//           apply the row and activation scales, round to BF16, coalesced stores.
+// Two accumulators (2 x N columns of TMEM) let the epilogue of one tile overlap the MMAs of
+// the next.  Every mbarrier wait is bounded and records a fault bit instead of hanging;
+// the allocating warp always frees its tensor memory before exit.
+#include "gemv_launch.h"
+#include "umma_common.cuh"
+
+namespace dlmh {
+namespace {
+
+using namespace umma;
+
+constexpr int kUmmaThreads = 192;
+constexpr int kKC = 2;  // 128-byte K-chunks per stage
+constexpr int kChunkBytesA = kBM * 128;
+constexpr int kMaxUStages = 6;
+
+static __device__ int umma_fault_word = 0;  // 1: producer, 2: MMA (stage), 4: MMA (tmem), 8: epilogue
+
+__device__ __forceinline__ void umma_f8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, int accum) {
+  asm volatile(
+      "{ .reg .pred p; setp.ne.b32 p, %4, 0; "
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p; }" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
+      : "memory");
+}
+
+struct UmmaParams {
+  int n, k, rows, npad;  // npad: rows rounded up to 16
+  int nb;                // MMA N = B rows: npad (W8A8) or 2 npad (W8A16 hi | lo)
+  int split;             // 1: W8A16 two-term epilogue
+  const float* w_scale;
+  const float* x_scale;  // sx[m] (W8A8) or 2^-e[m] (W8A16)
+  uint16_t* out;
+  int64_t ldc;
+  int ns;                // ring stages
+  int stage_bytes;       // A + B bytes of one stage
+};
+
+__global__ void __launch_bounds__(kUmmaThreads, 1)
+    umma_f8_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x,
+                     const UmmaParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t bar_full[kMaxUStages], bar_empty[kMaxUStages], bar_tfull[2], bar_tempty[2];
+  __shared__ uint32_t s_tmem;
+
+  const int ntiles = (p.n + kBM - 1) / kBM;
+  const int T0 = (int)((int64_t)blockIdx.x * ntiles / gridDim.x);
+  const int T1 = (int)((int64_t)(blockIdx.x + 1) * ntiles / gridDim.x);
+  if (T0 >= T1) return;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kchunks = p.k / 128;
+  const int spt = (kchunks + kKC - 1) / kKC;  // stages per tile
+  const int nstages = (T1 - T0) * spt;
+  const uint32_t ring_u32 = smem_u32(ring);
+  const uint32_t full0 = smem_u32(bar_full), empty0 = smem_u32(bar_empty);
+  const uint32_t tfull0 = smem_u32(bar_tfull), tempty0 = smem_u32(bar_tempty);
+  const int a_bytes = kKC * kChunkBytesA;
+  const int b_chunk = p.nb * 128;
+  const uint32_t tmem_cols = (uint32_t)tmem_cols_for(2 * p.nb);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < p.ns; ++i) {
+      bar_init(full0 + 8u * i, 1);
+      bar_init(empty0 + 8u * i, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      bar_init(tfull0 + 8u * i, 1);
+      bar_init(tempty0 + 8u * i, 4);  // the four epilogue warps
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) tmem_alloc(smem_u32(&s_tmem), tmem_cols);
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem_base = s_tmem;
+
+  if (warp == 0) {
+    // ---------------- producer
+    if (lane == 0) {
+      int slot = 0, phase = 0;
+      for (int s = 0; s < nstages; ++s) {
+        const int tile = T0 + s / spt, j = s % spt;
+        if (s >= p.ns && !wait(empty0 + 8u * slot, phase ^ 1)) atomicOr(&umma_fault_word, 1);
+        const uint32_t st = ring_u32 + slot * p.stage_bytes;
+        // the full box always lands (rows past n, rows past `rows` and a chunk past K are
+        // zero-filled), so every stage completes exactly stage_bytes
+        expect_tx(full0 + 8u * slot, (uint32_t)p.stage_bytes);
+        // A: weight rows [tile*128, +128) x chunks [j*KC, j*KC + KC); B: all activation rows
+        tma_load_3d(st, &map_w, 0, tile * kBM, j * kKC, full0 + 8u * slot);
+        tma_load_3d(st + a_bytes, &map_x, 0, 0, j * kKC, full0 + 8u * slot);
+        if (++slot == p.ns) {
+          slot = 0;
+          phase ^= 1;
+        }
+      }
+      // no copy may still be landing when the CTA exits: wait (bounded) for the last
+      // phase of every slot (already complete in a healthy run, where the MMAs consumed it)
+      for (int s = nstages - 1; s >= 0 && s >= nstages - p.ns; --s)
+        if (!wait(full0 + 8u * (s % p.ns), (s / p.ns) & 1)) atomicOr(&umma_fault_word, 1);
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_m128(p.nb);
+      int slot = 0, phase = 0;
+      for (int i = 0; T0 + i < T1; ++i) {
+        const int acc = i & 1;
+        if (i >= 2 && !wait(tempty0 + 8u * acc, ((i - 2) >> 1) & 1)) atomicOr(&umma_fault_word, 4);
+        fence_after();
+        const uint32_t tmem_d = tmem_base + (uint32_t)acc * (tmem_cols / 2);
+        for (int j = 0; j < spt; ++j) {
+          if (!wait(full0 + 8u * slot, phase)) atomicOr(&umma_fault_word, 2);
+          fence_after();
+          const int nch = min(kKC, kchunks - j * kKC);
+          const uint32_t st = ring_u32 + slot * p.stage_bytes;
+          for (int c = 0; c < nch; ++c) {
+            const uint32_t a0 = st + c * kChunkBytesA;
+            const uint32_t b0 = st + a_bytes + c * b_chunk;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)  // K = 32 bytes per MMA
+              umma_f8(tmem_d, desc_sw128(a0 + kk * 32), desc_sw128(b0 + kk * 32), idesc,
+                      (j | c | kk) != 0);
+          }
+          commit(empty0 + 8u * slot);  // the stage is free once these MMAs have read it
+          if (++slot == p.ns) {
+            slot = 0;
+            phase ^= 1;
+          }
+        }
+        commit(tfull0 + 8u * acc);  // the accumulator is complete
+      }
+    }
+  } else {
+    // ---------------- epilogue (warps 2..5)
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int lane_row = q * 32 + lane;
+    for (int i = 0; T0 + i < T1; ++i) {
+      const int tile = T0 + i, acc = i & 1;
+      if (!wait(tfull0 + 8u * acc, (i >> 1) & 1)) atomicOr(&umma_fault_word, 8);
+      fence_after();
+      const int row = tile * kBM + lane_row;
+      const float s = row < p.n ? p.w_scale[row] : 0.f;
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)acc * (tmem_cols / 2);
+      for (int c0 = 0; c0 < p.npad; c0 += 16) {
+        uint32_t v[16];
+        tmem_ld16(taddr + (uint32_t)c0, v);
+        if (p.split) {  // y = hi-term sum + lo-term sum / 16
+          uint32_t u[16];
+          tmem_ld16(taddr + (uint32_t)(p.npad + c0), u);
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj)
+            v[jj] = __float_as_uint(fmaf(__uint_as_float(u[jj]), 0.0625f, __uint_as_float(v[jj])));
+        }
+        if (row < p.n) {
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) {
+            const int m = c0 + jj;
+            if (m < p.rows) {
+              const float y = (__uint_as_float(v[jj]) * s) * p.x_scale[m];
+              p.out[(int64_t)m * p.ldc + row] = f32_to_bf16_bits(y);
+            }
+          }
+        }
+      }
+      fence_before();
+      __syncwarp();
+      if (lane == 0) arrive(tempty0 + 8u * acc);
+    }
+  }
+
+  fence_before();
+  __syncthreads();
+  fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem_base, tmem_cols);
+  }
+}
+
+constexpr size_t kUmmaSmemLimit = 232448 - 2048;
+
+// Per-row exponent e with max|x| * 2^e in [2^7, 2^8), clamped so that 2^e and 2^-e are
+// normal f32 values (rows whose maximum is below 2^-119 lose precision; zero rows give 0).
+__device__ __forceinline__ int e4m3_split_exponent(float amax) {
+  if (!(amax > 0.f)) return 0;
+  const uint32_t b = __float_as_uint(amax);
+  const int field = (int)((b >> 23) & 0xff);
+  const int E = field != 0 ? field - 127 : (31 - __clz((int)(b & 0x7fffff))) - 149;  // amax in [2^E, 2^(E+1))
+  return max(-126, min(126, 7 - E));
+}
+
+// W8A16 activation split: CTA m writes E4M3 rows codes[m] = hi(x'[m]) and codes[npad + m] =
+// lo(x'[m]) (zero rows for m >= rows) and x_mul[m] = 2^-e[m].  k a multiple of 8, x
+// 16-byte aligned with ldx a multiple of 8.
+__global__ void __launch_bounds__(256) w8a16_split_kernel(const uint16_t* __restrict__ x, int64_t ldx, int rows,
+                                                          int k, int npad, uint8_t* __restrict__ codes,
+                                                          float* __restrict__ x_mul) {
+  __shared__ float s_red[8];
+  const int m = blockIdx.x;
+  uint8_t* hi_row = codes + (int64_t)m * k;
+  uint8_t* lo_row = codes + (int64_t)(npad + m) * k;
+  if (m >= rows) {
+    for (int k8 = threadIdx.x * 8; k8 < k; k8 += 256 * 8) {
+      *reinterpret_cast<uint2*>(hi_row + k8) = make_uint2(0, 0);
+      *reinterpret_cast<uint2*>(lo_row + k8) = make_uint2(0, 0);
+    }
+    if (threadIdx.x == 0) x_mul[m] = 0.f;
+    return;
+  }
+  const uint16_t* xr = x + (int64_t)m * ldx;
+  float amax = 0.f;
+  for (int k8 = threadIdx.x * 8; k8 < k; k8 += 256 * 8) {
+    const uint4 v = ldg_nc(xr + k8);
+    const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      amax = fmaxf(amax, fabsf(bf16_bits_to_f32(wv[i] & 0xffffu)));
+      amax = fmaxf(amax, fabsf(bf16_bits_to_f32(wv[i] >> 16)));
+    }
+  }
+  amax = warp_max(amax);
+  if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  amax = s_red[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) amax = fmaxf(amax, s_red[i]);
+  const int e = e4m3_split_exponent(amax);
+  const float mul = __int_as_float((127 + e) << 23);
+  if (threadIdx.x == 0) x_mul[m] = __int_as_float((127 - e) << 23);
+  for (int k8 = threadIdx.x * 8; k8 < k; k8 += 256 * 8) {
+    const uint4 v = ldg_nc(xr + k8);
+    const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+    uint32_t hi[2] = {0, 0}, lo[2] = {0, 0};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {  // elements 2i, 2i+1 of this 8-element group
+      const float a = bf16_bits_to_f32(wv[i] & 0xffffu) * mul;  // exact (power of two)
+      const float b = bf16_bits_to_f32(wv[i] >> 16) * mul;
+      const uint32_t h2 = f32x2_to_e4m3x2(a, b);
+      const uint32_t hf = e4m3x2_to_f16x2((uint16_t)h2);
+      const float ra = a - f16_bits_to_f32(hf & 0xffffu);  // exact residual
+      const float rb = b - f16_bits_to_f32(hf >> 16);
+      const uint32_t l2 = f32x2_to_e4m3x2(ra * 16.f, rb * 16.f);
+      hi[i >> 1] |= h2 << (16 * (i & 1));
+      lo[i >> 1] |= l2 << (16 * (i & 1));
+    }
+    *reinterpret_cast<uint2*>(hi_row + k8) = make_uint2(hi[0], hi[1]);
+    *reinterpret_cast<uint2*>(lo_row + k8) = make_uint2(lo[0], lo[1]);
+  }
+}
+
+int launch_umma_f8(const uint8_t* w, const float* w_scale, int n, int k, const uint8_t* b_codes, int64_t ldb,
+                   int b_rows, const float* x_scale, int rows, int split, uint16_t* out, int64_t ldc, cudaStream_t s) {
+  const DeviceInfo di = device_info();
+  if (di.sms <= 0) return DLMH_ERR_CUDA;
+  UmmaParams p{};
+  p.n = n;
+  p.k = k;
+  p.rows = rows;
+  p.npad = (rows + 15) / 16 * 16;
+  p.nb = split ? 2 * p.npad : p.npad;
+  p.split = split;
+  p.w_scale = w_scale;
+  p.x_scale = x_scale;
+  p.out = out;
+  p.ldc = ldc;
+  p.stage_bytes = kKC * (kChunkBytesA + p.nb * 128);
+  int ns = (int)(kUmmaSmemLimit / (size_t)p.stage_bytes);
+  if (ns > kMaxUStages) ns = kMaxUStages;
+  if (ns < 2) return DLMH_ERR_UNSUPPORTED;
+  p.ns = ns;
+  CUtensorMap mw, mx;
+  if (!make_map_k128(&mw, w, 1, n, k, k, kBM, kKC) || !make_map_k128(&mx, b_codes, 1, b_rows, k, ldb, p.nb, kKC))
+    return DLMH_ERR_CUDA;
+  const size_t smem = (size_t)ns * p.stage_bytes + 1024;
+  if (cudaFuncSetAttribute(umma_f8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return DLMH_ERR_CUDA;
+  const int ntiles = (n + kBM - 1) / kBM;
+  const int grid = ntiles < di.sms ? ntiles : di.sms;
+  umma_f8_kernel<<<grid, kUmmaThreads, smem, s>>>(mw, mx, p);
+  return launch_status();
+}
+
+// Library-owned stream-ordered pool for the W8A16 activation codes (one per device; memory
+// is kept between calls so that steady-state calls map nothing).
+cudaMemPool_t scratch_pool(int dev) {
+  static std::mutex mu;
+  static cudaMemPool_t pools[64] = {};
+  if (dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!pools[dev]) {
+    cudaMemPoolProps props{};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pool = nullptr;
+    if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) return nullptr;
+    uint64_t keep = ~uint64_t(0);
+    cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+    pools[dev] = pool;
+  }
+  return pools[dev];
+}
+
+}  // namespace
+
+bool w8a8_umma_supported(int k) {
+  // whole 128-byte K chunks (the tensor map's innermost box); a pure function of k so that
+  // every row count of a given weight takes this kernel
+  return k > 0 && k % 128 == 0;
+}
+
+bool w8a16_umma_supported(int k) { return k > 0 && k % 128 == 0; }
+
+int w8a8_umma_pass(const uint8_t* w, const float* w_scale, int n, int k, const uint8_t* xq, int64_t ldq,
+                   const float* x_scale, int rows, uint16_t* out, int64_t ldc, cudaStream_t s) {
+  if (rows < 1 || rows > 128) return DLMH_ERR_ROWS;
+  if (!w8a8_umma_supported(k)) return DLMH_ERR_SHAPE;
+  if ((reinterpret_cast<uintptr_t>(w) & 15u) || (reinterpret_cast<uintptr_t>(xq) & 15u) || ldq % 16 != 0)
+    return DLMH_ERR_ALIGN;
+  return launch_umma_f8(w, w_scale, n, k, xq, ldq, rows, x_scale, rows, 0, out, ldc, s);
+}
+
+int w8a16_umma_run(const uint8_t* w, const float* w_scale, int n, int k, const uint16_t* x, int64_t ldx, int rows,
+                   uint16_t* out, int64_t ldc, cudaStream_t s) {
+  if (!w8a16_umma_supported(k)) return DLMH_ERR_SHAPE;
+  if (rows <= 0) return DLMH_OK;
+  if ((reinterpret_cast<uintptr_t>(w) & 15u) || (reinterpret_cast<uintptr_t>(x) & 15u) || ldx % 8 != 0)
+    return DLMH_ERR_ALIGN;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DLMH_ERR_CUDA;
+  cudaMemPool_t pool = scratch_pool(dev);
+  if (!pool) return DLMH_ERR_CUDA;
+  const int first = rows < 128 ? rows : 128;
+  const int npad_max = (first + 15) / 16 * 16;
+  const size_t code_bytes = (size_t)2 * npad_max * k;  // a multiple of 256 (k % 128 == 0)
+  void* scratch = nullptr;
+  if (cudaMallocFromPoolAsync(&scratch, code_bytes + 128 * sizeof(float), pool, s) != cudaSuccess)
+    return DLMH_ERR_CUDA;
+  uint8_t* codes = static_cast<uint8_t*>(scratch);
+  float* x_mul = reinterpret_cast<float*>(codes + code_bytes);
+  int rc = DLMH_OK;
+  for (int done = 0; done < rows && rc == DLMH_OK;) {
+    const int m = rows - done < 128 ? rows - done : 128;
+    const int npad = (m + 15) / 16 * 16;
+    w8a16_split_kernel<<<npad, 256, 0, s>>>(x + (int64_t)done * ldx, ldx, m, k, npad, codes, x_mul);
+    rc = launch_status();
+    if (rc == DLMH_OK)
+      rc = launch_umma_f8(w, w_scale, n, k, codes, k, 2 * npad, x_mul, m, 1, out + (int64_t)done * ldc, ldc, s);
+    done += m;
+  }
+  if (cudaFreeAsync(scratch, s) != cudaSuccess && rc == DLMH_OK) rc = DLMH_ERR_CUDA;
+  return rc;
+}
+
+int umma_fault(int reset) {
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, umma_fault_word, sizeof(int)) != cudaSuccess) return DLMH_ERR_CUDA;
+  if (reset) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(umma_fault_word, &zero, sizeof(int)) != cudaSuccess) return DLMH_ERR_CUDA;
+  }
+  return v;
+}
+
+}  // namespace dlmh

@@ -33,7 +33,7 @@ def test_error_strings_and_version():
     assert dl.error_string(-99) == "unknown status"
 
 
-@pytest.mark.parametrize("opid,k,width", [(dl.OP_W8A16, 5120, 16), (dl.OP_W8A16, 1024, 16), (dl.OP_W8A8, 5120, 128),
+@pytest.mark.parametrize("opid,k,width", [(dl.OP_W8A16, 5120, 128), (dl.OP_W8A16, 1040, 16), (dl.OP_W8A8, 5120, 128),
                                            (dl.OP_W8A8, 14336, 128), (dl.OP_W8A8, 1040, 32), (dl.OP_W4A16, 4096, 16),
                                            (dl.OP_Q6K, 7168, 8)])
 def test_plan_matches_oracle_rules(opid, k, width):
@@ -44,7 +44,7 @@ def test_plan_matches_oracle_rules(opid, k, width):
         assert [(o, c) for o, c, _ in plan] == ref
         if opid == dl.OP_Q6K:
             widths = [8]
-        elif opid == dl.OP_W8A8 and k % 128 == 0:
+        elif opid in (dl.OP_W8A8, dl.OP_W8A16) and k % 128 == 0:
             widths = list(range(16, 129, 16))  # tensor-core tier: MMA N in steps of 16
         else:
             widths = [8, 16, 32]
@@ -57,9 +57,10 @@ def test_plan_rejects():
     assert L.dlmh_plan_chunks(dl.OP_W4A16, 33, 4096, None, None, None, 0) == -4
     assert L.dlmh_plan_chunks(dl.OP_W8A16, -1, 5120, None, None, None, 0) == -4
     assert L.dlmh_plan_chunks(9, 1, 5120, None, None, None, 0) == -2
-    assert L.dlmh_plan_chunks(dl.OP_W8A16, 1, 65536, None, None, None, 0) == -7
+    # k % 128 != 0 keeps the register-fragment tiers, whose activation tile must fit on chip
+    assert L.dlmh_plan_chunks(dl.OP_W8A16, 1, 65552, None, None, None, 0) == -7
     arr = (ctypes.c_int * 1)()
-    assert L.dlmh_plan_chunks(dl.OP_W8A16, 40, 5120, arr, arr, arr, 1) == -8
+    assert L.dlmh_plan_chunks(dl.OP_W8A16, 140, 5120, arr, arr, arr, 1) == -8
 
 
 # Fake device addresses: the argument checks must reject these calls before any CUDA call
@@ -80,7 +81,7 @@ def test_w8a16_argument_errors():
     assert f(A, A, 16, 64, U, 64, 1, A, 16, None) == -3
     assert f(A, A, 16, 64, A, 68, 1, A, 16, None) == -3
     assert f(A, A, 16, 64, A, 64, -1, A, 16, None) == -4
-    assert f(A, A, 16, 8192, A, 8192, 1, A, 16, None) == -7
+    assert f(A, A, 16, 8208, A, 8208, 1, A, 16, None) == -7
 
 
 def test_w8a8_argument_errors():

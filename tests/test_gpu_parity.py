@@ -70,6 +70,45 @@ def test_w8a16_ragged_shapes_and_tiers(n, k):
     assert (rep == full[3][None, :]).all()
 
 
+@pytest.mark.parametrize("n,k", [(300, 1152), (9000, 384)])
+def test_w8a16_tensor_core_tier_wide_rows(n, k):
+    # k % 128 == 0: one tensor-core pass per 128 rows for every row count; 130 rows cross a
+    # pass boundary, n leaves a ragged 128-row tile, an odd chunk count a half-empty stage
+    w = synth.fp8_weight(n, k, 12, DEV)
+    s = synth.row_scales(n, 12, DEV)
+    x = synth.bf16_rows(130, k, 12, DEV, std=0.5)
+    ref = og.w8a16_gemv(bits(w), bits(s), bits(x))
+    full = bits(dl.lm_head_fp8_w8a16(w, s, x))
+    assert_bf16_close(full, ref, f"w8a16 tensor-core tier n={n} k={k} M=130")
+    for m in (1, 15, 16, 17, 64, 127, 128):
+        part = bits(dl.lm_head_fp8_w8a16(w, s, x[:m]))
+        assert np.array_equal(part, full[:m]), f"row invariance M={m}"
+    assert np.array_equal(bits(dl.lm_head_fp8_w8a16(w, s, x[128:])), full[128:])
+    assert dl.device_fault(reset=True) == 0
+
+
+def test_w8a16_one_hot_weights_reproduce_activations():
+    # W[n] = 1.0 at column n % k (scale 1): out[m, n] = x[m, n % k] exactly wherever
+    # |x| >= 2^-13 max|x_m| (the two-term E4M3 split is exact there), within 2^-20 max|x_m|
+    # elsewhere -- checks the K order, the hi/lo pairing and the row exponent end to end
+    n, k = 2304, 1024
+    cols = np.arange(n) % k
+    codes = np.zeros((n, k), dtype=np.uint8)
+    codes[np.arange(n), cols] = 0x38                     # E4M3 1.0
+    w = torch.from_numpy(codes).to(DEV)
+    s = torch.ones(n, dtype=torch.float32, device=DEV)
+    x = synth.bf16_rows(37, k, 14, DEV)
+    x[3] *= 1e-20
+    x[4] *= 1e20
+    out = nx.bf16_decode(bits(dl.lm_head_fp8_w8a16(w, s, x)))
+    xv = nx.bf16_decode(bits(x))
+    want = xv[:, cols]
+    amax = np.abs(xv).max(axis=1, keepdims=True)
+    big = np.abs(want) >= 2.0 ** -13 * amax
+    assert np.array_equal(out[big], want[big])
+    assert np.all(np.abs(out - want)[~big] <= 2.0 ** -20 * np.broadcast_to(amax, want.shape)[~big])
+
+
 def test_w8a16_strided_io_and_zero_rows():
     n, k = 515, 1024
     w = synth.fp8_weight(n, k, 6, DEV)
