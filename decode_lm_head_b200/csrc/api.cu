@@ -169,8 +169,9 @@ int w8a8_silu_quantize_rows(const dlmh_bf16* gate, const dlmh_bf16* up, int64_t 
   return dlmh::w8a8_silu_quantize_launch(gate, up, ld, rows, k, xq, ldq, x_scale, as_stream(stream));
 }
 
-int w8a8_gemv(const uint8_t* w, const float* w_scale, int n, int k, const uint8_t* xq, int64_t ldq,
-              const float* x_scale, int rows, dlmh_bf16* out, int64_t ldc, void* stream) {
+static int w8a8_gemv_impl(const uint8_t* w, const float* w_scale, int n, int k, const uint8_t* xq, int64_t ldq,
+                          const float* x_scale, int rows, dlmh_bf16* out, int64_t ldc, void* stream,
+                          float* partial_ws, size_t partial_cap, bool after_prepass = false) {
   DLMH_TRY(check_rows(rows, DLMH_W8A8_MAX_ROWS));
   DLMH_TRY(check_nk(n, k, 16));
   if (rows == 0) return DLMH_OK;
@@ -186,7 +187,8 @@ int w8a8_gemv(const uint8_t* w, const float* w_scale, int n, int k, const uint8_
     const int m = rows - done < width ? rows - done : width;
     if (dlmh::w8a8_umma_supported(k))
       DLMH_TRY(dlmh::w8a8_umma_pass(w, w_scale, n, k, xq + (int64_t)done * ldq, ldq, x_scale + done, m,
-                                    out + (int64_t)done * ldc, ldc, as_stream(stream)));
+                                    out + (int64_t)done * ldc, ldc, as_stream(stream), partial_ws, partial_cap,
+                                    after_prepass && done == 0));
     else
       DLMH_TRY(dlmh::w8a8_gemv_pass(w, w_scale, n, k, xq + (int64_t)done * ldq, ldq, x_scale + done, m,
                                     out + (int64_t)done * ldc, ldc, as_stream(stream)));
@@ -195,9 +197,14 @@ int w8a8_gemv(const uint8_t* w, const float* w_scale, int n, int k, const uint8_
   return DLMH_OK;
 }
 
+int w8a8_gemv(const uint8_t* w, const float* w_scale, int n, int k, const uint8_t* xq, int64_t ldq,
+              const float* x_scale, int rows, dlmh_bf16* out, int64_t ldc, void* stream) {
+  return w8a8_gemv_impl(w, w_scale, n, k, xq, ldq, x_scale, rows, out, ldc, stream, nullptr, 0);
+}
+
 static int w8a8_proj_impl(const uint8_t* w, const float* w_scale, int n, int k, const dlmh_bf16* x,
                           const dlmh_bf16* up, int64_t ldx, int rows, dlmh_bf16* out, int64_t ldc, uint8_t* xq,
-                          float* xs, void* stream) {
+                          float* xs, void* stream, float* partial_ws = nullptr, size_t partial_cap = 0) {
   DLMH_TRY(check_rows(rows, 0));
   DLMH_TRY(check_nk(n, k, 16));
   if (rows == 0) return DLMH_OK;
@@ -218,7 +225,8 @@ static int w8a8_proj_impl(const uint8_t* w, const float* w_scale, int n, int k, 
       DLMH_TRY(dlmh::w8a8_silu_quantize_launch(xc, up + (int64_t)done * ldx, ldx, m, k, xq, k, xs, s));
     else
       DLMH_TRY(dlmh::w8a8_quantize_launch(xc, ldx, m, k, xq, k, xs, s));
-    DLMH_TRY(w8a8_gemv(w, w_scale, n, k, xq, k, xs, m, out + (int64_t)done * ldc, ldc, stream));
+    DLMH_TRY(w8a8_gemv_impl(w, w_scale, n, k, xq, k, xs, m, out + (int64_t)done * ldc, ldc, stream, partial_ws,
+                            partial_cap, true));
     done += m;
   }
   return DLMH_OK;
@@ -309,3 +317,14 @@ int q6k_lm_head(const void* blocks, int n, int k, const dlmh_bf16* x, int64_t ld
 }
 
 }  // extern "C"
+
+namespace dlmh {
+
+int w8a8_proj_fixed_scratch(const uint8_t* w, const float* w_scale, int n, int k, const uint16_t* x, int64_t ldx,
+                            int rows, uint16_t* out, int64_t ldc, uint8_t* xq, float* xs, float* partial_ws,
+                            size_t partial_cap, cudaStream_t stream) {
+  return w8a8_proj_impl(w, w_scale, n, k, x, nullptr, ldx, rows, out, ldc, xq, xs, stream, partial_ws,
+                        partial_cap);
+}
+
+}  // namespace dlmh

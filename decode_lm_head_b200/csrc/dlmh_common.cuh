@@ -57,6 +57,13 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t v) {
   return r;
 }
 
+// Programmatic dependent launch.  grid_dependents_launch(): this grid no longer holds back
+// the next kernel of the stream launched with programmatic stream serialization (it may
+// start its prologue now).  grid_dependency_wait(): block until the preceding kernel of the
+// stream has completed and its memory is visible (returns at once without such a launch).
+__device__ __forceinline__ void grid_dependents_launch() { asm volatile("griddepcontrol.launch_dependents;"); }
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Two f32 values -> two E4M3 codes (round-to-nearest-even, saturating to +-448);
 // `lo` lands in the low byte.
 __device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {

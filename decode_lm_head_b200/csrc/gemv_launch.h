@@ -23,8 +23,18 @@ int w8a8_gemv_pass(const uint8_t* w, const float* w_scale, int n, int k, const u
 // Tensor-core W8A8 pass (tcgen05, TMA-fed): one weight pass for 1..128 rows.  Taken for every
 // row count whenever w8a8_umma_supported(k) holds (a pure function of k).
 bool w8a8_umma_supported(int k);
+// The stream-K remainder's partial sums go to `partial_ws` (capacity `partial_cap` bytes,
+// DLMH_ERR_UNSUPPORTED if too small) or, when it is NULL, to stream-ordered scratch from the
+// library's memory pool.  after_prepass: the preceding kernel on `s` is this library's
+// activation quantize (weight loads may then overlap its tail).
 int w8a8_umma_pass(const uint8_t* w, const float* w_scale, int n, int k, const uint8_t* xq, int64_t ldq,
-                   const float* x_scale, int rows, uint16_t* out, int64_t ldc, cudaStream_t s);
+                   const float* x_scale, int rows, uint16_t* out, int64_t ldc, cudaStream_t s,
+                   float* partial_ws = nullptr, size_t partial_cap = 0, bool after_prepass = false);
+// w8a8_proj with caller-fixed scratch for everything, including the partial sums: never
+// allocates (the allocation-free entry point).
+int w8a8_proj_fixed_scratch(const uint8_t* w, const float* w_scale, int n, int k, const uint16_t* x, int64_t ldx,
+                            int rows, uint16_t* out, int64_t ldc, uint8_t* xq, float* xs, float* partial_ws,
+                            size_t partial_cap, cudaStream_t stream);
 // Fault bits of the tensor-core kernel's bounded waits (read synchronously).
 int umma_fault(int reset);
 

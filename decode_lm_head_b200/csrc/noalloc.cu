@@ -17,15 +17,23 @@
 #include <mutex>
 
 #include "dlmh_common.cuh"
+#include "gemv_launch.h"
 
 namespace {
 
 constexpr size_t kCodeBytes = (size_t)DLMH_W8A8_MAX_ROWS * DLMH_NOALLOC_MAX_K;
 constexpr size_t kScaleOffset = kCodeBytes;  // 256-byte aligned: kCodeBytes is a multiple of 256
-constexpr size_t kScratchBytes = kCodeBytes + DLMH_W8A8_MAX_ROWS * sizeof(float);
+constexpr size_t kScaleBytes = DLMH_W8A8_MAX_ROWS * sizeof(float);  // 512, keeps 256-byte alignment
+constexpr size_t kPartialOffset = kCodeBytes + kScaleBytes;
+// Partial sums of the tensor-core pass's stream-K remainder: two slots per CTA, 128 weight
+// rows x up to 128 activation rows of f32 each, for up to DLMH_NOALLOC_MAX_SMS CTAs.
+constexpr size_t kPartialBytes = (size_t)2 * DLMH_NOALLOC_MAX_SMS * 128 * DLMH_W8A8_MAX_ROWS * sizeof(float);
+constexpr size_t kScratchBytes = kPartialOffset + kPartialBytes;
 static_assert(kCodeBytes % 256 == 0, "scale block must stay aligned");
+static_assert(kPartialOffset % 256 == 0, "partial area must stay aligned");
 
-// Codes of up to 128 rows x DLMH_NOALLOC_MAX_K (row stride k), then 128 float32 row scales.
+// Codes of up to 128 rows x DLMH_NOALLOC_MAX_K (row stride k), 128 float32 row scales, then
+// the partial-sum area.
 static __device__ __align__(256) uint8_t g_w8a8_noalloc_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
@@ -57,8 +65,12 @@ extern "C" int w8a8_proj_noalloc(const uint8_t* w, const float* w_scale, int n, 
   uint8_t* base = nullptr;
   const int rc = scratch_on_current_device(&base);
   if (rc != DLMH_OK) return rc;
-  // Each chunk's quantize writes every code and scale the following GEMV reads, so nothing
-  // in the shared array has to start at zero.
-  return w8a8_proj(w, w_scale, n, k, x, ldx, rows, out, ldc, base, reinterpret_cast<float*>(base + kScaleOffset),
-                   stream);
+  // Each chunk's quantize writes every code and scale the following GEMV reads, and every
+  // partial sum is written before the fixup reads it, so nothing in the shared array has to
+  // start at zero.  A device with more SMs than the partial area serves gets
+  // DLMH_ERR_UNSUPPORTED.
+  return dlmh::w8a8_proj_fixed_scratch(w, w_scale, n, k, x, ldx, rows, out, ldc, base,
+                                       reinterpret_cast<float*>(base + kScaleOffset),
+                                       reinterpret_cast<float*>(base + kPartialOffset), kPartialBytes,
+                                       static_cast<cudaStream_t>(stream));
 }

@@ -62,6 +62,7 @@ __global__ void __launch_bounds__(kQThreads) w8a8_quantize_kernel(const uint16_t
                                                                   uint8_t* __restrict__ xq, int64_t ldq,
                                                                   float* __restrict__ sx) {
   __shared__ float red[32];
+  grid_dependents_launch();  // a following tensor-core GEMV may start its weight loads
   const int m = blockIdx.x;
   const uint16_t* xr = x + (int64_t)m * ldx;
   quantize_row([&](int i) { return bf16_bits_to_f32(xr[i]); }, k, xq + (int64_t)m * ldq, sx + m, red);
@@ -75,6 +76,7 @@ __global__ void __launch_bounds__(kQThreads) w8a8_silu_quantize_kernel(const uin
                                                                        float* __restrict__ sx) {
   extern __shared__ __align__(16) float hbuf[];  // k floats (BF16-exact values)
   __shared__ float red[32];
+  grid_dependents_launch();  // a following tensor-core GEMV may start its weight loads
   const int m = blockIdx.x;
   const uint16_t* gr = gate + (int64_t)m * ld;
   const uint16_t* ur = up + (int64_t)m * ld;

@@ -36,6 +36,7 @@
 // the allocating warp always frees its tensor memory before exit.
 #include "gemv_launch.h"
 #include "umma_common.cuh"
+#include "umma_sched.h"
 
 namespace dlmh {
 namespace {
@@ -67,25 +68,31 @@ struct UmmaParams {
   int64_t ldc;
   int ns;                // ring stages
   int stage_bytes;       // A + B bytes of one stage
+  // Stream-K schedule (umma_sched.h) over G = gridDim.x CTAs, a pure function of n, k and
+  // the SM count, never of the row count; partial sums are laid out [slot][col][128 rows].
+  int spt, wt, rem;
+  float* partial;
+  int early_w;  // 1: the preceding kernel is this library's activation pre-pass (it writes
+                // neither W nor the outputs), so weight loads may start before it completes
 };
+
 
 __global__ void __launch_bounds__(kUmmaThreads, 1)
     umma_f8_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x,
-                     const UmmaParams p) {
+                   const UmmaParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   __shared__ __align__(8) uint64_t bar_full[kMaxUStages], bar_empty[kMaxUStages], bar_tfull[2], bar_tempty[2];
   __shared__ uint32_t s_tmem;
 
-  const int ntiles = (p.n + kBM - 1) / kBM;
-  const int T0 = (int)((int64_t)blockIdx.x * ntiles / gridDim.x);
-  const int T1 = (int)((int64_t)(blockIdx.x + 1) * ntiles / gridDim.x);
-  if (T0 >= T1) return;
+  const Sched sc{p.spt, p.wt, p.rem, (int)gridDim.x};
+  const int b = blockIdx.x;
+  int njobs = 0, nunits = 0;
+  for (int tile, u0, u1, slot; sc.job(b, njobs, tile, u0, u1, slot); ++njobs) nunits += u1 - u0;
+  if (njobs == 0) return;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kchunks = p.k / 128;
-  const int spt = (kchunks + kKC - 1) / kKC;  // stages per tile
-  const int nstages = (T1 - T0) * spt;
   const uint32_t ring_u32 = smem_u32(ring);
   const uint32_t full0 = smem_u32(bar_full), empty0 = smem_u32(bar_empty);
   const uint32_t tfull0 = smem_u32(bar_tfull), tempty0 = smem_u32(bar_tempty);
@@ -109,45 +116,70 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
   __syncthreads();
   fence_after();
   const uint32_t tmem_base = s_tmem;
+  grid_dependents_launch();  // the fixup may be scheduled; it waits for this grid to finish
 
   if (warp == 0) {
     // ---------------- producer
     if (lane == 0) {
-      int slot = 0, phase = 0;
-      for (int s = 0; s < nstages; ++s) {
-        const int tile = T0 + s / spt, j = s % spt;
-        if (s >= p.ns && !wait(empty0 + 8u * slot, phase ^ 1)) atomicOr(&umma_fault_word, 1);
-        const uint32_t st = ring_u32 + slot * p.stage_bytes;
-        // the full box always lands (rows past n, rows past `rows` and a chunk past K are
-        // zero-filled), so every stage completes exactly stage_bytes
-        expect_tx(full0 + 8u * slot, (uint32_t)p.stage_bytes);
-        // A: weight rows [tile*128, +128) x chunks [j*KC, j*KC + KC); B: all activation rows
-        tma_load_3d(st, &map_w, 0, tile * kBM, j * kKC, full0 + 8u * slot);
-        tma_load_3d(st + a_bytes, &map_x, 0, 0, j * kKC, full0 + 8u * slot);
-        if (++slot == p.ns) {
-          slot = 0;
-          phase ^= 1;
+      const uint64_t pol_w = l2_policy_evict_first(), pol_x = l2_policy_evict_last();
+      // The first ring's weight tiles may be requested before the preceding kernel has
+      // finished (early_w); activation tiles only after it.
+      const int npre = p.early_w ? min(p.ns, nunits) : 0;
+      {
+        int s = 0;
+        for (int j = 0; j < njobs && s < npre; ++j) {
+          int tile, u0, u1, ps;
+          sc.job(b, j, tile, u0, u1, ps);
+          for (int u = u0; u < u1 && s < npre; ++u, ++s) {
+            expect_tx(full0 + 8u * s, (uint32_t)p.stage_bytes);
+            tma_load_3d(ring_u32 + s * p.stage_bytes, &map_w, 0, tile * kBM, u * kKC, full0 + 8u * s, pol_w);
+          }
+        }
+      }
+      grid_dependency_wait();
+      int slot = 0, phase = 0, s = 0;
+      for (int j = 0; j < njobs; ++j) {
+        int tile, u0, u1, ps;
+        sc.job(b, j, tile, u0, u1, ps);
+        for (int u = u0; u < u1; ++u, ++s) {
+          if (s >= p.ns && !wait(empty0 + 8u * slot, phase ^ 1)) atomicOr(&umma_fault_word, 1);
+          const uint32_t st = ring_u32 + slot * p.stage_bytes;
+          // the full boxes always land (rows past n, rows past `rows` and a chunk past K are
+          // zero-filled), so every stage completes exactly stage_bytes
+          if (s >= npre) {
+            expect_tx(full0 + 8u * slot, (uint32_t)p.stage_bytes);
+            // A: weight rows [tile*128, +128) x chunks [u*KC, u*KC + KC)
+            tma_load_3d(st, &map_w, 0, tile * kBM, u * kKC, full0 + 8u * slot, pol_w);
+          }
+          // B: all activation rows, the same chunks
+          tma_load_3d(st + a_bytes, &map_x, 0, 0, u * kKC, full0 + 8u * slot, pol_x);
+          if (++slot == p.ns) {
+            slot = 0;
+            phase ^= 1;
+          }
         }
       }
       // no copy may still be landing when the CTA exits: wait (bounded) for the last
       // phase of every slot (already complete in a healthy run, where the MMAs consumed it)
-      for (int s = nstages - 1; s >= 0 && s >= nstages - p.ns; --s)
-        if (!wait(full0 + 8u * (s % p.ns), (s / p.ns) & 1)) atomicOr(&umma_fault_word, 1);
+      for (int t = nunits - 1; t >= 0 && t >= nunits - p.ns; --t)
+        if (!wait(full0 + 8u * (t % p.ns), (t / p.ns) & 1)) atomicOr(&umma_fault_word, 1);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer
     if (lane == 0) {
       const uint32_t idesc = idesc_m128(p.nb);
       int slot = 0, phase = 0;
-      for (int i = 0; T0 + i < T1; ++i) {
+      for (int i = 0; i < njobs; ++i) {
+        int tile, u0, u1, ps;
+        sc.job(b, i, tile, u0, u1, ps);
         const int acc = i & 1;
         if (i >= 2 && !wait(tempty0 + 8u * acc, ((i - 2) >> 1) & 1)) atomicOr(&umma_fault_word, 4);
         fence_after();
         const uint32_t tmem_d = tmem_base + (uint32_t)acc * (tmem_cols / 2);
-        for (int j = 0; j < spt; ++j) {
+        for (int u = u0; u < u1; ++u) {
           if (!wait(full0 + 8u * slot, phase)) atomicOr(&umma_fault_word, 2);
           fence_after();
-          const int nch = min(kKC, kchunks - j * kKC);
+          const int nch = min(kKC, kchunks - u * kKC);
           const uint32_t st = ring_u32 + slot * p.stage_bytes;
           for (int c = 0; c < nch; ++c) {
             const uint32_t a0 = st + c * kChunkBytesA;
@@ -155,7 +187,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)  // K = 32 bytes per MMA
               umma_f8(tmem_d, desc_sw128(a0 + kk * 32), desc_sw128(b0 + kk * 32), idesc,
-                      (j | c | kk) != 0);
+                      ((u - u0) | c | kk) != 0);
           }
           commit(empty0 + 8u * slot);  // the stage is free once these MMAs have read it
           if (++slot == p.ns) {
@@ -170,30 +202,48 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
     // ---------------- epilogue (warps 2..5)
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const int lane_row = q * 32 + lane;
-    for (int i = 0; T0 + i < T1; ++i) {
-      const int tile = T0 + i, acc = i & 1;
+    grid_dependency_wait();  // x_scale comes from the preceding kernel
+    for (int i = 0; i < njobs; ++i) {
+      int tile, u0, u1, ps;
+      sc.job(b, i, tile, u0, u1, ps);
+      const int acc = i & 1;
       if (!wait(tfull0 + 8u * acc, (i >> 1) & 1)) atomicOr(&umma_fault_word, 8);
       fence_after();
       const int row = tile * kBM + lane_row;
-      const float s = row < p.n ? p.w_scale[row] : 0.f;
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)acc * (tmem_cols / 2);
-      for (int c0 = 0; c0 < p.npad; c0 += 16) {
-        uint32_t v[16];
-        tmem_ld16(taddr + (uint32_t)c0, v);
-        if (p.split) {  // y = hi-term sum + lo-term sum / 16
-          uint32_t u[16];
-          tmem_ld16(taddr + (uint32_t)(p.npad + c0), u);
+      if (ps >= 0) {
+        // partial tile: raw f32 sums of the used columns, [slot][col][128 rows]
+        float* dst = p.partial + (int64_t)ps * p.nb * kBM + lane_row;
+        for (int half = 0; half <= p.split; ++half) {
+          const int cb = half * p.npad;
+          for (int c0 = 0; c0 < p.npad; c0 += 16) {
+            uint32_t v[16];
+            tmem_ld16(taddr + (uint32_t)(cb + c0), v);
 #pragma unroll
-          for (int jj = 0; jj < 16; ++jj)
-            v[jj] = __float_as_uint(fmaf(__uint_as_float(u[jj]), 0.0625f, __uint_as_float(v[jj])));
+            for (int jj = 0; jj < 16; ++jj)
+              if (c0 + jj < p.rows) dst[(int64_t)(cb + c0 + jj) * kBM] = __uint_as_float(v[jj]);
+          }
         }
-        if (row < p.n) {
+      } else {
+        const float s = row < p.n ? p.w_scale[row] : 0.f;
+        for (int c0 = 0; c0 < p.npad; c0 += 16) {
+          uint32_t v[16];
+          tmem_ld16(taddr + (uint32_t)c0, v);
+          if (p.split) {  // y = hi-term sum + lo-term sum / 16
+            uint32_t u[16];
+            tmem_ld16(taddr + (uint32_t)(p.npad + c0), u);
 #pragma unroll
-          for (int jj = 0; jj < 16; ++jj) {
-            const int m = c0 + jj;
-            if (m < p.rows) {
-              const float y = (__uint_as_float(v[jj]) * s) * p.x_scale[m];
-              p.out[(int64_t)m * p.ldc + row] = f32_to_bf16_bits(y);
+            for (int jj = 0; jj < 16; ++jj)
+              v[jj] = __float_as_uint(fmaf(__uint_as_float(u[jj]), 0.0625f, __uint_as_float(v[jj])));
+          }
+          if (row < p.n) {
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) {
+              const int m = c0 + jj;
+              if (m < p.rows) {
+                const float y = (__uint_as_float(v[jj]) * s) * p.x_scale[m];
+                p.out[(int64_t)m * p.ldc + row] = f32_to_bf16_bits(y);
+              }
             }
           }
         }
@@ -211,6 +261,57 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
     __syncwarp();
     tmem_dealloc(tmem_base, tmem_cols);
   }
+}
+
+// Remainder tiles: CTA (t, m) finishes remainder tile t for activation row m; thread r owns
+// weight row r.  All partial sums of (r, m) are loaded first, then added in K order (the
+// CTAs that ran the tile's units, lowest first), so the result does not depend on which CTA
+// finished first, and the loads take one round trip.
+constexpr int kMaxParts = 512;  // >= G (the host checks)
+constexpr int kFixupBatch = 16;
+
+__global__ void __launch_bounds__(kBM) umma_f8_fixup_kernel(const UmmaParams p, int G) {
+  __shared__ int s_slot[kMaxParts];
+  __shared__ int s_nparts;
+  const Sched sc{p.spt, p.wt, p.rem, G};
+  const int t_rem = blockIdx.x, m = blockIdx.y;
+  if (threadIdx.x == 0) {  // contributors of this tile: independent of the main kernel's data
+    const int64_t tu0 = (int64_t)t_rem * p.spt, tu1 = tu0 + p.spt;
+    int np = 0;
+    for (int bb = sc.owner(tu0); bb < G && sc.r0(bb) < tu1 && np < kMaxParts; ++bb)
+      if (sc.r0(bb + 1) > sc.r0(bb)) s_slot[np++] = 2 * bb + (sc.r0(bb) / p.spt == t_rem ? 0 : 1);
+    s_nparts = np;
+  }
+  __syncthreads();
+  grid_dependency_wait();  // the partial sums and scales of the preceding kernels
+  const int row = (p.wt * G + t_rem) * kBM + threadIdx.x;
+  if (row >= p.n) return;
+  const int np = s_nparts;
+  const float* base = p.partial + threadIdx.x;
+  const int64_t slot_stride = (int64_t)p.nb * kBM;
+  const int64_t off_hi = (int64_t)m * kBM, off_lo = (int64_t)(p.npad + m) * kBM;
+  float hi = 0.f, lo = 0.f;
+  for (int q0 = 0; q0 < np; q0 += kFixupBatch) {
+    float vh[kFixupBatch], vl[kFixupBatch];
+#pragma unroll
+    for (int j = 0; j < kFixupBatch; ++j) {
+      vh[j] = vl[j] = 0.f;
+      if (q0 + j < np) {
+        const float* src = base + s_slot[q0 + j] * slot_stride;
+        vh[j] = src[off_hi];
+        if (p.split) vl[j] = src[off_lo];
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kFixupBatch; ++j) {
+      if (q0 + j < np) {
+        hi += vh[j];
+        lo += vl[j];
+      }
+    }
+  }
+  const float acc = p.split ? fmaf(lo, 0.0625f, hi) : hi;
+  p.out[(int64_t)m * p.ldc + row] = f32_to_bf16_bits((acc * p.w_scale[row]) * p.x_scale[m]);
 }
 
 constexpr size_t kUmmaSmemLimit = 232448 - 2048;
@@ -232,6 +333,7 @@ __global__ void __launch_bounds__(256) w8a16_split_kernel(const uint16_t* __rest
                                                           int k, int npad, uint8_t* __restrict__ codes,
                                                           float* __restrict__ x_mul) {
   __shared__ float s_red[8];
+  grid_dependents_launch();  // the GEMV may start its prologue and weight loads now
   const int m = blockIdx.x;
   uint8_t* hi_row = codes + (int64_t)m * k;
   uint8_t* lo_row = codes + (int64_t)(npad + m) * k;
@@ -284,39 +386,8 @@ __global__ void __launch_bounds__(256) w8a16_split_kernel(const uint16_t* __rest
   }
 }
 
-int launch_umma_f8(const uint8_t* w, const float* w_scale, int n, int k, const uint8_t* b_codes, int64_t ldb,
-                   int b_rows, const float* x_scale, int rows, int split, uint16_t* out, int64_t ldc, cudaStream_t s) {
-  const DeviceInfo di = device_info();
-  if (di.sms <= 0) return DLMH_ERR_CUDA;
-  UmmaParams p{};
-  p.n = n;
-  p.k = k;
-  p.rows = rows;
-  p.npad = (rows + 15) / 16 * 16;
-  p.nb = split ? 2 * p.npad : p.npad;
-  p.split = split;
-  p.w_scale = w_scale;
-  p.x_scale = x_scale;
-  p.out = out;
-  p.ldc = ldc;
-  p.stage_bytes = kKC * (kChunkBytesA + p.nb * 128);
-  int ns = (int)(kUmmaSmemLimit / (size_t)p.stage_bytes);
-  if (ns > kMaxUStages) ns = kMaxUStages;
-  if (ns < 2) return DLMH_ERR_UNSUPPORTED;
-  p.ns = ns;
-  CUtensorMap mw, mx;
-  if (!make_map_k128(&mw, w, 1, n, k, k, kBM, kKC) || !make_map_k128(&mx, b_codes, 1, b_rows, k, ldb, p.nb, kKC))
-    return DLMH_ERR_CUDA;
-  const size_t smem = (size_t)ns * p.stage_bytes + 1024;
-  if (cudaFuncSetAttribute(umma_f8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-    return DLMH_ERR_CUDA;
-  const int ntiles = (n + kBM - 1) / kBM;
-  const int grid = ntiles < di.sms ? ntiles : di.sms;
-  umma_f8_kernel<<<grid, kUmmaThreads, smem, s>>>(mw, mx, p);
-  return launch_status();
-}
-
-// Library-owned stream-ordered pool for the W8A16 activation codes (one per device; memory
+// Library-owned stream-ordered pool for the W8A16 activation codes and the stream-K partial
+// sums (one per device; memory
 // is kept between calls so that steady-state calls map nothing).
 cudaMemPool_t scratch_pool(int dev) {
   static std::mutex mu;
@@ -337,6 +408,64 @@ cudaMemPool_t scratch_pool(int dev) {
   return pools[dev];
 }
 
+int launch_umma_f8(const uint8_t* w, const float* w_scale, int n, int k, const uint8_t* b_codes, int64_t ldb,
+                   int b_rows, const float* x_scale, int rows, int split, uint16_t* out, int64_t ldc, cudaStream_t s,
+                   float* partial_ws, size_t partial_cap, int early_w) {
+  const DeviceInfo di = device_info();
+  if (di.sms <= 0) return DLMH_ERR_CUDA;
+  UmmaParams p{};
+  p.n = n;
+  p.k = k;
+  p.rows = rows;
+  p.npad = (rows + 15) / 16 * 16;
+  p.nb = split ? 2 * p.npad : p.npad;
+  p.split = split;
+  p.early_w = early_w;
+  p.w_scale = w_scale;
+  p.x_scale = x_scale;
+  p.out = out;
+  p.ldc = ldc;
+  p.stage_bytes = kKC * (kChunkBytesA + p.nb * 128);
+  int ns = (int)(kUmmaSmemLimit / (size_t)p.stage_bytes);
+  if (ns > kMaxUStages) ns = kMaxUStages;
+  if (ns < 2) return DLMH_ERR_UNSUPPORTED;
+  p.ns = ns;
+  CUtensorMap mw, mx;
+  if (!make_map_k128(&mw, w, 1, n, k, k, kBM, kKC) || !make_map_k128(&mx, b_codes, 1, b_rows, k, ldb, p.nb, kKC))
+    return DLMH_ERR_CUDA;
+  const size_t smem = (size_t)ns * p.stage_bytes + 1024;
+  if (cudaFuncSetAttribute(umma_f8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return DLMH_ERR_CUDA;
+  // schedule: whole tiles in full waves over the SMs, the rest split into units
+  const int ntiles = (n + kBM - 1) / kBM;
+  p.spt = (k / 128 + kKC - 1) / kKC;
+  const Sched sched = make_sched(ntiles, p.spt, di.sms);
+  const int G = sched.G;
+  if (G > kMaxParts) return DLMH_ERR_UNSUPPORTED;
+  p.wt = sched.wt;
+  p.rem = sched.rem;
+  void* ws = nullptr;
+  const size_t need = (size_t)2 * G * p.nb * kBM * sizeof(float);
+  if (p.rem > 0 && partial_ws) {
+    if (partial_cap < need) return DLMH_ERR_UNSUPPORTED;
+    p.partial = partial_ws;
+  } else if (p.rem > 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return DLMH_ERR_CUDA;
+    cudaMemPool_t pool = scratch_pool(dev);
+    if (!pool) return DLMH_ERR_CUDA;
+    if (cudaMallocFromPoolAsync(&ws, need, pool, s) != cudaSuccess)
+      return DLMH_ERR_CUDA;
+    p.partial = static_cast<float*>(ws);
+  }
+  int rc = launch_pdl(umma_f8_kernel, dim3(G), dim3(kUmmaThreads), smem, s, mw, mx, p);
+  if (rc == DLMH_OK && p.rem > 0) {
+    rc = launch_pdl(umma_f8_fixup_kernel, dim3(p.rem, rows), dim3(kBM), 0, s, p, G);
+  }
+  if (ws && cudaFreeAsync(ws, s) != cudaSuccess && rc == DLMH_OK) rc = DLMH_ERR_CUDA;
+  return rc;
+}
+
 }  // namespace
 
 bool w8a8_umma_supported(int k) {
@@ -348,12 +477,14 @@ bool w8a8_umma_supported(int k) {
 bool w8a16_umma_supported(int k) { return k > 0 && k % 128 == 0; }
 
 int w8a8_umma_pass(const uint8_t* w, const float* w_scale, int n, int k, const uint8_t* xq, int64_t ldq,
-                   const float* x_scale, int rows, uint16_t* out, int64_t ldc, cudaStream_t s) {
+                   const float* x_scale, int rows, uint16_t* out, int64_t ldc, cudaStream_t s, float* partial_ws,
+                   size_t partial_cap, bool after_prepass) {
   if (rows < 1 || rows > 128) return DLMH_ERR_ROWS;
   if (!w8a8_umma_supported(k)) return DLMH_ERR_SHAPE;
   if ((reinterpret_cast<uintptr_t>(w) & 15u) || (reinterpret_cast<uintptr_t>(xq) & 15u) || ldq % 16 != 0)
     return DLMH_ERR_ALIGN;
-  return launch_umma_f8(w, w_scale, n, k, xq, ldq, rows, x_scale, rows, 0, out, ldc, s);
+  return launch_umma_f8(w, w_scale, n, k, xq, ldq, rows, x_scale, rows, 0, out, ldc, s, partial_ws, partial_cap,
+                        after_prepass ? 1 : 0);
 }
 
 int w8a16_umma_run(const uint8_t* w, const float* w_scale, int n, int k, const uint16_t* x, int64_t ldx, int rows,
@@ -381,7 +512,8 @@ int w8a16_umma_run(const uint8_t* w, const float* w_scale, int n, int k, const u
     w8a16_split_kernel<<<npad, 256, 0, s>>>(x + (int64_t)done * ldx, ldx, m, k, npad, codes, x_mul);
     rc = launch_status();
     if (rc == DLMH_OK)
-      rc = launch_umma_f8(w, w_scale, n, k, codes, k, 2 * npad, x_mul, m, 1, out + (int64_t)done * ldc, ldc, s);
+      rc = launch_umma_f8(w, w_scale, n, k, codes, k, 2 * npad, x_mul, m, 1, out + (int64_t)done * ldc, ldc, s,
+                          nullptr, 0, 1);
     done += m;
   }
   if (cudaFreeAsync(scratch, s) != cudaSuccess && rc == DLMH_OK) rc = DLMH_ERR_CUDA;

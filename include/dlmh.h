@@ -19,7 +19,13 @@
  * ----------------------------------------
  *   - Every pointer argument named w*, x*, gate, up, out*, xq*, *scale*, q8*, blocks or
  *     *scratch is a DEVICE pointer on the current CUDA device.  The caller owns all of
- *     them; the library allocates no device memory and keeps no pointer after return.
+ *     them; the library keeps no pointer after return.
+ *   - Internal scratch: the tensor-core passes (k % 128 == 0) of lm_head_fp8_w8a16 and of
+ *     the W8A8 GEMV take stream-ordered scratch (W8A16 activation codes; stream-K partial
+ *     sums) from a library-owned memory pool of the current device, with
+ *     cudaMallocFromPoolAsync / cudaFreeAsync on `stream`.  The pool keeps its memory between
+ *     calls, so steady-state calls map nothing and never synchronize; concurrent calls on
+ *     different streams get distinct scratch.  w8a8_proj_noalloc never uses the pool.
  *   - BF16 values are passed as raw 16-bit patterns (dlmh_bf16).
  *   - Matrices are row-major.  Leading dimensions (ld*) count ELEMENTS of the pointed-to
  *     type, so row r of x starts at x + r * ldx.
@@ -94,14 +100,21 @@ typedef enum dlmh_status {
  *   w_scale [n] float32, one per output row.
  *   x       [rows, ldx] BF16, ldx >= k, ldx % 8 == 0, 16-byte aligned.
  *   out     [rows, ldc] BF16, ldc >= n.
- *   k % 16 == 0.  Any rows >= 0: one weight pass per 16 rows (rows above 16 run as
- *   consecutive 16-row chunks, the last one ragged).
- *   Numerics: E4M3 weights are exact in f16; each x row is scaled by a power of two into
- *   f16 (exact for every |x| >= 2^-31 * max|x| of the row), products are exact and summed
- *   in f32; the row scale and the power of two are applied to the f32 sum, then rounded
- *   to BF16 (round-to-nearest-even).
- *   k above the shared-memory limit of a 16-row chunk (k > 6144) returns
+ *   k % 16 == 0.  Any rows >= 0.
+ *   k % 128 == 0 (the tensor-core path, every FP8 head): one weight pass per 128 rows (the
+ *   last pass ragged).  Each x row is scaled by a power of two 2^e with max|x| 2^e in
+ *   [2^7, 2^8) and split into two E4M3 terms hi = e4m3(x'), lo = e4m3(16 (x' - hi)); then
+ *   out = bf16(s[n] 2^-e (sum_k w hi + (sum_k w lo) / 16)) with f32 sums.  hi + lo/16 equals
+ *   x' exactly for every element with |x| >= 2^-13 max|x| of its row (every BF16 value has
+ *   8 significant bits, E4M3 4); smaller elements keep an error below 2^-21 max|x|.
+ *   Scratch: 2 * roundup16(min(rows, 128)) * k bytes + 512 B, plus the stream-K partial
+ *   sums (at most 2 * #SMs * 128 * 256 * 4 bytes), from the library pool (see above).
+ *   Other k: one weight pass per 16 rows; E4M3 weights decoded exactly to f16 and each x row
+ *   scaled by a power of two into f16 (exact for every |x| >= 2^-31 max|x|), products
+ *   summed in f32.  k above the shared-memory limit of a 16-row chunk (k > 6144) returns
  *   DLMH_ERR_UNSUPPORTED.
+ *   Either way the row scale and the power of two are applied to the f32 sum, then rounded
+ *   to BF16 (round-to-nearest-even).
  * ------------------------------------------------------------------------------------- */
 DLMH_API int lm_head_fp8_w8a16(const uint8_t* w, const float* w_scale, int n, int k, const dlmh_bf16* x,
                       int64_t ldx, int rows, dlmh_bf16* out, int64_t ldc, void* stream);
@@ -130,8 +143,10 @@ DLMH_API int w8a8_silu_quantize_rows(const dlmh_bf16* gate, const dlmh_bf16* up,
  * W8A8 GEMV on already-quantized rows
  *   out[m, n] = bf16( s[n] * sx[m] * sum_k e4m3(w[n, k]) * e4m3(xq[m, k]) )
  * lm_head_fp8_rows.rs (W8A8 branch), w8a8_layer.rs (ops::w8a8_gemv).
- *   rows <= 128; one weight pass per call.  xq [rows, ldq] as written by the quantize
- *   entry points; x_scale [rows].  k % 16 == 0 and k <= 16384.
+ *   rows <= 128; one weight pass per call when k % 128 == 0 (tensor cores; stream-K partial
+ *   sums in pool scratch, see above), else passes of up to 32 rows (k bounded by the
+ *   shared-memory activation tile, DLMH_ERR_UNSUPPORTED beyond).  xq [rows, ldq] as written
+ *   by the quantize entry points; x_scale [rows].  k % 16 == 0.
  * ------------------------------------------------------------------------------------- */
 DLMH_API int w8a8_gemv(const uint8_t* w, const float* w_scale, int n, int k, const uint8_t* xq, int64_t ldq,
               const float* x_scale, int rows, dlmh_bf16* out, int64_t ldc, void* stream);
@@ -162,8 +177,11 @@ DLMH_API int w8a8_silu_proj(const uint8_t* w, const float* w_scale, int n, int k
  *   loops that cannot afford cudaMalloc's implicit device synchronization.  They still pass
  *   w, w_scale, x and out.
  *
- *   Limit: k <= DLMH_NOALLOC_MAX_K (16384), else DLMH_ERR_UNSUPPORTED.  Every GPU that loads
- *   the library holds the 2 MiB + 512 B array until the process exits.
+ *   Limits: k <= DLMH_NOALLOC_MAX_K (16384), else DLMH_ERR_UNSUPPORTED; a device with more
+ *   than DLMH_NOALLOC_MAX_SMS (160) SMs gets DLMH_ERR_UNSUPPORTED for shapes whose
+ *   tensor-core pass needs stream-K partial sums.  Every GPU that loads the library holds
+ *   the array until the process exits: 2 MiB of codes, 512 B of scales and 20 MiB of
+ *   partial sums (22 MiB + 512 B).
  *
  *   Set-up: a device's first call looks the array's device address up
  *   (cudaGetSymbolAddress, with that device current).  Make that first call before any
@@ -176,6 +194,7 @@ DLMH_API int w8a8_silu_proj(const uint8_t* w, const float* w_scale, int n, int k
  *   No cudaMalloc, cudaFree or allocating library routine is called.
  * ------------------------------------------------------------------------------------- */
 #define DLMH_NOALLOC_MAX_K 16384
+#define DLMH_NOALLOC_MAX_SMS 160
 DLMH_API int w8a8_proj_noalloc(const uint8_t* w, const float* w_scale, int n, int k, const dlmh_bf16* x,
                                int64_t ldx, int rows, dlmh_bf16* out, int64_t ldc, void* stream);
 
@@ -236,8 +255,10 @@ typedef enum dlmh_op {
 /* The weight passes an entry point runs for `rows` at reduction length k: pass i covers rows
  * [offsets[i], offsets[i] + counts[i]) and runs the kernel tier of width tiers[i] (the
  * narrowest compiled tier that covers counts[i], w4a16_gemv_tiers.rs select_tier).
- * The pass width is a pure function of (op, k) (which activation tile fits on chip), so
- * this needs no GPU.  Returns the number of passes (0 for rows == 0), DLMH_ERR_ROWS for
+ * For W8A16 and W8A8 with k % 128 == 0 the tensor-core tier serves 128 rows per pass and
+ * its width is counts[i] rounded up to 16 (the MMA's N, doubled inside for W8A16).
+ * The pass width is a pure function of (op, k) (which kernel serves k, and which activation
+ * tile fits on chip), so this needs no GPU.  Returns the number of passes (0 for rows == 0), DLMH_ERR_ROWS for
  * rows < 0 or above the op's cap, DLMH_ERR_SHAPE for an unknown op or k <= 0,
  * DLMH_ERR_UNSUPPORTED when no tier fits k, DLMH_ERR_CAPACITY when more than `cap`
  * passes are needed.  Arrays may be NULL when cap == 0 (count only). */
