@@ -9,13 +9,14 @@
 // rounding it to E4M3's 4 leaves a residual of at most 4 bits, so hi + lo/16 == x' exactly
 // whenever |x'| >= 2^-6 (every element within 2^-13 of the row maximum); below that the
 // error is at most 2^-14 in x' units.  The two terms are the B operand's first and second
-// npad columns, so the weights stay E4M3 in the A operand: the tensor core takes an M=128,
+// roundup8(rows) columns, so the weights stay E4M3 in the A operand: the tensor core takes an M=128,
 // K=32-byte instruction in the same ~142 clocks whatever N <= 256, i.e. it consumes A at
 // ~29 bytes/clock/SM, above the HBM share of an SM (~24); a 16-bit A operand would halve
 // the weight rate and make the kernel MMA-bound.
 //
 // Swap-AB: the weight is the MMA's A operand (M = 128 weight rows per tile) and the
-// activation codes are its B operand (N = rows rounded up to 16, twice that for W8A16).
+// activation codes are its B operand (N = rows rounded up to 16; for W8A16 twice the rows
+// rounded up to 8).
 // Both operands are E4M3 bytes used as stored (kind::f8f6f4, f32 accumulation in TMEM).
 //
 // Operand staging: both matrices are read through 3-D tensor maps over [rows][K] bytes,
@@ -59,9 +60,11 @@ __device__ __forceinline__ void umma_f8(uint32_t tmem_d, uint64_t adesc, uint64_
 }
 
 struct UmmaParams {
-  int n, k, rows, npad;  // npad: rows rounded up to 16
-  int nb;                // MMA N = B rows: npad (W8A8) or 2 npad (W8A16 hi | lo)
+  int n, k, rows, npad;  // npad: rows rounded up to 16 (the epilogue's column loop)
+  int nb;                // MMA N = B rows: npad (W8A8) or 2 * roundup8(rows) (W8A16 hi | lo)
   int split;             // 1: W8A16 two-term epilogue
+  int lo_off;            // W8A16: column of row 0's lo term (roundup8(rows))
+  int accw;              // TMEM columns per accumulator (a power of two >= 32)
   const float* w_scale;
   const float* x_scale;  // sx[m] (W8A8) or 2^-e[m] (W8A16)
   uint16_t* out;
@@ -98,7 +101,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
   const uint32_t tfull0 = smem_u32(bar_tfull), tempty0 = smem_u32(bar_tempty);
   const int a_bytes = kKC * kChunkBytesA;
   const int b_chunk = p.nb * 128;
-  const uint32_t tmem_cols = (uint32_t)tmem_cols_for(2 * p.nb);
+  const uint32_t tmem_cols = 2u * (uint32_t)p.accw;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < p.ns; ++i) {
@@ -175,7 +178,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
         const int acc = i & 1;
         if (i >= 2 && !wait(tempty0 + 8u * acc, ((i - 2) >> 1) & 1)) atomicOr(&umma_fault_word, 4);
         fence_after();
-        const uint32_t tmem_d = tmem_base + (uint32_t)acc * (tmem_cols / 2);
+        const uint32_t tmem_d = tmem_base + (uint32_t)(acc * p.accw);
         for (int u = u0; u < u1; ++u) {
           if (!wait(full0 + 8u * slot, phase)) atomicOr(&umma_fault_word, 2);
           fence_after();
@@ -210,12 +213,12 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
       if (!wait(tfull0 + 8u * acc, (i >> 1) & 1)) atomicOr(&umma_fault_word, 8);
       fence_after();
       const int row = tile * kBM + lane_row;
-      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)acc * (tmem_cols / 2);
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * p.accw);
       if (ps >= 0) {
         // partial tile: raw f32 sums of the used columns, [slot][col][128 rows]
         float* dst = p.partial + (int64_t)ps * p.nb * kBM + lane_row;
         for (int half = 0; half <= p.split; ++half) {
-          const int cb = half * p.npad;
+          const int cb = half * p.lo_off;
           for (int c0 = 0; c0 < p.npad; c0 += 16) {
             uint32_t v[16];
             tmem_ld16(taddr + (uint32_t)(cb + c0), v);
@@ -231,7 +234,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
           tmem_ld16(taddr + (uint32_t)c0, v);
           if (p.split) {  // y = hi-term sum + lo-term sum / 16
             uint32_t u[16];
-            tmem_ld16(taddr + (uint32_t)(p.npad + c0), u);
+            tmem_ld16(taddr + (uint32_t)(p.lo_off + c0), u);
 #pragma unroll
             for (int jj = 0; jj < 16; ++jj)
               v[jj] = __float_as_uint(fmaf(__uint_as_float(u[jj]), 0.0625f, __uint_as_float(v[jj])));
@@ -275,12 +278,25 @@ __global__ void __launch_bounds__(kBM) umma_f8_fixup_kernel(const UmmaParams p, 
   __shared__ int s_nparts;
   const Sched sc{p.spt, p.wt, p.rem, G};
   const int t_rem = blockIdx.x, m = blockIdx.y;
-  if (threadIdx.x == 0) {  // contributors of this tile: independent of the main kernel's data
+  // Contributors of this tile (independent of the main kernel's data, so computed before the
+  // dependency wait): consecutive CTAs from the owner of its first unit; thread i checks
+  // candidate owner + i, i.e. the list is built in parallel, in K order.
+  if (threadIdx.x == 0) s_nparts = 0;
+  __syncthreads();
+  {
     const int64_t tu0 = (int64_t)t_rem * p.spt, tu1 = tu0 + p.spt;
-    int np = 0;
-    for (int bb = sc.owner(tu0); bb < G && sc.r0(bb) < tu1 && np < kMaxParts; ++bb)
-      if (sc.r0(bb + 1) > sc.r0(bb)) s_slot[np++] = 2 * bb + (sc.r0(bb) / p.spt == t_rem ? 0 : 1);
-    s_nparts = np;
+    const int b0 = sc.owner(tu0);
+    for (int i = threadIdx.x; i < kMaxParts && b0 + i < G; i += kBM) {
+      const int bb = b0 + i;
+      const int64_t a = sc.r0(bb), e = sc.r0(bb + 1);
+      if (a < tu1 && e > a) {  // non-empty range starting before the tile's end (it ends after tu0)
+        s_slot[i] = 2 * bb + (a / p.spt == t_rem ? 0 : 1);
+        atomicMax(&s_nparts, i + 1);
+      } else if (a < tu1) {
+        s_slot[i] = -1;  // empty range inside the run: skipped
+      }
+      if (a >= tu1) break;
+    }
   }
   __syncthreads();
   grid_dependency_wait();  // the partial sums and scales of the preceding kernels
@@ -289,14 +305,16 @@ __global__ void __launch_bounds__(kBM) umma_f8_fixup_kernel(const UmmaParams p, 
   const int np = s_nparts;
   const float* base = p.partial + threadIdx.x;
   const int64_t slot_stride = (int64_t)p.nb * kBM;
-  const int64_t off_hi = (int64_t)m * kBM, off_lo = (int64_t)(p.npad + m) * kBM;
+  const int64_t off_hi = (int64_t)m * kBM, off_lo = (int64_t)(p.lo_off + m) * kBM;
   float hi = 0.f, lo = 0.f;
   for (int q0 = 0; q0 < np; q0 += kFixupBatch) {
     float vh[kFixupBatch], vl[kFixupBatch];
+    bool ok[kFixupBatch];
 #pragma unroll
     for (int j = 0; j < kFixupBatch; ++j) {
       vh[j] = vl[j] = 0.f;
-      if (q0 + j < np) {
+      ok[j] = q0 + j < np && s_slot[q0 + j] >= 0;
+      if (ok[j]) {
         const float* src = base + s_slot[q0 + j] * slot_stride;
         vh[j] = src[off_hi];
         if (p.split) vl[j] = src[off_lo];
@@ -304,7 +322,7 @@ __global__ void __launch_bounds__(kBM) umma_f8_fixup_kernel(const UmmaParams p, 
     }
 #pragma unroll
     for (int j = 0; j < kFixupBatch; ++j) {
-      if (q0 + j < np) {
+      if (ok[j]) {
         hi += vh[j];
         lo += vl[j];
       }
@@ -326,17 +344,17 @@ __device__ __forceinline__ int e4m3_split_exponent(float amax) {
   return max(-126, min(126, 7 - E));
 }
 
-// W8A16 activation split: CTA m writes E4M3 rows codes[m] = hi(x'[m]) and codes[npad + m] =
+// W8A16 activation split: CTA m writes E4M3 rows codes[m] = hi(x'[m]) and codes[half + m] =
 // lo(x'[m]) (zero rows for m >= rows) and x_mul[m] = 2^-e[m].  k a multiple of 8, x
 // 16-byte aligned with ldx a multiple of 8.
 __global__ void __launch_bounds__(256) w8a16_split_kernel(const uint16_t* __restrict__ x, int64_t ldx, int rows,
-                                                          int k, int npad, uint8_t* __restrict__ codes,
+                                                          int k, int half, uint8_t* __restrict__ codes,
                                                           float* __restrict__ x_mul) {
   __shared__ float s_red[8];
   grid_dependents_launch();  // the GEMV may start its prologue and weight loads now
   const int m = blockIdx.x;
   uint8_t* hi_row = codes + (int64_t)m * k;
-  uint8_t* lo_row = codes + (int64_t)(npad + m) * k;
+  uint8_t* lo_row = codes + (int64_t)(half + m) * k;
   if (m >= rows) {
     for (int k8 = threadIdx.x * 8; k8 < k; k8 += 256 * 8) {
       *reinterpret_cast<uint2*>(hi_row + k8) = make_uint2(0, 0);
@@ -418,7 +436,12 @@ int launch_umma_f8(const uint8_t* w, const float* w_scale, int n, int k, const u
   p.k = k;
   p.rows = rows;
   p.npad = (rows + 15) / 16 * 16;
-  p.nb = split ? 2 * p.npad : p.npad;
+  p.lo_off = (rows + 7) / 8 * 8;
+  p.nb = split ? 2 * p.lo_off : p.npad;
+  // the epilogue reads 16 columns from lo_off + c0 (c0 < npad): keep that inside the
+  // accumulator when lo_off is not a multiple of 16
+  p.accw = tmem_cols_for(split && (p.lo_off % 16) ? p.nb + 16 : p.nb);
+  if (2 * p.accw > 512) return DLMH_ERR_UNSUPPORTED;
   p.split = split;
   p.early_w = early_w;
   p.w_scale = w_scale;
@@ -498,8 +521,8 @@ int w8a16_umma_run(const uint8_t* w, const float* w_scale, int n, int k, const u
   cudaMemPool_t pool = scratch_pool(dev);
   if (!pool) return DLMH_ERR_CUDA;
   const int first = rows < 128 ? rows : 128;
-  const int npad_max = (first + 15) / 16 * 16;
-  const size_t code_bytes = (size_t)2 * npad_max * k;  // a multiple of 256 (k % 128 == 0)
+  const int half_max = (first + 7) / 8 * 8;
+  const size_t code_bytes = (size_t)2 * half_max * k;  // a multiple of 256 (k % 128 == 0)
   void* scratch = nullptr;
   if (cudaMallocFromPoolAsync(&scratch, code_bytes + 128 * sizeof(float), pool, s) != cudaSuccess)
     return DLMH_ERR_CUDA;
@@ -508,11 +531,11 @@ int w8a16_umma_run(const uint8_t* w, const float* w_scale, int n, int k, const u
   int rc = DLMH_OK;
   for (int done = 0; done < rows && rc == DLMH_OK;) {
     const int m = rows - done < 128 ? rows - done : 128;
-    const int npad = (m + 15) / 16 * 16;
-    w8a16_split_kernel<<<npad, 256, 0, s>>>(x + (int64_t)done * ldx, ldx, m, k, npad, codes, x_mul);
+    const int half = (m + 7) / 8 * 8;  // hi rows [0, half), lo rows [half, 2 half)
+    w8a16_split_kernel<<<half, 256, 0, s>>>(x + (int64_t)done * ldx, ldx, m, k, half, codes, x_mul);
     rc = launch_status();
     if (rc == DLMH_OK)
-      rc = launch_umma_f8(w, w_scale, n, k, codes, k, 2 * npad, x_mul, m, 1, out + (int64_t)done * ldc, ldc, s,
+      rc = launch_umma_f8(w, w_scale, n, k, codes, k, 2 * half, x_mul, m, 1, out + (int64_t)done * ldc, ldc, s,
                           nullptr, 0, 1);
     done += m;
   }

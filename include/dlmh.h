@@ -107,7 +107,7 @@ typedef enum dlmh_status {
  *   out = bf16(s[n] 2^-e (sum_k w hi + (sum_k w lo) / 16)) with f32 sums.  hi + lo/16 equals
  *   x' exactly for every element with |x| >= 2^-13 max|x| of its row (every BF16 value has
  *   8 significant bits, E4M3 4); smaller elements keep an error below 2^-21 max|x|.
- *   Scratch: 2 * roundup16(min(rows, 128)) * k bytes + 512 B, plus the stream-K partial
+ *   Scratch: 2 * roundup8(min(rows, 128)) * k bytes + 512 B, plus the stream-K partial
  *   sums (at most 2 * #SMs * 128 * 256 * 4 bytes), from the library pool (see above).
  *   Other k: one weight pass per 16 rows; E4M3 weights decoded exactly to f16 and each x row
  *   scaled by a power of two into f16 (exact for every |x| >= 2^-31 max|x|), products
