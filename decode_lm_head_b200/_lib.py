@@ -105,10 +105,17 @@ def _check(rc, what):
         raise DlmhError(rc, what)
 
 
-def _stream(stream):
-    if stream is None:
-        stream = torch.cuda.current_stream()
-    return ctypes.c_void_p(stream.cuda_stream)
+_raw_current_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
+def _stream(stream, device=None):
+    """The cudaStream_t to launch on, as an int (the current stream of `device` if None)."""
+    if stream is not None:
+        return stream.cuda_stream
+    if _raw_current_stream is not None:
+        index = device.index if device is not None and device.index is not None else torch.cuda.current_device()
+        return _raw_current_stream(index)
+    return torch.cuda.current_stream().cuda_stream
 
 
 def _cuda(t, dtype, name, ndim):
@@ -130,7 +137,7 @@ def _ld(t):
 
 
 def _ptr(t):
-    return ctypes.c_void_p(t.data_ptr())
+    return t.data_ptr()
 
 
 def plan_chunks(op, rows, k):
@@ -164,7 +171,7 @@ def lm_head_fp8_w8a16(w, w_scale, x, out=None, stream=None):
         out = torch.empty(rows, n, dtype=torch.bfloat16, device=x.device)
     _cuda(out, torch.bfloat16, "out", 2)
     _check(lib().lm_head_fp8_w8a16(_ptr(w), _ptr(w_scale), n, k, _ptr(x), _ld(x), rows, _ptr(out), _ld(out),
-                                   _stream(stream)), "lm_head_fp8_w8a16")
+                                   _stream(stream, x.device)), "lm_head_fp8_w8a16")
     return out
 
 
@@ -175,8 +182,8 @@ def w8a8_quantize_rows(x, xq=None, x_scale=None, stream=None):
         xq = torch.empty(rows, k, dtype=torch.uint8, device=x.device)
     if x_scale is None:
         x_scale = torch.empty(rows, dtype=torch.float32, device=x.device)
-    _check(lib().w8a8_quantize_rows(_ptr(x), _ld(x), rows, k, _ptr(xq), _ld(xq), _ptr(x_scale), _stream(stream)),
-           "w8a8_quantize_rows")
+    _check(lib().w8a8_quantize_rows(_ptr(x), _ld(x), rows, k, _ptr(xq), _ld(xq), _ptr(x_scale),
+                                    _stream(stream, x.device)), "w8a8_quantize_rows")
     return xq, x_scale
 
 
@@ -191,7 +198,7 @@ def w8a8_silu_quantize_rows(gate, up, xq=None, x_scale=None, stream=None):
     if x_scale is None:
         x_scale = torch.empty(rows, dtype=torch.float32, device=gate.device)
     _check(lib().w8a8_silu_quantize_rows(_ptr(gate), _ptr(up), _ld(gate), rows, k, _ptr(xq), _ld(xq),
-                                         _ptr(x_scale), _stream(stream)), "w8a8_silu_quantize_rows")
+                                         _ptr(x_scale), _stream(stream, gate.device)), "w8a8_silu_quantize_rows")
     return xq, x_scale
 
 
@@ -205,7 +212,7 @@ def w8a8_gemv(w, w_scale, xq, x_scale, out=None, stream=None):
     if out is None:
         out = torch.empty(rows, n, dtype=torch.bfloat16, device=w.device)
     _check(lib().w8a8_gemv(_ptr(w), _ptr(w_scale), n, k, _ptr(xq), _ld(xq), _ptr(x_scale), rows, _ptr(out),
-                           _ld(out), _stream(stream)), "w8a8_gemv")
+                           _ld(out), _stream(stream, xq.device)), "w8a8_gemv")
     return out
 
 
@@ -227,7 +234,7 @@ def w8a8_proj(w, w_scale, x, out=None, xq_scratch=None, xscale_scratch=None, str
         out = torch.empty(rows, n, dtype=torch.bfloat16, device=x.device)
     xq_scratch, xscale_scratch = _w8a8_scratch(k, x.device, xq_scratch, xscale_scratch)
     _check(lib().w8a8_proj(_ptr(w), _ptr(w_scale), n, k, _ptr(x), _ld(x), rows, _ptr(out), _ld(out),
-                           _ptr(xq_scratch), _ptr(xscale_scratch), _stream(stream)), "w8a8_proj")
+                           _ptr(xq_scratch), _ptr(xscale_scratch), _stream(stream, x.device)), "w8a8_proj")
     return out
 
 
@@ -242,7 +249,7 @@ def w8a8_proj_noalloc(w, w_scale, x, out=None, stream=None):
     if out is None:
         out = torch.empty(rows, n, dtype=torch.bfloat16, device=x.device)
     _check(lib().w8a8_proj_noalloc(_ptr(w), _ptr(w_scale), n, k, _ptr(x), _ld(x), rows, _ptr(out), _ld(out),
-                                   _stream(stream)), "w8a8_proj_noalloc")
+                                   _stream(stream, x.device)), "w8a8_proj_noalloc")
     return out
 
 
@@ -259,7 +266,8 @@ def w8a8_silu_proj(w, w_scale, gate, up, out=None, xq_scratch=None, xscale_scrat
         out = torch.empty(rows, n, dtype=torch.bfloat16, device=gate.device)
     xq_scratch, xscale_scratch = _w8a8_scratch(k, gate.device, xq_scratch, xscale_scratch)
     _check(lib().w8a8_silu_proj(_ptr(w), _ptr(w_scale), n, k, _ptr(gate), _ptr(up), _ld(gate), rows, _ptr(out),
-                                _ld(out), _ptr(xq_scratch), _ptr(xscale_scratch), _stream(stream)), "w8a8_silu_proj")
+                                _ld(out), _ptr(xq_scratch), _ptr(xscale_scratch), _stream(stream, gate.device)),
+           "w8a8_silu_proj")
     return out
 
 
@@ -275,7 +283,7 @@ def w4a16_gemv(w_packed, w_block_scale, global_scale, x, out=None, stream=None):
     if out is None:
         out = torch.empty(rows, n, dtype=torch.bfloat16, device=x.device)
     _check(lib().w4a16_gemv(_ptr(w_packed), _ptr(w_block_scale), float(global_scale), n, k, _ptr(x), _ld(x), rows,
-                            _ptr(out), _ld(out), _stream(stream)), "w4a16_gemv")
+                            _ptr(out), _ld(out), _stream(stream, x.device)), "w4a16_gemv")
     return out
 
 
@@ -284,7 +292,8 @@ def q8_1_quantize_rows(x, q8=None, stream=None):
     rows, k = x.shape
     if q8 is None:
         q8 = torch.empty(rows, k // 32, Q8_1_BLOCK_BYTES, dtype=torch.uint8, device=x.device)
-    _check(lib().q8_1_quantize_rows(_ptr(x), _ld(x), rows, k, _ptr(q8), _stream(stream)), "q8_1_quantize_rows")
+    _check(lib().q8_1_quantize_rows(_ptr(x), _ld(x), rows, k, _ptr(q8), _stream(stream, x.device)),
+           "q8_1_quantize_rows")
     return q8
 
 
@@ -298,7 +307,8 @@ def q6k_mmvq(blocks, q8, out=None, stream=None):
     rows = q8.shape[0]
     if out is None:
         out = torch.empty(rows, n, dtype=torch.bfloat16, device=blocks.device)
-    _check(lib().q6k_mmvq(_ptr(blocks), n, k, _ptr(q8), rows, _ptr(out), _ld(out), _stream(stream)), "q6k_mmvq")
+    _check(lib().q6k_mmvq(_ptr(blocks), n, k, _ptr(q8), rows, _ptr(out), _ld(out), _stream(stream, q8.device)),
+           "q6k_mmvq")
     return out
 
 
@@ -315,5 +325,5 @@ def q6k_lm_head(blocks, x, out=None, q8_scratch=None, stream=None):
     if q8_scratch is None:
         q8_scratch = torch.empty(Q6K_CHUNK_ROWS * (k // 32) * Q8_1_BLOCK_BYTES, dtype=torch.uint8, device=x.device)
     _check(lib().q6k_lm_head(_ptr(blocks), n, k, _ptr(x), _ld(x), rows, _ptr(out), _ld(out), _ptr(q8_scratch),
-                             _stream(stream)), "q6k_lm_head")
+                             _stream(stream, x.device)), "q6k_lm_head")
     return out

@@ -216,7 +216,6 @@ static int w8a8_proj_impl(const uint8_t* w, const float* w_scale, int n, int k, 
   if (!xq || !xs) return DLMH_ERR_NULL;
   if (!aligned16(xq) || k % 16 != 0) return DLMH_ERR_ALIGN;
   if (pass_rows(DLMH_OP_W8A8, k) <= 0) return DLMH_ERR_UNSUPPORTED;
-  if (up && (size_t)k * sizeof(float) > 200 * 1024) return DLMH_ERR_UNSUPPORTED;
   cudaStream_t s = as_stream(stream);
   for (int done = 0; done < rows;) {
     const int m = rows - done < DLMH_W8A8_MAX_ROWS ? rows - done : DLMH_W8A8_MAX_ROWS;

@@ -164,6 +164,10 @@ struct DeviceInfo {
 // Per-device properties, queried once per device (thread-safe after first call per device).
 DeviceInfo device_info();
 
+// cudaFuncAttributeMaxDynamicSharedMemorySize of `fn` on the current device raised to at
+// least `bytes`, set once per (function, device) and remembered (thread-safe).
+int ensure_dynamic_smem(const void* fn, int bytes);
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 inline int launch_status() {

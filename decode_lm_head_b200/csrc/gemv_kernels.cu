@@ -25,6 +25,28 @@ DeviceInfo device_info() {
   return cache[dev];
 }
 
+int ensure_dynamic_smem(const void* fn, int bytes) {
+  struct Entry {
+    const void* fn;
+    int dev;
+    int bytes;
+  };
+  static std::mutex mu;
+  static Entry done[256];
+  static int count = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DLMH_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  Entry* e = nullptr;
+  for (int i = 0; i < count; ++i)
+    if (done[i].fn == fn && done[i].dev == dev) e = &done[i];
+  if (e && e->bytes >= bytes) return DLMH_OK;
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return DLMH_ERR_CUDA;
+  if (!e && count < 256) e = &done[count++];
+  if (e) *e = Entry{fn, dev, bytes};
+  return DLMH_OK;
+}
+
 // The tier table is a pure function of the shape, so the host plan (dlmh_plan_chunks, no
 // GPU needed) and the launches agree: it uses the sm_100 shared-memory limit per block.
 constexpr size_t kSmemLimit = 232448 - 1024;
@@ -51,8 +73,7 @@ int launch_rowtile(const RowTileParams& p, cudaStream_t stream) {
   if (smem > kSmemLimit || smem + 256 > (size_t)di.smem_optin) return DLMH_ERR_UNSUPPORTED;
   auto kern = rowtile_gemv_kernel<F, NT, prefetch_depth<F, NT>()>;
   // Setting the attribute is cheap and idempotent; do it per call so every device is covered.
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-    return DLMH_ERR_CUDA;
+  if (ensure_dynamic_smem(reinterpret_cast<const void*>(kern), (int)smem) != DLMH_OK) return DLMH_ERR_CUDA;
   const int ntiles = (p.n + kTileRows - 1) / kTileRows;
   const int grid = ntiles < di.sms ? ntiles : di.sms;
   kern<<<grid, kThreads, smem, stream>>>(p);
@@ -102,8 +123,7 @@ int launch_stream_nkb(const RowTileParams& p, cudaStream_t stream) {
   if (di.sms <= 0) return DLMH_ERR_CUDA;
   const size_t smem = stream_smem_bytes<F, NT, C, NS>();
   auto kern = stream_gemv_kernel<F, NT, NKB, C, NS>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-    return DLMH_ERR_CUDA;
+  if (ensure_dynamic_smem(reinterpret_cast<const void*>(kern), (int)smem) != DLMH_OK) return DLMH_ERR_CUDA;
   const int ntiles = (p.n + kTileRows - 1) / kTileRows;
   const int grid = ntiles < di.sms ? ntiles : di.sms;
   kern<<<grid, kThreads, smem, stream>>>(p);

@@ -53,6 +53,10 @@ int w8a8_quantize_launch(const uint16_t* x, int64_t ldx, int rows, int k, uint8_
                          cudaStream_t s);
 int w8a8_silu_quantize_launch(const uint16_t* gate, const uint16_t* up, int64_t ld, int rows, int k, uint8_t* xq,
                               int64_t ldq, float* sx, cudaStream_t s);
+// W8A16 two-term split (act_quant.cu): rows [0, half) of `codes` get hi(x'), rows
+// [half, 2 half) lo(x'), padding rows zeros; x_mul[m] = 2^-e[m].
+int w8a16_split_launch(const uint16_t* x, int64_t ldx, int rows, int k, int half, uint8_t* codes, float* x_mul,
+                       cudaStream_t s);
 int q8_1_quantize_launch(const uint16_t* x, int64_t ldx, int rows, int k, uint8_t* q8, cudaStream_t s);
 int q6k_mmvq_launch(const uint8_t* blocks, int n, int k, const uint8_t* q8, int rows, uint16_t* out, int64_t ldc,
                     cudaStream_t s);

@@ -181,8 +181,7 @@ int q6k_mmvq_launch(const uint8_t* blocks, int n, int k, const uint8_t* q8, int 
   if (di.sms <= 0) return DLMH_ERR_CUDA;
   const size_t smem = q6k_smem_bytes(k);
   if (smem + 1024 > (size_t)di.smem_optin) return DLMH_ERR_UNSUPPORTED;
-  if (cudaFuncSetAttribute(q6k_mmvq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-    return DLMH_ERR_CUDA;
+  if (ensure_dynamic_smem(reinterpret_cast<const void*>(q6k_mmvq_kernel), (int)smem) != DLMH_OK) return DLMH_ERR_CUDA;
   Q6Params p{blocks, n, k, q8, rows, out, ldc};
   const int ntiles = (n + kQ6TileRows - 1) / kQ6TileRows;
   const int grid = ntiles < di.sms ? ntiles : di.sms;

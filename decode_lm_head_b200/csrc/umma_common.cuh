@@ -151,6 +151,42 @@ inline bool make_map_k128(CUtensorMap* m, const void* base, int elem_bytes, int 
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// make_map_k128 through a small cache keyed by (device, address, geometry): a tensor map
+// holds only the address and the geometry, so an equal key gives an equal map (thread-safe).
+inline bool cached_map_k128(CUtensorMap* m, const void* base, int elem_bytes, int rows, int64_t row_bytes,
+                            int64_t ld_bytes, int box_rows, int box_chunks) {
+  struct Entry {
+    const void* base;
+    int dev, elem_bytes, rows, box_rows, box_chunks;
+    int64_t row_bytes, ld_bytes;
+    CUtensorMap map;
+  };
+  constexpr int kEntries = 64;
+  static std::mutex mu;
+  static Entry cache[kEntries];
+  static int used = 0, next = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < used; ++i) {
+      const Entry& e = cache[i];
+      if (e.base == base && e.dev == dev && e.elem_bytes == elem_bytes && e.rows == rows && e.row_bytes == row_bytes &&
+          e.ld_bytes == ld_bytes && e.box_rows == box_rows && e.box_chunks == box_chunks) {
+        *m = e.map;
+        return true;
+      }
+    }
+  }
+  if (!make_map_k128(m, base, elem_bytes, rows, row_bytes, ld_bytes, box_rows, box_chunks)) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  Entry& e = cache[next];
+  e = Entry{base, dev, elem_bytes, rows, box_rows, box_chunks, row_bytes, ld_bytes, *m};
+  next = (next + 1) % kEntries;
+  if (used < kEntries) ++used;
+  return true;
+}
+
 // Launch with programmatic stream serialization: the kernel may start while the preceding
 // kernel of the stream finishes; it must call grid_dependency_wait() before touching
 // anything that kernel writes.

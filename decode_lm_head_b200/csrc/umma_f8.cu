@@ -334,79 +334,8 @@ __global__ void __launch_bounds__(kBM) umma_f8_fixup_kernel(const UmmaParams p, 
 
 constexpr size_t kUmmaSmemLimit = 232448 - 2048;
 
-// Per-row exponent e with max|x| * 2^e in [2^7, 2^8), clamped so that 2^e and 2^-e are
-// normal f32 values (rows whose maximum is below 2^-119 lose precision; zero rows give 0).
-__device__ __forceinline__ int e4m3_split_exponent(float amax) {
-  if (!(amax > 0.f)) return 0;
-  const uint32_t b = __float_as_uint(amax);
-  const int field = (int)((b >> 23) & 0xff);
-  const int E = field != 0 ? field - 127 : (31 - __clz((int)(b & 0x7fffff))) - 149;  // amax in [2^E, 2^(E+1))
-  return max(-126, min(126, 7 - E));
-}
-
-// W8A16 activation split: CTA m writes E4M3 rows codes[m] = hi(x'[m]) and codes[half + m] =
-// lo(x'[m]) (zero rows for m >= rows) and x_mul[m] = 2^-e[m].  k a multiple of 8, x
-// 16-byte aligned with ldx a multiple of 8.
-__global__ void __launch_bounds__(256) w8a16_split_kernel(const uint16_t* __restrict__ x, int64_t ldx, int rows,
-                                                          int k, int half, uint8_t* __restrict__ codes,
-                                                          float* __restrict__ x_mul) {
-  __shared__ float s_red[8];
-  grid_dependents_launch();  // the GEMV may start its prologue and weight loads now
-  const int m = blockIdx.x;
-  uint8_t* hi_row = codes + (int64_t)m * k;
-  uint8_t* lo_row = codes + (int64_t)(half + m) * k;
-  if (m >= rows) {
-    for (int k8 = threadIdx.x * 8; k8 < k; k8 += 256 * 8) {
-      *reinterpret_cast<uint2*>(hi_row + k8) = make_uint2(0, 0);
-      *reinterpret_cast<uint2*>(lo_row + k8) = make_uint2(0, 0);
-    }
-    if (threadIdx.x == 0) x_mul[m] = 0.f;
-    return;
-  }
-  const uint16_t* xr = x + (int64_t)m * ldx;
-  float amax = 0.f;
-  for (int k8 = threadIdx.x * 8; k8 < k; k8 += 256 * 8) {
-    const uint4 v = ldg_nc(xr + k8);
-    const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      amax = fmaxf(amax, fabsf(bf16_bits_to_f32(wv[i] & 0xffffu)));
-      amax = fmaxf(amax, fabsf(bf16_bits_to_f32(wv[i] >> 16)));
-    }
-  }
-  amax = warp_max(amax);
-  if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = amax;
-  __syncthreads();
-  amax = s_red[0];
-#pragma unroll
-  for (int i = 1; i < 8; ++i) amax = fmaxf(amax, s_red[i]);
-  const int e = e4m3_split_exponent(amax);
-  const float mul = __int_as_float((127 + e) << 23);
-  if (threadIdx.x == 0) x_mul[m] = __int_as_float((127 - e) << 23);
-  for (int k8 = threadIdx.x * 8; k8 < k; k8 += 256 * 8) {
-    const uint4 v = ldg_nc(xr + k8);
-    const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-    uint32_t hi[2] = {0, 0}, lo[2] = {0, 0};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {  // elements 2i, 2i+1 of this 8-element group
-      const float a = bf16_bits_to_f32(wv[i] & 0xffffu) * mul;  // exact (power of two)
-      const float b = bf16_bits_to_f32(wv[i] >> 16) * mul;
-      const uint32_t h2 = f32x2_to_e4m3x2(a, b);
-      const uint32_t hf = e4m3x2_to_f16x2((uint16_t)h2);
-      const float ra = a - f16_bits_to_f32(hf & 0xffffu);  // exact residual
-      const float rb = b - f16_bits_to_f32(hf >> 16);
-      const uint32_t l2 = f32x2_to_e4m3x2(ra * 16.f, rb * 16.f);
-      hi[i >> 1] |= h2 << (16 * (i & 1));
-      lo[i >> 1] |= l2 << (16 * (i & 1));
-    }
-    *reinterpret_cast<uint2*>(hi_row + k8) = make_uint2(hi[0], hi[1]);
-    *reinterpret_cast<uint2*>(lo_row + k8) = make_uint2(lo[0], lo[1]);
-  }
-}
-
 // Library-owned stream-ordered pool for the W8A16 activation codes and the stream-K partial
-// sums (one per device; memory
-// is kept between calls so that steady-state calls map nothing).
+// sums (one per device; memory is kept between calls so that steady-state calls map nothing).
 cudaMemPool_t scratch_pool(int dev) {
   static std::mutex mu;
   static cudaMemPool_t pools[64] = {};
@@ -454,11 +383,10 @@ int launch_umma_f8(const uint8_t* w, const float* w_scale, int n, int k, const u
   if (ns < 2) return DLMH_ERR_UNSUPPORTED;
   p.ns = ns;
   CUtensorMap mw, mx;
-  if (!make_map_k128(&mw, w, 1, n, k, k, kBM, kKC) || !make_map_k128(&mx, b_codes, 1, b_rows, k, ldb, p.nb, kKC))
+  if (!cached_map_k128(&mw, w, 1, n, k, k, kBM, kKC) || !cached_map_k128(&mx, b_codes, 1, b_rows, k, ldb, p.nb, kKC))
     return DLMH_ERR_CUDA;
   const size_t smem = (size_t)ns * p.stage_bytes + 1024;
-  if (cudaFuncSetAttribute(umma_f8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-    return DLMH_ERR_CUDA;
+  if (ensure_dynamic_smem(reinterpret_cast<const void*>(umma_f8_kernel), (int)smem) != DLMH_OK) return DLMH_ERR_CUDA;
   // schedule: whole tiles in full waves over the SMs, the rest split into units
   const int ntiles = (n + kBM - 1) / kBM;
   p.spt = (k / 128 + kKC - 1) / kKC;
@@ -532,8 +460,7 @@ int w8a16_umma_run(const uint8_t* w, const float* w_scale, int n, int k, const u
   for (int done = 0; done < rows && rc == DLMH_OK;) {
     const int m = rows - done < 128 ? rows - done : 128;
     const int half = (m + 7) / 8 * 8;  // hi rows [0, half), lo rows [half, 2 half)
-    w8a16_split_kernel<<<half, 256, 0, s>>>(x + (int64_t)done * ldx, ldx, m, k, half, codes, x_mul);
-    rc = launch_status();
+    rc = w8a16_split_launch(x + (int64_t)done * ldx, ldx, m, k, half, codes, x_mul, s);
     if (rc == DLMH_OK)
       rc = launch_umma_f8(w, w_scale, n, k, codes, k, 2 * half, x_mul, m, 1, out + (int64_t)done * ldc, ldc, s,
                           nullptr, 0, 1);
