@@ -264,7 +264,9 @@ int device_fault(int reset) {
   }
   const int u = umma_fault(reset);
   if (u < 0) return u;
-  return v | (u << 8);
+  const int q6 = q6k_fault(reset);
+  if (q6 < 0) return q6;
+  return v | (u << 8) | (q6 << 16);
 }
 
 int max_tier_rows(int op, int k) {

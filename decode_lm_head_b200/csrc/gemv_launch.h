@@ -58,6 +58,8 @@ int w8a8_silu_quantize_launch(const uint16_t* gate, const uint16_t* up, int64_t 
 int w8a16_split_launch(const uint16_t* x, int64_t ldx, int rows, int k, int half, uint8_t* codes, float* x_mul,
                        cudaStream_t s);
 int q8_1_quantize_launch(const uint16_t* x, int64_t ldx, int rows, int k, uint8_t* q8, cudaStream_t s);
+// Fault bits of the streamed Q6_K kernel's bounded waits (read synchronously).
+int q6k_fault(int reset);
 int q6k_mmvq_launch(const uint8_t* blocks, int n, int k, const uint8_t* q8, int rows, uint16_t* out, int64_t ldc,
                     cudaStream_t s);
 

@@ -17,6 +17,7 @@
 // 16-bit read-only loads (each 32-byte sector still comes from DRAM once).
 #include "dlmh_common.cuh"
 #include "gemv_launch.h"
+#include "umma_common.cuh"
 
 namespace dlmh {
 namespace {
@@ -168,6 +169,195 @@ __global__ void __launch_bounds__(kQ6Threads, 1) q6k_mmvq_kernel(const Q6Params 
   }
 }
 
+// ---------------------------------------------------------------------------------------
+// Streamed variant: the weight reaches shared memory through 1-D bulk copies (TMA) of 8-row
+// stages.  8 rows of Q6_K are 8 * 210 * (k / 256) = 1680 * (k / 256) bytes, a multiple of 16,
+// so every full stage starts and ends 16-byte aligned for any k; a ragged last stage copies
+// its 16-byte-multiple prefix in bulk and its last few bytes with plain loads.  A 16-row MMA
+// tile is two consecutive stages; the ring holds NS >= 3 stages, so the next tile is in
+// flight while this one is computed.  Each lane reads its bytes from shared memory as aligned
+// 32-bit pairs joined by a funnel shift (super-blocks are only 2-byte aligned).  The
+// arithmetic, its order and the warp split are those of q6k_mmvq_kernel, so the two give the
+// same bits.
+constexpr int kQ6StageRows = 8;
+constexpr int kQ6MaxStages = 6;
+static __device__ int q6_fault_word = 0;
+
+__device__ __forceinline__ uint32_t lds_u32_a2(uint32_t saddr) {  // 2-byte aligned 32-bit load
+  const uint32_t a = saddr & ~3u;
+  uint32_t w0, w1;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w0) : "r"(a));
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w1) : "r"(a + 4));
+  return __funnelshift_r(w0, w1, (saddr & 3u) * 8u);
+}
+__device__ __forceinline__ uint32_t lds_u16(uint32_t saddr) {
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(saddr));
+  return v;
+}
+
+struct Q6StreamParams {
+  Q6Params q;
+  int ns;             // ring stages
+  int stage_stride;   // bytes per stage slot (>= 8 rows, multiple of 128)
+  int ring_offset;    // byte offset of the ring in dynamic shared memory
+};
+
+__global__ void __launch_bounds__(kQ6Threads, 1) q6k_stream_kernel(const Q6StreamParams sp) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ __align__(8) uint64_t full[kQ6MaxStages];
+  const Q6Params& p = sp.q;
+  const int nsb = p.k / 256;
+  const int nb32 = p.k / 32;
+  const int rs = q6_row_stride(p.k);
+  const int64_t row_bytes = (int64_t)nsb * 210;
+  int8_t* xs = reinterpret_cast<int8_t*>(smem);                              // [8][rs]
+  float* dx = reinterpret_cast<float*>(smem + kQ6MaxRows * rs);              // [8][nb32]
+  float* red = dx + kQ6MaxRows * nb32;                                       // [2][16 warps][32 lanes][4]
+  const uint32_t ring = smem_u32(smem + sp.ring_offset);
+  const uint32_t full0 = smem_u32(full);
+
+  const int ntiles = (p.n + kQ6TileRows - 1) / kQ6TileRows;
+  const int T0 = (int)((int64_t)blockIdx.x * ntiles / gridDim.x);
+  const int T1 = (int)((int64_t)(blockIdx.x + 1) * ntiles / gridDim.x);
+  const int nstages = 2 * (T1 - T0);
+
+  // Stage s of this CTA: rows [16 (T0 + s/2) + 8 (s%2), +8) clipped to n, into slot s % NS.
+  auto produce = [&](int s) {
+    const int slot = s % sp.ns;
+    const int64_t r0 = (int64_t)(T0 + s / 2) * kQ6TileRows + (s % 2) * kQ6StageRows;
+    const int64_t nr = r0 >= p.n ? 0 : (p.n - r0 < kQ6StageRows ? p.n - r0 : kQ6StageRows);
+    const uint32_t bytes = (uint32_t)(nr * row_bytes);
+    const uint32_t bulk = bytes & ~15u;
+    const uint32_t dst = ring + (uint32_t)slot * sp.stage_stride;
+    const uint8_t* src = p.blocks + r0 * row_bytes;
+    for (uint32_t o = bulk; o < bytes; o += 2) {  // ragged tail: at most 7 half-words
+      const uint32_t v = ldg_u16(src + o);
+      asm volatile("st.shared.u16 [%0], %1;" ::"r"(dst + o), "h"((unsigned short)v) : "memory");
+    }
+    umma::expect_tx(full0 + 8u * slot, bulk);
+    if (bulk) umma::bulk_load(dst, src, bulk, full0 + 8u * slot, umma::l2_policy_evict_first());
+  };
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < sp.ns; ++i) umma::bar_init(full0 + 8u * i, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    for (int s = 0; s < sp.ns && s < nstages; ++s) produce(s);
+  }
+
+  // ---- stage the q8_1 rows (while the first weight stages are in flight)
+  for (int it = threadIdx.x; it < kQ6MaxRows * nb32; it += kQ6Threads) {
+    const int m = it / nb32, b = it % nb32;
+    uint32_t w[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    float d = 0.f;
+    if (m < p.rows) {
+      const uint8_t* blk = p.q8 + ((int64_t)m * nb32 + b) * 36;
+      const uint32_t* bw = reinterpret_cast<const uint32_t*>(blk);
+      d = f16_bits_to_f32(bw[0] & 0xffff);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) w[i] = bw[1 + i];
+    }
+    dx[m * nb32 + b] = d;
+    uint4* dst = reinterpret_cast<uint4*>(xs + m * rs + b * 32);
+    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  }
+  __syncthreads();
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int nsbw = (nsb + kQ6Warps - 1) / kQ6Warps;
+  const int8_t* xrow = xs + g * rs;  // B column g
+  int parity = 0;
+
+  for (int i = 0; T0 + i < T1; ++i) {
+    const int tile = T0 + i;
+    const int sa = 2 * i, sb2 = 2 * i + 1;
+    const bool oka = umma::wait(full0 + 8u * (sa % sp.ns), (sa / sp.ns) & 1);
+    const bool okb = umma::wait(full0 + 8u * (sb2 % sp.ns), (sb2 / sp.ns) & 1);
+    if (!(oka && okb)) atomicOr(&q6_fault_word, 1);
+    const uint32_t base_a = ring + (uint32_t)(sa % sp.ns) * sp.stage_stride + (uint32_t)(g * row_bytes);
+    const uint32_t base_b = ring + (uint32_t)(sb2 % sp.ns) * sp.stage_stride + (uint32_t)(g * row_bytes);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    const int r0 = tile * kQ6TileRows + g;
+    const bool va = r0 < p.n, vb = r0 + 8 < p.n;
+    for (int s = 0; s < nsbw; ++s) {
+      const int sb = warp * nsbw + s;
+      if (sb >= nsb) break;
+      const uint32_t ba = base_a + (uint32_t)sb * 210u;
+      const uint32_t bb = base_b + (uint32_t)sb * 210u;
+      uint32_t qla[8], qlb[8], qha[4], qhb[4], sca[4], scb[4];
+      float da = 0.f, db = 0.f;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {  // ql bytes 16q + 4t
+        qla[q] = va ? lds_u32_a2(ba + 16 * q + 4 * t) : 0u;
+        qlb[q] = vb ? lds_u32_a2(bb + 16 * q + 4 * t) : 0u;
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {  // qh bytes 128 + 16q + 4t, scales 192 + 4q
+        qha[q] = va ? lds_u32_a2(ba + 128 + 16 * q + 4 * t) : 0u;
+        qhb[q] = vb ? lds_u32_a2(bb + 128 + 16 * q + 4 * t) : 0u;
+        sca[q] = va ? lds_u32_a2(ba + 192 + 4 * q) : 0u;
+        scb[q] = vb ? lds_u32_a2(bb + 192 + 4 * q) : 0u;
+      }
+      if (va) da = f16_bits_to_f32(lds_u16(ba + 208));
+      if (vb) db = f16_bits_to_f32(lds_u16(bb + 208));
+
+      const int8_t* xsb = xrow + sb * 256;
+#pragma unroll
+      for (int blk = 0; blk < 8; ++blk) {  // q8_1 block = sub-blocks 2blk, 2blk+1
+        float part[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int hj = 0; hj < 2; ++hj) {
+          const int j = 2 * blk + hj;
+          const int h = j >> 3, u = (j & 7) >> 1;
+          const int qi = 4 * h + 2 * (u & 1) + (j & 1);
+          const int hi = 2 * h + (j & 1);
+          const int nsh = (u >> 1) * 4, hsh = 2 * u;
+          const uint32_t qa = ((qla[qi] >> nsh) & 0x0f0f0f0fu) | (((qha[hi] >> hsh) & 0x03030303u) << 4);
+          const uint32_t qb = ((qlb[qi] >> nsh) & 0x0f0f0f0fu) | (((qhb[hi] >> hsh) & 0x03030303u) << 4);
+          const uint32_t bx = *reinterpret_cast<const uint32_t*>(xsb + 16 * j + 4 * t);
+          int d4[4] = {0, 0, 0, 0};
+          mma_s8_16816(d4, q6_to_s8x4(qa), q6_to_s8x4(qb), bx);
+          const float ra = da * (float)(int8_t)((sca[j >> 2] >> (8 * (j & 3))) & 0xff);
+          const float rb = db * (float)(int8_t)((scb[j >> 2] >> (8 * (j & 3))) & 0xff);
+          part[0] += (float)d4[0] * ra;
+          part[1] += (float)d4[1] * ra;
+          part[2] += (float)d4[2] * rb;
+          part[3] += (float)d4[3] * rb;
+        }
+        const int b32 = sb * 8 + blk;
+        const float dx0 = dx[(2 * t) * nb32 + b32], dx1 = dx[(2 * t + 1) * nb32 + b32];
+        acc[0] += part[0] * dx0;
+        acc[1] += part[1] * dx1;
+        acc[2] += part[2] * dx0;
+        acc[3] += part[3] * dx1;
+      }
+    }
+    // ---- fixed-order reduction over warps; after its barrier the tile's stages are free
+    float* rb_ = red + parity * (kQ6Warps * 32 * 4);
+    reinterpret_cast<float4*>(rb_)[warp * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      if (sa + sp.ns < nstages) produce(sa + sp.ns);
+      if (sb2 + sp.ns < nstages) produce(sb2 + sp.ns);
+    }
+    if (threadIdx.x < kQ6TileRows * kQ6MaxRows) {
+      const int rr = threadIdx.x % kQ6TileRows, cc = threadIdx.x / kQ6TileRows;
+      const int row = tile * kQ6TileRows + rr;
+      if (cc < p.rows && row < p.n) {
+        const int gg = rr & 7, up = rr >> 3;
+        const int ln = gg * 4 + (cc >> 1), comp = up * 2 + (cc & 1);
+        float sum = 0.f;
+#pragma unroll
+        for (int ww = 0; ww < kQ6Warps; ++ww) sum += rb_[(ww * 32 + ln) * 4 + comp];
+        p.out[(int64_t)cc * p.ldc + row] = f32_to_bf16_bits(sum);
+      }
+    }
+    parity ^= 1;
+  }
+}
+
 size_t q6k_smem_bytes(int k) {
   int rs = k + ((16 - k % 128) + 128) % 128;
   return (size_t)kQ6MaxRows * rs + (size_t)kQ6MaxRows * (k / 32) * 4 + 2ull * kQ6Warps * 32 * 4 * 4;
@@ -179,14 +369,40 @@ int q6k_mmvq_launch(const uint8_t* blocks, int n, int k, const uint8_t* q8, int 
                     cudaStream_t s) {
   const DeviceInfo di = device_info();
   if (di.sms <= 0) return DLMH_ERR_CUDA;
-  const size_t smem = q6k_smem_bytes(k);
-  if (smem + 1024 > (size_t)di.smem_optin) return DLMH_ERR_UNSUPPORTED;
-  if (ensure_dynamic_smem(reinterpret_cast<const void*>(q6k_mmvq_kernel), (int)smem) != DLMH_OK) return DLMH_ERR_CUDA;
+  const size_t base_smem = q6k_smem_bytes(k);
   Q6Params p{blocks, n, k, q8, rows, out, ldc};
   const int ntiles = (n + kQ6TileRows - 1) / kQ6TileRows;
   const int grid = ntiles < di.sms ? ntiles : di.sms;
-  q6k_mmvq_kernel<<<grid, kQ6Threads, smem, s>>>(p);
+  // streamed variant when the ring holds at least three 8-row stages and the blocks start
+  // 16-byte aligned (then every 8-row stage does); both variants give the same bits
+  const size_t ring_offset = (base_smem + 127) / 128 * 128;
+  const size_t stage_stride = ((size_t)kQ6StageRows * (k / 256) * 210 + 127) / 128 * 128;
+  const size_t limit = (size_t)di.smem_optin > 2048 ? (size_t)di.smem_optin - 2048 : 0;
+  int ns = limit > ring_offset ? (int)((limit - ring_offset) / stage_stride) : 0;
+  if (ns > kQ6MaxStages) ns = kQ6MaxStages;
+  if (ns >= 3 && (reinterpret_cast<uintptr_t>(blocks) & 15u) == 0) {
+    const size_t smem = ring_offset + (size_t)ns * stage_stride;
+    if (ensure_dynamic_smem(reinterpret_cast<const void*>(q6k_stream_kernel), (int)smem) != DLMH_OK)
+      return DLMH_ERR_CUDA;
+    Q6StreamParams sp{p, ns, (int)stage_stride, (int)ring_offset};
+    q6k_stream_kernel<<<grid, kQ6Threads, smem, s>>>(sp);
+    return launch_status();
+  }
+  if (base_smem + 1024 > (size_t)di.smem_optin) return DLMH_ERR_UNSUPPORTED;
+  if (ensure_dynamic_smem(reinterpret_cast<const void*>(q6k_mmvq_kernel), (int)base_smem) != DLMH_OK)
+    return DLMH_ERR_CUDA;
+  q6k_mmvq_kernel<<<grid, kQ6Threads, base_smem, s>>>(p);
   return launch_status();
+}
+
+int q6k_fault(int reset) {
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, q6_fault_word, sizeof(int)) != cudaSuccess) return DLMH_ERR_CUDA;
+  if (reset) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(q6_fault_word, &zero, sizeof(int)) != cudaSuccess) return DLMH_ERR_CUDA;
+  }
+  return v;
 }
 
 }  // namespace dlmh

@@ -310,6 +310,24 @@ def test_q6k_mmvq_and_head(n, k):
         assert np.array_equal(part, full[:m]), f"row invariance M={m}"
 
 
+@pytest.mark.parametrize("n,k", [(1000, 7168), (37, 512), (45, 1280)])
+def test_q6k_streamed_and_register_kernels_agree(n, k):
+    # 16-byte-aligned blocks take the TMA-streamed kernel, 2-byte-aligned ones the
+    # register-load kernel; both use the same arithmetic in the same order
+    blocks = synth.q6k_blocks(n, k, 6, DEV)
+    flat = torch.zeros(blocks.numel() + 16, dtype=torch.uint8, device=DEV)
+    flat[2:2 + blocks.numel()] = blocks.reshape(-1)
+    shifted = flat[2:2 + blocks.numel()].view(blocks.shape)
+    assert shifted.data_ptr() % 16 == 2
+    x = synth.bf16_rows(8, k, 6, DEV)
+    q8 = dl.q8_1_quantize_rows(x)
+    a = bits(dl.q6k_mmvq(blocks, q8))
+    b = bits(dl.q6k_mmvq(shifted, q8))
+    assert np.array_equal(a, b)
+    assert_bf16_close(a, og.q6k_mmvq(bits(blocks), bits(q8)), f"q6k streamed n={n} k={k}")
+    assert dl.device_fault(reset=True) == 0
+
+
 # ---------------------------------------------------------------------------
 # full-size heads, sampled outputs
 # ---------------------------------------------------------------------------
