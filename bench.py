@@ -150,7 +150,9 @@ class ClockSampler:
                 "reasons": sorted(reasons)}
 
 
-def dist_setup(args):
+def dist_setup(args, backend="nccl"):
+    """Join the process group when launched with WORLD_SIZE > 1 (torchrun); one GPU per rank
+    for NCCL, none for gloo (the host-side path the CPU tests exercise)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -159,10 +161,13 @@ def dist_setup(args):
 
         import torch.distributed as dist
 
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    else:
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif backend == "nccl":
         torch.cuda.set_device(0)
     return world, rank, local
 
@@ -175,13 +180,20 @@ def barrier(world):
 
 
 def max_over_ranks(v, world):
+    """The largest of every rank's value (the job's device time is its slowest rank's)."""
     if world == 1:
         return v
     import torch.distributed as dist
 
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_value(world, steps, step_bytes, elapsed_ms):
+    """Whole-job weight GB/s: every rank streams step_bytes per step; time is the max over ranks."""
+    return world * steps * step_bytes / (elapsed_ms * 1e-3) / 1e9
 
 
 # ---------------------------------------------------------------------------------------
@@ -400,7 +412,7 @@ def run_ours(args):
     clocks = clk.summary()
 
     step_bytes = sum(passes(m) * weight_bytes() for m in ROWS)
-    value = world * args.steps * step_bytes / (elapsed_ms * 1e-3) / 1e9
+    value = job_value(world, args.steps, step_bytes, elapsed_ms)
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     passes_per_step = sum(passes(m) for m in ROWS)
     launches_per_step = sum(launches_per_call(m, sms) for m in ROWS)
@@ -438,7 +450,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     barrier(world)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-    e2e_value = world * args.steps * step_bytes / (e2e_ms * 1e-3) / 1e9
+    e2e_value = job_value(world, args.steps, step_bytes, e2e_ms)
 
     formats = None
     if args.all_formats:
