@@ -11,6 +11,7 @@ from ._lib import (  # noqa: F401
     OP_W4A16,
     OP_W8A8,
     OP_W8A16,
+    check_bounded_wait,
     device_fault,
     error_string,
     lib,

@@ -55,6 +55,7 @@ _SIGNATURES = {
     "q6k_lm_head": [_P, _I, _I, _P, _L, _I, _P, _L, _P, _P],
     "dlmh_plan_chunks": [_I, _I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I), _I],
     "dlmh_device_fault": [_I],
+    "dlmh_check_bounded_wait": [_P],
     "dlmh_version": [],
 }
 
@@ -98,6 +99,11 @@ def device_fault(reset=False):
     if rc < 0:
         raise DlmhError(rc, "dlmh_device_fault")
     return rc
+
+
+def check_bounded_wait(stream=None):
+    """Run the library's bounded-wait check on the current device (see dlmh.h)."""
+    _check(lib().dlmh_check_bounded_wait(_stream(stream)), "dlmh_check_bounded_wait")
 
 
 def _check(rc, what):

@@ -76,6 +76,8 @@ int dlmh_version(void) { return 100; }
 
 int dlmh_device_fault(int reset) { return dlmh::device_fault(reset); }
 
+int dlmh_check_bounded_wait(void* stream) { return dlmh::bounded_wait_check(as_stream(stream)); }
+
 const char* dlmh_error_string(int code) {
   switch (code) {
     case DLMH_OK: return "ok";

@@ -37,6 +37,9 @@ int w8a8_proj_fixed_scratch(const uint8_t* w, const float* w_scale, int n, int k
                             size_t partial_cap, cudaStream_t stream);
 // Fault bits of the tensor-core kernel's bounded waits (read synchronously).
 int umma_fault(int reset);
+// Runs one bounded mbarrier wait that can never complete; DLMH_OK if it gave up and recorded
+// its fault bit (then cleared again), synchronizes `s`.
+int bounded_wait_check(cudaStream_t s);
 
 // Tensor-core W8A16 (the same kernel; activations split into two exact E4M3 terms): one
 // weight pass per 128 rows, taken for every row count whenever w8a16_umma_supported(k)

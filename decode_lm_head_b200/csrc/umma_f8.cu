@@ -50,6 +50,7 @@ constexpr int kChunkBytesA = kBM * 128;
 constexpr int kMaxUStages = 6;
 
 static __device__ int umma_fault_word = 0;  // 1: producer, 2: MMA (stage), 4: MMA (tmem), 8: epilogue
+constexpr int kWaitProbeBit = 0x40;         // set only by the bounded-wait check
 
 __device__ __forceinline__ void umma_f8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, int accum) {
   asm volatile(
@@ -468,6 +469,31 @@ int w8a16_umma_run(const uint8_t* w, const float* w_scale, int n, int k, const u
   }
   if (cudaFreeAsync(scratch, s) != cudaSuccess && rc == DLMH_OK) rc = DLMH_ERR_CUDA;
   return rc;
+}
+
+namespace {
+
+// One thread waits (bounded) on an mbarrier that nothing will ever complete.
+__global__ void bounded_wait_probe_kernel() {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = smem_u32(&bar);
+  bar_init(b, 1);
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  if (!wait(b, 0)) atomicOr(&umma_fault_word, kWaitProbeBit);
+}
+
+}  // namespace
+
+int bounded_wait_check(cudaStream_t s) {
+  int before = 0;
+  if (cudaMemcpyFromSymbol(&before, umma_fault_word, sizeof(int)) != cudaSuccess) return DLMH_ERR_CUDA;
+  bounded_wait_probe_kernel<<<1, 1, 0, s>>>();
+  if (launch_status() != DLMH_OK || cudaStreamSynchronize(s) != cudaSuccess) return DLMH_ERR_CUDA;
+  int after = 0;
+  if (cudaMemcpyFromSymbol(&after, umma_fault_word, sizeof(int)) != cudaSuccess) return DLMH_ERR_CUDA;
+  const int restored = before & ~kWaitProbeBit;  // leave the other bits as they were
+  if (cudaMemcpyToSymbol(umma_fault_word, &restored, sizeof(int)) != cudaSuccess) return DLMH_ERR_CUDA;
+  return (after & kWaitProbeBit) ? DLMH_OK : DLMH_ERR_CUDA;
 }
 
 int umma_fault(int reset) {

@@ -271,6 +271,13 @@ DLMH_API int dlmh_plan_chunks(int op, int rows, int k, int* offsets, int* counts
  * (Library diagnostic, no counterpart on the pages.) */
 DLMH_API int dlmh_device_fault(int reset);
 
+/* Failure-detection check (library diagnostic, no counterpart on the pages): runs one bounded
+ * mbarrier wait on a barrier that nothing completes, the same wait every TMA / tensor-core
+ * kernel here uses instead of an unbounded spin, and returns DLMH_OK when it gave up (after
+ * 2^22 polls, well under a second) and recorded its fault bit; the bit is cleared again and the
+ * other bits are left as they were.  Synchronizes `stream`; DLMH_ERR_CUDA otherwise. */
+DLMH_API int dlmh_check_bounded_wait(void* stream);
+
 /* Static description of a status code (never NULL). */
 DLMH_API const char* dlmh_error_string(int code);
 
