@@ -38,6 +38,48 @@ __device__ __forceinline__ uint32_t q6_to_s8x4(uint32_t q) {
   return x | (s * 6u);                          // sign-extend bit 5 into bits 6, 7
 }
 
+// One super-block for rows g (a) and g+8 (b) of a 16-row tile against activation columns 2t
+// and 2t+1 (acc[0..1]: row a, acc[2..3]: row b).  Per q8_1 block (sub-blocks j0, j1) the two
+// exact int32 sub-block dots are scaled by their int8 sub-scales and summed in int32 -- exact,
+// |sum| < 2^24 so its f32 conversion is exact too -- then multiplied by the super-block d and
+// the q8_1 d in f32.  Shared by both Q6_K kernels so that they give the same bits.
+__device__ __forceinline__ void q6_superblock(float (&acc)[4], const uint32_t (&qla)[8], const uint32_t (&qlb)[8],
+                                              const uint32_t (&qha)[4], const uint32_t (&qhb)[4],
+                                              const uint32_t (&sca)[4], const uint32_t (&scb)[4], float da, float db,
+                                              const int8_t* xsb, const float* dx, int nb32, int sb, int t) {
+#pragma unroll
+  for (int blk = 0; blk < 8; ++blk) {  // q8_1 block = sub-blocks 2blk, 2blk+1
+    int is0 = 0, is1 = 0, is2 = 0, is3 = 0;
+#pragma unroll
+    for (int hj = 0; hj < 2; ++hj) {
+      const int j = 2 * blk + hj;
+      const int h = j >> 3, u = (j & 7) >> 1;
+      // ql word index: 64h + 32(u&1) + 16(j&1) -> q = 4h + 2(u&1) + (j&1); qh: 32h + 16(j&1)
+      const int qi = 4 * h + 2 * (u & 1) + (j & 1);
+      const int hi = 2 * h + (j & 1);
+      const int nsh = (u >> 1) * 4, hsh = 2 * u;
+      const uint32_t qa = ((qla[qi] >> nsh) & 0x0f0f0f0fu) | (((qha[hi] >> hsh) & 0x03030303u) << 4);
+      const uint32_t qb = ((qlb[qi] >> nsh) & 0x0f0f0f0fu) | (((qhb[hi] >> hsh) & 0x03030303u) << 4);
+      const uint32_t bx = *reinterpret_cast<const uint32_t*>(xsb + 16 * j + 4 * t);
+      int d4[4] = {0, 0, 0, 0};
+      mma_s8_16816(d4, q6_to_s8x4(qa), q6_to_s8x4(qb), bx);
+      const int sha = 24 - 8 * (j & 3);  // sign-extend byte j&3 of the scale word
+      const int ra = (int)(sca[j >> 2] << sha) >> 24;
+      const int rb = (int)(scb[j >> 2] << sha) >> 24;
+      is0 += d4[0] * ra;
+      is1 += d4[1] * ra;
+      is2 += d4[2] * rb;
+      is3 += d4[3] * rb;
+    }
+    const int b32 = sb * 8 + blk;
+    const float dx0 = dx[(2 * t) * nb32 + b32], dx1 = dx[(2 * t + 1) * nb32 + b32];
+    acc[0] += ((float)is0 * da) * dx0;
+    acc[1] += ((float)is1 * da) * dx1;
+    acc[2] += ((float)is2 * db) * dx0;
+    acc[3] += ((float)is3 * db) * dx1;
+  }
+}
+
 struct Q6Params {
   const uint8_t* blocks;
   int n, k;
@@ -117,37 +159,7 @@ __global__ void __launch_bounds__(kQ6Threads, 1) q6k_mmvq_kernel(const Q6Params 
       if (va) da = f16_bits_to_f32(ldg_u16(ba + 208));
       if (vb) db = f16_bits_to_f32(ldg_u16(bb + 208));
 
-      const int8_t* xsb = xrow + sb * 256;
-#pragma unroll
-      for (int blk = 0; blk < 8; ++blk) {  // q8_1 block = sub-blocks 2blk, 2blk+1
-        float part[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int hj = 0; hj < 2; ++hj) {
-          const int j = 2 * blk + hj;
-          const int h = j >> 3, u = (j & 7) >> 1;
-          // ql word index: 64h + 32(u&1) + 16(j&1) -> i = 4h + 2(u&1) + (j&1)
-          const int qi = 4 * h + 2 * (u & 1) + (j & 1);
-          const int hi = 2 * h + (j & 1);  // qh: 32h + 16(j&1)
-          const int nsh = (u >> 1) * 4, hsh = 2 * u;
-          const uint32_t qa = ((qla[qi] >> nsh) & 0x0f0f0f0fu) | (((qha[hi] >> hsh) & 0x03030303u) << 4);
-          const uint32_t qb = ((qlb[qi] >> nsh) & 0x0f0f0f0fu) | (((qhb[hi] >> hsh) & 0x03030303u) << 4);
-          const uint32_t bx = *reinterpret_cast<const uint32_t*>(xsb + 16 * j + 4 * t);
-          int d4[4] = {0, 0, 0, 0};
-          mma_s8_16816(d4, q6_to_s8x4(qa), q6_to_s8x4(qb), bx);
-          const float ra = da * (float)(int8_t)((sca[j >> 2] >> (8 * (j & 3))) & 0xff);
-          const float rb = db * (float)(int8_t)((scb[j >> 2] >> (8 * (j & 3))) & 0xff);
-          part[0] += (float)d4[0] * ra;
-          part[1] += (float)d4[1] * ra;
-          part[2] += (float)d4[2] * rb;
-          part[3] += (float)d4[3] * rb;
-        }
-        const int b32 = sb * 8 + blk;
-        const float dx0 = dx[(2 * t) * nb32 + b32], dx1 = dx[(2 * t + 1) * nb32 + b32];
-        acc[0] += part[0] * dx0;
-        acc[1] += part[1] * dx1;
-        acc[2] += part[2] * dx0;
-        acc[3] += part[3] * dx1;
-      }
+      q6_superblock(acc, qla, qlb, qha, qhb, sca, scb, da, db, xrow + sb * 256, dx, nb32, sb, t);
     }
     // ---- fixed-order reduction over warps
     float* rb_ = red + parity * (kQ6Warps * 32 * 4);
@@ -303,36 +315,7 @@ __global__ void __launch_bounds__(kQ6Threads, 1) q6k_stream_kernel(const Q6Strea
       if (va) da = f16_bits_to_f32(lds_u16(ba + 208));
       if (vb) db = f16_bits_to_f32(lds_u16(bb + 208));
 
-      const int8_t* xsb = xrow + sb * 256;
-#pragma unroll
-      for (int blk = 0; blk < 8; ++blk) {  // q8_1 block = sub-blocks 2blk, 2blk+1
-        float part[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int hj = 0; hj < 2; ++hj) {
-          const int j = 2 * blk + hj;
-          const int h = j >> 3, u = (j & 7) >> 1;
-          const int qi = 4 * h + 2 * (u & 1) + (j & 1);
-          const int hi = 2 * h + (j & 1);
-          const int nsh = (u >> 1) * 4, hsh = 2 * u;
-          const uint32_t qa = ((qla[qi] >> nsh) & 0x0f0f0f0fu) | (((qha[hi] >> hsh) & 0x03030303u) << 4);
-          const uint32_t qb = ((qlb[qi] >> nsh) & 0x0f0f0f0fu) | (((qhb[hi] >> hsh) & 0x03030303u) << 4);
-          const uint32_t bx = *reinterpret_cast<const uint32_t*>(xsb + 16 * j + 4 * t);
-          int d4[4] = {0, 0, 0, 0};
-          mma_s8_16816(d4, q6_to_s8x4(qa), q6_to_s8x4(qb), bx);
-          const float ra = da * (float)(int8_t)((sca[j >> 2] >> (8 * (j & 3))) & 0xff);
-          const float rb = db * (float)(int8_t)((scb[j >> 2] >> (8 * (j & 3))) & 0xff);
-          part[0] += (float)d4[0] * ra;
-          part[1] += (float)d4[1] * ra;
-          part[2] += (float)d4[2] * rb;
-          part[3] += (float)d4[3] * rb;
-        }
-        const int b32 = sb * 8 + blk;
-        const float dx0 = dx[(2 * t) * nb32 + b32], dx1 = dx[(2 * t + 1) * nb32 + b32];
-        acc[0] += part[0] * dx0;
-        acc[1] += part[1] * dx1;
-        acc[2] += part[2] * dx0;
-        acc[3] += part[3] * dx1;
-      }
+      q6_superblock(acc, qla, qlb, qha, qhb, sca, scb, da, db, xrow + sb * 256, dx, nb32, sb, t);
     }
     // ---- fixed-order reduction over warps; after its barrier the tile's stages are free
     float* rb_ = red + parity * (kQ6Warps * 32 * 4);

@@ -358,10 +358,45 @@ def test_fp8_head_full_size_sampled():
 
 
 def test_q6k_head_full_size_sampled():
+    # the Q6_K head config: 8-row launches, swept to 64 rows
     n, k = 129280, 7168
     blocks = synth.q6k_blocks(n, k, 4, DEV)
-    x = synth.bf16_rows(16, k, 4, DEV)
+    x = synth.bf16_rows(64, k, 4, DEV)
     idx = _sample_rows(n)
     out = bits(dl.q6k_lm_head(blocks, x))
     ref = og.q6k_mmvq(bits(blocks[torch.from_numpy(idx).to(DEV)]), og.q8_1_quantize_rows(bits(x)))
-    assert_bf16_close(out[:, idx], ref, "q6k head M=16 sampled")
+    assert_bf16_close(out[:, idx], ref, "q6k head M=64 sampled")
+    for m in (1, 8, 9, 16):
+        part = bits(dl.q6k_lm_head(blocks, x[:m]))
+        assert np.array_equal(part, out[:m]), f"row invariance M={m}"
+
+
+def test_nvfp4_full_size_all_tiers():
+    # the NVFP4 config: 14336 x 4096, M in {1,4,5,6,7,8,16,32}; the oracle covers every output
+    n, k = 14336, 4096
+    wp, ws, gl = synth.nvfp4_weight(n, k, 20, DEV)
+    x = synth.bf16_rows(32, k, 4, DEV)
+    full = bits(dl.w4a16_gemv(wp, ws, gl, x))
+    ref = og.w4a16_gemv(bits(wp), bits(ws), np.float32(gl), bits(x))
+    assert_bf16_close(full, ref, "nvfp4 14336x4096 M=32")
+    for m in (1, 4, 5, 6, 7, 8, 16):
+        part = bits(dl.w4a16_gemv(wp, ws, gl, x[:m]))
+        assert np.array_equal(part, full[:m]), f"row invariance M={m}"
+
+
+def test_w8a8_silu_down_full_size_128_rows():
+    # the W8A8 down-projection config: 4096 x 14336, one 128-row call from bf16(silu(g)*u)
+    n, k = 4096, 14336
+    w = synth.fp8_weight(n, k, 10, DEV)
+    s = synth.row_scales(n, 10, DEV)
+    gate = synth.bf16_rows(128, k, 3, DEV, tensor_id=4)
+    up = synth.bf16_rows(128, k, 3, DEV, tensor_id=5)
+    out = bits(dl.w8a8_silu_proj(w, s, gate, up))
+    xq, sx = dl.w8a8_silu_quantize_rows(gate, up)
+    sub = slice(0, n, 3)
+    ref = og.w8a8_gemv(bits(w)[sub], bits(s)[sub], bits(xq), bits(sx))
+    assert_bf16_close(out[:, sub], ref, "w8a8 silu down M=128")
+    for m in (1, 16, 64):
+        part = bits(dl.w8a8_silu_proj(w, s, gate[:m], up[:m]))
+        assert np.array_equal(part, out[:m]), f"row invariance M={m}"
+    assert dl.device_fault(reset=True) == 0
