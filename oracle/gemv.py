@@ -143,6 +143,50 @@ def w4a16_gemv(w_packed, w_block_scale, global_scale, x):
 
 
 # ----------------------------------------------------------------------------
+# NEXT 3  load-time FP4 dequant to BF16 (the step before the path)
+# ----------------------------------------------------------------------------
+
+
+def nvfp4_dequant_bf16(w_packed, w_block_scale, global_scale, is_reciprocal):
+    """BF16 bits [N, K] of ``e2m1(W) * e4m3(S) * g``.
+
+    fp8_lut.rs, ``dequant_nvfp4_to_bf16``: the stored global is folded into one
+    float32 multiplier ``g`` (compressed-tensors: ``1 / global``, a zero global
+    giving 0; ModelOpt: ``global``), and one BF16 value is written per weight.
+    The kernel body is not printed; the reading is float32 arithmetic:
+    ``e2m1 * e4m3`` is exact in float32 (at most 6 significant bits), its
+    product with ``g`` is rounded once to float32, then to BF16 (nearest-even).
+    w_packed uint8 [N, K/2], w_block_scale uint8 [N, K/16] -> uint16 [N, K].
+    """
+    g = float(nx.nvfp4_fold_global(global_scale, is_reciprocal))
+    v = nvfp4_dequant(w_packed, w_block_scale)      # exact float64
+    with np.errstate(over="ignore"):
+        return nx.bf16_rn(nx.f32(v * g))
+
+
+def e8m0_fp4_dequant_bf16(w_packed, scales, n, k):
+    """BF16 bits [N, K] of ``e2m1(W) * e8m0(scale[group])``.
+
+    fp8_lut.rs, ``dequant_nvfp4_e8m0_to_bf16``: two E2M1 values per byte (an
+    even flat index is the low nibble), one E8M0 byte per group, the group size
+    ``block = N*K / #scales`` over flat (row-major) indices, no global scale;
+    ``f32_to_bf16(e2m1_table[code] * block_scale)``: a float32 product (exact
+    unless it leaves the float32 range) rounded to BF16.  E8M0 codes 0 and 255
+    decode to 0 (``FP8_E8M0_LUT``, pinned by ``tests/golden``).
+    w_packed uint8 [N*K/2] (any shape), scales uint8 [#scales] -> uint16 [N, K].
+    """
+    total = n * k
+    scales = np.asarray(scales, dtype=np.uint8).reshape(-1)
+    if scales.size == 0 or total % scales.size != 0:
+        raise ValueError("N*K must be a multiple of the number of E8M0 scales")
+    block = total // scales.size
+    codes = nx.unpack_nibbles(np.asarray(w_packed, dtype=np.uint8).reshape(-1))
+    vals = nx.e2m1_decode(codes) * nx.E8M0_TABLE[np.repeat(scales, block)]
+    with np.errstate(over="ignore"):
+        return nx.bf16_rn(nx.f32(vals)).reshape(n, k)
+
+
+# ----------------------------------------------------------------------------
 # a6  block_q8_1 row quantize
 # ----------------------------------------------------------------------------
 
