@@ -354,6 +354,30 @@ def other_formats(dev, stream, peak):
     entry("nvfp4_w4a16", f"{n}x{k}", n * k // 2 + n * k // 16, [(lambda m=m: fp4(m)) for m in rows_list], rows_list)
     del wf
 
+    # load-time NVFP4 / E8M0 dequant to BF16 (HBM stream: codes + scales in, BF16 out)
+    n, k = 14336, 4096
+    wq = rotating(lambda i: synth.nvfp4_weight(n, k, 40 + i, dev), n * k // 2)
+    outq = torch.empty(n, k, dtype=torch.bfloat16, device=dev)
+    e8 = [torch.randint(110, 140, (n * k // 32,), dtype=torch.int32, device=dev).to(torch.uint8) for _ in wq]
+
+    def dq_nvfp4():
+        wp, sc, _ = wq[ctr[0] % len(wq)]
+        ctr[0] += 1
+        dl.nvfp4_dequant_bf16(wp, sc, 448.0, True, out=outq, stream=stream)
+
+    def dq_e8m0():
+        i = ctr[0] % len(wq)
+        ctr[0] += 1
+        dl.e8m0_fp4_dequant_bf16(wq[i][0].reshape(-1), e8[i], n, k, out=outq, stream=stream)
+
+    for name, fn, sbytes in (("nvfp4_dequant_bf16", dq_nvfp4, n * k // 16), ("e8m0_fp4_dequant_bf16", dq_e8m0, n * k // 32)):
+        us = time_calls([fn], 20, stream)[0]
+        nbytes = n * k // 2 + sbytes + 2 * n * k
+        gbs = nbytes / (us * 1e-6) / 1e9
+        res[name] = {"shape": f"{n}x{k}", "bytes_per_call": nbytes,
+                     "per_call": {"us": round(us, 2), "gbs": round(gbs, 1), "frac_of_copy_peak": round(gbs / peak, 3)}}
+    del wq, e8
+
     # Q6_K head
     n, k = 129280, 7168
     blocks = synth.q6k_blocks(n, k, 4, dev)

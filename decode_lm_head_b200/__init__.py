@@ -13,9 +13,11 @@ from ._lib import (  # noqa: F401
     OP_W8A16,
     check_bounded_wait,
     device_fault,
+    e8m0_fp4_dequant_bf16,
     error_string,
     lib,
     lm_head_fp8_w8a16,
+    nvfp4_dequant_bf16,
     plan_chunks,
     q6k_lm_head,
     q6k_mmvq,

@@ -53,6 +53,8 @@ _SIGNATURES = {
     "q8_1_quantize_rows": [_P, _L, _I, _I, _P, _P],
     "q6k_mmvq": [_P, _I, _I, _P, _I, _P, _L, _P],
     "q6k_lm_head": [_P, _I, _I, _P, _L, _I, _P, _L, _P, _P],
+    "nvfp4_dequant_bf16": [_P, _P, _F, _I, _I, _I, _P, _L, _P],
+    "e8m0_fp4_dequant_bf16": [_P, _P, _L, _I, _I, _P, _L, _P],
     "dlmh_plan_chunks": [_I, _I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I), _I],
     "dlmh_device_fault": [_I],
     "dlmh_check_bounded_wait": [_P],
@@ -332,4 +334,40 @@ def q6k_lm_head(blocks, x, out=None, q8_scratch=None, stream=None):
         q8_scratch = torch.empty(Q6K_CHUNK_ROWS * (k // 32) * Q8_1_BLOCK_BYTES, dtype=torch.uint8, device=x.device)
     _check(lib().q6k_lm_head(_ptr(blocks), n, k, _ptr(x), _ld(x), rows, _ptr(out), _ld(out), _ptr(q8_scratch),
                              _stream(stream, x.device)), "q6k_lm_head")
+    return out
+
+
+# ---------------------------------------------------------------------------
+# load-time FP4 dequant
+# ---------------------------------------------------------------------------
+
+
+def nvfp4_dequant_bf16(w_packed, w_block_scale, global_scale, is_reciprocal, out=None, stream=None):
+    """NVFP4 [n, k/2] codes + [n, k/16] E4M3 block scales -> BF16 [n, k] (see dlmh.h)."""
+    _cuda(w_packed, torch.uint8, "w_packed", 2)
+    _cuda(w_block_scale, torch.uint8, "w_block_scale", 2)
+    n, k2 = w_packed.shape
+    k = 2 * k2
+    if tuple(w_block_scale.shape) != (n, k // 16):
+        raise ValueError("w_block_scale must be [n, k/16]")
+    if out is None:
+        out = torch.empty(n, k, dtype=torch.bfloat16, device=w_packed.device)
+    _check(lib().nvfp4_dequant_bf16(_ptr(w_packed), _ptr(w_block_scale), float(global_scale),
+                                    1 if is_reciprocal else 0, n, k, _ptr(out), _ld(out),
+                                    _stream(stream, w_packed.device)), "nvfp4_dequant_bf16")
+    return out
+
+
+def e8m0_fp4_dequant_bf16(w_packed, scales, n, k, out=None, stream=None):
+    """E2M1 pairs (n*k/2 bytes) + E8M0 group scales -> BF16 [n, k] (see dlmh.h)."""
+    if not isinstance(w_packed, torch.Tensor) or not w_packed.is_cuda or w_packed.dtype != torch.uint8:
+        raise TypeError("w_packed must be a CUDA uint8 tensor")
+    if not isinstance(scales, torch.Tensor) or not scales.is_cuda or scales.dtype != torch.uint8:
+        raise TypeError("scales must be a CUDA uint8 tensor")
+    if not w_packed.is_contiguous() or not scales.is_contiguous() or w_packed.numel() * 2 != n * k:
+        raise ValueError("w_packed must be n*k/2 contiguous bytes and scales contiguous")
+    if out is None:
+        out = torch.empty(n, k, dtype=torch.bfloat16, device=w_packed.device)
+    _check(lib().e8m0_fp4_dequant_bf16(_ptr(w_packed), _ptr(scales), scales.numel(), n, k, _ptr(out), _ld(out),
+                                       _stream(stream, w_packed.device)), "e8m0_fp4_dequant_bf16")
     return out

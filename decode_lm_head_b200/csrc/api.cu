@@ -319,6 +319,36 @@ int q6k_lm_head(const void* blocks, int n, int k, const dlmh_bf16* x, int64_t ld
 
 }  // extern "C"
 
+extern "C" {
+
+int nvfp4_dequant_bf16(const uint8_t* w_packed, const uint8_t* w_block_scale, float global_scale, int is_reciprocal,
+                       int n, int k, dlmh_bf16* out, int64_t ldo, void* stream) {
+  DLMH_TRY(check_nk(n, k, 16));
+  if (!w_packed || !w_block_scale) return DLMH_ERR_NULL;
+  if (!aligned16(w_packed) || !aligned16(w_block_scale)) return DLMH_ERR_ALIGN;
+  if (!out) return DLMH_ERR_NULL;
+  if (ldo < k) return DLMH_ERR_LD;
+  if (!aligned16(out) || ldo % 8 != 0) return DLMH_ERR_ALIGN;
+  // fold the stored global into one float32 multiplier, as the loader does
+  const float g = is_reciprocal ? (global_scale != 0.f ? 1.0f / global_scale : 0.f) : global_scale;
+  return dlmh::nvfp4_dequant_launch(w_packed, w_block_scale, g, n, k, out, ldo, as_stream(stream));
+}
+
+int e8m0_fp4_dequant_bf16(const uint8_t* w_packed, const uint8_t* scales, int64_t num_scales, int n, int k,
+                          dlmh_bf16* out, int64_t ldo, void* stream) {
+  DLMH_TRY(check_nk(n, k, 16));
+  if (!w_packed || !scales) return DLMH_ERR_NULL;
+  const int64_t total = (int64_t)n * k;
+  if (num_scales <= 0 || total % num_scales != 0) return DLMH_ERR_SHAPE;
+  if (!aligned16(w_packed)) return DLMH_ERR_ALIGN;
+  if (!out) return DLMH_ERR_NULL;
+  if (ldo < k) return DLMH_ERR_LD;
+  if (!aligned16(out) || ldo % 8 != 0) return DLMH_ERR_ALIGN;
+  return dlmh::e8m0_dequant_launch(w_packed, scales, total / num_scales, n, k, out, ldo, as_stream(stream));
+}
+
+}  // extern "C"
+
 namespace dlmh {
 
 int w8a8_proj_fixed_scratch(const uint8_t* w, const float* w_scale, int n, int k, const uint16_t* x, int64_t ldx,

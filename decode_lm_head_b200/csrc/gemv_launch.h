@@ -61,6 +61,12 @@ int w8a8_silu_quantize_launch(const uint16_t* gate, const uint16_t* up, int64_t 
 int w8a16_split_launch(const uint16_t* x, int64_t ldx, int rows, int k, int half, uint8_t* codes, float* x_mul,
                        cudaStream_t s);
 int q8_1_quantize_launch(const uint16_t* x, int64_t ldx, int rows, int k, uint8_t* q8, cudaStream_t s);
+// Load-time FP4 dequant to BF16 (dequant.cu); k % 16 == 0, out 16-byte aligned, ldo % 8 == 0.
+int nvfp4_dequant_launch(const uint8_t* packed, const uint8_t* bscale, float g, int n, int k, uint16_t* out,
+                         int64_t ldo, cudaStream_t s);
+int e8m0_dequant_launch(const uint8_t* packed, const uint8_t* scales, int64_t block, int n, int k, uint16_t* out,
+                        int64_t ldo, cudaStream_t s);
+
 // Fault bits of the streamed Q6_K kernel's bounded waits (read synchronously).
 int q6k_fault(int reset);
 int q6k_mmvq_launch(const uint8_t* blocks, int n, int k, const uint8_t* q8, int rows, uint16_t* out, int64_t ldc,

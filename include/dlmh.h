@@ -241,6 +241,31 @@ DLMH_API int q6k_lm_head(const void* blocks, int n, int k, const dlmh_bf16* x, i
                 dlmh_bf16* out, int64_t ldc, void* q8_scratch, void* stream);
 
 /* ---------------------------------------------------------------------------------------
+ * Load-time FP4 dequant to BF16 (the step before the path)
+ *
+ * NVFP4:  out[n, k] = bf16( e2m1(w[n, k]) * e4m3(s[n, k/16]) * g )
+ *   fp8_lut.rs, dequant_nvfp4_to_bf16.  The stored global is folded into one float32
+ *   multiplier: is_reciprocal != 0 (compressed-tensors weight_global_scale) gives
+ *   g = 1 / global_scale, or 0 when global_scale == 0; is_reciprocal == 0 (ModelOpt
+ *   weight_scale_2) gives g = global_scale.  Float32 arithmetic: e2m1 * e4m3 is exact, its
+ *   product with g is rounded once to float32, then to BF16 (round-to-nearest-even).
+ *   w_packed [n, k/2] E2M1 pairs (element 2i in the low nibble), w_block_scale [n, k/16]
+ *   E4M3, both 16-byte aligned; out [n, ldo] BF16, ldo >= k, ldo % 8 == 0, 16-byte aligned.
+ *   k % 16 == 0.  Errors as for the GEMV entry points.
+ * ------------------------------------------------------------------------------------- */
+DLMH_API int nvfp4_dequant_bf16(const uint8_t* w_packed, const uint8_t* w_block_scale, float global_scale,
+                                int is_reciprocal, int n, int k, dlmh_bf16* out, int64_t ldo, void* stream);
+
+/* E8M0-scaled FP4:  out[f] = bf16( e2m1(w[f]) * 2^(e[f / block] - 127) ), f the flat (row-major)
+ * index, block = n * k / num_scales (DLMH_ERR_SHAPE unless it divides exactly); E8M0 codes 0
+ * and 255 decode to 0; no global scale.  fp8_lut.rs, dequant_nvfp4_e8m0_to_bf16 (there a
+ * host-side loop; here the same values on the GPU).  The float32 product is exact unless it
+ * leaves the float32 range (then +-inf).  w_packed [n * k / 2] 16-byte aligned, scales
+ * [num_scales] bytes; out as above; k % 16 == 0. */
+DLMH_API int e8m0_fp4_dequant_bf16(const uint8_t* w_packed, const uint8_t* scales, int64_t num_scales, int n, int k,
+                                   dlmh_bf16* out, int64_t ldo, void* stream);
+
+/* ---------------------------------------------------------------------------------------
  * Host helpers (no device work; callable without a GPU)
  * ------------------------------------------------------------------------------------- */
 

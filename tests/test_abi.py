@@ -115,3 +115,17 @@ def test_zero_rows_launch_nothing():
     # valid arguments with rows == 0 return OK without touching CUDA
     assert L.w8a8_quantize_rows(A, 64, 0, 64, A, 64, A, None) == 0
     assert L.q8_1_quantize_rows(A, 64, 0, 64, A, None) == 0
+
+
+def test_dequant_argument_errors():
+    f = L.nvfp4_dequant_bf16
+    assert f(None, A, 1.0, 0, 16, 64, A, 64, None) == -1
+    assert f(A, A, 1.0, 0, 16, 40, A, 64, None) == -2      # k % 16
+    assert f(A, A, 1.0, 0, 16, 64, A, 32, None) == -5      # ldo < k
+    assert f(A, U, 1.0, 0, 16, 64, A, 64, None) == -3
+    assert f(A, A, 1.0, 0, 16, 64, A, 68, None) == -3      # ldo % 8
+    e = L.e8m0_fp4_dequant_bf16
+    assert e(A, None, 4, 16, 64, A, 64, None) == -1
+    assert e(A, A, 7, 16, 64, A, 64, None) == -2           # 1024 elements not a multiple of 7 groups
+    assert e(A, A, 0, 16, 64, A, 64, None) == -2
+    assert e(U, A, 4, 16, 64, A, 64, None) == -3

@@ -281,6 +281,40 @@ def test_w4a16_tiers(n, k):
 
 
 # ---------------------------------------------------------------------------
+# load-time FP4 dequant (bit-exact)
+# ---------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("n,k", [(14336, 4096), (37, 48), (300, 1152)])
+def test_nvfp4_dequant_bit_exact_both_conventions(n, k):
+    wp, ws, _ = synth.nvfp4_weight(n, k, 30, DEV)
+    for stored, reciprocal in [(448.0, True), (1.0 / 448.0, False), (3.0, True), (0.0, True)]:
+        out = bits(dl.nvfp4_dequant_bf16(wp, ws, stored, reciprocal))
+        ref = og.nvfp4_dequant_bf16(bits(wp), bits(ws), stored, reciprocal)
+        assert np.array_equal(out, ref), (stored, reciprocal)
+    # strided output: the padding columns stay untouched
+    outb = torch.full((n, k + 24), 7.0, dtype=torch.bfloat16, device=DEV)
+    dl.nvfp4_dequant_bf16(wp, ws, 448.0, True, out=outb[:, :k])
+    assert np.array_equal(bits(outb[:, :k]), og.nvfp4_dequant_bf16(bits(wp), bits(ws), 448.0, True))
+    assert (outb[:, k:] == 7.0).all()
+
+
+@pytest.mark.parametrize("n,k,groups", [(64, 4096, 64 * 4096 // 32), (3, 80, 5), (7, 32, 1), (256, 512, 1024)])
+def test_e8m0_fp4_dequant_bit_exact(n, k, groups):
+    g = torch.Generator(device="cpu").manual_seed(31)
+    wp = torch.randint(0, 256, (n * k // 2,), generator=g, dtype=torch.int32).to(torch.uint8)
+    sc = torch.randint(100, 160, (groups,), generator=g, dtype=torch.int32).to(torch.uint8)
+    sc[0] = 0                                             # special codes decode to 0
+    sc[-1] = 255
+    if groups > 2:
+        sc[1] = 254                                       # 6 * 2^127 overflows float32 -> inf
+    wp, sc = wp.to(DEV), sc.to(DEV)
+    out = bits(dl.e8m0_fp4_dequant_bf16(wp, sc, n, k))
+    ref = og.e8m0_fp4_dequant_bf16(bits(wp), bits(sc), n, k)
+    assert np.array_equal(out, ref)
+
+
+# ---------------------------------------------------------------------------
 # q8_1 and Q6_K
 # ---------------------------------------------------------------------------
 
