@@ -59,17 +59,37 @@ def w8a8_quantize_rows(x):
     return q, sx
 
 
-def silu_mul_bf16(gate, up):
-    """``h = bf16_rn(silu(gate) * up)``, ``silu(g) = g / (1 + e^-g)``, in float64.
+def silu_exp_neg_f32(g):
+    """``e^-g`` correctly rounded to float32, as float64 values.
 
-    w8a8_layer.rs, ``W8a8Ctx::silu_proj``: the down projection's input is
-    ``bf16(silu(gate) * up)`` of BF16 gate and up rows.  Returns uint16.
+    The float64 exp (error below one float64 ulp) is rounded once to float32; this is the
+    correctly rounded float32 value unless e^-g lies within a float64 ulp of a float32
+    rounding midpoint (``tests/test_oracle_pins.py`` checks every finite BF16 g against a
+    60-digit evaluation).  Overflow gives inf, as in float32.
+    """
+    with np.errstate(over="ignore"):
+        return nx.f32(np.exp(-np.asarray(g, dtype=np.float64)))
+
+
+def silu_mul_bf16(gate, up):
+    """``h = bf16_rn(silu(gate) * up)``, ``silu(g) = g / (1 + e^-g)``, in float32 steps.
+
+    w8a8_layer.rs, ``W8a8Ctx::silu_proj`` (``ops::w8a8_act_quant_silu``): the down
+    projection's input is ``bf16(silu(gate) * up)`` of BF16 gate and up rows, computed by
+    the fused quantize kernel.  h decides the E4M3 codes, so it is evaluated in that
+    kernel's float32: ``e = rn32(e^-g)`` (``silu_exp_neg_f32``), ``d = rn32(1 + e)``,
+    ``s = rn32(g / d)``, ``p = rn32(s * u)``, then one round-to-nearest-even to BF16.
+    Each float32 step is the float64 operation rounded once to float32, which equals the
+    IEEE float32 operation (53 >= 2*24 + 2 bits: double rounding is innocuous for
+    +, -, *, /).  Returns uint16.
     """
     g = nx.bf16_decode(gate)
     u = nx.bf16_decode(up)
-    with np.errstate(over="ignore"):
-        s = g / (1.0 + np.exp(-g))
-    return nx.bf16_rn(s * u)
+    e = silu_exp_neg_f32(g)
+    d = nx.f32(1.0 + e)
+    with np.errstate(invalid="ignore"):
+        s = nx.f32(g / d)
+    return nx.bf16_rn(nx.f32(s * u))
 
 
 def silu_quantize_rows(gate, up):

@@ -304,6 +304,85 @@ def test_silu_product_matches_torch_silu():
     assert (got == ref).mean() > 0.999
 
 
+def _finite_bf16_bits():
+    b = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    return b[(b & 0x7F80) != 0x7F80]
+
+
+def _mp_round_f32(v):
+    """Nearest float32 to the mpmath value v (no ties: v is transcendental), inf on overflow."""
+    import mpmath as mp
+
+    if v > mp.mpf(float(np.finfo(np.float32).max)) * (1 + mp.mpf(2) ** -25):
+        return math.inf
+    c = np.float32(float(v))
+    best, bd = None, None
+    for cand in (np.nextafter(c, np.float32(-np.inf)), c, np.nextafter(c, np.float32(np.inf))):
+        if not np.isfinite(cand) or cand < 0:
+            continue
+        d = abs(v - mp.mpf(float(cand)))
+        if bd is None or d < bd:
+            best, bd = float(cand), d
+    return best
+
+
+def test_silu_exp_step_is_correctly_rounded_for_every_bf16():
+    # e^-g rounded to float32, for every finite BF16 g, against a 200-bit mpmath evaluation
+    import mpmath as mp
+
+    gb = _finite_bf16_bits()
+    g = nx.bf16_decode(gb)
+    got = og.silu_exp_neg_f32(g)
+    mp.mp.prec = 200
+    for gi, e in zip(g, got):
+        if gi > 104.0:                      # e^-g < 2^-150: rounds to +0
+            assert e == 0.0, gi
+        elif gi < -89.0:                    # e^-g > float32 max: inf
+            assert e == math.inf, gi
+        else:
+            assert e == _mp_round_f32(mp.exp(-mp.mpf(float(gi)))), gi
+
+
+def test_silu_agrees_with_float64_definition_off_midpoints():
+    # The float32 chain (four correctly rounded steps, relative error < 2^-22) must round to
+    # the BF16 of the float64 definition wherever that is farther than 2^-20 from a midpoint.
+    rng = np.random.default_rng(81)
+    gb = _finite_bf16_bits()
+    g = nx.bf16_decode(gb)
+    keep = np.abs(g) < 60.0
+    gb, g = gb[keep], g[keep]
+    ub = _rand_bf16(rng, gb.shape)
+    u = nx.bf16_decode(ub)
+    h = nx.bf16_decode(og.silu_mul_bf16(gb, ub))
+    p = g / (1.0 + np.exp(-g)) * u                      # float64 definition
+    a = np.abs(p)
+    _, ex = np.frexp(a)
+    quantum = np.ldexp(1.0, np.maximum(ex - 1, -126) - 7)
+    frac = a / quantum - np.floor(a / quantum)
+    near = (np.abs(frac - 0.5) * quantum <= a * 2.0 ** -20) & (a > 0)
+    ref = torch.from_numpy(p).float().to(torch.bfloat16).double().numpy()
+    # torch rounds float64 -> float32 -> BF16; off midpoints that is the BF16 of p
+    assert np.array_equal(h[~near], ref[~near])
+    # for large g, silu(g)*u is nearly the exact product of two 8-bit significands, which
+    # lands on a BF16 midpoint about once in 128; the band stays a small minority
+    assert near.mean() < 0.03
+    ulp = np.ldexp(1.0, np.maximum(np.frexp(np.abs(ref))[1] - 1, -126) - 7)
+    assert np.all(np.abs(h[near] - ref[near]) <= ulp[near])
+
+
+def test_silu_special_values():
+    one = np.array([0x3F80], np.uint16)
+    def h(gbits, ubits=one):
+        return nx.bf16_decode(og.silu_mul_bf16(np.array([gbits], np.uint16), np.asarray(ubits, np.uint16)))[0]
+    assert h(0x0000) == 0.0                               # silu(0) = 0
+    assert h(0x42C8) == 100.0                             # e^-100 is far below half an ulp of 1
+    z = h(0xC2C8)                                         # g = -100: e^100 overflows float32 -> -0
+    assert z == 0.0 and math.copysign(1.0, z) < 0
+    assert h(0x3F80) == 0.73046875                        # silu(1) = 0.7310585786...
+    assert h(0xBF80) == -0.26953125                       # silu(-1) = -0.2689414214...
+    assert h(0x4000, np.array([0xC000], np.uint16)) == -3.515625  # silu(2) * -2 = -3.5231883...
+
+
 def test_w4a16_brute_force_exact():
     rng = np.random.default_rng(9)
     N, K, M = 3, 64, 2
