@@ -336,6 +336,35 @@ def other_formats(dev, stream, peak):
     entry("w8a8_silu_down", f"{n}x{k}", n * k + 4 * n, [(lambda m=m: down(m)) for m in rows_list], rows_list)
     del ws
 
+    # W8A8 FFN gate + up on one quantized x (one launch over both weights), against the same
+    # two projections as two w8a8_proj calls
+    n, k = 14336, 4096
+    pairs = rotating(lambda i: (synth.fp8_weight(n, k, 50 + i, dev, tensor_id=1), synth.row_scales(n, 50 + i, dev),
+                                synth.fp8_weight(n, k, 50 + i, dev, tensor_id=6),
+                                synth.row_scales(n, 50 + i, dev, tensor_id=7)), 2 * n * k)
+    xg = synth.bf16_rows(128, k, 5, dev)
+    xq = torch.empty(128 * k, dtype=torch.uint8, device=dev)
+    og_, ou_ = torch.empty(128, n, dtype=torch.bfloat16, device=dev), torch.empty(128, n, dtype=torch.bfloat16,
+                                                                                  device=dev)
+    rows_list = [1, 16, 128]
+    gviews = {m: (xg[:m], og_[:m], ou_[:m]) for m in rows_list}
+
+    def gate_up(m, paired):
+        wg, sg, wu, su = pairs[ctr[0] % len(pairs)]
+        ctr[0] += 1
+        xm, gm, um = gviews[m]
+        if paired:
+            dl.w8a8_gate_up_proj(wg, sg, wu, su, xm, gate_out=gm, up_out=um, xq_scratch=xq, xscale_scratch=xs,
+                                 stream=stream)
+        else:
+            dl.w8a8_proj(wg, sg, xm, out=gm, xq_scratch=xq, xscale_scratch=xs, stream=stream)
+            dl.w8a8_proj(wu, su, xm, out=um, xq_scratch=xq, xscale_scratch=xs, stream=stream)
+
+    for name, paired in (("w8a8_gate_up_pair", True), ("w8a8_gate_up_two_calls", False)):
+        entry(name, f"2x{n}x{k}", 2 * (n * k + 4 * n), [(lambda m=m, p=paired: gate_up(m, p)) for m in rows_list],
+              rows_list)
+    del pairs
+
     # NVFP4 W4A16
     n, k = 14336, 4096
     wf = rotating(lambda i: synth.nvfp4_weight(n, k, 20 + i, dev), n * k // 2)

@@ -24,6 +24,7 @@ from ._lib import (  # noqa: F401
     q8_1_quantize_rows,
     version,
     w4a16_gemv,
+    w8a8_gate_up_proj,
     w8a8_gemv,
     w8a8_proj,
     w8a8_proj_noalloc,

@@ -48,6 +48,7 @@ _SIGNATURES = {
     "w8a8_gemv": [_P, _P, _I, _I, _P, _L, _P, _I, _P, _L, _P],
     "w8a8_proj": [_P, _P, _I, _I, _P, _L, _I, _P, _L, _P, _P, _P],
     "w8a8_silu_proj": [_P, _P, _I, _I, _P, _P, _L, _I, _P, _L, _P, _P, _P],
+    "w8a8_gate_up_proj": [_P, _P, _P, _P, _I, _I, _P, _L, _I, _P, _P, _L, _P, _P, _P],
     "w8a8_proj_noalloc": [_P, _P, _I, _I, _P, _L, _I, _P, _L, _P],
     "w4a16_gemv": [_P, _P, _F, _I, _I, _P, _L, _I, _P, _L, _P],
     "q8_1_quantize_rows": [_P, _L, _I, _I, _P, _P],
@@ -277,6 +278,32 @@ def w8a8_silu_proj(w, w_scale, gate, up, out=None, xq_scratch=None, xscale_scrat
                                 _ld(out), _ptr(xq_scratch), _ptr(xscale_scratch), _stream(stream, gate.device)),
            "w8a8_silu_proj")
     return out
+
+
+def w8a8_gate_up_proj(w_gate, s_gate, w_up, s_up, x, gate_out=None, up_out=None, xq_scratch=None,
+                      xscale_scratch=None, stream=None):
+    """(gate, up) = the two W8A8 projections of x on one quantized copy of it."""
+    for t, name in ((w_gate, "w_gate"), (w_up, "w_up")):
+        _cuda(t, torch.uint8, name, 2)
+    for t, name in ((s_gate, "s_gate"), (s_up, "s_up")):
+        _cuda(t, torch.float32, name, 1)
+    _cuda(x, torch.bfloat16, "x", 2)
+    if w_gate.shape != w_up.shape:
+        raise ValueError("w_gate and w_up must have the same shape")
+    n, k = w_gate.shape
+    rows = x.shape[0]
+    if gate_out is None:
+        gate_out = torch.empty(rows, n, dtype=torch.bfloat16, device=x.device)
+    if up_out is None:
+        up_out = torch.empty(rows, n, dtype=torch.bfloat16, device=x.device)
+    if _ld(gate_out) != _ld(up_out):
+        raise ValueError("gate_out and up_out must have the same row stride")
+    xq_scratch, xscale_scratch = _w8a8_scratch(k, x.device, xq_scratch, xscale_scratch)
+    _check(lib().w8a8_gate_up_proj(_ptr(w_gate), _ptr(s_gate), _ptr(w_up), _ptr(s_up), n, k, _ptr(x), _ld(x), rows,
+                                   _ptr(gate_out), _ptr(up_out), _ld(gate_out), _ptr(xq_scratch),
+                                   _ptr(xscale_scratch), _stream(stream, x.device)),
+           "w8a8_gate_up_proj")
+    return gate_out, up_out
 
 
 def w4a16_gemv(w_packed, w_block_scale, global_scale, x, out=None, stream=None):

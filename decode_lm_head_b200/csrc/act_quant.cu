@@ -8,7 +8,7 @@
 // cluster of kQC CTAs shares a row: every CTA takes a contiguous 1/kQC of the row's 8-element
 // groups, keeps its values in registers, reduces its maximum, and the cluster combines the
 // kQC maxima through distributed shared memory.  The arithmetic is the same as a one-CTA
-// pass (IEEE division, one BF16 rounding of silu(g)*u, round-to-nearest-even codes), so the
+// pass (correctly rounded f32 steps for silu(g)*u, round-to-nearest-even codes), so the
 // codes do not depend on the split.
 #include <utility>
 
@@ -41,11 +41,14 @@ __device__ __forceinline__ float ld_cluster_f32(const float* local, uint32_t ran
   return v;
 }
 
-// h = bf16(silu(g) * u) as BF16 bits: silu in f32 as g / (1 + e^-g) with an IEEE division,
-// one product, one rounding.
+// h = bf16(silu(g) * u) as BF16 bits, in f32 steps: e = e^-g correctly rounded to f32 (the
+// double exp, below one double ulp, rounded once), d = 1 + e, s = g / d (IEEE division),
+// p = s * u, then one round-to-nearest-even to BF16.  Every step is a correctly rounded f32
+// operation, so h is a function of (g, u) alone and the codes that follow are reproducible.
 __device__ __forceinline__ uint32_t silu_mul_bf16_bits(float g, float u) {
-  const float s = __fdiv_rn(g, 1.0f + expf(-g));
-  return f32_to_bf16_bits(s * u);
+  const float e = __double2float_rn(exp(-(double)g));
+  const float s = __fdiv_rn(g, __fadd_rn(1.0f, e));
+  return f32_to_bf16_bits(__fmul_rn(s, u));
 }
 
 // The 8 BF16 values of group `g` of a row, packed two per word (element 2i low).

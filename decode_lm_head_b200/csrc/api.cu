@@ -247,6 +247,38 @@ int w8a8_silu_proj(const uint8_t* w, const float* w_scale, int n, int k, const d
   return w8a8_proj_impl(w, w_scale, n, k, gate, up, ld, rows, out, ldc, xq_scratch, xscale_scratch, stream);
 }
 
+int w8a8_gate_up_proj(const uint8_t* w_gate, const float* s_gate, const uint8_t* w_up, const float* s_up, int n,
+                      int k, const dlmh_bf16* x, int64_t ldx, int rows, dlmh_bf16* gate_out, dlmh_bf16* up_out,
+                      int64_t ldc, uint8_t* xq_scratch, float* xscale_scratch, void* stream) {
+  DLMH_TRY(check_rows(rows, 0));
+  DLMH_TRY(check_nk(n, k, 16));
+  if (rows == 0) return DLMH_OK;
+  if (!w_gate || !s_gate || !w_up || !s_up) return DLMH_ERR_NULL;
+  if (!aligned16(w_gate) || !aligned16(w_up)) return DLMH_ERR_ALIGN;
+  DLMH_TRY(check_bf16_in(x, ldx, k));
+  DLMH_TRY(check_out(gate_out, ldc, n));
+  DLMH_TRY(check_out(up_out, ldc, n));
+  if (!xq_scratch || !xscale_scratch) return DLMH_ERR_NULL;
+  if (!aligned16(xq_scratch) || k % 16 != 0) return DLMH_ERR_ALIGN;
+  if (pass_rows(DLMH_OP_W8A8, k) <= 0) return DLMH_ERR_UNSUPPORTED;
+  cudaStream_t s = as_stream(stream);
+  for (int done = 0; done < rows;) {
+    const int m = rows - done < DLMH_W8A8_MAX_ROWS ? rows - done : DLMH_W8A8_MAX_ROWS;
+    DLMH_TRY(dlmh::w8a8_quantize_launch(x + (int64_t)done * ldx, ldx, m, k, xq_scratch, k, xscale_scratch, s));
+    dlmh_bf16* g = gate_out + (int64_t)done * ldc;
+    dlmh_bf16* u = up_out + (int64_t)done * ldc;
+    if (dlmh::w8a8_umma_supported(k)) {
+      DLMH_TRY(dlmh::w8a8_umma_pair_pass(w_gate, s_gate, n, g, ldc, w_up, s_up, n, u, ldc, k, xq_scratch, k,
+                                         xscale_scratch, m, s, true));
+    } else {
+      DLMH_TRY(w8a8_gemv_impl(w_gate, s_gate, n, k, xq_scratch, k, xscale_scratch, m, g, ldc, stream, nullptr, 0));
+      DLMH_TRY(w8a8_gemv_impl(w_up, s_up, n, k, xq_scratch, k, xscale_scratch, m, u, ldc, stream, nullptr, 0));
+    }
+    done += m;
+  }
+  return DLMH_OK;
+}
+
 int w4a16_gemv(const uint8_t* w_packed, const uint8_t* w_block_scale, float global_scale, int n, int k,
                const dlmh_bf16* x, int64_t ldx, int rows, dlmh_bf16* out, int64_t ldc, void* stream) {
   DLMH_TRY(check_rows(rows, DLMH_W4A16_MAX_ROWS));

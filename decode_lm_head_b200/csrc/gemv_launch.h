@@ -30,6 +30,13 @@ bool w8a8_umma_supported(int k);
 int w8a8_umma_pass(const uint8_t* w, const float* w_scale, int n, int k, const uint8_t* xq, int64_t ldq,
                    const float* x_scale, int rows, uint16_t* out, int64_t ldc, cudaStream_t s,
                    float* partial_ws = nullptr, size_t partial_cap = 0, bool after_prepass = false);
+// Two weight matrices (same k) against the same activation codes in ONE tensor-core launch
+// (an FFN's gate and up): the tiles of both share one stream-K schedule over the SMs, a pure
+// function of (n1, n2, k, #SMs).  Partial sums from the library's pool.
+int w8a8_umma_pair_pass(const uint8_t* w1, const float* s1, int n1, uint16_t* out1, int64_t ldc1,
+                        const uint8_t* w2, const float* s2, int n2, uint16_t* out2, int64_t ldc2, int k,
+                        const uint8_t* xq, int64_t ldq, const float* x_scale, int rows, cudaStream_t s,
+                        bool after_prepass);
 // w8a8_proj with caller-fixed scratch for everything, including the partial sums: never
 // allocates (the allocation-free entry point).
 int w8a8_proj_fixed_scratch(const uint8_t* w, const float* w_scale, int n, int k, const uint16_t* x, int64_t ldx,

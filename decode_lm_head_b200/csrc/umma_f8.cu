@@ -78,12 +78,32 @@ struct UmmaParams {
   float* partial;
   int early_w;  // 1: the preceding kernel is this library's activation pre-pass (it writes
                 // neither W nor the outputs), so weight loads may start before it completes
+  // A second weight matrix against the same activations (an FFN's gate and up) runs in the
+  // same launch: tiles [t1, ...) read map_w2 and write out2 with w_scale2.  Without one, t1
+  // is the tile count.
+  int t1, n2;
+  const float* w_scale2;
+  uint16_t* out2;
+  int64_t ldc2;
 };
+
+// Where tile `tile`'s 128 output columns go.
+struct TileDst {
+  int row0, n;
+  const float* scale;
+  uint16_t* out;
+  int64_t ldc;
+};
+
+__device__ __forceinline__ TileDst tile_dst(const UmmaParams& p, int tile) {
+  if (tile < p.t1) return TileDst{tile * kBM, p.n, p.w_scale, p.out, p.ldc};
+  return TileDst{(tile - p.t1) * kBM, p.n2, p.w_scale2, p.out2, p.ldc2};
+}
 
 
 __global__ void __launch_bounds__(kUmmaThreads, 1)
-    umma_f8_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x,
-                   const UmmaParams p) {
+    umma_f8_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_w2,
+                   const __grid_constant__ CUtensorMap map_x, const UmmaParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   __shared__ __align__(8) uint64_t bar_full[kMaxUStages], bar_empty[kMaxUStages], bar_tfull[2], bar_tempty[2];
@@ -136,7 +156,9 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
           sc.job(b, j, tile, u0, u1, ps);
           for (int u = u0; u < u1 && s < npre; ++u, ++s) {
             expect_tx(full0 + 8u * s, (uint32_t)p.stage_bytes);
-            tma_load_3d(ring_u32 + s * p.stage_bytes, &map_w, 0, tile * kBM, u * kKC, full0 + 8u * s, pol_w);
+            const bool first = tile < p.t1;
+            tma_load_3d(ring_u32 + s * p.stage_bytes, first ? &map_w : &map_w2, 0, (first ? tile : tile - p.t1) * kBM,
+                        u * kKC, full0 + 8u * s, pol_w);
           }
         }
       }
@@ -152,8 +174,10 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
           // zero-filled), so every stage completes exactly stage_bytes
           if (s >= npre) {
             expect_tx(full0 + 8u * slot, (uint32_t)p.stage_bytes);
-            // A: weight rows [tile*128, +128) x chunks [u*KC, u*KC + KC)
-            tma_load_3d(st, &map_w, 0, tile * kBM, u * kKC, full0 + 8u * slot, pol_w);
+            // A: weight rows [tile*128, +128) x chunks [u*KC, u*KC + KC) of the tile's matrix
+            const bool first = tile < p.t1;
+            tma_load_3d(st, first ? &map_w : &map_w2, 0, (first ? tile : tile - p.t1) * kBM, u * kKC,
+                        full0 + 8u * slot, pol_w);
           }
           // B: all activation rows, the same chunks
           tma_load_3d(st + a_bytes, &map_x, 0, 0, u * kKC, full0 + 8u * slot, pol_x);
@@ -213,7 +237,6 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
       const int acc = i & 1;
       if (!wait(tfull0 + 8u * acc, (i >> 1) & 1)) atomicOr(&umma_fault_word, 8);
       fence_after();
-      const int row = tile * kBM + lane_row;
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * p.accw);
       if (ps >= 0) {
         // partial tile: raw f32 sums of the used columns, [slot][col][128 rows]
@@ -229,7 +252,9 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
           }
         }
       } else {
-        const float s = row < p.n ? p.w_scale[row] : 0.f;
+        const TileDst d = tile_dst(p, tile);
+        const int row = d.row0 + lane_row;
+        const float s = row < d.n ? d.scale[row] : 0.f;
         for (int c0 = 0; c0 < p.npad; c0 += 16) {
           uint32_t v[16];
           tmem_ld16(taddr + (uint32_t)c0, v);
@@ -240,13 +265,13 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
             for (int jj = 0; jj < 16; ++jj)
               v[jj] = __float_as_uint(fmaf(__uint_as_float(u[jj]), 0.0625f, __uint_as_float(v[jj])));
           }
-          if (row < p.n) {
+          if (row < d.n) {
 #pragma unroll
             for (int jj = 0; jj < 16; ++jj) {
               const int m = c0 + jj;
               if (m < p.rows) {
                 const float y = (__uint_as_float(v[jj]) * s) * p.x_scale[m];
-                p.out[(int64_t)m * p.ldc + row] = f32_to_bf16_bits(y);
+                d.out[(int64_t)m * d.ldc + row] = f32_to_bf16_bits(y);
               }
             }
           }
@@ -301,8 +326,9 @@ __global__ void __launch_bounds__(kBM) umma_f8_fixup_kernel(const UmmaParams p, 
   }
   __syncthreads();
   grid_dependency_wait();  // the partial sums and scales of the preceding kernels
-  const int row = (p.wt * G + t_rem) * kBM + threadIdx.x;
-  if (row >= p.n) return;
+  const TileDst d = tile_dst(p, p.wt * G + t_rem);
+  const int row = d.row0 + threadIdx.x;
+  if (row >= d.n) return;
   const int np = s_nparts;
   const float* base = p.partial + threadIdx.x;
   const int64_t slot_stride = (int64_t)p.nb * kBM;
@@ -330,7 +356,7 @@ __global__ void __launch_bounds__(kBM) umma_f8_fixup_kernel(const UmmaParams p, 
     }
   }
   const float acc = p.split ? fmaf(lo, 0.0625f, hi) : hi;
-  p.out[(int64_t)m * p.ldc + row] = f32_to_bf16_bits((acc * p.w_scale[row]) * p.x_scale[m]);
+  d.out[(int64_t)m * d.ldc + row] = f32_to_bf16_bits((acc * d.scale[row]) * p.x_scale[m]);
 }
 
 constexpr size_t kUmmaSmemLimit = 232448 - 2048;
@@ -356,9 +382,18 @@ cudaMemPool_t scratch_pool(int dev) {
   return pools[dev];
 }
 
+// The optional second weight matrix of a paired launch (same k, same activations).
+struct SecondWeight {
+  const uint8_t* w;
+  const float* w_scale;
+  int n;
+  uint16_t* out;
+  int64_t ldc;
+};
+
 int launch_umma_f8(const uint8_t* w, const float* w_scale, int n, int k, const uint8_t* b_codes, int64_t ldb,
                    int b_rows, const float* x_scale, int rows, int split, uint16_t* out, int64_t ldc, cudaStream_t s,
-                   float* partial_ws, size_t partial_cap, int early_w) {
+                   float* partial_ws, size_t partial_cap, int early_w, const SecondWeight* second = nullptr) {
   const DeviceInfo di = device_info();
   if (di.sms <= 0) return DLMH_ERR_CUDA;
   UmmaParams p{};
@@ -383,13 +418,23 @@ int launch_umma_f8(const uint8_t* w, const float* w_scale, int n, int k, const u
   if (ns > kMaxUStages) ns = kMaxUStages;
   if (ns < 2) return DLMH_ERR_UNSUPPORTED;
   p.ns = ns;
-  CUtensorMap mw, mx;
+  CUtensorMap mw, mw2, mx;
   if (!cached_map_k128(&mw, w, 1, n, k, k, kBM, kKC) || !cached_map_k128(&mx, b_codes, 1, b_rows, k, ldb, p.nb, kKC))
     return DLMH_ERR_CUDA;
+  p.t1 = (n + kBM - 1) / kBM;
+  if (second) {
+    if (!cached_map_k128(&mw2, second->w, 1, second->n, k, k, kBM, kKC)) return DLMH_ERR_CUDA;
+    p.n2 = second->n;
+    p.w_scale2 = second->w_scale;
+    p.out2 = second->out;
+    p.ldc2 = second->ldc;
+  } else {
+    mw2 = mw;
+  }
   const size_t smem = (size_t)ns * p.stage_bytes + 1024;
   if (ensure_dynamic_smem(reinterpret_cast<const void*>(umma_f8_kernel), (int)smem) != DLMH_OK) return DLMH_ERR_CUDA;
   // schedule: whole tiles in full waves over the SMs, the rest split into units
-  const int ntiles = (n + kBM - 1) / kBM;
+  const int ntiles = p.t1 + (second ? (second->n + kBM - 1) / kBM : 0);
   p.spt = (k / 128 + kKC - 1) / kKC;
   const Sched sched = make_sched(ntiles, p.spt, di.sms);
   const int G = sched.G;
@@ -410,7 +455,7 @@ int launch_umma_f8(const uint8_t* w, const float* w_scale, int n, int k, const u
       return DLMH_ERR_CUDA;
     p.partial = static_cast<float*>(ws);
   }
-  int rc = launch_pdl(umma_f8_kernel, dim3(G), dim3(kUmmaThreads), smem, s, mw, mx, p);
+  int rc = launch_pdl(umma_f8_kernel, dim3(G), dim3(kUmmaThreads), smem, s, mw, mw2, mx, p);
   if (rc == DLMH_OK && p.rem > 0) {
     rc = launch_pdl(umma_f8_fixup_kernel, dim3(p.rem, rows), dim3(kBM), 0, s, p, G);
   }
@@ -437,6 +482,20 @@ int w8a8_umma_pass(const uint8_t* w, const float* w_scale, int n, int k, const u
     return DLMH_ERR_ALIGN;
   return launch_umma_f8(w, w_scale, n, k, xq, ldq, rows, x_scale, rows, 0, out, ldc, s, partial_ws, partial_cap,
                         after_prepass ? 1 : 0);
+}
+
+int w8a8_umma_pair_pass(const uint8_t* w1, const float* s1, int n1, uint16_t* out1, int64_t ldc1,
+                        const uint8_t* w2, const float* s2, int n2, uint16_t* out2, int64_t ldc2, int k,
+                        const uint8_t* xq, int64_t ldq, const float* x_scale, int rows, cudaStream_t s,
+                        bool after_prepass) {
+  if (rows < 1 || rows > 128) return DLMH_ERR_ROWS;
+  if (!w8a8_umma_supported(k)) return DLMH_ERR_SHAPE;
+  if ((reinterpret_cast<uintptr_t>(w1) & 15u) || (reinterpret_cast<uintptr_t>(w2) & 15u) ||
+      (reinterpret_cast<uintptr_t>(xq) & 15u) || ldq % 16 != 0)
+    return DLMH_ERR_ALIGN;
+  const SecondWeight second{w2, s2, n2, out2, ldc2};
+  return launch_umma_f8(w1, s1, n1, k, xq, ldq, rows, x_scale, rows, 0, out1, ldc1, s, nullptr, 0,
+                        after_prepass ? 1 : 0, &second);
 }
 
 int w8a16_umma_run(const uint8_t* w, const float* w_scale, int n, int k, const uint16_t* x, int64_t ldx, int rows,

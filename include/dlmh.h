@@ -133,7 +133,8 @@ DLMH_API int w8a8_quantize_rows(const dlmh_bf16* x, int64_t ldx, int rows, int k
                        float* x_scale, void* stream);
 
 /* Fused SiLU quantize: h[m, k] = bf16( silu(gate[m, k]) * up[m, k] ), silu(g) = g / (1 + e^-g),
- * computed in f32 and rounded once to BF16, then quantized per row exactly as
+ * in correctly rounded f32 steps (e = rn32(e^-g), d = rn32(1 + e), s = rn32(g / d),
+ * p = rn32(s * up)) and one round-to-nearest-even to BF16, then quantized per row exactly as
  * w8a8_quantize_rows; h is never written to memory.  w8a8_layer.rs, W8a8Ctx::silu_proj
  * (ops::w8a8_act_quant_silu).  gate and up [rows, ld] BF16; rows <= 128. */
 DLMH_API int w8a8_silu_quantize_rows(const dlmh_bf16* gate, const dlmh_bf16* up, int64_t ld, int rows, int k,
@@ -165,6 +166,24 @@ DLMH_API int w8a8_proj(const uint8_t* w, const float* w_scale, int n, int k, con
 DLMH_API int w8a8_silu_proj(const uint8_t* w, const float* w_scale, int n, int k, const dlmh_bf16* gate,
                    const dlmh_bf16* up, int64_t ld, int rows, dlmh_bf16* out, int64_t ldc,
                    uint8_t* xq_scratch, float* xscale_scratch, void* stream);
+
+/* Gate and up projections of a SiLU FFN on ONE quantized copy of x (w8a8_layer.rs, W8a8Ffn:
+ * gate and up read the same input).  Per 128-row chunk: w8a8_quantize_rows once, then
+ *   gate_out[m, n] = bf16( s_gate[n] * sx[m] * sum_k e4m3(w_gate[n, k]) * xq[m, k] )
+ *   up_out[m, n]   = bf16( s_up[n]   * sx[m] * sum_k e4m3(w_up[n, k])   * xq[m, k] )
+ * in one launch over the tiles of both weights when k % 128 == 0 (two register-kernel GEMVs
+ * on the same codes otherwise).  Same numerics as w8a8_proj of each weight; a row's bits do
+ * not depend on `rows`, and they may differ in the last place from a lone w8a8_proj of the
+ * same weight (the two weights share one split-K schedule).
+ *   w_gate, w_up   [n, k] E4M3 bytes (16-byte aligned), s_gate, s_up [n] float32.
+ *   x              [rows, ldx] BF16, any rows >= 0 (chunks of 128).
+ *   gate_out, up_out  [rows, ldc] BF16 (ldc >= n); they feed w8a8_silu_proj with ld = ldc.
+ *   xq_scratch, xscale_scratch  as for w8a8_proj.
+ * Errors as w8a8_proj (DLMH_ERR_NULL for a NULL weight, scale or output of either). */
+DLMH_API int w8a8_gate_up_proj(const uint8_t* w_gate, const float* s_gate, const uint8_t* w_up,
+                               const float* s_up, int n, int k, const dlmh_bf16* x, int64_t ldx, int rows,
+                               dlmh_bf16* gate_out, dlmh_bf16* up_out, int64_t ldc, uint8_t* xq_scratch,
+                               float* xscale_scratch, void* stream);
 
 /* ---------------------------------------------------------------------------------------
  * W8A8 projection that allocates nothing, not even caller scratch

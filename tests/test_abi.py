@@ -92,6 +92,14 @@ def test_w8a8_argument_errors():
     assert L.w8a8_gemv(A, A, 16, 64, A, 64, A, 129, A, 16, None) == -4
     assert L.w8a8_proj(A, A, 16, 64, A, 64, 1, A, 16, None, A, None) == -1
     assert L.w8a8_silu_proj(A, A, 16, 64, A, None, 64, 1, A, 16, A, A, None) == -1
+    # gate+up pair: every pointer of both weights is checked before anything launches
+    assert L.w8a8_gate_up_proj(A, A, None, A, 16, 64, A, 64, 1, A, A, 16, A, A, None) == -1
+    assert L.w8a8_gate_up_proj(A, A, A, None, 16, 64, A, 64, 1, A, A, 16, A, A, None) == -1
+    assert L.w8a8_gate_up_proj(A, A, U, A, 16, 64, A, 64, 1, A, A, 16, A, A, None) == -3
+    assert L.w8a8_gate_up_proj(A, A, A, A, 16, 64, A, 64, 1, A, None, 16, A, A, None) == -1
+    assert L.w8a8_gate_up_proj(A, A, A, A, 16, 64, A, 64, 1, A, A, 8, A, A, None) == -5
+    assert L.w8a8_gate_up_proj(A, A, A, A, 16, 64, A, 64, -1, A, A, 16, A, A, None) == -4
+    assert L.w8a8_gate_up_proj(A, A, A, A, 16, 64, A, 64, 0, A, A, 16, A, A, None) == 0
 
 
 def test_w4a16_argument_errors():
