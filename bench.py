@@ -411,9 +411,9 @@ def other_formats(dev, stream, peak):
     n, k = 129280, 7168
     blocks = synth.q6k_blocks(n, k, 4, dev)
     xk = synth.bf16_rows(64, k, 4, dev)
-    q8s = torch.empty(8 * (k // 32) * 36, dtype=torch.uint8, device=dev)
+    q8s = torch.empty(64 * (k // 32) * 36, dtype=torch.uint8, device=dev)  # one pass per 64 rows
     outk = torch.empty(64, n, dtype=torch.bfloat16, device=dev)
-    rows_list = [1, 8, 16, 64]
+    rows_list = [1, 8, 16, 32, 64]
     calls = [(lambda xm=xk[:m], om=outk[:m]: dl.q6k_lm_head(blocks, xm, out=om, q8_scratch=q8s, stream=stream))
              for m in rows_list]
     entry("q6k_head", f"{n}x{k}", n * (k // 256) * 210, calls, rows_list)

@@ -24,6 +24,7 @@ W8A8_MAX_ROWS = 128
 W8A16_CHUNK_ROWS = 16
 W4A16_MAX_ROWS = 32
 Q6K_CHUNK_ROWS = 8
+Q6K_MAX_ROWS = 64
 Q8_1_BLOCK_BYTES = 36
 Q6K_BLOCK_BYTES = 210
 
@@ -358,7 +359,8 @@ def q6k_lm_head(blocks, x, out=None, q8_scratch=None, stream=None):
     if out is None:
         out = torch.empty(rows, n, dtype=torch.bfloat16, device=x.device)
     if q8_scratch is None:
-        q8_scratch = torch.empty(Q6K_CHUNK_ROWS * (k // 32) * Q8_1_BLOCK_BYTES, dtype=torch.uint8, device=x.device)
+        q8_scratch = torch.empty(min(rows, Q6K_MAX_ROWS) * (k // 32) * Q8_1_BLOCK_BYTES, dtype=torch.uint8,
+                                 device=x.device)
     _check(lib().q6k_lm_head(_ptr(blocks), n, k, _ptr(x), _ld(x), rows, _ptr(out), _ld(out), _ptr(q8_scratch),
                              _stream(stream, x.device)), "q6k_lm_head")
     return out

@@ -56,7 +56,7 @@ int pass_rows(int op, int k) {
     case DLMH_OP_W8A8:
       return dlmh::w8a8_umma_supported(k) ? DLMH_W8A8_MAX_ROWS : dlmh::max_tier_rows(DLMH_OP_W8A8, k);
     case DLMH_OP_W4A16: return dlmh::max_tier_rows(DLMH_OP_W4A16, k);
-    case DLMH_OP_Q6K: return DLMH_Q6K_CHUNK_ROWS;
+    case DLMH_OP_Q6K: return DLMH_Q6K_MAX_ROWS;
     default: return 0;
   }
 }
@@ -107,7 +107,7 @@ int dlmh_plan_chunks(int op, int rows, int k, int* offsets, int* counts, int* ti
       offsets[nchunks] = done;
       counts[nchunks] = m;
       if (op == DLMH_OP_Q6K)
-        tiers[nchunks] = DLMH_Q6K_CHUNK_ROWS;
+        tiers[nchunks] = dlmh::q6k_wide_rows(m);
       else if ((op == DLMH_OP_W8A8 && dlmh::w8a8_umma_supported(k)) ||
                (op == DLMH_OP_W8A16 && dlmh::w8a16_umma_supported(k)))
         tiers[nchunks] = (m + 15) / 16 * 16;  // tensor-core tier: MMA N = rows rounded up to 16
@@ -317,8 +317,9 @@ int q6k_mmvq(const void* blocks, int n, int k, const void* q8, int rows, dlmh_bf
   if ((reinterpret_cast<uintptr_t>(blocks) & 1u) || (reinterpret_cast<uintptr_t>(q8) & 3u)) return DLMH_ERR_ALIGN;
   DLMH_TRY(check_out(out, ldc, n));
   const int64_t q8_row = (int64_t)(k / 32) * DLMH_Q8_1_BLOCK_BYTES;
+  const int width = aligned16(q8) && aligned16(blocks) ? DLMH_Q6K_MAX_ROWS : DLMH_Q6K_CHUNK_ROWS;
   for (int done = 0; done < rows;) {
-    const int m = rows - done < DLMH_Q6K_CHUNK_ROWS ? rows - done : DLMH_Q6K_CHUNK_ROWS;
+    const int m = rows - done < width ? rows - done : width;
     DLMH_TRY(dlmh::q6k_mmvq_launch(static_cast<const uint8_t*>(blocks), n, k,
                                    static_cast<const uint8_t*>(q8) + done * q8_row, m, out + (int64_t)done * ldc, ldc,
                                    as_stream(stream)));
@@ -339,8 +340,9 @@ int q6k_lm_head(const void* blocks, int n, int k, const dlmh_bf16* x, int64_t ld
     return DLMH_ERR_ALIGN;
   DLMH_TRY(check_out(out, ldc, n));
   cudaStream_t s = as_stream(stream);
+  const int width = aligned16(q8_scratch) && aligned16(blocks) ? DLMH_Q6K_MAX_ROWS : DLMH_Q6K_CHUNK_ROWS;
   for (int done = 0; done < rows;) {
-    const int m = rows - done < DLMH_Q6K_CHUNK_ROWS ? rows - done : DLMH_Q6K_CHUNK_ROWS;
+    const int m = rows - done < width ? rows - done : width;
     DLMH_TRY(dlmh::q8_1_quantize_launch(x + (int64_t)done * ldx, ldx, m, k, static_cast<uint8_t*>(q8_scratch), s));
     DLMH_TRY(dlmh::q6k_mmvq_launch(static_cast<const uint8_t*>(blocks), n, k,
                                    static_cast<const uint8_t*>(q8_scratch), m, out + (int64_t)done * ldc, ldc, s));

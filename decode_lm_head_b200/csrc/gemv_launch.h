@@ -76,6 +76,9 @@ int e8m0_dequant_launch(const uint8_t* packed, const uint8_t* scales, int64_t bl
 
 // Fault bits of the streamed Q6_K kernel's bounded waits (read synchronously).
 int q6k_fault(int reset);
+// Q6_K GEMV of 1..64 q8_1 rows in one weight pass: the 8-row kernels up to 8 rows, the wide
+// kernel (tiers 16 / 32 / 64, q8 16-byte aligned, else DLMH_ERR_ALIGN) above; same bits.
+int q6k_wide_rows(int rows);
 int q6k_mmvq_launch(const uint8_t* blocks, int n, int k, const uint8_t* q8, int rows, uint16_t* out, int64_t ldc,
                     cudaStream_t s);
 

@@ -38,6 +38,12 @@ __device__ __forceinline__ uint32_t q6_to_s8x4(uint32_t q) {
   return x | (s * 6u);                          // sign-extend bit 5 into bits 6, 7
 }
 
+// acc + (is * d) * dx with one rounding per step (a product, then a fused multiply-add), the
+// same in every Q6_K kernel whatever the compiler would contract.
+__device__ __forceinline__ float q6_block_step(float acc, int is, float d, float dx) {
+  return __fmaf_rn(__fmul_rn((float)is, d), dx, acc);
+}
+
 // One super-block for rows g (a) and g+8 (b) of a 16-row tile against activation columns 2t
 // and 2t+1 (acc[0..1]: row a, acc[2..3]: row b).  Per q8_1 block (sub-blocks j0, j1) the two
 // exact int32 sub-block dots are scaled by their int8 sub-scales and summed in int32 -- exact,
@@ -73,10 +79,10 @@ __device__ __forceinline__ void q6_superblock(float (&acc)[4], const uint32_t (&
     }
     const int b32 = sb * 8 + blk;
     const float dx0 = dx[(2 * t) * nb32 + b32], dx1 = dx[(2 * t + 1) * nb32 + b32];
-    acc[0] += ((float)is0 * da) * dx0;
-    acc[1] += ((float)is1 * da) * dx1;
-    acc[2] += ((float)is2 * db) * dx0;
-    acc[3] += ((float)is3 * db) * dx1;
+    acc[0] = q6_block_step(acc[0], is0, da, dx0);
+    acc[1] = q6_block_step(acc[1], is1, da, dx1);
+    acc[2] = q6_block_step(acc[2], is2, db, dx0);
+    acc[3] = q6_block_step(acc[3], is3, db, dx1);
   }
 }
 
@@ -173,7 +179,7 @@ __global__ void __launch_bounds__(kQ6Threads, 1) q6k_mmvq_kernel(const Q6Params 
         const int ln = gg * 4 + (cc >> 1), comp = up * 2 + (cc & 1);
         float sum = 0.f;
 #pragma unroll
-        for (int ww = 0; ww < kQ6Warps; ++ww) sum += rb_[(ww * 32 + ln) * 4 + comp];
+        for (int ww = 0; ww < kQ6Warps; ++ww) sum = __fadd_rn(sum, rb_[(ww * 32 + ln) * 4 + comp]);
         p.out[(int64_t)cc * p.ldc + row] = f32_to_bf16_bits(sum);
       }
     }
@@ -333,11 +339,285 @@ __global__ void __launch_bounds__(kQ6Threads, 1) q6k_stream_kernel(const Q6Strea
         const int ln = gg * 4 + (cc >> 1), comp = up * 2 + (cc & 1);
         float sum = 0.f;
 #pragma unroll
-        for (int ww = 0; ww < kQ6Warps; ++ww) sum += rb_[(ww * 32 + ln) * 4 + comp];
+        for (int ww = 0; ww < kQ6Warps; ++ww) sum = __fadd_rn(sum, rb_[(ww * 32 + ln) * 4 + comp]);
         p.out[(int64_t)cc * p.ldc + row] = f32_to_bf16_bits(sum);
       }
     }
     parity ^= 1;
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Wide variant: 9..64 q8_1 rows in one weight pass.  Whole activation rows no longer fit in
+// shared memory (64 rows of codes at K = 7168 take 458 KB), so the loop order is turned
+// around: a CTA takes its 16-row weight tiles in row-blocks of up to kQWWarps tiles, one tile
+// per consumer warp, and the row-block walks K one super-block at a time.
+//   - Activations: a producer warp copies each super-block's q8_1 blocks of every activation
+//     row (288 contiguous bytes per row) into a ring shared by the row-block's warps, with
+//     16-byte cp.async and one mbarrier arrival per lane; the activations are re-read (from
+//     L2) once per row-block, not once per tile.
+//   - Weights: every consumer warp streams its own tile through a private ring of kQWDepth
+//     stages with 16-byte cp.async (Ampere-style multistage pipeline, no registers held):
+//     per row the 16-byte aligned span that covers the super-block's 210 bytes (at most 224;
+//     super-blocks are only 2-byte aligned), read back at the span's offset with
+//     funnel-shifted 32-bit shared loads.  The buffer's last bytes past its last 16-byte
+//     boundary are stored with plain loads, so no copy reads past the weight buffer.
+// Each consumer warp runs NT 8-column MMAs per sub-block on one decoded A fragment.
+// The per-output arithmetic and its order are those of the 8-row kernels: K is cut into the
+// same 16 slices of nsbw super-blocks, each slice is accumulated alone from 0 with the same
+// per-block step, and the slices are added to 0 in order -- so a row's bits do not depend on
+// which kernel, or how many rows, served it.
+// 15 consumer warps + 1 producer: 16 warps, 4 per SM sub-partition, so 128 registers a thread
+constexpr int kQWWarps = 15;
+constexpr int kQWThreads = (kQWWarps + 1) * 32;
+constexpr int kQWRowBytes = 288;   // one super-block of one q8_1 row: 8 blocks
+constexpr int kQWRowStride = 304;  // 76 words: the 8 B-fragment rows hit 32 banks
+constexpr int kQWSpan = 240;       // staged bytes per weight row and super-block (>= 224)
+constexpr int kQWTileBytes = kQ6TileRows * kQWSpan;
+constexpr int kQWMaxActStages = 4;
+
+struct Q6WideParams {
+  Q6Params q;
+  int act_stages;  // activation ring stages of NT * 8 * kQWRowStride bytes
+  int depth;       // weight stages per consumer warp (>= 2)
+};
+
+__device__ __forceinline__ uint32_t lds_u32(uint32_t saddr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(saddr));
+  return v;
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+// The mbarrier receives one arrival when this thread's earlier cp.async copies have landed.
+__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+// One super-block of one warp's 16-row tile against NT 8-column groups of the staged chunk at
+// `xs` (row stride kQWRowStride, block b of row m at m * stride + 36 b: f16 d, f16 s, 32 codes).
+// Per (row, column) the same integer and float steps, in the same order, as q6_superblock.
+template <int NT>
+__device__ __forceinline__ void q6_superblock_wide(float (&acc)[NT][4], const uint32_t (&qla)[8],
+                                                   const uint32_t (&qlb)[8], const uint32_t (&qha)[4],
+                                                   const uint32_t (&qhb)[4], const uint32_t (&sca)[4],
+                                                   const uint32_t (&scb)[4], float da, float db, uint32_t xs, int g,
+                                                   int t) {
+#pragma unroll
+  for (int blk = 0; blk < 8; ++blk) {  // unrolled: the fragment arrays stay in registers
+    uint32_t a0[2], a1[2];
+    int ra[2], rb[2];
+#pragma unroll
+    for (int hj = 0; hj < 2; ++hj) {
+      const int j = 2 * blk + hj;
+      const int h = j >> 3, u = (j & 7) >> 1;
+      const int qi = 4 * h + 2 * (u & 1) + (j & 1);
+      const int hi = 2 * h + (j & 1);
+      const int nsh = (u >> 1) * 4, hsh = 2 * u;
+      a0[hj] = q6_to_s8x4(((qla[qi] >> nsh) & 0x0f0f0f0fu) | (((qha[hi] >> hsh) & 0x03030303u) << 4));
+      a1[hj] = q6_to_s8x4(((qlb[qi] >> nsh) & 0x0f0f0f0fu) | (((qhb[hi] >> hsh) & 0x03030303u) << 4));
+      const int sha = 24 - 8 * (j & 3);
+      ra[hj] = (int)(sca[j >> 2] << sha) >> 24;
+      rb[hj] = (int)(scb[j >> 2] << sha) >> 24;
+    }
+#pragma unroll
+    for (int ct = 0; ct < NT; ++ct) {
+      const uint32_t brow = xs + (uint32_t)((8 * ct + g) * kQWRowStride + 36 * blk + 4 + 4 * t);
+      int d0[4] = {0, 0, 0, 0}, d1[4] = {0, 0, 0, 0};
+      mma_s8_16816(d0, a0[0], a1[0], lds_u32(brow));
+      mma_s8_16816(d1, a0[1], a1[1], lds_u32(brow + 16));
+      const int is0 = d0[0] * ra[0] + d1[0] * ra[1];
+      const int is1 = d0[1] * ra[0] + d1[1] * ra[1];
+      const int is2 = d0[2] * rb[0] + d1[2] * rb[1];
+      const int is3 = d0[3] * rb[0] + d1[3] * rb[1];
+      const uint32_t drow = xs + (uint32_t)((8 * ct + 2 * t) * kQWRowStride + 36 * blk);
+      const float dx0 = f16_bits_to_f32(lds_u16(drow));
+      const float dx1 = f16_bits_to_f32(lds_u16(drow + kQWRowStride));
+      acc[ct][0] = q6_block_step(acc[ct][0], is0, da, dx0);
+      acc[ct][1] = q6_block_step(acc[ct][1], is1, da, dx1);
+      acc[ct][2] = q6_block_step(acc[ct][2], is2, db, dx0);
+      acc[ct][3] = q6_block_step(acc[ct][3], is3, db, dx1);
+    }
+  }
+}
+
+// Stage super-block sb of the 16 rows of tile `tile` into `dst` (row i at i * kQWSpan) with
+// this lane's share of the 16-byte pieces; rows at or past n are skipped.
+__device__ __forceinline__ void q6_stage_tile(const Q6Params& p, int64_t row_bytes, uintptr_t buf_end, int tile,
+                                              int sb, uint32_t dst, int lane) {
+  for (int c = lane; c < kQ6TileRows * (kQWSpan / 16); c += 32) {
+    const int i = c / (kQWSpan / 16), piece = c % (kQWSpan / 16);
+    const int row = tile * kQ6TileRows + i;
+    if (row >= p.n) continue;
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p.blocks) + (uintptr_t)((int64_t)row * row_bytes + 210 * sb);
+    const uintptr_t a16 = a & ~uintptr_t(15);
+    const uintptr_t src = a16 + 16u * piece;
+    if (src >= a + 210) continue;  // past the span
+    const uint32_t d = dst + (uint32_t)(i * kQWSpan + 16 * piece);
+    if (src + 16 <= buf_end) {
+      cp_async16(d, reinterpret_cast<const void*>(src));
+    } else {  // the buffer's last bytes: plain 16-bit loads up to its end
+      for (uintptr_t o = src; o < buf_end; o += 2)
+        asm volatile("st.shared.u16 [%0], %1;" ::"r"(d + (uint32_t)(o - src)),
+                     "h"((unsigned short)ldg_u16(reinterpret_cast<const void*>(o)))
+                     : "memory");
+    }
+  }
+}
+
+template <int NT>
+__global__ void __launch_bounds__(kQWThreads, 1) q6k_wide_kernel(const Q6WideParams wp) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ __align__(8) uint64_t full[kQWMaxActStages], empty[kQWMaxActStages];
+  const Q6Params& p = wp.q;
+  const int nsb = p.k / 256;
+  const int nb32 = p.k / 32;
+  const int nsbw = (nsb + kQ6Warps - 1) / kQ6Warps;  // slice length of the 8-row kernels
+  const int64_t row_bytes = (int64_t)nsb * 210;
+  const uintptr_t buf_end = reinterpret_cast<uintptr_t>(p.blocks) + (uintptr_t)((int64_t)p.n * row_bytes);
+  constexpr int kRows = NT * 8;
+  constexpr uint32_t kActBytes = kRows * kQWRowStride;
+  const int ns = wp.act_stages, depth = wp.depth;
+  const uint32_t act_ring = smem_u32(smem);
+  const uint32_t w_rings = act_ring + (uint32_t)ns * kActBytes;
+  const uint32_t full0 = smem_u32(full), empty0 = smem_u32(empty);
+
+  const int ntiles = (p.n + kQ6TileRows - 1) / kQ6TileRows;
+  const int T0 = (int)((int64_t)blockIdx.x * ntiles / gridDim.x);
+  const int T1 = (int)((int64_t)(blockIdx.x + 1) * ntiles / gridDim.x);
+  const int nt = T1 - T0;
+  const int nrb = (nt + kQWWarps - 1) / kQWWarps;  // row-blocks, as even as possible
+  const int nchunks = nrb * nsb;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // padding activation rows [rows, kRows) of every stage stay zero (never copied)
+  for (int i = threadIdx.x; i < ns * (int)(kActBytes / 4); i += blockDim.x) {
+    const int w = i % (int)(kActBytes / 4);
+    if (w / (kQWRowStride / 4) >= p.rows) reinterpret_cast<uint32_t*>(smem)[i] = 0u;
+  }
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < ns; ++i) {
+      umma::bar_init(full0 + 8u * i, 32);  // one arrival per producer lane, when its copies land
+      umma::bar_init(empty0 + 8u * i, kQWWarps);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+
+  if (warp == kQWWarps) {
+    // ---------------- producer: chunk c = (row-block c / nsb, super-block c % nsb)
+    constexpr int kPieces = kQWRowBytes / 16;
+    for (int c = 0; c < nchunks; ++c) {
+      const int slot = c % ns, sb = c % nsb;
+      if (c >= ns && !umma::wait(empty0 + 8u * slot, ((c / ns) - 1) & 1)) atomicOr(&q6_fault_word, 4);
+      __syncwarp();
+      const uint32_t st = act_ring + (uint32_t)slot * kActBytes;
+      for (int q = lane; q < p.rows * kPieces; q += 32) {
+        const int m = q / kPieces, piece = q % kPieces;
+        cp_async16(st + (uint32_t)(m * kQWRowStride + 16 * piece),
+                   p.q8 + ((int64_t)m * nb32 + 8 * sb) * 36 + 16 * piece);
+      }
+      cp_async_arrive(full0 + 8u * slot);
+    }
+    cp_async_wait<0>();  // nothing of this thread in flight at exit
+    return;
+  }
+
+  // ---------------- consumers
+  const int g = lane >> 2, t = lane & 3;
+  const uint32_t my_ring = w_rings + (uint32_t)(warp * depth * kQWTileBytes);
+  int c = 0;
+  for (int r = 0; r < nrb; ++r) {
+    const int tb0 = T0 + (int)((int64_t)r * nt / nrb), tb1 = T0 + (int)((int64_t)(r + 1) * nt / nrb);
+    const int tile = tb0 + warp;
+    const bool active = tile < tb1;
+    const int r0 = tile * kQ6TileRows + g;
+    const bool va = active && r0 < p.n, vb = active && r0 + 8 < p.n;
+    // weight pipeline: stages 0 .. depth-2 in flight before the loop (one group each)
+    for (int s = 0; s < depth - 1; ++s) {
+      if (active && s < nsb) q6_stage_tile(p, row_bytes, buf_end, tile, s, my_ring + (uint32_t)(s * kQWTileBytes), lane);
+      cp_async_commit();
+    }
+    float tot[NT][4], sl[NT][4];
+#pragma unroll
+    for (int ct = 0; ct < NT; ++ct)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) tot[ct][i] = sl[ct][i] = 0.f;
+    for (int sb = 0; sb < nsb; ++sb, ++c) {
+      const int slot = c % ns;
+      const uint32_t st = act_ring + (uint32_t)slot * kActBytes;
+      // keep depth - 1 weight stages in flight: issue sb + depth - 1, wait for sb
+      {
+        const int s2 = sb + depth - 1;
+        if (active && s2 < nsb)
+          q6_stage_tile(p, row_bytes, buf_end, tile, s2, my_ring + (uint32_t)((s2 % depth) * kQWTileBytes), lane);
+        cp_async_commit();
+      }
+      if (depth == 3) cp_async_wait<2>(); else cp_async_wait<1>();
+      __syncwarp();
+      if (!umma::wait(full0 + 8u * slot, (c / ns) & 1)) atomicOr(&q6_fault_word, 2);
+      if (active) {
+        const uint32_t wbase = my_ring + (uint32_t)((sb % depth) * kQWTileBytes);
+        const uint32_t ba = wbase + (uint32_t)(g * kQWSpan) +
+                            (uint32_t)((reinterpret_cast<uintptr_t>(p.blocks) + (uintptr_t)((int64_t)r0 * row_bytes + 210 * sb)) & 15u);
+        const uint32_t bb = wbase + (uint32_t)((g + 8) * kQWSpan) +
+                            (uint32_t)((reinterpret_cast<uintptr_t>(p.blocks) + (uintptr_t)((int64_t)(r0 + 8) * row_bytes + 210 * sb)) & 15u);
+        uint32_t qla[8], qlb[8], qha[4], qhb[4], sca[4], scb[4];
+        float da = 0.f, db = 0.f;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          qla[q] = va ? lds_u32_a2(ba + 16 * q + 4 * t) : 0u;
+          qlb[q] = vb ? lds_u32_a2(bb + 16 * q + 4 * t) : 0u;
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          qha[q] = va ? lds_u32_a2(ba + 128 + 16 * q + 4 * t) : 0u;
+          qhb[q] = vb ? lds_u32_a2(bb + 128 + 16 * q + 4 * t) : 0u;
+          sca[q] = va ? lds_u32_a2(ba + 192 + 4 * q) : 0u;
+          scb[q] = vb ? lds_u32_a2(bb + 192 + 4 * q) : 0u;
+        }
+        if (va) da = f16_bits_to_f32(lds_u16(ba + 208));
+        if (vb) db = f16_bits_to_f32(lds_u16(bb + 208));
+        q6_superblock_wide<NT>(sl, qla, qlb, qha, qhb, sca, scb, da, db, st, g, t);
+      }
+      __syncwarp();  // the weight stage and the activation slot are read
+      if (lane == 0) umma::arrive(empty0 + 8u * slot);
+      // end of a slice of the 8-row kernels: add it to the total and restart
+      if ((sb + 1) % nsbw == 0 || sb + 1 == nsb) {
+#pragma unroll
+        for (int ct = 0; ct < NT; ++ct)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            tot[ct][i] = __fadd_rn(tot[ct][i], sl[ct][i]);
+            sl[ct][i] = 0.f;
+          }
+      }
+    }
+    cp_async_wait<0>();
+    __syncwarp();
+    // slices past K (empty warps of the 8-row kernels) add +0
+    for (int w = (nsb + nsbw - 1) / nsbw; w < kQ6Warps; ++w)
+#pragma unroll
+      for (int ct = 0; ct < NT; ++ct)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) tot[ct][i] = __fadd_rn(tot[ct][i], 0.f);
+    if (active) {
+#pragma unroll
+      for (int ct = 0; ct < NT; ++ct) {
+        const int m0 = 8 * ct + 2 * t;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int m = m0 + (i & 1), row = r0 + 8 * (i >> 1);
+          if (m < p.rows && row < p.n) p.out[(int64_t)m * p.ldc + row] = f32_to_bf16_bits(tot[ct][i]);
+        }
+      }
+    }
   }
 }
 
@@ -348,10 +628,46 @@ size_t q6k_smem_bytes(int k) {
 
 }  // namespace
 
+namespace {
+
+template <int NT>
+int launch_wide(const Q6Params& p, int sms, int smem_optin, cudaStream_t s) {
+  const size_t act = (size_t)NT * 8 * kQWRowStride;
+  const size_t limit = (size_t)smem_optin > 1024 ? (size_t)smem_optin - 1024 : 0;  // static smem < 1 KB
+  // three weight stages per warp when they fit beside at least two activation stages
+  int depth = 3;
+  if ((size_t)kQWWarps * depth * kQWTileBytes + 2 * act > limit) depth = 2;
+  const size_t wbytes = (size_t)kQWWarps * depth * kQWTileBytes;
+  if (wbytes + 2 * act > limit) return DLMH_ERR_UNSUPPORTED;
+  int ns = (int)((limit - wbytes) / act);
+  if (ns > kQWMaxActStages) ns = kQWMaxActStages;
+  const size_t smem = (size_t)ns * act + wbytes;
+  if (ensure_dynamic_smem(reinterpret_cast<const void*>(q6k_wide_kernel<NT>), (int)smem) != DLMH_OK)
+    return DLMH_ERR_CUDA;
+  const int ntiles = (p.n + kQ6TileRows - 1) / kQ6TileRows;
+  const int grid = ntiles < sms ? ntiles : sms;
+  q6k_wide_kernel<NT><<<grid, kQWThreads, smem, s>>>(Q6WideParams{p, ns, depth});
+  return launch_status();
+}
+
+}  // namespace
+
+int q6k_wide_rows(int rows) { return rows <= 8 ? 8 : rows <= 16 ? 16 : rows <= 32 ? 32 : 64; }
+
 int q6k_mmvq_launch(const uint8_t* blocks, int n, int k, const uint8_t* q8, int rows, uint16_t* out, int64_t ldc,
                     cudaStream_t s) {
   const DeviceInfo di = device_info();
   if (di.sms <= 0) return DLMH_ERR_CUDA;
+  if (rows > kQ6MaxRows) {  // 9..64 rows: one pass of the wide kernel (16-byte aligned blocks, q8_1 rows)
+    if (rows > 64) return DLMH_ERR_ROWS;
+    if ((reinterpret_cast<uintptr_t>(q8) & 15u) || (reinterpret_cast<uintptr_t>(blocks) & 15u)) return DLMH_ERR_ALIGN;
+    const Q6Params p{blocks, n, k, q8, rows, out, ldc};
+    switch (q6k_wide_rows(rows)) {
+      case 16: return launch_wide<2>(p, di.sms, di.smem_optin, s);
+      case 32: return launch_wide<4>(p, di.sms, di.smem_optin, s);
+      default: return launch_wide<8>(p, di.sms, di.smem_optin, s);
+    }
+  }
   const size_t base_smem = q6k_smem_bytes(k);
   Q6Params p{blocks, n, k, q8, rows, out, ldc};
   const int ntiles = (n + kQ6TileRows - 1) / kQ6TileRows;

@@ -86,8 +86,10 @@ typedef enum dlmh_status {
 /* Largest row count of one NVFP4 W4A16 call (w4a16_gemv_tiers.rs, kernel_within:
  * more than 32 rows is refused). */
 #define DLMH_W4A16_MAX_ROWS 32
-/* Rows per Q6_K launch (MAX_M / KQ_MAX_M in lm_head_q6k.rs). */
+/* Rows of the pages' Q6_K launch (MAX_M / KQ_MAX_M in lm_head_q6k.rs): the narrowest tier. */
 #define DLMH_Q6K_CHUNK_ROWS 8
+/* Rows per Q6_K weight pass here (tiers 8 / 16 / 32 / 64; the pages run 8-row launches). */
+#define DLMH_Q6K_MAX_ROWS 64
 /* Bytes of one block_q8_1 (32 values) and one Q6_K super-block (256 values). */
 #define DLMH_Q8_1_BLOCK_BYTES 36
 #define DLMH_Q6K_BLOCK_BYTES 210
@@ -248,14 +250,18 @@ DLMH_API int q8_1_quantize_rows(const dlmh_bf16* x, int64_t ldx, int rows, int k
  * 2 bits from bits 2t..2t+1 of qh[32h + l]; element i uses scales[i/16].
  *   blocks [n][k/256] super-blocks, row stride k/256 * 210 bytes (the raw store layout).
  *   q8     [rows][k/32] block_q8_1 as written by q8_1_quantize_rows.
- *   k % 256 == 0 (set_lm_head_q6k requires hidden % 256 == 0).  Any rows (8-row launches).
+ *   k % 256 == 0 (set_lm_head_q6k requires hidden % 256 == 0).  Any rows: one weight pass per
+ *   64 rows, through the narrowest tier of 8 / 16 / 32 / 64 that covers them (above 8 rows the
+ *   q8_1 rows must start 16-byte aligned, else the pass falls back to 8-row launches).  Every
+ *   tier adds the same products in the same order, so a row's bits do not depend on `rows`.
  * ------------------------------------------------------------------------------------- */
 DLMH_API int q6k_mmvq(const void* blocks, int n, int k, const void* q8, int rows, dlmh_bf16* out, int64_t ldc,
              void* stream);
 
 /* The Q6_K head for BF16 rows (lm_head_q6k.rs, lm_head_q6k_run): for each chunk of up to
- * 8 rows, q8_1_quantize_rows into q8_scratch, then q6k_mmvq.  q8_scratch holds at least
- * 8 * k/32 * 36 bytes. */
+ * DLMH_Q6K_MAX_ROWS rows, q8_1_quantize_rows into q8_scratch, then q6k_mmvq.  q8_scratch holds
+ * at least min(rows, 64) * k/32 * 36 bytes (16-byte aligned for one pass per 64 rows; a
+ * 4-byte aligned scratch runs 8-row passes). */
 DLMH_API int q6k_lm_head(const void* blocks, int n, int k, const dlmh_bf16* x, int64_t ldx, int rows,
                 dlmh_bf16* out, int64_t ldc, void* q8_scratch, void* stream);
 

@@ -35,7 +35,7 @@ def test_error_strings_and_version():
 
 @pytest.mark.parametrize("opid,k,width", [(dl.OP_W8A16, 5120, 128), (dl.OP_W8A16, 1040, 16), (dl.OP_W8A8, 5120, 128),
                                            (dl.OP_W8A8, 14336, 128), (dl.OP_W8A8, 1040, 32), (dl.OP_W4A16, 4096, 16),
-                                           (dl.OP_Q6K, 7168, 8)])
+                                           (dl.OP_Q6K, 7168, 64)])
 def test_plan_matches_oracle_rules(opid, k, width):
     cap = 32 if opid == dl.OP_W4A16 else 300
     for rows in range(0, cap + 1):
@@ -43,7 +43,7 @@ def test_plan_matches_oracle_rules(opid, k, width):
         ref = op.chunk_plan(rows, width)
         assert [(o, c) for o, c, _ in plan] == ref
         if opid == dl.OP_Q6K:
-            widths = [8]
+            widths = [8, 16, 32, 64]
         elif opid in (dl.OP_W8A8, dl.OP_W8A16) and k % 128 == 0:
             widths = list(range(16, 129, 16))  # tensor-core tier: MMA N in steps of 16
         else:

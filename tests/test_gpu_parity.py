@@ -380,6 +380,35 @@ def test_q6k_streamed_and_register_kernels_agree(n, k):
     assert dl.device_fault(reset=True) == 0
 
 
+@pytest.mark.parametrize("n,k", [(1000, 7168), (45, 1280), (300, 512)])
+def test_q6k_wide_tiers_one_pass(n, k):
+    # (45 x 1280: the weight buffer ends off a 16-byte boundary, so its last bytes are staged
+    # with plain loads)
+    # 9..64 rows take one pass of the wide kernel (tiers 16 / 32 / 64); every row count must
+    # give the 8-row kernels' bits (same slices, same order), and the oracle's values
+    blocks = synth.q6k_blocks(n, k, 7, DEV)
+    x = synth.bf16_rows(64, k, 7, DEV)
+    full = bits(dl.q6k_lm_head(blocks, x))
+    ref = og.q6k_mmvq(bits(blocks), og.q8_1_quantize_rows(bits(x)))
+    assert_bf16_close(full, ref, f"q6k wide n={n} k={k} M=64")
+    for m in (1, 8, 9, 15, 16, 17, 32, 33, 63):
+        part = bits(dl.q6k_lm_head(blocks, x[:m]))
+        assert np.array_equal(part, full[:m]), f"row invariance M={m}"
+    # q8_1 rows that are only 4-byte aligned: 8-row passes, the same bits
+    q8 = dl.q8_1_quantize_rows(x[:40])
+    flat = torch.zeros(q8.numel() + 16, dtype=torch.uint8, device=DEV)
+    flat[4:4 + q8.numel()] = q8.reshape(-1)
+    shifted = flat[4:4 + q8.numel()].view(q8.shape)
+    assert shifted.data_ptr() % 16 == 4
+    assert np.array_equal(bits(dl.q6k_mmvq(blocks, shifted)), full[:40])
+    # super-blocks that start only 2-byte aligned as a whole: 8-row passes as well
+    fb = torch.zeros(blocks.numel() + 16, dtype=torch.uint8, device=DEV)
+    fb[2:2 + blocks.numel()] = blocks.reshape(-1)
+    bshift = fb[2:2 + blocks.numel()].view(blocks.shape)
+    assert np.array_equal(bits(dl.q6k_mmvq(bshift, q8)), full[:40])
+    assert dl.device_fault(reset=True) == 0
+
+
 # ---------------------------------------------------------------------------
 # full-size heads, sampled outputs
 # ---------------------------------------------------------------------------
