@@ -163,6 +163,68 @@ def w4a16_gemv(w_packed, w_block_scale, global_scale, x):
 
 
 # ----------------------------------------------------------------------------
+# NEXT 4  NVFP4 W4A4: FP4 activations for the wider row edge
+# ----------------------------------------------------------------------------
+
+NVFP4_ACT_GLOBAL_DIV = 2688.0   # 6 (largest E2M1) x 448 (largest E4M3)
+
+
+def nvfp4_quantize_rows(x):
+    """Per-row dynamic NVFP4 quantize of BF16 rows (the W4A4 activations).
+
+    w4a16_gemv_tiers.rs, ``W4a16BatchmTiers`` (``a4_rows``, ``w4a4_proj``): a
+    weight that declares FP4 activations runs its narrow projections W4A4 up
+    to ``W4A4_MAX_M`` rows; the NVFP4 layout is fp8_lut.rs's (E2M1 pairs,
+    even index in the low nibble, one E4M3 scale per 16 values, a float32
+    global).  The pages do not print the quantize; this is the plain NVFP4
+    recipe, every decision in float32 as the kernel takes it:
+      g     = amax(row) / 2688                      (IEEE float32 division)
+      s_b   = e4m3_rn_sat( amax(block b) / rn32(6 g) )
+      S_b   = rn32( e4m3(s_b) * g )
+      code  = e2m1_rn_sat( rn32(x / S_b) ),  0 where S_b == 0.
+    Returns (codes packed uint8 [M, K/2], block scales uint8 [M, K/16],
+    globals float32 [M]).  x: uint16 [M, K], K % 16 == 0.
+    """
+    X = nx.bf16_decode(x)
+    M, K = X.shape
+    if K % NVFP4_BLOCK:
+        raise ValueError("K must be a multiple of 16")
+    g = nx.f32(np.abs(X).max(axis=1) / NVFP4_ACT_GLOBAL_DIV) if K else np.zeros(M)
+    B = np.abs(X).reshape(M, K // NVFP4_BLOCK, NVFP4_BLOCK).max(axis=2)
+    d6 = nx.f32(6.0 * g)[:, None]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        sf = np.where(d6 > 0, nx.f32(B / np.where(d6 > 0, d6, 1.0)), 0.0)
+    s_code = nx.e4m3_rn_sat(sf)
+    S = nx.f32(nx.e4m3_decode(s_code) * g[:, None])
+    S_full = np.repeat(S, NVFP4_BLOCK, axis=1)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        q = np.where(S_full > 0, nx.f32(X / np.where(S_full > 0, S_full, 1.0)), 0.0)
+    codes = np.where(S_full > 0, nx.e2m1_rn_sat(q), 0).astype(np.uint8)
+    return nx.pack_nibbles(codes), s_code, g.astype(np.float32)
+
+
+def w4a4_gemv(w_packed, w_block_scale, global_scale, xq, x_block_scale, x_global):
+    """``out[m, n] = bf16_rn(g_w * g_x[m] * sum_b e4m3(S[n, b]) e4m3(s[m, b]) sum_{k in b} e2m1(W) e2m1(X))``.
+
+    The W4A4 projection (w4a16_gemv_tiers.rs, ``w4a4_proj``): both operands
+    NVFP4, decoded exactly, the dot in float64, the two globals applied once,
+    one BF16 rounding.  xq uint8 [M, K/2], x_block_scale uint8 [M, K/16],
+    x_global float32 [M].
+    """
+    Wd = nvfp4_dequant(w_packed, w_block_scale)
+    Xd = nvfp4_dequant(xq, x_block_scale)
+    acc = Xd @ Wd.T
+    gx = np.asarray(x_global, dtype=np.float32).astype(np.float64)[:, None]
+    return nx.bf16_rn(acc * float(np.float32(global_scale)) * gx)
+
+
+def w4a4_proj(w_packed, w_block_scale, global_scale, x):
+    """BF16 rows -> nvfp4_quantize_rows -> w4a4_gemv."""
+    q, s, g = nvfp4_quantize_rows(x)
+    return w4a4_gemv(w_packed, w_block_scale, global_scale, q, s, g)
+
+
+# ----------------------------------------------------------------------------
 # NEXT 3  load-time FP4 dequant to BF16 (the step before the path)
 # ----------------------------------------------------------------------------
 

@@ -149,6 +149,29 @@ def e2m1_decode(codes):
     return E2M1_TABLE[np.asarray(codes, dtype=np.uint8) & 0xF]
 
 
+def e2m1_rn_sat(v):
+    """Values (float64, typically float32-exact) -> 4-bit E2M1 codes (0..15).
+
+    Round-to-nearest-even on the E2M1 grid (1 mantissa bit, subnormal quantum
+    0.5: 0, 0.5, 1, 1.5, 2, 3, 4, 6), then saturate: magnitudes above 6 give
+    6.  A negative value that rounds to zero gives -0 (code 8).  NaN input is
+    outside the contract.
+    """
+    v = np.asarray(v, dtype=np.float64)
+    r = _round_to_format(v, 1, 0, 6.0, False)
+    mag = np.abs(r)
+    code = np.searchsorted(E2M1_TABLE[:8], mag)
+    if not np.array_equal(E2M1_TABLE[np.minimum(code, 7)], mag):
+        raise AssertionError("rounded value is not on the E2M1 grid")
+    return (code.astype(np.uint8) | np.where(np.signbit(r), 8, 0).astype(np.uint8)).astype(np.uint8)
+
+
+def pack_nibbles(codes):
+    """Codes [..., K] (0..15) -> packed bytes [..., K/2], even index in the low nibble."""
+    c = np.asarray(codes, dtype=np.uint8)
+    return (c[..., 0::2] | (c[..., 1::2] << 4)).astype(np.uint8)
+
+
 def unpack_nibbles(packed):
     """Packed FP4 bytes [..., K/2] -> codes [..., K].
 
