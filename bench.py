@@ -381,6 +381,20 @@ def other_formats(dev, stream, peak):
         dl.w4a16_gemv(wp, sc, gl, xm, out=om, stream=stream)
 
     entry("nvfp4_w4a16", f"{n}x{k}", n * k // 2 + n * k // 16, [(lambda m=m: fp4(m)) for m in rows_list], rows_list)
+
+    # NVFP4 W4A4: the same weights against per-row NVFP4-quantized activations (quantize + GEMV)
+    rows_list = [1, 8, 16, 32]
+    xq4 = torch.empty(32 * k // 2, dtype=torch.uint8, device=dev)
+    xs4 = torch.empty(32 * k // 16, dtype=torch.uint8, device=dev)
+    xg4 = torch.empty(32, dtype=torch.float32, device=dev)
+
+    def fp4a4(m):
+        wp, sc, gl = wf[ctr[0] % len(wf)]
+        ctr[0] += 1
+        xm, om = fviews[m]
+        dl.w4a4_proj(wp, sc, gl, xm, out=om, xq_scratch=xq4, xs_scratch=xs4, xg_scratch=xg4, stream=stream)
+
+    entry("nvfp4_w4a4", f"{n}x{k}", n * k // 2 + n * k // 16, [(lambda m=m: fp4a4(m)) for m in rows_list], rows_list)
     del wf
 
     # load-time NVFP4 / E8M0 dequant to BF16 (HBM stream: codes + scales in, BF16 out)

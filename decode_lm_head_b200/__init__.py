@@ -8,6 +8,7 @@ generators used by the tests and the benchmark.
 from ._lib import (  # noqa: F401
     DlmhError,
     OP_Q6K,
+    OP_W4A4,
     OP_W4A16,
     OP_W8A8,
     OP_W8A16,
@@ -18,12 +19,15 @@ from ._lib import (  # noqa: F401
     lib,
     lm_head_fp8_w8a16,
     nvfp4_dequant_bf16,
+    nvfp4_quantize_rows,
     plan_chunks,
     q6k_lm_head,
     q6k_mmvq,
     q8_1_quantize_rows,
     version,
     w4a16_gemv,
+    w4a4_gemv,
+    w4a4_proj,
     w8a8_gate_up_proj,
     w8a8_gemv,
     w8a8_proj,

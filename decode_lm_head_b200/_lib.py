@@ -18,7 +18,8 @@ LIB_PATH = os.environ.get("DLMH_LIBRARY") or os.path.join(_HERE, "libdlmh.so")
 HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "dlmh.h")
 
 # op ids of dlmh_plan_chunks (dlmh_op in dlmh.h)
-OP_W8A16, OP_W8A8, OP_W4A16, OP_Q6K = 0, 1, 2, 3
+OP_W8A16, OP_W8A8, OP_W4A16, OP_Q6K, OP_W4A4 = 0, 1, 2, 3, 4
+W4A4_MAX_ROWS = 32
 
 W8A8_MAX_ROWS = 128
 W8A16_CHUNK_ROWS = 16
@@ -52,6 +53,9 @@ _SIGNATURES = {
     "w8a8_gate_up_proj": [_P, _P, _P, _P, _I, _I, _P, _L, _I, _P, _P, _L, _P, _P, _P],
     "w8a8_proj_noalloc": [_P, _P, _I, _I, _P, _L, _I, _P, _L, _P],
     "w4a16_gemv": [_P, _P, _F, _I, _I, _P, _L, _I, _P, _L, _P],
+    "nvfp4_quantize_rows": [_P, _L, _I, _I, _P, _P, _P, _P],
+    "w4a4_gemv": [_P, _P, _F, _I, _I, _P, _P, _P, _I, _P, _L, _P],
+    "w4a4_proj": [_P, _P, _F, _I, _I, _P, _L, _I, _P, _L, _P, _P, _P, _P],
     "q8_1_quantize_rows": [_P, _L, _I, _I, _P, _P],
     "q6k_mmvq": [_P, _I, _I, _P, _I, _P, _L, _P],
     "q6k_lm_head": [_P, _I, _I, _P, _L, _I, _P, _L, _P, _P],
@@ -320,6 +324,66 @@ def w4a16_gemv(w_packed, w_block_scale, global_scale, x, out=None, stream=None):
         out = torch.empty(rows, n, dtype=torch.bfloat16, device=x.device)
     _check(lib().w4a16_gemv(_ptr(w_packed), _ptr(w_block_scale), float(global_scale), n, k, _ptr(x), _ld(x), rows,
                             _ptr(out), _ld(out), _stream(stream, x.device)), "w4a16_gemv")
+    return out
+
+
+def nvfp4_quantize_rows(x, xq=None, x_block_scale=None, x_global=None, stream=None):
+    """(codes [rows, k/2] uint8, block scales [rows, k/16] uint8, globals [rows] f32)."""
+    _cuda(x, torch.bfloat16, "x", 2)
+    rows, k = x.shape
+    if xq is None:
+        xq = torch.empty(rows, k // 2, dtype=torch.uint8, device=x.device)
+    if x_block_scale is None:
+        x_block_scale = torch.empty(rows, k // 16, dtype=torch.uint8, device=x.device)
+    if x_global is None:
+        x_global = torch.empty(rows, dtype=torch.float32, device=x.device)
+    _check(lib().nvfp4_quantize_rows(_ptr(x), _ld(x), rows, k, _ptr(xq), _ptr(x_block_scale), _ptr(x_global),
+                                     _stream(stream, x.device)), "nvfp4_quantize_rows")
+    return xq, x_block_scale, x_global
+
+
+def _w4a4_weight(w_packed, w_block_scale):
+    _cuda(w_packed, torch.uint8, "w_packed", 2)
+    _cuda(w_block_scale, torch.uint8, "w_block_scale", 2)
+    n, k2 = w_packed.shape
+    k = 2 * k2
+    if tuple(w_block_scale.shape) != (n, k // 16):
+        raise ValueError("w_block_scale must be [n, k/16]")
+    return n, k
+
+
+def w4a4_gemv(w_packed, w_block_scale, global_scale, xq, x_block_scale, x_global, out=None, stream=None):
+    n, k = _w4a4_weight(w_packed, w_block_scale)
+    _cuda(xq, torch.uint8, "xq", 2)
+    rows = xq.shape[0]
+    if tuple(xq.shape) != (rows, k // 2) or tuple(x_block_scale.shape) != (rows, k // 16) or \
+            tuple(x_global.shape) != (rows,) or not xq.is_contiguous() or not x_block_scale.is_contiguous():
+        raise ValueError("xq [rows, k/2], x_block_scale [rows, k/16] (contiguous), x_global [rows]")
+    if out is None:
+        out = torch.empty(rows, n, dtype=torch.bfloat16, device=xq.device)
+    _check(lib().w4a4_gemv(_ptr(w_packed), _ptr(w_block_scale), float(global_scale), n, k, _ptr(xq),
+                           _ptr(x_block_scale), _ptr(x_global), rows, _ptr(out), _ld(out),
+                           _stream(stream, xq.device)), "w4a4_gemv")
+    return out
+
+
+def w4a4_proj(w_packed, w_block_scale, global_scale, x, out=None, xq_scratch=None, xs_scratch=None,
+              xg_scratch=None, stream=None):
+    n, k = _w4a4_weight(w_packed, w_block_scale)
+    _cuda(x, torch.bfloat16, "x", 2)
+    rows = x.shape[0]
+    r = max(1, min(rows, W4A4_MAX_ROWS))
+    if out is None:
+        out = torch.empty(rows, n, dtype=torch.bfloat16, device=x.device)
+    if xq_scratch is None:
+        xq_scratch = torch.empty(r * k // 2, dtype=torch.uint8, device=x.device)
+    if xs_scratch is None:
+        xs_scratch = torch.empty(r * k // 16, dtype=torch.uint8, device=x.device)
+    if xg_scratch is None:
+        xg_scratch = torch.empty(r, dtype=torch.float32, device=x.device)
+    _check(lib().w4a4_proj(_ptr(w_packed), _ptr(w_block_scale), float(global_scale), n, k, _ptr(x), _ld(x), rows,
+                           _ptr(out), _ld(out), _ptr(xq_scratch), _ptr(xs_scratch), _ptr(xg_scratch),
+                           _stream(stream, x.device)), "w4a4_proj")
     return out
 
 

@@ -249,6 +249,106 @@ __global__ void __launch_bounds__(kQT) w8a16_split_cluster_kernel(const uint16_t
   cluster_sync();
 }
 
+// Four pairs of values -> eight packed E2M1 codes (element 2i in the low nibble of byte i),
+// round-to-nearest-even with saturation to +-6 (cvt.rn.satfinite.e2m1x2: first source in the
+// high nibble).
+__device__ __forceinline__ uint32_t f32x8_to_e2m1x8(const float (&v)[8]) {
+  uint32_t r;
+  asm("{ .reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3}; }"
+      : "=r"(r)
+      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+  return r;
+}
+
+// NVFP4 quantize of row blockIdx.y (the W4A4 activations), each decision in f32:
+//   g = amax / 2688;  per 16-value block b:  s_b = e4m3_rn_sat(bmax / (6 g)),
+//   S_b = e4m3(s_b) * g,  codes = e2m1_rn_sat(x / S_b)  (all zero where S_b == 0).
+// One thread per block of 16 values (two 16-byte loads), a cluster of kQC CTAs per row.
+__global__ void __launch_bounds__(kQT) nvfp4_quant_cluster_kernel(const uint16_t* __restrict__ x, int64_t ldx,
+                                                                  int k, uint8_t* __restrict__ xq,
+                                                                  uint8_t* __restrict__ xbs, float* __restrict__ xg) {
+  __shared__ float red[kQT / 32];
+  __shared__ float cta_max;
+  grid_dependents_launch();
+  const int m = blockIdx.y;
+  const uint16_t* xr = x + (int64_t)m * ldx;
+  int b0, b1;
+  cta_range(k / 16, b0, b1);
+  constexpr int kCache = 2;  // blocks a thread keeps in registers
+  uint32_t h[kCache][8];
+  auto load_block = [&](int b, uint32_t (&v)[8]) {
+    const uint4 lo = ldg_nc(xr + 16 * b), hi = ldg_nc(xr + 16 * b + 8);
+    v[0] = lo.x, v[1] = lo.y, v[2] = lo.z, v[3] = lo.w, v[4] = hi.x, v[5] = hi.y, v[6] = hi.z, v[7] = hi.w;
+  };
+  auto block_max = [&](const uint32_t (&v)[8]) {
+    float a = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      a = fmaxf(a, fabsf(bf16_bits_to_f32(v[i] & 0xffffu)));
+      a = fmaxf(a, fabsf(bf16_bits_to_f32(v[i] >> 16)));
+    }
+    return a;
+  };
+  float amax = 0.f;
+#pragma unroll
+  for (int c = 0; c < kCache; ++c) {
+    const int b = b0 + threadIdx.x + c * kQT;
+    if (b < b1) {
+      load_block(b, h[c]);
+      amax = fmaxf(amax, block_max(h[c]));
+    }
+  }
+  for (int b = b0 + threadIdx.x + kCache * kQT; b < b1; b += kQT) {
+    uint32_t t[8];
+    load_block(b, t);
+    amax = fmaxf(amax, block_max(t));
+  }
+  amax = cluster_row_max(amax, red, &cta_max);
+  const float g = __fdiv_rn(amax, 2688.0f);
+  const float d6 = __fmul_rn(6.0f, g);
+  if (cluster_rank() == 0 && threadIdx.x == 0) xg[m] = g;
+  uint8_t* qrow = xq + (int64_t)m * (k / 2);
+  uint8_t* srow = xbs + (int64_t)m * (k / 16);
+  auto emit = [&](int b, const uint32_t (&v)[8]) {
+    const float bmax = block_max(v);
+    const float sf = d6 > 0.f ? __fdiv_rn(bmax, d6) : 0.f;
+    const uint32_t scode = f32x2_to_e4m3x2(sf, 0.f) & 0xffu;
+    const float S = __fmul_rn(f16_bits_to_f32(e4m3x2_to_f16x2((uint16_t)scode) & 0xffffu), g);
+    uint32_t w[2] = {0u, 0u};
+    if (S > 0.f) {
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        float q[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t pair = v[4 * half + i];
+          q[2 * i] = __fdiv_rn(bf16_bits_to_f32(pair & 0xffffu), S);
+          q[2 * i + 1] = __fdiv_rn(bf16_bits_to_f32(pair >> 16), S);
+        }
+        w[half] = f32x8_to_e2m1x8(q);
+      }
+    }
+    *reinterpret_cast<uint2*>(qrow + 8 * b) = make_uint2(w[0], w[1]);
+    srow[b] = (uint8_t)scode;
+  };
+#pragma unroll
+  for (int c = 0; c < kCache; ++c) {
+    const int b = b0 + threadIdx.x + c * kQT;
+    if (b < b1) emit(b, h[c]);
+  }
+  for (int b = b0 + threadIdx.x + kCache * kQT; b < b1; b += kQT) {
+    uint32_t t[8];
+    load_block(b, t);
+    emit(b, t);
+  }
+  cluster_sync();
+}
+
 template <typename... KArgs, typename... Args>
 int launch_cluster(void (*kernel)(KArgs...), int rows, cudaStream_t s, Args&&... args) {
   cudaLaunchConfig_t cfg{};
@@ -283,6 +383,12 @@ int w8a8_silu_quantize_launch(const uint16_t* gate, const uint16_t* up, int64_t 
                               int64_t ldq, float* sx, cudaStream_t s) {
   if (rows <= 0) return DLMH_OK;
   return launch_cluster(w8a8_quant_cluster_kernel<Src::Silu>, rows, s, gate, up, ld, k, xq, ldq, sx);
+}
+
+int nvfp4_quantize_launch(const uint16_t* x, int64_t ldx, int rows, int k, uint8_t* xq, uint8_t* xbs, float* xg,
+                          cudaStream_t s) {
+  if (rows <= 0) return DLMH_OK;
+  return launch_cluster(nvfp4_quant_cluster_kernel, rows, s, x, ldx, k, xq, xbs, xg);
 }
 
 int w8a16_split_launch(const uint16_t* x, int64_t ldx, int rows, int k, int half, uint8_t* codes, float* x_mul,

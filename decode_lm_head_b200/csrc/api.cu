@@ -56,6 +56,7 @@ int pass_rows(int op, int k) {
     case DLMH_OP_W8A8:
       return dlmh::w8a8_umma_supported(k) ? DLMH_W8A8_MAX_ROWS : dlmh::max_tier_rows(DLMH_OP_W8A8, k);
     case DLMH_OP_W4A16: return dlmh::max_tier_rows(DLMH_OP_W4A16, k);
+    case DLMH_OP_W4A4: return k % 256 == 0 ? dlmh::max_tier_rows(DLMH_OP_W4A4, k) : 0;
     case DLMH_OP_Q6K: return DLMH_Q6K_MAX_ROWS;
     default: return 0;
   }
@@ -94,7 +95,7 @@ const char* dlmh_error_string(int code) {
 }
 
 int dlmh_plan_chunks(int op, int rows, int k, int* offsets, int* counts, int* tiers, int cap) {
-  if (op < DLMH_OP_W8A16 || op > DLMH_OP_Q6K) return DLMH_ERR_SHAPE;
+  if (op < DLMH_OP_W8A16 || op > DLMH_OP_W4A4) return DLMH_ERR_SHAPE;
   if (k <= 0) return DLMH_ERR_SHAPE;
   DLMH_TRY(check_rows(rows, op_row_cap(op)));
   const int width = pass_rows(op, k);
@@ -294,6 +295,70 @@ int w4a16_gemv(const uint8_t* w_packed, const uint8_t* w_block_scale, float glob
     const int m = rows - done < width ? rows - done : width;
     DLMH_TRY(dlmh::w4a16_pass(w_packed, w_block_scale, global_scale, n, k, x + (int64_t)done * ldx, ldx, m,
                               out + (int64_t)done * ldc, ldc, as_stream(stream)));
+    done += m;
+  }
+  return DLMH_OK;
+}
+
+int nvfp4_quantize_rows(const dlmh_bf16* x, int64_t ldx, int rows, int k, uint8_t* xq, uint8_t* x_block_scale,
+                        float* x_global, void* stream) {
+  DLMH_TRY(check_rows(rows, 0));
+  if (k <= 0 || k > kMaxK || k % 16) return DLMH_ERR_SHAPE;
+  if (rows == 0) return DLMH_OK;
+  DLMH_TRY(check_bf16_in(x, ldx, k));
+  if (!xq || !x_block_scale || !x_global) return DLMH_ERR_NULL;
+  if (!aligned16(xq) || (reinterpret_cast<uintptr_t>(x_global) & 3u)) return DLMH_ERR_ALIGN;
+  return dlmh::nvfp4_quantize_launch(x, ldx, rows, k, xq, x_block_scale, x_global, as_stream(stream));
+}
+
+static int check_w4a4(const uint8_t* w_packed, const uint8_t* w_block_scale, int n, int k, int rows, dlmh_bf16* out,
+                      int64_t ldc) {
+  DLMH_TRY(check_rows(rows, 0));
+  DLMH_TRY(check_nk(n, k, 256));
+  if (!w_packed || !w_block_scale) return DLMH_ERR_NULL;
+  if (!aligned16(w_packed) || !aligned16(w_block_scale)) return DLMH_ERR_ALIGN;
+  return check_out(out, ldc, n);
+}
+
+int w4a4_gemv(const uint8_t* w_packed, const uint8_t* w_block_scale, float global_scale, int n, int k,
+              const uint8_t* xq, const uint8_t* x_block_scale, const float* x_global, int rows, dlmh_bf16* out,
+              int64_t ldc, void* stream) {
+  if (rows == 0 && check_rows(rows, 0) == DLMH_OK && check_nk(n, k, 256) == DLMH_OK) return DLMH_OK;
+  DLMH_TRY(check_w4a4(w_packed, w_block_scale, n, k, rows, out, ldc));
+  if (!xq || !x_block_scale || !x_global) return DLMH_ERR_NULL;
+  if (!aligned16(xq) || (reinterpret_cast<uintptr_t>(x_block_scale) & 1u) ||
+      (reinterpret_cast<uintptr_t>(x_global) & 3u))
+    return DLMH_ERR_ALIGN;
+  const int width = pass_rows(DLMH_OP_W4A4, k);
+  if (width <= 0) return DLMH_ERR_UNSUPPORTED;
+  for (int done = 0; done < rows;) {
+    const int m = rows - done < width ? rows - done : width;
+    DLMH_TRY(dlmh::w4a4_pass(w_packed, w_block_scale, global_scale, n, k, xq + (int64_t)done * (k / 2),
+                             x_block_scale + (int64_t)done * (k / 16), x_global + done, m, out + (int64_t)done * ldc,
+                             ldc, as_stream(stream)));
+    done += m;
+  }
+  return DLMH_OK;
+}
+
+int w4a4_proj(const uint8_t* w_packed, const uint8_t* w_block_scale, float global_scale, int n, int k,
+              const dlmh_bf16* x, int64_t ldx, int rows, dlmh_bf16* out, int64_t ldc, uint8_t* xq_scratch,
+              uint8_t* xs_scratch, float* xg_scratch, void* stream) {
+  if (rows == 0 && check_rows(rows, 0) == DLMH_OK && check_nk(n, k, 256) == DLMH_OK) return DLMH_OK;
+  DLMH_TRY(check_w4a4(w_packed, w_block_scale, n, k, rows, out, ldc));
+  DLMH_TRY(check_bf16_in(x, ldx, k));
+  if (!xq_scratch || !xs_scratch || !xg_scratch) return DLMH_ERR_NULL;
+  if (!aligned16(xq_scratch) || (reinterpret_cast<uintptr_t>(xs_scratch) & 1u) ||
+      (reinterpret_cast<uintptr_t>(xg_scratch) & 3u))
+    return DLMH_ERR_ALIGN;
+  const int width = pass_rows(DLMH_OP_W4A4, k);
+  if (width <= 0) return DLMH_ERR_UNSUPPORTED;
+  cudaStream_t s = as_stream(stream);
+  for (int done = 0; done < rows;) {
+    const int m = rows - done < width ? rows - done : width;
+    DLMH_TRY(dlmh::nvfp4_quantize_launch(x + (int64_t)done * ldx, ldx, m, k, xq_scratch, xs_scratch, xg_scratch, s));
+    DLMH_TRY(dlmh::w4a4_pass(w_packed, w_block_scale, global_scale, n, k, xq_scratch, xs_scratch, xg_scratch, m,
+                             out + (int64_t)done * ldc, ldc, s));
     done += m;
   }
   return DLMH_OK;

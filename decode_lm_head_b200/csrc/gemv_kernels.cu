@@ -87,7 +87,8 @@ int launch_rowtile(const RowTileParams& p, cudaStream_t stream) {
 // 512-thread CTA without spills (checked with -Xptxas -v).
 template <class F, int NT>
 constexpr int stream_max_nkb() {
-  if constexpr (F::kBlockScale) return NT == 1 ? 5 : (NT == 2 ? 2 : 0);
+  if constexpr (F::kXBytes == 0) return NT == 1 ? 7 : (NT == 2 ? 3 : 2);  // W4A4: 5 words per (k-block, n-tile)
+  else if constexpr (F::kBlockScale) return NT == 1 ? 5 : (NT == 2 ? 2 : 0);
   else if constexpr (F::kXBytes == 1) return NT <= 2 ? 8 : 3;
   else return NT == 1 ? 7 : (NT == 2 ? 5 : 2);
 }
@@ -187,6 +188,19 @@ int launch_tier(int nt, const RowTileParams& p, cudaStream_t s) {
   }
 }
 
+// The streamed kernel alone (W4A4 has no register-tile fallback).
+template <class F>
+int launch_tier_stream(int nt, const RowTileParams& p, cudaStream_t s) {
+  if (!stream_fits<F>(nt, p.k)) return DLMH_ERR_UNSUPPORTED;
+  const int nkb = stream_nkb<F>(p.k);
+  switch (nt) {
+    case 1: return launch_stream<F, 1>(nkb, p, s);
+    case 2: return launch_stream<F, 2>(nkb, p, s);
+    case 4: return launch_stream<F, 4>(nkb, p, s);
+    default: return DLMH_ERR_UNSUPPORTED;
+  }
+}
+
 template <class F>
 bool tier_fits(int nt, int k) {
   if (stream_fits<F>(nt, k)) return true;
@@ -255,6 +269,25 @@ int w4a16_pass(const uint8_t* wp, const uint8_t* wbs, float g, int n, int k, con
   return launch_tier<FmtW4A16>(tier_ntiles(rows), p, s);
 }
 
+int w4a4_pass(const uint8_t* wp, const uint8_t* wbs, float g, int n, int k, const uint8_t* xq,
+              const uint8_t* xbs, const float* xg, int rows, uint16_t* out, int64_t ldc, cudaStream_t s) {
+  RowTileParams p{};
+  p.w = wp;
+  p.w_row_bytes = k / 2;
+  p.w_bscale = wbs;
+  p.gscale = g;
+  p.n = n;
+  p.k = k;
+  p.x = xq;
+  p.ldx = k;  // codes row stride: k/2 bytes
+  p.x_bscale = xbs;
+  p.x_scale = xg;
+  p.rows = rows;
+  p.out = out;
+  p.ldc = ldc;
+  return launch_tier_stream<FmtW4A4>(tier_ntiles(rows), p, s);
+}
+
 int device_fault(int reset) {
   int v = 0;
   if (cudaMemcpyFromSymbol(&v, dlmh_fault_word, sizeof(int)) != cudaSuccess) return DLMH_ERR_CUDA;
@@ -280,6 +313,7 @@ int max_tier_rows(int op, int k) {
     case DLMH_OP_W8A16: return widest([&](int nt) { return tier_fits<FmtW8A16>(nt, k); });
     case DLMH_OP_W8A8: return widest([&](int nt) { return tier_fits<FmtW8A8>(nt, k); });
     case DLMH_OP_W4A16: return widest([&](int nt) { return tier_fits<FmtW4A16>(nt, k); });
+    case DLMH_OP_W4A4: return widest([&](int nt) { return stream_fits<FmtW4A4>(nt, k); });
     default: return 0;
   }
 }

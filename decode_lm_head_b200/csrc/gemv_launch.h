@@ -12,6 +12,14 @@ namespace dlmh {
 int max_tier_rows(int op, int k);
 // Fault bits recorded by bounded device waits since the last reset (0 in a healthy run);
 // reads synchronously.
+// NVFP4 W4A4 pass (streamed kernel, k % 256 == 0): NVFP4 weights against NVFP4 activation rows
+// xq [rows][k/2], xbs [rows][k/16], xg [rows] as written by nvfp4_quantize_launch.
+int w4a4_pass(const uint8_t* wp, const uint8_t* wbs, float g, int n, int k, const uint8_t* xq,
+              const uint8_t* xbs, const float* xg, int rows, uint16_t* out, int64_t ldc, cudaStream_t s);
+// Per-row NVFP4 quantize of BF16 rows (one 8-CTA cluster per row): codes [rows][k/2] (row
+// stride k/2), block scales [rows][k/16], globals [rows].  k % 16 == 0.
+int nvfp4_quantize_launch(const uint16_t* x, int64_t ldx, int rows, int k, uint8_t* xq, uint8_t* xbs, float* xg,
+                          cudaStream_t s);
 int device_fault(int reset);
 // Width (8, 16 or 32) of the narrowest compiled tier that covers `rows` (1..32).
 inline int tier_width(int rows) { return rows <= 8 ? 8 : (rows <= 16 ? 16 : 32); }

@@ -39,7 +39,8 @@ struct RowTileParams {
   int n, k;                // output rows, reduction length (elements)
   const void* x;           // activations (bf16 for A16, e4m3 codes for W8A8)
   int64_t ldx;             // elements
-  const float* x_scale;    // W8A8: per-row activation scale
+  const float* x_scale;    // W8A8: per-row activation scale; W4A4: per-row NVFP4 global
+  const uint8_t* x_bscale; // W4A4: per-16 E4M3 activation block scales [rows, k/16]
   int rows;                // activation rows in this pass (<= 8*NT)
   uint16_t* out;           // bf16 out [rows, ldc]
   int64_t ldc;
@@ -63,6 +64,16 @@ struct FmtW4A16 {
   static constexpr int kElemsPerKB = 128;  // two values per byte
   static constexpr int kXBytes = 2;
   static constexpr int kXChunks = 4;
+  static constexpr bool kBlockScale = true;
+};
+
+// NVFP4 weight x NVFP4 activations (W4A4): both operands E2M1 x E4M3 block scale -> f16
+// (exact: at most 6 significant bits, range 2^-10 .. 2688), f16 MMA; the activation codes stay
+// packed in registers (kXBytes == 0) and are decoded per MMA step.  Streamed kernel only.
+struct FmtW4A4 {
+  static constexpr int kElemsPerKB = 128;
+  static constexpr int kXBytes = 0;
+  static constexpr int kXChunks = 1;
   static constexpr bool kBlockScale = true;
 };
 

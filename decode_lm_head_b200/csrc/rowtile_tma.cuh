@@ -46,7 +46,9 @@ struct StageLayout {
 // 32-bit words of the activation fragment per lane, k-block and n-tile.
 template <class F>
 constexpr int x_words() {
-  return F::kXBytes == 1 ? 4 : (F::kElemsPerKB / 4) / 2;
+  // W8A8: 16 codes; W4A4: 32 packed FP4 codes (4 words) + the two block scales as f16x2;
+  // A16: 32 f16 values
+  return F::kXBytes == 1 ? 4 : (F::kXBytes == 0 ? 5 : (F::kElemsPerKB / 4) / 2);
 }
 
 template <class F, int NT, int C, int NS>
@@ -142,6 +144,39 @@ __device__ __forceinline__ void kb_w4a16_reg(float (&acc)[NT][4], const uint4& r
     const uint32_t a3 = hmul2(e2m1x2_to_f16x2((word_b >> (sh + 8)) & 0xff), ssb);
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) mma_f16_16816(acc[nt], a0, a1, a2, a3, xr[nt][2 * j], xr[nt][2 * j + 1]);
+  }
+}
+
+// W4A4: the activation side decoded like the weight side -- MMA step j takes bytes 2j, 2j+1
+// of the lane's 16 code bytes (values 4j..4j+3 of its 32), times the block scale of values
+// 0..15 (j < 4) or 16..31; every product of two such f16 values is exact in the f32 sum.
+template <int NT, int XW>
+__device__ __forceinline__ void kb_w4a4_reg(float (&acc)[NT][4], const uint4& ra, const uint4& rb, uint32_t s2a,
+                                            uint32_t s2b, const uint32_t (&xr)[NT][XW]) {
+  const uint32_t wa[4] = {ra.x, ra.y, ra.z, ra.w};
+  const uint32_t wb[4] = {rb.x, rb.y, rb.z, rb.w};
+  const uint32_t sa = e4m3x2_to_f16x2((uint16_t)s2a);
+  const uint32_t sb = e4m3x2_to_f16x2((uint16_t)s2b);
+  const uint32_t sa0 = __byte_perm(sa, 0, 0x1010), sa1 = __byte_perm(sa, 0, 0x3232);
+  const uint32_t sb0 = __byte_perm(sb, 0, 0x1010), sb1 = __byte_perm(sb, 0, 0x3232);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint32_t word_a = wa[j >> 1], word_b = wb[j >> 1];
+    const int sh = (j & 1) * 16;
+    const uint32_t ssa = (j < 4) ? sa0 : sa1;
+    const uint32_t ssb = (j < 4) ? sb0 : sb1;
+    const uint32_t a0 = hmul2(e2m1x2_to_f16x2((word_a >> sh) & 0xff), ssa);
+    const uint32_t a2 = hmul2(e2m1x2_to_f16x2((word_a >> (sh + 8)) & 0xff), ssa);
+    const uint32_t a1 = hmul2(e2m1x2_to_f16x2((word_b >> sh) & 0xff), ssb);
+    const uint32_t a3 = hmul2(e2m1x2_to_f16x2((word_b >> (sh + 8)) & 0xff), ssb);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const uint32_t cw = xr[nt][j >> 1];
+      const uint32_t sx = (j < 4) ? __byte_perm(xr[nt][4], 0, 0x1010) : __byte_perm(xr[nt][4], 0, 0x3232);
+      const uint32_t b0 = hmul2(e2m1x2_to_f16x2((cw >> sh) & 0xff), sx);
+      const uint32_t b1 = hmul2(e2m1x2_to_f16x2((cw >> (sh + 8)) & 0xff), sx);
+      mma_f16_16816(acc[nt], a0, a1, a2, a3, b0, b1);
+    }
   }
 }
 
@@ -285,6 +320,30 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemv_kernel(const RowTileP
         }
       }
     }
+  } else if constexpr (F::kXBytes == 0) {
+    // W4A4: the lane's 32 values of each k-block as 16 packed code bytes + two block scales;
+    // the row's NVFP4 global goes to the epilogue
+    const uint8_t* xq = static_cast<const uint8_t*>(p.x);
+    if (threadIdx.x < MT) rowmul[threadIdx.x] = threadIdx.x < p.rows ? p.x_scale[threadIdx.x] : 0.f;
+#pragma unroll
+    for (int j = 0; j < NKB; ++j) {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const int m = nt * 8 + g;
+        const int k0 = (j * kWarps + warp) * F::kElemsPerKB + t * EL;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        uint32_t sc = 0;
+        if (m < p.rows && k0 < p.k) {
+          v = ldg_nc(xq + (int64_t)m * (p.ldx / 2) + k0 / 2);
+          sc = e4m3x2_to_f16x2((uint16_t)ldg_u16(p.x_bscale + (int64_t)m * (p.k / 16) + k0 / 16));
+        }
+        xr[j][nt][0] = v.x;
+        xr[j][nt][1] = v.y;
+        xr[j][nt][2] = v.z;
+        xr[j][nt][3] = v.w;
+        xr[j][nt][4] = sc;
+      }
+    }
   } else {
     const uint8_t* x = static_cast<const uint8_t*>(p.x);
     if (threadIdx.x < MT) rowmul[threadIdx.x] = threadIdx.x < p.rows ? p.x_scale[threadIdx.x] : 0.f;
@@ -351,7 +410,9 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemv_kernel(const RowTileP
                 sb = vb;
               }
             }
-            if constexpr (F::kBlockScale)
+            if constexpr (F::kXBytes == 0)
+              kb_w4a4_reg<NT, XW>(acc, ra, rb, sa, sb, xr[q]);
+            else if constexpr (F::kBlockScale)
               kb_w4a16_reg<NT, XW>(acc, ra, rb, sa, sb, xr[q]);
             else if constexpr (F::kXBytes == 1)
               kb_w8a8_reg<NT, XW>(acc, ra, rb, xr[q]);

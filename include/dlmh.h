@@ -86,6 +86,8 @@ typedef enum dlmh_status {
 /* Largest row count of one NVFP4 W4A16 call (w4a16_gemv_tiers.rs, kernel_within:
  * more than 32 rows is refused). */
 #define DLMH_W4A16_MAX_ROWS 32
+/* Widest W4A4 pass (w4a4_proj::W4A4_MAX_M in w4a16_gemv_tiers.rs). */
+#define DLMH_W4A4_MAX_ROWS 32
 /* Rows of the pages' Q6_K launch (MAX_M / KQ_MAX_M in lm_head_q6k.rs): the narrowest tier. */
 #define DLMH_Q6K_CHUNK_ROWS 8
 /* Rows per Q6_K weight pass here (tiers 8 / 16 / 32 / 64; the pages run 8-row launches). */
@@ -233,6 +235,45 @@ DLMH_API int w4a16_gemv(const uint8_t* w_packed, const uint8_t* w_block_scale, f
                const dlmh_bf16* x, int64_t ldx, int rows, dlmh_bf16* out, int64_t ldc, void* stream);
 
 /* ---------------------------------------------------------------------------------------
+ * NVFP4 W4A4: FP4 activations for the wider row edge (w4a16_gemv_tiers.rs,
+ * W4a16BatchmTiers: a weight that declares FP4 activations runs its narrow projections
+ * W4A4, up to W4A4_MAX_M = 32 rows; NVFP4 layout of fp8_lut.rs).
+ *
+ * nvfp4_quantize_rows: per row m, every decision in float32 (the pages do not print the
+ * activation quantize; this is the plain NVFP4 recipe):
+ *   g[m] = amax_k |x[m, k]| / 2688                       (IEEE division; 2688 = 6 * 448)
+ *   per 16-value block b:  s[m, b] = e4m3_rn_sat( amax_b / (6 g[m]) )   (6 g: one f32 product)
+ *                          S = e4m3(s[m, b]) * g[m]      (one f32 product)
+ *                          code = e2m1_rn_sat( x / S )   (IEEE division; ties to even,
+ *                          magnitudes above 6 give 6, a negative zero keeps its sign);
+ *                          all codes 0 where S == 0.
+ *   x      [rows, ldx] BF16, 16-byte aligned, ldx % 8 == 0.  k % 16 == 0.
+ *   xq     [rows][k/2] packed codes (row stride k/2, element 2i in the low nibble of byte i),
+ *          16-byte aligned.  x_block_scale [rows][k/16] E4M3.  x_global [rows] float32.
+ *
+ * w4a4_gemv: out[m, n] = bf16( g_w * g[m] * sum_b e4m3(S[n, b]) e4m3(s[m, b])
+ *                                           * sum_{k in b} e2m1(W[n, k]) e2m1(X[m, k]) )
+ *   Both operands are decoded exactly to f16 (E2M1 x E4M3 has at most 6 significant bits)
+ *   and multiplied on the tensor cores with f32 accumulation; one BF16 rounding.
+ *   w_packed [n, k/2] and w_block_scale [n, k/16] as for w4a16_gemv (16-byte aligned);
+ *   xq / x_block_scale / x_global as written by nvfp4_quantize_rows (x_block_scale 2-byte
+ *   aligned).  k % 256 == 0.  Any rows: weight passes of up to DLMH_W4A4_MAX_ROWS (fewer when
+ *   k is long: dlmh_plan_chunks(DLMH_OP_W4A4, ...)); DLMH_ERR_UNSUPPORTED when no pass fits k.
+ *
+ * w4a4_proj: per pass, nvfp4_quantize_rows into the scratch, then w4a4_gemv.  xq_scratch
+ *   holds min(rows, 32) * k/2 bytes (16-byte aligned), xs_scratch min(rows, 32) * k/16,
+ *   xg_scratch min(rows, 32) floats.
+ * ------------------------------------------------------------------------------------- */
+DLMH_API int nvfp4_quantize_rows(const dlmh_bf16* x, int64_t ldx, int rows, int k, uint8_t* xq,
+                                 uint8_t* x_block_scale, float* x_global, void* stream);
+DLMH_API int w4a4_gemv(const uint8_t* w_packed, const uint8_t* w_block_scale, float global_scale, int n, int k,
+                       const uint8_t* xq, const uint8_t* x_block_scale, const float* x_global, int rows,
+                       dlmh_bf16* out, int64_t ldc, void* stream);
+DLMH_API int w4a4_proj(const uint8_t* w_packed, const uint8_t* w_block_scale, float global_scale, int n, int k,
+                       const dlmh_bf16* x, int64_t ldx, int rows, dlmh_bf16* out, int64_t ldc, uint8_t* xq_scratch,
+                       uint8_t* xs_scratch, float* xg_scratch, void* stream);
+
+/* ---------------------------------------------------------------------------------------
  * block_q8_1 row quantize (lm_head_q6k.rs, lm_head_q6k_run: kquant_q8_1_rows_bf16)
  *   Block layout (36 bytes per 32 values): { f16 d; f16 s; int8 qs[32] }.
  *   d = amax / 127 (f32 division), qs = round-half-away( x / d ) (f32 division; 0 when
@@ -299,7 +340,8 @@ typedef enum dlmh_op {
   DLMH_OP_W8A16 = 0, /* lm_head_fp8_w8a16 */
   DLMH_OP_W8A8 = 1,  /* w8a8_proj / w8a8_silu_proj */
   DLMH_OP_W4A16 = 2, /* w4a16_gemv */
-  DLMH_OP_Q6K = 3    /* q6k_mmvq / q6k_lm_head */
+  DLMH_OP_Q6K = 3,   /* q6k_mmvq / q6k_lm_head */
+  DLMH_OP_W4A4 = 4   /* w4a4_gemv / w4a4_proj */
 } dlmh_op;
 
 /* The weight passes an entry point runs for `rows` at reduction length k: pass i covers rows

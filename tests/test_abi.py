@@ -35,7 +35,8 @@ def test_error_strings_and_version():
 
 @pytest.mark.parametrize("opid,k,width", [(dl.OP_W8A16, 5120, 128), (dl.OP_W8A16, 1040, 16), (dl.OP_W8A8, 5120, 128),
                                            (dl.OP_W8A8, 14336, 128), (dl.OP_W8A8, 1040, 32), (dl.OP_W4A16, 4096, 16),
-                                           (dl.OP_Q6K, 7168, 64)])
+                                           (dl.OP_Q6K, 7168, 64),
+                                           (dl.OP_W4A4, 4096, 32), (dl.OP_W4A4, 14336, 8), (dl.OP_W4A4, 6144, 16)])
 def test_plan_matches_oracle_rules(opid, k, width):
     cap = 32 if opid == dl.OP_W4A16 else 300
     for rows in range(0, cap + 1):
@@ -44,6 +45,8 @@ def test_plan_matches_oracle_rules(opid, k, width):
         assert [(o, c) for o, c, _ in plan] == ref
         if opid == dl.OP_Q6K:
             widths = [8, 16, 32, 64]
+        elif opid == dl.OP_W4A4:
+            widths = [8, 16, 32]
         elif opid in (dl.OP_W8A8, dl.OP_W8A16) and k % 128 == 0:
             widths = list(range(16, 129, 16))  # tensor-core tier: MMA N in steps of 16
         else:
@@ -123,6 +126,27 @@ def test_zero_rows_launch_nothing():
     # valid arguments with rows == 0 return OK without touching CUDA
     assert L.w8a8_quantize_rows(A, 64, 0, 64, A, 64, A, None) == 0
     assert L.q8_1_quantize_rows(A, 64, 0, 64, A, None) == 0
+
+
+def test_w4a4_argument_errors():
+    # nvfp4_quantize_rows(x, ldx, rows, k, xq, xs, xg, stream)
+    assert L.nvfp4_quantize_rows(A, 64, 1, 40, A, A, A, None) == -2          # k % 16
+    assert L.nvfp4_quantize_rows(A, 64, -1, 64, A, A, A, None) == -4
+    assert L.nvfp4_quantize_rows(A, 64, 1, 64, A, None, A, None) == -1
+    assert L.nvfp4_quantize_rows(A, 64, 1, 64, U, A, A, None) == -3          # codes 16-byte aligned
+    assert L.nvfp4_quantize_rows(A, 64, 0, 64, None, None, None, None) == 0
+    # w4a4_gemv(wp, ws, g, n, k, xq, xs, xg, rows, out, ldc, stream)
+    assert L.w4a4_gemv(A, A, 1.0, 16, 128, A, A, A, 1, A, 16, None) == -2    # k % 256
+    assert L.w4a4_gemv(None, A, 1.0, 16, 256, A, A, A, 1, A, 16, None) == -1
+    assert L.w4a4_gemv(A, U, 1.0, 16, 256, A, A, A, 1, A, 16, None) == -3
+    assert L.w4a4_gemv(A, A, 1.0, 16, 256, A, A + 1, A, 1, A, 16, None) == -3
+    assert L.w4a4_gemv(A, A, 1.0, 16, 256, A, A, A, 1, A, 8, None) == -5
+    assert L.w4a4_gemv(A, A, 1.0, 16, 256, None, None, None, 0, None, 16, None) == 0
+    assert L.w4a4_gemv(A, A, 1.0, 16, 1 << 18, A, A, A, 1, A, 16, None) == -7  # no pass fits this k
+    # w4a4_proj(wp, ws, g, n, k, x, ldx, rows, out, ldc, xq, xs, xg, stream)
+    assert L.w4a4_proj(A, A, 1.0, 16, 256, A, 256, 1, A, 16, None, A, A, None) == -1
+    assert L.w4a4_proj(A, A, 1.0, 16, 256, A, 256, 1, A, 16, U, A, A, None) == -3
+    assert L.w4a4_proj(A, A, 1.0, 16, 256, A, 128, 1, A, 16, A, A, A, None) == -5
 
 
 def test_dequant_argument_errors():

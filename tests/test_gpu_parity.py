@@ -410,6 +410,49 @@ def test_q6k_wide_tiers_one_pass(n, k):
 
 
 # ---------------------------------------------------------------------------
+# NVFP4 W4A4 (FP4 activations)
+# ---------------------------------------------------------------------------
+
+
+def _w4a4_rows(m, k, seed):
+    # N(0,1) rows at a spread of magnitudes, a zero row, -0 values and tiny values
+    x = synth.bf16_rows(m, k, seed, DEV) * torch.logspace(-3, 2, m, device=DEV).to(torch.bfloat16)[:, None]
+    if m > 2:
+        x[1] = 0
+        x[2, ::7] = -0.0
+        x[2, 1::7] = 1e-30
+    return x
+
+
+@pytest.mark.parametrize("m,k", [(40, 4096), (5, 1040), (130, 256)])
+def test_nvfp4_quantize_rows_bit_exact(m, k):
+    x = _w4a4_rows(m, k, 14)
+    q, s, g = dl.nvfp4_quantize_rows(x)
+    q_ref, s_ref, g_ref = og.nvfp4_quantize_rows(bits(x))
+    assert np.array_equal(bits(g), g_ref)
+    assert np.array_equal(bits(s), s_ref)
+    assert np.array_equal(bits(q), q_ref)
+
+
+@pytest.mark.parametrize("n,k", [(14336, 4096), (300, 1024), (77, 512), (130, 14336)])
+def test_w4a4_gemv_and_proj(n, k):
+    wp, ws, gw = synth.nvfp4_weight(n, k, 15, DEV)
+    x = _w4a4_rows(70, k, 15)
+    full = bits(dl.w4a4_proj(wp, ws, gw, x))                     # passes of up to 32 rows
+    sub = slice(None) if n <= 1000 else slice(0, n, 9)
+    q_ref, s_ref, g_ref = og.nvfp4_quantize_rows(bits(x))
+    ref = og.w4a4_gemv(bits(wp)[sub], bits(ws)[sub], float(gw), q_ref, s_ref, g_ref)
+    assert_bf16_close(full[:, sub], ref, f"w4a4 n={n} k={k} M=70")
+    for m in (1, 7, 8, 9, 16, 17, 32, 33):
+        part = bits(dl.w4a4_proj(wp, ws, gw, x[:m]))
+        assert np.array_equal(part, full[:m]), f"row invariance M={m}"
+    q, sc, g = dl.nvfp4_quantize_rows(x)
+    direct = bits(dl.w4a4_gemv(wp, ws, gw, q, sc, g))
+    assert np.array_equal(direct, full)
+    assert dl.device_fault(reset=True) == 0
+
+
+# ---------------------------------------------------------------------------
 # full-size heads, sampled outputs
 # ---------------------------------------------------------------------------
 
