@@ -358,7 +358,7 @@ int w4a4_proj(const uint8_t* w_packed, const uint8_t* w_block_scale, float globa
     const int m = rows - done < width ? rows - done : width;
     DLMH_TRY(dlmh::nvfp4_quantize_launch(x + (int64_t)done * ldx, ldx, m, k, xq_scratch, xs_scratch, xg_scratch, s));
     DLMH_TRY(dlmh::w4a4_pass(w_packed, w_block_scale, global_scale, n, k, xq_scratch, xs_scratch, xg_scratch, m,
-                             out + (int64_t)done * ldc, ldc, s));
+                             out + (int64_t)done * ldc, ldc, s, true));
     done += m;
   }
   return DLMH_OK;

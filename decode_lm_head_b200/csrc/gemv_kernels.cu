@@ -4,6 +4,7 @@
 #include "gemv_launch.h"
 #include "rowtile_gemv.cuh"
 #include "rowtile_tma.cuh"
+#include "umma_common.cuh"
 
 namespace dlmh {
 
@@ -127,8 +128,7 @@ int launch_stream_nkb(const RowTileParams& p, cudaStream_t stream) {
   if (ensure_dynamic_smem(reinterpret_cast<const void*>(kern), (int)smem) != DLMH_OK) return DLMH_ERR_CUDA;
   const int ntiles = (p.n + kTileRows - 1) / kTileRows;
   const int grid = ntiles < di.sms ? ntiles : di.sms;
-  kern<<<grid, kThreads, smem, stream>>>(p);
-  return launch_status();
+  return umma::launch_pdl(kern, dim3(grid), dim3(kThreads), smem, stream, p);
 }
 
 template <class F, int NT>
@@ -270,7 +270,8 @@ int w4a16_pass(const uint8_t* wp, const uint8_t* wbs, float g, int n, int k, con
 }
 
 int w4a4_pass(const uint8_t* wp, const uint8_t* wbs, float g, int n, int k, const uint8_t* xq,
-              const uint8_t* xbs, const float* xg, int rows, uint16_t* out, int64_t ldc, cudaStream_t s) {
+              const uint8_t* xbs, const float* xg, int rows, uint16_t* out, int64_t ldc, cudaStream_t s,
+              bool after_prepass) {
   RowTileParams p{};
   p.w = wp;
   p.w_row_bytes = k / 2;
@@ -285,6 +286,7 @@ int w4a4_pass(const uint8_t* wp, const uint8_t* wbs, float g, int n, int k, cons
   p.rows = rows;
   p.out = out;
   p.ldc = ldc;
+  p.early_w = after_prepass ? 1 : 0;
   return launch_tier_stream<FmtW4A4>(tier_ntiles(rows), p, s);
 }
 

@@ -14,8 +14,10 @@ int max_tier_rows(int op, int k);
 // reads synchronously.
 // NVFP4 W4A4 pass (streamed kernel, k % 256 == 0): NVFP4 weights against NVFP4 activation rows
 // xq [rows][k/2], xbs [rows][k/16], xg [rows] as written by nvfp4_quantize_launch.
+// after_prepass: the preceding kernel on `s` is nvfp4_quantize_launch (weight loads may overlap it).
 int w4a4_pass(const uint8_t* wp, const uint8_t* wbs, float g, int n, int k, const uint8_t* xq,
-              const uint8_t* xbs, const float* xg, int rows, uint16_t* out, int64_t ldc, cudaStream_t s);
+              const uint8_t* xbs, const float* xg, int rows, uint16_t* out, int64_t ldc, cudaStream_t s,
+              bool after_prepass = false);
 // Per-row NVFP4 quantize of BF16 rows (one 8-CTA cluster per row): codes [rows][k/2] (row
 // stride k/2), block scales [rows][k/16], globals [rows].  k % 16 == 0.
 int nvfp4_quantize_launch(const uint16_t* x, int64_t ldx, int rows, int k, uint8_t* xq, uint8_t* xbs, float* xg,

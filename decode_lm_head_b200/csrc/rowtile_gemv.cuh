@@ -44,6 +44,9 @@ struct RowTileParams {
   int rows;                // activation rows in this pass (<= 8*NT)
   uint16_t* out;           // bf16 out [rows, ldc]
   int64_t ldc;
+  int early_w;             // streamed kernel: 1 when the preceding kernel on the stream is this
+                           // library's activation pre-pass (writes neither weights nor outputs), so
+                           // the weight ring may fill before that kernel completes
 };
 
 // ---------------------------------------------------------------------------------------

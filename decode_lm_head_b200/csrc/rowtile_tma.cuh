@@ -51,9 +51,22 @@ constexpr int x_words() {
   return F::kXBytes == 1 ? 4 : (F::kXBytes == 0 ? 5 : (F::kElemsPerKB / 4) / 2);
 }
 
+// Register-light configurations (8-row tier, at most 40 words of activation fragments per
+// lane) run two tiles per reduction round when a tile is one stage, and load x in one pass.
+template <int NT, int NKB, int XW>
+__host__ __device__ constexpr bool register_light() {
+  return NT == 1 && NKB * XW <= 40;
+}
+template <int NT, int NKB, int XW, int NST>
+__host__ __device__ constexpr int tiles_per_round() {
+  return (register_light<NT, NKB, XW>() && NST == 1) ? 2 : 1;
+}
+
+// Shared memory of the streamed kernel; the partial-sum buffer holds two rounds (parity) of
+// up to two tiles for the 8-row tier.
 template <class F, int NT, int C, int NS>
 __host__ __device__ constexpr size_t stream_smem_bytes() {
-  return (size_t)NS * StageLayout<F, C>::kBytes + 2ull * kWarps * kTileRows * (8 * NT) * sizeof(float) +
+  return (size_t)NS * StageLayout<F, C>::kBytes + 2ull * (NT == 1 ? 2 : 1) * kWarps * kTileRows * (8 * NT) * sizeof(float) +
          2 * 8 * NT * sizeof(float) + 2 * NS * sizeof(uint64_t) + 64;
 }
 
@@ -192,11 +205,14 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemv_kernel(const RowTileP
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* ring = smem;
   float* red = reinterpret_cast<float*>(smem + (size_t)NS * L::kBytes);
-  float* rowmul = red + 2 * kWarps * kTileRows * MT;
+  float* rowmul = red + 2 * (NT == 1 ? 2 : 1) * kWarps * kTileRows * MT;  // after two rounds of partials
   int* rowexp = reinterpret_cast<int*>(rowmul + MT);
   uint64_t* bars = reinterpret_cast<uint64_t*>(rowexp + MT + ((MT & 1) ? 1 : 0));  // full[NS], empty[NS]
   __shared__ int s_fault;
 
+  // Programmatic dependent launch: the next kernel on the stream may start its prologue now;
+  // this one touches nothing a preceding kernel may write before grid_dependency_wait().
+  grid_dependents_launch();
   const int ntiles = (p.n + kTileRows - 1) / kTileRows;
   const int T0 = (int)((int64_t)blockIdx.x * ntiles / gridDim.x);
   const int T1 = (int)((int64_t)(blockIdx.x + 1) * ntiles / gridDim.x);
@@ -268,13 +284,17 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemv_kernel(const RowTileP
     }
   };
 
+  if (!p.early_w) grid_dependency_wait();  // weights may come from the preceding kernel
   if (warp == 0) {
     for (int s = 0; s < NS && s < nstages; ++s) produce(s);
   }
+  grid_dependency_wait();  // activations (and the outputs) belong to the preceding kernel
 
   // ---- activation fragments into registers (while the first stages are in flight)
   uint32_t xr[NKB][NT][XW];
-  if constexpr (F::kXBytes == 2) {
+  if constexpr (F::kXBytes == 2 && !register_light<NT, NKB, XW>()) {
+    // Two passes over x (the wider tiers keep fewer registers live): each row's maximum from
+    // its own warp, then the fragments converted as they load.
     const uint16_t* x = static_cast<const uint16_t*>(p.x);
     for (int m = warp; m < MT; m += kWarps) {  // per-row power of two into f16 range
       float amax = 0.f;
@@ -317,6 +337,65 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemv_kernel(const RowTileP
             const uint32_t hi = f32_to_f16_bits(bf16_bits_to_f32(wv[i] >> 16) * mul);
             xr[j][nt][4 * c + i] = lo | (hi << 16);
           }
+        }
+      }
+    }
+  } else if constexpr (F::kXBytes == 2) {
+    // One pass over x: the lane's fragments are loaded as raw BF16 pairs while each row's
+    // maximum is reduced (lanes of a row, then warps through shared memory); the row's power
+    // of two into f16 range then converts the fragments in registers.
+    const uint16_t* x = static_cast<const uint16_t*>(p.x);
+    float pmax[NT];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) pmax[nt] = 0.f;
+#pragma unroll
+    for (int j = 0; j < NKB; ++j) {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const int m = nt * 8 + g;
+        const int k0 = (j * kWarps + warp) * F::kElemsPerKB + t * EL;
+#pragma unroll
+        for (int c = 0; c < EL / 8; ++c) {  // 8 values per 16-byte load
+          uint4 v = make_uint4(0, 0, 0, 0);
+          if (m < p.rows && k0 + 8 * c < p.k) v = ldg_nc(x + (int64_t)m * p.ldx + k0 + 8 * c);
+          const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            xr[j][nt][4 * c + i] = wv[i];
+            pmax[nt] = fmaxf(pmax[nt], fabsf(bf16_bits_to_f32(wv[i] & 0xffffu)));
+            pmax[nt] = fmaxf(pmax[nt], fabsf(bf16_bits_to_f32(wv[i] >> 16)));
+          }
+        }
+      }
+    }
+    float* wmax = red;  // [kWarps][MT], free until the first tile ends
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      float v = pmax[nt];
+      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
+      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
+      if (t == 0) wmax[warp * MT + nt * 8 + g] = v;
+    }
+    __syncthreads();
+    if (threadIdx.x < MT) {
+      float amax = 0.f;
+      for (int w = 0; w < kWarps; ++w) amax = fmaxf(amax, wmax[w * MT + threadIdx.x]);
+      const int e = f16_row_exponent(amax);
+      rowexp[threadIdx.x] = e;
+      rowmul[threadIdx.x] = __int_as_float((127 - e) << 23);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const float mul = __int_as_float((127 + rowexp[nt * 8 + g]) << 23);
+#pragma unroll
+      for (int j = 0; j < NKB; ++j) {
+#pragma unroll
+        for (int w = 0; w < XW; ++w) {
+          const uint32_t raw = xr[j][nt][w];
+          const uint32_t lo = f32_to_f16_bits(bf16_bits_to_f32(raw & 0xffffu) * mul);
+          const uint32_t hi = f32_to_f16_bits(bf16_bits_to_f32(raw >> 16) * mul);
+          xr[j][nt][w] = lo | (hi << 16);
         }
       }
     }
@@ -364,93 +443,109 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemv_kernel(const RowTileP
   }
   __syncthreads();
 
-  // ---- main loop
-  const bool reducer = threadIdx.x < kTileRows * MT;
-  const int red_rr = threadIdx.x % kTileRows, red_cc = threadIdx.x / kTileRows;
+  // ---- main loop: rounds of TPR tiles, one cross-warp reduction (one CTA barrier) per round.
+  // Two independent tiles per round (8-row tier, one stage per tile) halve the barriers and
+  // let the two tiles' MMA chains interleave; the per-output sum is the same either way.
+  constexpr int TPR = tiles_per_round<NT, NKB, XW, NST>();
+  constexpr int kRed = kWarps * kTileRows * MT;  // floats of one tile's partial sums
+  const int red_tt = threadIdx.x / (kTileRows * MT);
+  const bool reducer = red_tt < TPR;
+  const int red_rr = threadIdx.x % kTileRows, red_cc = (threadIdx.x / kTileRows) % MT;
   float wscale_cur = 0.f;
   if constexpr (!F::kBlockScale) {
-    const int row = T0 * kTileRows + red_rr;
-    if (reducer && row < p.n) wscale_cur = p.w_scale[row];
+    const int row = (T0 + red_tt) * kTileRows + red_rr;
+    if (reducer && T0 + red_tt < T1 && row < p.n) wscale_cur = p.w_scale[row];
   }
-  float acc[NT][4];
+  float acc[TPR][NT][4];
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt)
+  for (int tt = 0; tt < TPR; ++tt)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[tt][nt][i] = 0.f;
 
   int s = 0, parity = 0;
-  for (int tile = T0; tile < T1; ++tile) {
+  for (int tile0 = T0; tile0 < T1; tile0 += TPR) {
+    const int ntl = min(TPR, T1 - tile0);
 #pragma unroll
-    for (int j = 0; j < NST; ++j, ++s) {
-      const int slot = s % NS;
-      if (!mbar_wait(full_bar(slot), (s / NS) & 1)) {
-        record_fault(2);
-        s_fault = 1;
-      }
-      const uint32_t stage = ring_u32 + slot * L::kBytes;
+    for (int tt = 0; tt < TPR; ++tt) {
+      if (tt < ntl) {
 #pragma unroll
-      for (int i = 0; i < C; ++i) {
-        const int q = j * C + i;  // the warp's slot index: k-block 16 q + warp
-        if (q < NKB) {
-          const int kb = q * kWarps + warp;
-          if (kb < kb_total) {
-            const int col = kb * kKBlockBytes + 16 * t;  // lane's byte column in the row
-            const uint32_t st = stage + g * wpitch + (i * kWarps + warp) * kKBlockBytes + 16 * t;
-            uint4 ra = make_uint4(0, 0, 0, 0), rb = ra;
-            uint32_t sa = 0, sb = 0;
-            if (col < wrb) {
-              ra = lds128(st);
-              rb = lds128(st + 8 * wpitch);
-              if constexpr (F::kBlockScale) {
-                const uint32_t ss = stage + L::kWeightBytes + g * spitch + (i * kWarps + warp) * 8 + 2 * t;
-                uint16_t va, vb;
-                asm volatile("ld.shared.u16 %0, [%1];" : "=h"(va) : "r"(ss));
-                asm volatile("ld.shared.u16 %0, [%1];" : "=h"(vb) : "r"(ss + 8 * spitch));
-                sa = va;
-                sb = vb;
+        for (int j = 0; j < NST; ++j, ++s) {
+          const int slot = s % NS;
+          if (!mbar_wait(full_bar(slot), (s / NS) & 1)) {
+            record_fault(2);
+            s_fault = 1;
+          }
+          const uint32_t stage = ring_u32 + slot * L::kBytes;
+#pragma unroll
+          for (int i = 0; i < C; ++i) {
+            const int q = j * C + i;  // the warp's slot index: k-block 16 q + warp
+            if (q < NKB) {
+              const int kb = q * kWarps + warp;
+              if (kb < kb_total) {
+                const int col = kb * kKBlockBytes + 16 * t;  // lane's byte column in the row
+                const uint32_t st = stage + g * wpitch + (i * kWarps + warp) * kKBlockBytes + 16 * t;
+                uint4 ra = make_uint4(0, 0, 0, 0), rb = ra;
+                uint32_t sa = 0, sb = 0;
+                if (col < wrb) {
+                  ra = lds128(st);
+                  rb = lds128(st + 8 * wpitch);
+                  if constexpr (F::kBlockScale) {
+                    const uint32_t ss = stage + L::kWeightBytes + g * spitch + (i * kWarps + warp) * 8 + 2 * t;
+                    uint16_t va, vb;
+                    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(va) : "r"(ss));
+                    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(vb) : "r"(ss + 8 * spitch));
+                    sa = va;
+                    sb = vb;
+                  }
+                }
+                if constexpr (F::kXBytes == 0)
+                  kb_w4a4_reg<NT, XW>(acc[tt], ra, rb, sa, sb, xr[q]);
+                else if constexpr (F::kBlockScale)
+                  kb_w4a16_reg<NT, XW>(acc[tt], ra, rb, sa, sb, xr[q]);
+                else if constexpr (F::kXBytes == 1)
+                  kb_w8a8_reg<NT, XW>(acc[tt], ra, rb, xr[q]);
+                else
+                  kb_w8a16_reg<NT, XW>(acc[tt], ra, rb, xr[q]);
               }
             }
-            if constexpr (F::kXBytes == 0)
-              kb_w4a4_reg<NT, XW>(acc, ra, rb, sa, sb, xr[q]);
-            else if constexpr (F::kBlockScale)
-              kb_w4a16_reg<NT, XW>(acc, ra, rb, sa, sb, xr[q]);
-            else if constexpr (F::kXBytes == 1)
-              kb_w8a8_reg<NT, XW>(acc, ra, rb, xr[q]);
-            else
-              kb_w8a16_reg<NT, XW>(acc, ra, rb, xr[q]);
           }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(empty_bar(slot));
+          if (warp == 0 && s + NS < nstages) produce(s + NS);
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(empty_bar(slot));
-      if (warp == 0 && s + NS < nstages) produce(s + NS);
     }
 
-    // ---- end of tile: fixed-order cross-warp reduction
-    float* rb_ = red + parity * (kWarps * kTileRows * MT);
+    // ---- end of round: fixed-order cross-warp reduction of each tile
+    float* rb_ = red + parity * (TPR * kRed);
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      reinterpret_cast<float4*>(rb_)[(warp * NT + nt) * 32 + lane] =
-          make_float4(acc[nt][0], acc[nt][1], acc[nt][2], acc[nt][3]);
-      acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-    }
+    for (int tt = 0; tt < TPR; ++tt)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        reinterpret_cast<float4*>(rb_ + tt * kRed)[(warp * NT + nt) * 32 + lane] =
+            make_float4(acc[tt][nt][0], acc[tt][nt][1], acc[tt][nt][2], acc[tt][nt][3]);
+        acc[tt][nt][0] = acc[tt][nt][1] = acc[tt][nt][2] = acc[tt][nt][3] = 0.f;
+      }
     __syncthreads();
     if (reducer) {
-      const int rr = red_rr, cc = red_cc;
+      const int rr = red_rr, cc = red_cc, tile = tile0 + red_tt;
       const int row = tile * kTileRows + rr;
+      const float* rt = rb_ + red_tt * kRed;
       float wsc = 0.f;
       if constexpr (!F::kBlockScale) {
         wsc = wscale_cur;
-        const int nrow = row + kTileRows;
-        if (tile + 1 < T1 && nrow < p.n) wscale_cur = p.w_scale[nrow];
+        const int nrow = row + TPR * kTileRows;
+        if (tile + TPR < T1 && nrow < p.n) wscale_cur = p.w_scale[nrow];
       }
-      if (cc < p.rows && row < p.n) {
+      if (red_tt < ntl && cc < p.rows && row < p.n) {
         const int gg = rr & 7, up = rr >> 3;
         const int nt = cc >> 3, cl = cc & 7;
         const int ln = gg * 4 + (cl >> 1), comp = up * 2 + (cl & 1);
         float sum = 0.f;
 #pragma unroll
-        for (int ww = 0; ww < kWarps; ++ww) sum += rb_[((ww * NT + nt) * 32 + ln) * 4 + comp];
+        for (int ww = 0; ww < kWarps; ++ww) sum += rt[((ww * NT + nt) * 32 + ln) * 4 + comp];
         float y;
         if constexpr (F::kBlockScale)
           y = (sum * p.gscale) * rowmul[cc];
