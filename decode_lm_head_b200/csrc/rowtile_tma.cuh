@@ -284,11 +284,15 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemv_kernel(const RowTileP
     }
   };
 
-  if (!p.early_w) grid_dependency_wait();  // weights may come from the preceding kernel
-  if (warp == 0) {
-    for (int s = 0; s < NS && s < nstages; ++s) produce(s);
-  }
-  grid_dependency_wait();  // activations (and the outputs) belong to the preceding kernel
+  // The first NS stages.  After this library's own pre-pass (early_w) they are requested at
+  // once; otherwise after the preceding kernel, and after this CTA's activation loads, so that
+  // the few x bytes are not queued behind the ring's ~180 KB per SM.
+  auto prefill = [&]() {
+    if (warp == 0)
+      for (int s = 0; s < NS && s < nstages; ++s) produce(s);
+  };
+  if (p.early_w) prefill();
+  grid_dependency_wait();  // activations, outputs (and otherwise the weights) follow the preceding kernel
 
   // ---- activation fragments into registers (while the first stages are in flight)
   uint32_t xr[NKB][NT][XW];
@@ -318,6 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemv_kernel(const RowTileP
         rowmul[m] = __int_as_float((127 - e) << 23);
       }
     }
+    if (!p.early_w) prefill();
     __syncthreads();
 #pragma unroll
     for (int j = 0; j < NKB; ++j) {
@@ -358,16 +363,23 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemv_kernel(const RowTileP
         for (int c = 0; c < EL / 8; ++c) {  // 8 values per 16-byte load
           uint4 v = make_uint4(0, 0, 0, 0);
           if (m < p.rows && k0 + 8 * c < p.k) v = ldg_nc(x + (int64_t)m * p.ldx + k0 + 8 * c);
-          const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            xr[j][nt][4 * c + i] = wv[i];
-            pmax[nt] = fmaxf(pmax[nt], fabsf(bf16_bits_to_f32(wv[i] & 0xffffu)));
-            pmax[nt] = fmaxf(pmax[nt], fabsf(bf16_bits_to_f32(wv[i] >> 16)));
-          }
+          xr[j][nt][4 * c + 0] = v.x;
+          xr[j][nt][4 * c + 1] = v.y;
+          xr[j][nt][4 * c + 2] = v.z;
+          xr[j][nt][4 * c + 3] = v.w;
         }
       }
     }
+    if (!p.early_w) prefill();
+#pragma unroll
+    for (int j = 0; j < NKB; ++j)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int w = 0; w < XW; ++w) {
+          pmax[nt] = fmaxf(pmax[nt], fabsf(bf16_bits_to_f32(xr[j][nt][w] & 0xffffu)));
+          pmax[nt] = fmaxf(pmax[nt], fabsf(bf16_bits_to_f32(xr[j][nt][w] >> 16)));
+        }
     float* wmax = red;  // [kWarps][MT], free until the first tile ends
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
@@ -414,7 +426,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemv_kernel(const RowTileP
         uint32_t sc = 0;
         if (m < p.rows && k0 < p.k) {
           v = ldg_nc(xq + (int64_t)m * (p.ldx / 2) + k0 / 2);
-          sc = e4m3x2_to_f16x2((uint16_t)ldg_u16(p.x_bscale + (int64_t)m * (p.k / 16) + k0 / 16));
+          sc = ldg_u16(p.x_bscale + (int64_t)m * (p.k / 16) + k0 / 16);
         }
         xr[j][nt][0] = v.x;
         xr[j][nt][1] = v.y;
@@ -423,6 +435,11 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemv_kernel(const RowTileP
         xr[j][nt][4] = sc;
       }
     }
+    if (!p.early_w) prefill();
+#pragma unroll
+    for (int j = 0; j < NKB; ++j)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) xr[j][nt][4] = e4m3x2_to_f16x2((uint16_t)xr[j][nt][4]);
   } else {
     const uint8_t* x = static_cast<const uint8_t*>(p.x);
     if (threadIdx.x < MT) rowmul[threadIdx.x] = threadIdx.x < p.rows ? p.x_scale[threadIdx.x] : 0.f;
@@ -440,6 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemv_kernel(const RowTileP
         xr[j][nt][3] = v.w;
       }
     }
+    if (!p.early_w) prefill();
   }
   __syncthreads();
 
