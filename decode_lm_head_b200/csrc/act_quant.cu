@@ -118,6 +118,7 @@ __global__ void __launch_bounds__(kQT) w8a8_quant_cluster_kernel(const uint16_t*
   __shared__ float red[kQT / 32];
   __shared__ float cta_max;
   grid_dependents_launch();  // a following tensor-core GEMV may start its weight loads
+  grid_dependency_wait();    // launched early (programmatic): x and the outputs follow the preceding kernel
   const int m = blockIdx.y;
   const uint16_t* ar = a + (int64_t)m * ld;
   const uint16_t* br = S == Src::Silu ? b + (int64_t)m * ld : nullptr;
@@ -186,6 +187,7 @@ __global__ void __launch_bounds__(kQT) w8a16_split_cluster_kernel(const uint16_t
   __shared__ float red[kQT / 32];
   __shared__ float cta_max;
   grid_dependents_launch();  // the GEMV may start its prologue and weight loads now
+  grid_dependency_wait();    // launched early (programmatic): x and the codes follow the preceding kernel
   const int m = blockIdx.y;
   uint8_t* hi_row = codes + (int64_t)m * k;
   uint8_t* lo_row = codes + (int64_t)(half + m) * k;
@@ -275,6 +277,7 @@ __global__ void __launch_bounds__(kQT) nvfp4_quant_cluster_kernel(const uint16_t
   __shared__ float red[kQT / 32];
   __shared__ float cta_max;
   grid_dependents_launch();
+  grid_dependency_wait();  // launched early (programmatic): x and the codes follow the preceding kernel
   const int m = blockIdx.y;
   const uint16_t* xr = x + (int64_t)m * ldx;
   int b0, b1;
@@ -356,13 +359,17 @@ int launch_cluster(void (*kernel)(KArgs...), int rows, cudaStream_t s, Args&&...
   cfg.blockDim = dim3(kQT);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  // a cluster per row; programmatic stream serialization lets the launch (and CTA set-up)
+  // overlap the preceding kernel's tail: the kernels wait for it before touching memory
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = kQC;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   if (cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) != cudaSuccess) {
     (void)cudaGetLastError();
     return DLMH_ERR_CUDA;

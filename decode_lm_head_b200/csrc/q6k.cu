@@ -103,6 +103,8 @@ __device__ __forceinline__ int q6_row_stride(int k) {  // qs bytes per staged ro
 
 __global__ void __launch_bounds__(kQ6Threads, 1) q6k_mmvq_kernel(const Q6Params p) {
   extern __shared__ __align__(128) uint8_t smem[];
+  grid_dependents_launch();
+  grid_dependency_wait();  // launched early (programmatic): q8, blocks and out follow the preceding kernel
   const int nsb = p.k / 256;
   const int nb32 = p.k / 32;
   const int rs = q6_row_stride(p.k);
@@ -223,6 +225,8 @@ struct Q6StreamParams {
 
 __global__ void __launch_bounds__(kQ6Threads, 1) q6k_stream_kernel(const Q6StreamParams sp) {
   extern __shared__ __align__(128) uint8_t smem[];
+  grid_dependents_launch();
+  grid_dependency_wait();  // launched early (programmatic): q8, blocks and out follow the preceding kernel
   __shared__ __align__(8) uint64_t full[kQ6MaxStages];
   const Q6Params& p = sp.q;
   const int nsb = p.k / 256;
@@ -474,6 +478,8 @@ __device__ __forceinline__ void q6_stage_tile(const Q6Params& p, int64_t row_byt
 template <int NT>
 __global__ void __launch_bounds__(kQWThreads, 1) q6k_wide_kernel(const Q6WideParams wp) {
   extern __shared__ __align__(128) uint8_t smem[];
+  grid_dependents_launch();
+  grid_dependency_wait();  // launched early (programmatic): q8, blocks and out follow the preceding kernel
   __shared__ __align__(8) uint64_t full[kQWMaxActStages], empty[kQWMaxActStages];
   const Q6Params& p = wp.q;
   const int nsb = p.k / 256;
@@ -646,8 +652,7 @@ int launch_wide(const Q6Params& p, int sms, int smem_optin, cudaStream_t s) {
     return DLMH_ERR_CUDA;
   const int ntiles = (p.n + kQ6TileRows - 1) / kQ6TileRows;
   const int grid = ntiles < sms ? ntiles : sms;
-  q6k_wide_kernel<NT><<<grid, kQWThreads, smem, s>>>(Q6WideParams{p, ns, depth});
-  return launch_status();
+  return umma::launch_pdl(q6k_wide_kernel<NT>, dim3(grid), dim3(kQWThreads), smem, s, Q6WideParams{p, ns, depth});
 }
 
 }  // namespace
@@ -684,14 +689,12 @@ int q6k_mmvq_launch(const uint8_t* blocks, int n, int k, const uint8_t* q8, int 
     if (ensure_dynamic_smem(reinterpret_cast<const void*>(q6k_stream_kernel), (int)smem) != DLMH_OK)
       return DLMH_ERR_CUDA;
     Q6StreamParams sp{p, ns, (int)stage_stride, (int)ring_offset};
-    q6k_stream_kernel<<<grid, kQ6Threads, smem, s>>>(sp);
-    return launch_status();
+    return umma::launch_pdl(q6k_stream_kernel, dim3(grid), dim3(kQ6Threads), smem, s, sp);
   }
   if (base_smem + 1024 > (size_t)di.smem_optin) return DLMH_ERR_UNSUPPORTED;
   if (ensure_dynamic_smem(reinterpret_cast<const void*>(q6k_mmvq_kernel), (int)base_smem) != DLMH_OK)
     return DLMH_ERR_CUDA;
-  q6k_mmvq_kernel<<<grid, kQ6Threads, base_smem, s>>>(p);
-  return launch_status();
+  return umma::launch_pdl(q6k_mmvq_kernel, dim3(grid), dim3(kQ6Threads), base_smem, s, p);
 }
 
 int q6k_fault(int reset) {

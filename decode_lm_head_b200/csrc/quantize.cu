@@ -3,6 +3,7 @@
 // act_quant.cu.
 #include "dlmh_common.cuh"
 #include "gemv_launch.h"
+#include "umma_common.cuh"
 
 namespace dlmh {
 namespace {
@@ -12,6 +13,8 @@ constexpr int kQThreads = 256;
 // block_q8_1: one warp per 32-value block.  Layout {f16 d; f16 s; int8 qs[32]}.
 __global__ void __launch_bounds__(kQThreads) q8_1_quantize_kernel(const uint16_t* __restrict__ x, int64_t ldx,
                                                                   int rows, int k, uint8_t* __restrict__ q8) {
+  grid_dependents_launch();  // the Q6_K GEMV may launch and set up now
+  grid_dependency_wait();    // launched early (programmatic): x and q8 follow the preceding kernel
   const int nb = k / 32;
   const int64_t blk = (int64_t)blockIdx.x * (kQThreads / 32) + (threadIdx.x >> 5);
   if (blk >= (int64_t)rows * nb) return;
@@ -39,8 +42,7 @@ __global__ void __launch_bounds__(kQThreads) q8_1_quantize_kernel(const uint16_t
 int q8_1_quantize_launch(const uint16_t* x, int64_t ldx, int rows, int k, uint8_t* q8, cudaStream_t s) {
   const int64_t blocks = (int64_t)rows * (k / 32);
   const int64_t grid = (blocks + (kQThreads / 32) - 1) / (kQThreads / 32);
-  q8_1_quantize_kernel<<<(unsigned)grid, kQThreads, 0, s>>>(x, ldx, rows, k, q8);
-  return launch_status();
+  return umma::launch_pdl(q8_1_quantize_kernel, dim3((unsigned)grid), dim3(kQThreads), 0, s, x, ldx, rows, k, q8);
 }
 
 }  // namespace dlmh

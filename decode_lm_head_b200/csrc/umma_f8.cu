@@ -302,6 +302,7 @@ constexpr int kFixupBatch = 16;
 __global__ void __launch_bounds__(kBM) umma_f8_fixup_kernel(const UmmaParams p, int G) {
   __shared__ int s_slot[kMaxParts];
   __shared__ int s_nparts;
+  grid_dependents_launch();  // the next call's pre-pass may launch; it waits for this grid
   const Sched sc{p.spt, p.wt, p.rem, G};
   const int t_rem = blockIdx.x, m = blockIdx.y;
   // Contributors of this tile (independent of the main kernel's data, so computed before the
