@@ -311,10 +311,9 @@ int nvfp4_quantize_rows(const dlmh_bf16* x, int64_t ldx, int rows, int k, uint8_
   return dlmh::nvfp4_quantize_launch(x, ldx, rows, k, xq, x_block_scale, x_global, as_stream(stream));
 }
 
-static int check_w4a4(const uint8_t* w_packed, const uint8_t* w_block_scale, int n, int k, int rows, dlmh_bf16* out,
-                      int64_t ldc) {
-  DLMH_TRY(check_rows(rows, 0));
-  DLMH_TRY(check_nk(n, k, 256));
+// NVFP4 weight and output checks shared by the W4A4 entry points (after the shape checks).
+static int check_w4a4_weight_out(const uint8_t* w_packed, const uint8_t* w_block_scale, int n, dlmh_bf16* out,
+                                 int64_t ldc) {
   if (!w_packed || !w_block_scale) return DLMH_ERR_NULL;
   if (!aligned16(w_packed) || !aligned16(w_block_scale)) return DLMH_ERR_ALIGN;
   return check_out(out, ldc, n);
@@ -323,8 +322,10 @@ static int check_w4a4(const uint8_t* w_packed, const uint8_t* w_block_scale, int
 int w4a4_gemv(const uint8_t* w_packed, const uint8_t* w_block_scale, float global_scale, int n, int k,
               const uint8_t* xq, const uint8_t* x_block_scale, const float* x_global, int rows, dlmh_bf16* out,
               int64_t ldc, void* stream) {
-  if (rows == 0 && check_rows(rows, 0) == DLMH_OK && check_nk(n, k, 256) == DLMH_OK) return DLMH_OK;
-  DLMH_TRY(check_w4a4(w_packed, w_block_scale, n, k, rows, out, ldc));
+  DLMH_TRY(check_rows(rows, 0));
+  DLMH_TRY(check_nk(n, k, 256));
+  if (rows == 0) return DLMH_OK;
+  DLMH_TRY(check_w4a4_weight_out(w_packed, w_block_scale, n, out, ldc));
   if (!xq || !x_block_scale || !x_global) return DLMH_ERR_NULL;
   if (!aligned16(xq) || (reinterpret_cast<uintptr_t>(x_block_scale) & 1u) ||
       (reinterpret_cast<uintptr_t>(x_global) & 3u))
@@ -344,8 +345,10 @@ int w4a4_gemv(const uint8_t* w_packed, const uint8_t* w_block_scale, float globa
 int w4a4_proj(const uint8_t* w_packed, const uint8_t* w_block_scale, float global_scale, int n, int k,
               const dlmh_bf16* x, int64_t ldx, int rows, dlmh_bf16* out, int64_t ldc, uint8_t* xq_scratch,
               uint8_t* xs_scratch, float* xg_scratch, void* stream) {
-  if (rows == 0 && check_rows(rows, 0) == DLMH_OK && check_nk(n, k, 256) == DLMH_OK) return DLMH_OK;
-  DLMH_TRY(check_w4a4(w_packed, w_block_scale, n, k, rows, out, ldc));
+  DLMH_TRY(check_rows(rows, 0));
+  DLMH_TRY(check_nk(n, k, 256));
+  if (rows == 0) return DLMH_OK;
+  DLMH_TRY(check_w4a4_weight_out(w_packed, w_block_scale, n, out, ldc));
   DLMH_TRY(check_bf16_in(x, ldx, k));
   if (!xq_scratch || !xs_scratch || !xg_scratch) return DLMH_ERR_NULL;
   if (!aligned16(xq_scratch) || (reinterpret_cast<uintptr_t>(xs_scratch) & 1u) ||
