@@ -48,6 +48,7 @@ constexpr int kUmmaThreads = 192;
 constexpr int kKC = 2;  // 128-byte K-chunks per stage
 constexpr int kChunkBytesA = kBM * 128;
 constexpr int kMaxUStages = 6;
+constexpr int kJobRing = 4;  // job descriptors in flight from the producer to the MMA and epilogue warps
 
 static __device__ int umma_fault_word = 0;  // 1: producer, 2: MMA (stage), 4: MMA (tmem), 8: epilogue
 constexpr int kWaitProbeBit = 0x40;         // set only by the bounded-wait check
@@ -76,6 +77,11 @@ struct UmmaParams {
   // the SM count, never of the row count; partial sums are laid out [slot][col][128 rows].
   int spt, wt, rem;
   float* partial;
+  // Dynamic hand-out of the whole tiles (null: the static order of the schedule).  queue[0]
+  // counts tiles claimed beyond each CTA's first, queue[1] the CTAs that have finished; the
+  // last CTA to finish puts both back to 0 for the next launch on the stream.  A whole tile's
+  // bits do not depend on which CTA ran it, so both orders give the same outputs.
+  int* queue;
   int early_w;  // 1: the preceding kernel is this library's activation pre-pass (it writes
                 // neither W nor the outputs), so weight loads may start before it completes
   // A second weight matrix against the same activations (an FFN's gate and up) runs in the
@@ -107,13 +113,18 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   __shared__ __align__(8) uint64_t bar_full[kMaxUStages], bar_empty[kMaxUStages], bar_tfull[2], bar_tempty[2];
+  __shared__ __align__(8) uint64_t bar_jfull[kJobRing], bar_jempty[kJobRing];
+  __shared__ int4 s_job[kJobRing];  // (tile, first unit, end unit, partial slot); tile < 0 ends
   __shared__ uint32_t s_tmem;
 
   const Sched sc{p.spt, p.wt, p.rem, (int)gridDim.x};
   const int b = blockIdx.x;
-  int njobs = 0, nunits = 0;
-  for (int tile, u0, u1, slot; sc.job(b, njobs, tile, u0, u1, slot); ++njobs) nunits += u1 - u0;
-  if (njobs == 0) return;
+  const int G = (int)gridDim.x;
+  {
+    int tile, u0, u1, slot;
+    if (!sc.job(b, 0, tile, u0, u1, slot)) return;  // no work at all (uniform over the CTA)
+  }
+  const bool dyn = p.queue != nullptr && p.wt > 0;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kchunks = p.k / 128;
@@ -133,6 +144,10 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
       bar_init(tfull0 + 8u * i, 1);
       bar_init(tempty0 + 8u * i, 4);  // the four epilogue warps
     }
+    for (int i = 0; i < kJobRing; ++i) {
+      bar_init(smem_u32(&bar_jfull[i]), 1);
+      bar_init(smem_u32(&bar_jempty[i]), 5);  // the MMA thread and the four epilogue warps
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) tmem_alloc(smem_u32(&s_tmem), tmem_cols);
@@ -143,31 +158,64 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
   grid_dependents_launch();  // the fixup may be scheduled; it waits for this grid to finish
 
   if (warp == 0) {
-    // ---------------- producer
+    // ---------------- producer: hands out the jobs and streams their stages
     if (lane == 0) {
       const uint64_t pol_w = l2_policy_evict_first(), pol_x = l2_policy_evict_last();
-      // The first ring's weight tiles may be requested before the preceding kernel has
-      // finished (early_w); activation tiles only after it.
-      const int npre = p.early_w ? min(p.ns, nunits) : 0;
-      {
-        int s = 0;
-        for (int j = 0; j < njobs && s < npre; ++j) {
-          int tile, u0, u1, ps;
-          sc.job(b, j, tile, u0, u1, ps);
-          for (int u = u0; u < u1 && s < npre; ++u, ++s) {
-            expect_tx(full0 + 8u * s, (uint32_t)p.stage_bytes);
-            const bool first = tile < p.t1;
-            tma_load_3d(ring_u32 + s * p.stage_bytes, first ? &map_w : &map_w2, 0, (first ? tile : tile - p.t1) * kBM,
-                        u * kKC, full0 + 8u * s, pol_w);
+      // Job sequence: the whole tiles (the first static -- tile b, or b*wt in the static
+      // order -- the rest claimed from the queue or taken in order), then the CTA's remainder
+      // segments, then an end marker.
+      bool whole = p.wt > 0;  // still handing out whole tiles
+      int wj = 0;             // whole tiles taken so far
+      int rj = p.wt;          // schedule index of the next remainder segment
+      auto next_job = [&](int4& jb) -> bool {
+        if (whole) {
+          int tile;
+          if (dyn)
+            tile = wj == 0 ? b : G + atomicAdd(p.queue, 1);
+          else
+            tile = wj < p.wt ? b * p.wt + wj : -1;
+          if (tile >= 0 && tile < p.wt * G) {
+            ++wj;
+            jb = make_int4(tile, 0, p.spt, -1);
+            return true;
           }
+          whole = false;
         }
+        int tile, u0, u1, ps;
+        if (sc.job(b, rj, tile, u0, u1, ps)) {
+          ++rj;
+          jb = make_int4(tile, u0, u1, ps);
+          return true;
+        }
+        return false;
+      };
+      int nj = 0;  // jobs published
+      auto publish = [&](const int4& jb) {
+        const int r = nj % kJobRing;
+        if (nj >= kJobRing && !wait(smem_u32(&bar_jempty[r]), ((nj / kJobRing) - 1) & 1))
+          atomicOr(&umma_fault_word, 16);
+        s_job[r] = jb;
+        arrive(smem_u32(&bar_jfull[r]));  // release: the descriptor is visible to the waiters
+        ++nj;
+      };
+      // The first job is static: its first ring of weight tiles may be requested before the
+      // preceding kernel has finished (early_w); activation tiles only after it.
+      int4 jb;
+      next_job(jb);
+      publish(jb);
+      const int npre = p.early_w ? min(p.ns, jb.z - jb.y) : 0;
+      for (int s = 0; s < npre; ++s) {
+        const int u = jb.y + s;
+        expect_tx(full0 + 8u * s, (uint32_t)p.stage_bytes);
+        const bool first = jb.x < p.t1;
+        tma_load_3d(ring_u32 + s * p.stage_bytes, first ? &map_w : &map_w2, 0, (first ? jb.x : jb.x - p.t1) * kBM,
+                    u * kKC, full0 + 8u * s, pol_w);
       }
       grid_dependency_wait();
       int slot = 0, phase = 0, s = 0;
-      for (int j = 0; j < njobs; ++j) {
-        int tile, u0, u1, ps;
-        sc.job(b, j, tile, u0, u1, ps);
-        for (int u = u0; u < u1; ++u, ++s) {
+      for (bool have = true; have;) {
+        const int tile = jb.x;
+        for (int u = jb.y; u < jb.z; ++u, ++s) {
           if (s >= p.ns && !wait(empty0 + 8u * slot, phase ^ 1)) atomicOr(&umma_fault_word, 1);
           const uint32_t st = ring_u32 + slot * p.stage_bytes;
           // the full boxes always land (rows past n, rows past `rows` and a chunk past K are
@@ -186,7 +234,10 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
             phase ^= 1;
           }
         }
+        have = next_job(jb);
+        publish(have ? jb : make_int4(-1, 0, 0, -1));
       }
+      const int nunits = s;
       // no copy may still be landing when the CTA exits: wait (bounded) for the last
       // phase of every slot (already complete in a healthy run, where the MMAs consumed it)
       for (int t = nunits - 1; t >= 0 && t >= nunits - p.ns; --t)
@@ -197,9 +248,16 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
     if (lane == 0) {
       const uint32_t idesc = idesc_m128(p.nb);
       int slot = 0, phase = 0;
-      for (int i = 0; i < njobs; ++i) {
-        int tile, u0, u1, ps;
-        sc.job(b, i, tile, u0, u1, ps);
+      for (int i = 0;; ++i) {
+        const int r = i % kJobRing;
+        if (!wait(smem_u32(&bar_jfull[r]), (i / kJobRing) & 1)) {
+          atomicOr(&umma_fault_word, 16);
+          break;
+        }
+        const int4 jb = s_job[r];
+        arrive(smem_u32(&bar_jempty[r]));
+        if (jb.x < 0) break;
+        const int u0 = jb.y, u1 = jb.z;
         const int acc = i & 1;
         if (i >= 2 && !wait(tempty0 + 8u * acc, ((i - 2) >> 1) & 1)) atomicOr(&umma_fault_word, 4);
         fence_after();
@@ -231,9 +289,17 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const int lane_row = q * 32 + lane;
     grid_dependency_wait();  // x_scale comes from the preceding kernel
-    for (int i = 0; i < njobs; ++i) {
-      int tile, u0, u1, ps;
-      sc.job(b, i, tile, u0, u1, ps);
+    for (int i = 0;; ++i) {
+      const int r = i % kJobRing;
+      if (!wait(smem_u32(&bar_jfull[r]), (i / kJobRing) & 1)) {
+        atomicOr(&umma_fault_word, 16);
+        break;
+      }
+      const int4 jb = s_job[r];
+      __syncwarp();
+      if (lane == 0) arrive(smem_u32(&bar_jempty[r]));
+      if (jb.x < 0) break;
+      const int tile = jb.x, ps = jb.w;
       const int acc = i & 1;
       if (!wait(tfull0 + 8u * acc, (i >> 1) & 1)) atomicOr(&umma_fault_word, 8);
       fence_after();
@@ -289,6 +355,13 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
   if (warp == 1) {
     __syncwarp();
     tmem_dealloc(tmem_base, tmem_cols);
+  }
+  if (dyn && threadIdx.x == 0) {  // this CTA claims no more tiles; the last one resets the queue
+    __threadfence();
+    if (atomicAdd(p.queue + 1, 1) == G - 1) {
+      p.queue[0] = 0;
+      p.queue[1] = 0;
+    }
   }
 }
 
@@ -392,6 +465,44 @@ struct SecondWeight {
   int64_t ldc;
 };
 
+// Whole-tile queue of a stream (two ints, zero between launches): one per (device, stream),
+// so that launches on different streams never share one.  Allocated on the stream's first
+// call (cudaMalloc, then zeroed in stream order); a stream that is being captured into a
+// graph and has none yet gets nullptr, i.e. the static order (same outputs).
+int* tile_queue(cudaStream_t s) {
+  struct Entry {
+    int dev;
+    cudaStream_t stream;
+    int* q;
+  };
+  static std::mutex mu;
+  static Entry entries[256];
+  static int count = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < count; ++i)
+    if (entries[i].dev == dev && entries[i].stream == s) return entries[i].q;
+  if (count == 256) return nullptr;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  void* q = nullptr;
+  if (cudaMalloc(&q, 256) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  if (cudaMemsetAsync(q, 0, 256, s) != cudaSuccess) {
+    (void)cudaGetLastError();
+    cudaFree(q);
+    return nullptr;
+  }
+  entries[count++] = Entry{dev, s, static_cast<int*>(q)};
+  return static_cast<int*>(q);
+}
+
 int launch_umma_f8(const uint8_t* w, const float* w_scale, int n, int k, const uint8_t* b_codes, int64_t ldb,
                    int b_rows, const float* x_scale, int rows, int split, uint16_t* out, int64_t ldc, cudaStream_t s,
                    float* partial_ws, size_t partial_cap, int early_w, const SecondWeight* second = nullptr) {
@@ -442,6 +553,9 @@ int launch_umma_f8(const uint8_t* w, const float* w_scale, int n, int k, const u
   if (G > kMaxParts) return DLMH_ERR_UNSUPPORTED;
   p.wt = sched.wt;
   p.rem = sched.rem;
+  // whole tiles from a per-stream queue, except for callers with fixed scratch (they must not
+  // allocate); both orders give the same outputs
+  p.queue = (p.wt > 0 && partial_ws == nullptr) ? tile_queue(s) : nullptr;
   void* ws = nullptr;
   const size_t need = (size_t)2 * G * p.nb * kBM * sizeof(float);
   if (p.rem > 0 && partial_ws) {
