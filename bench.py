@@ -72,6 +72,25 @@ def measured_peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
+def read_peak_gbs(dev, stream):
+    """A measured read-only HBM rate: torch's sum over a 2 GiB float32 tensor (a plain
+    reduction, reads only), median of 5 after 3 warm-ups, outside the timed region."""
+    t = torch.ones(1 << 29, dtype=torch.float32, device=dev)
+    times = []
+    with torch.cuda.stream(stream):
+        for i in range(8):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            r = t.sum()
+            b.record(stream)
+            torch.cuda.synchronize()
+            if i >= 3:
+                times.append(a.elapsed_time(b))
+    del t, r
+    torch.cuda.empty_cache()
+    return (1 << 31) / (statistics.median(times) * 1e-3) / 1e9
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
     for f in ("umma_f8.cu", "umma_common.cuh", "umma_sched.h", "dlmh_common.cuh"):
@@ -474,6 +493,7 @@ def run_ours(args):
         barrier(world)
     elapsed_ms = max_over_ranks(ev0.elapsed_time(ev1), world)
     clocks = clk.summary()
+    read_peak = read_peak_gbs(dev, stream)
     per_m_events = {m: [] for m in ROWS}
     for _ in range(args.steps):
         for m in ROWS:
@@ -569,7 +589,10 @@ def run_ours(args):
                        "rows_per_pass": 128, "l2": "weight 1.27 GB > 126 MB L2: no flush needed",
                        "parallelism": f"replica per GPU (vocab-shard layout), {world} rank(s)"},
             "hbm_fraction": {"of_measured_copy": round(value / world / peak, 4),
-                             "of_spec_8tbs": round(value / world / SPEC_HBM_GBS, 4)},
+                             "of_spec_8tbs": round(value / world / SPEC_HBM_GBS, 4),
+                             "of_measured_read": round(value / world / read_peak, 4),
+                             "read_peak_gbs": round(read_peak, 1),
+                             "read_peak_how": "torch.sum over a 2 GiB float32 tensor, median of 5"},
             "per_m": per_m,
             "rows_nk_per_s": round(rows_nk, 1),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
