@@ -465,30 +465,42 @@ struct SecondWeight {
   int64_t ldc;
 };
 
-// Whole-tile queue of a stream (two ints, zero between launches): one per (device, stream),
-// so that launches on different streams never share one.  Allocated on the stream's first
-// call (cudaMalloc, then zeroed in stream order); a stream that is being captured into a
-// graph and has none yet gets nullptr, i.e. the static order (same outputs).
+// Whole-tile queue of a stream (two ints, zero between launches): one per stream, keyed by
+// the device and the stream's id (cudaStreamGetId: unique within the context, never reused
+// after the stream is destroyed), so that launches on different streams never share one.
+// Allocated on the stream's first eager call (cudaMalloc, then zeroed in stream order).  A
+// launch being captured into a graph gets nullptr, i.e. the static order (same outputs), so
+// no graph holds a counter that its replays on other streams could share; so does a stream
+// past the table's capacity.
 int* tile_queue(cudaStream_t s) {
   struct Entry {
     int dev;
-    cudaStream_t stream;
+    unsigned long long id;
     int* q;
   };
+  constexpr int kMaxQueues = 1024;
   static std::mutex mu;
-  static Entry entries[256];
+  static Entry entries[kMaxQueues];
   static int count = 0;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
-  std::lock_guard<std::mutex> lock(mu);
-  for (int i = 0; i < count; ++i)
-    if (entries[i].dev == dev && entries[i].stream == s) return entries[i].q;
-  if (count == 256) return nullptr;
   cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
   if (cudaStreamIsCapturing(s, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) {
     (void)cudaGetLastError();
     return nullptr;
   }
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  unsigned long long id = 0;
+  if (cudaStreamGetId(s, &id) != cudaSuccess) {
+    (void)cudaGetLastError();
+    // the legacy default stream (this library is built with it as stream 0) is never
+    // destroyed: its handle is a key of its own.  Anything else takes the static order.
+    if (s != nullptr && s != cudaStreamLegacy) return nullptr;
+    id = ~0ull;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < count; ++i)
+    if (entries[i].dev == dev && entries[i].id == id) return entries[i].q;
+  if (count == kMaxQueues) return nullptr;
   void* q = nullptr;
   if (cudaMalloc(&q, 256) != cudaSuccess) {
     (void)cudaGetLastError();
@@ -499,7 +511,7 @@ int* tile_queue(cudaStream_t s) {
     cudaFree(q);
     return nullptr;
   }
-  entries[count++] = Entry{dev, s, static_cast<int*>(q)};
+  entries[count++] = Entry{dev, id, static_cast<int*>(q)};
   return static_cast<int*>(q);
 }
 

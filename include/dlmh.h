@@ -27,13 +27,12 @@
  *     calls, so steady-state calls map nothing and never synchronize; concurrent calls on
  *     different streams get distinct scratch.  w8a8_proj_noalloc never uses the pool.
  *   - Tile queue: when a tensor-core pass has more weight tiles than SMs, its CTAs take the
- *     whole tiles from an atomic counter, one per (device, stream), allocated on the
- *     stream's first such call (cudaMalloc, so that first call synchronizes the device) and
- *     left at zero by every launch.  A stream being captured into a CUDA graph before its
- *     first eager call, and w8a8_proj_noalloc, use the static tile order instead; both give
- *     the same outputs.  Replaying one captured call on two streams at the same time, or
- *     reusing a destroyed stream's handle while its last call still runs, would share a
- *     counter: order such launches.
+ *     whole tiles from an atomic counter, one per stream (keyed by the device and
+ *     cudaStreamGetId, which is never reused within a context), allocated on the stream's
+ *     first eager such call (cudaMalloc, so that first call synchronizes the device) and
+ *     left at zero by every launch.  Launches captured into a CUDA graph, and
+ *     w8a8_proj_noalloc, use the static tile order instead, so a graph holds no counter
+ *     and its replays may run on any streams at once; both orders give the same outputs.
  *   - BF16 values are passed as raw 16-bit patterns (dlmh_bf16).
  *   - Matrices are row-major.  Leading dimensions (ld*) count ELEMENTS of the pointed-to
  *     type, so row r of x starts at x + r * ldx.
