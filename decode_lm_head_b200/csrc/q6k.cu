@@ -1,7 +1,8 @@
 // Q6_K super-blocks x block_q8_1 rows on int8 warp MMAs.
 //
 // Same decomposition as the row-tile GEMV: one persistent 512-thread CTA per SM over
-// 16-row weight tiles, the super-blocks of a tile split across 16 warps, a fixed-order
+// 16-row weight tiles, the super-blocks of a tile split across 16 warps as evenly as
+// possible (q6_slice_begin), a fixed-order
 // cross-warp reduction at the end of each tile.  Per 16-value sub-block j a warp runs one
 // s8 m16n8k16 MMA: the weight codes (q - 32) times the q8_1 codes, an exact int32 dot;
 // the dot is then scaled in f32 by d(super-block) * scales[j] of the weight row, and
@@ -42,6 +43,24 @@ __device__ __forceinline__ uint32_t q6_to_s8x4(uint32_t q) {
 // same in every Q6_K kernel whatever the compiler would contract.
 __device__ __forceinline__ float q6_block_step(float acc, int is, float d, float dx) {
   return __fmaf_rn(__fmul_rn((float)is, d), dx, acc);
+}
+
+// First super-block of K-slice w (w <= kQ6Warps): the nsb super-blocks of a row split into
+// kQ6Warps slices as evenly as possible, the longer slices first.  The 8-row kernels run
+// slice w on warp w; at nsb = 28 (K = 7168) slices 0..11 hold two super-blocks and 12..15
+// one, so each SM sub-partition (warps w, w+4, w+8, w+12) gets seven.  Every Q6_K kernel
+// accumulates each slice alone from 0 and adds the slices in order: the split is part of the
+// arithmetic they share.
+__device__ __forceinline__ int q6_slice_begin(int nsb, int w) {
+  const int q = nsb / kQ6Warps, r = nsb % kQ6Warps;
+  return w * q + (w < r ? w : r);
+}
+// Whether a slice of q6_slice_begin's split ends with super-block sb: the r slices of q + 1
+// end at multiples of q + 1, the rest every q super-blocks after them (q = 0: every sb).
+__device__ __forceinline__ bool q6_slice_ends(int nsb, int sb) {
+  const int q = nsb / kQ6Warps, r = nsb % kQ6Warps;
+  const int e = sb + 1, long_end = r * (q + 1);
+  return e <= long_end ? e % (q + 1) == 0 : (e - long_end) % q == 0;
 }
 
 // One super-block for rows g (a) and g+8 (b) of a 16-row tile against activation columns 2t
@@ -136,7 +155,7 @@ __global__ void __launch_bounds__(kQ6Threads, 1) q6k_mmvq_kernel(const Q6Params 
   const int T1 = (int)((int64_t)(blockIdx.x + 1) * ntiles / gridDim.x);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
-  const int nsbw = (nsb + kQ6Warps - 1) / kQ6Warps;
+  const int sb_begin = q6_slice_begin(nsb, warp), sb_end = q6_slice_begin(nsb, warp + 1);
   const int64_t row_bytes = (int64_t)nsb * 210;
   const int8_t* xrow = xs + g * rs;  // B column g
   int parity = 0;
@@ -145,9 +164,7 @@ __global__ void __launch_bounds__(kQ6Threads, 1) q6k_mmvq_kernel(const Q6Params 
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     const int r0 = tile * kQ6TileRows + g;
     const bool va = r0 < p.n, vb = r0 + 8 < p.n;
-    for (int s = 0; s < nsbw; ++s) {
-      const int sb = warp * nsbw + s;
-      if (sb >= nsb) break;
+    for (int sb = sb_begin; sb < sb_end; ++sb) {
       const uint8_t* ba = p.blocks + (int64_t)r0 * row_bytes + (int64_t)sb * 210;
       const uint8_t* bb = ba + 8 * row_bytes;
       uint32_t qla[8], qlb[8], qha[4], qhb[4], sca[4], scb[4];
@@ -288,7 +305,7 @@ __global__ void __launch_bounds__(kQ6Threads, 1) q6k_stream_kernel(const Q6Strea
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
-  const int nsbw = (nsb + kQ6Warps - 1) / kQ6Warps;
+  const int sb_begin = q6_slice_begin(nsb, warp), sb_end = q6_slice_begin(nsb, warp + 1);
   const int8_t* xrow = xs + g * rs;  // B column g
   int parity = 0;
 
@@ -303,9 +320,7 @@ __global__ void __launch_bounds__(kQ6Threads, 1) q6k_stream_kernel(const Q6Strea
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     const int r0 = tile * kQ6TileRows + g;
     const bool va = r0 < p.n, vb = r0 + 8 < p.n;
-    for (int s = 0; s < nsbw; ++s) {
-      const int sb = warp * nsbw + s;
-      if (sb >= nsb) break;
+    for (int sb = sb_begin; sb < sb_end; ++sb) {
       const uint32_t ba = base_a + (uint32_t)sb * 210u;
       const uint32_t bb = base_b + (uint32_t)sb * 210u;
       uint32_t qla[8], qlb[8], qha[4], qhb[4], sca[4], scb[4];
@@ -368,7 +383,7 @@ __global__ void __launch_bounds__(kQ6Threads, 1) q6k_stream_kernel(const Q6Strea
 //     boundary are stored with plain loads, so no copy reads past the weight buffer.
 // Each consumer warp runs NT 8-column MMAs per sub-block on one decoded A fragment.
 // The per-output arithmetic and its order are those of the 8-row kernels: K is cut into the
-// same 16 slices of nsbw super-blocks, each slice is accumulated alone from 0 with the same
+// same 16 slices (q6_slice_begin), each slice is accumulated alone from 0 with the same
 // per-block step, and the slices are added to 0 in order -- so a row's bits do not depend on
 // which kernel, or how many rows, served it.
 // 15 consumer warps + 1 producer: 16 warps, 4 per SM sub-partition, so 128 registers a thread
@@ -484,7 +499,6 @@ __global__ void __launch_bounds__(kQWThreads, 1) q6k_wide_kernel(const Q6WidePar
   const Q6Params& p = wp.q;
   const int nsb = p.k / 256;
   const int nb32 = p.k / 32;
-  const int nsbw = (nsb + kQ6Warps - 1) / kQ6Warps;  // slice length of the 8-row kernels
   const int64_t row_bytes = (int64_t)nsb * 210;
   const uintptr_t buf_end = reinterpret_cast<uintptr_t>(p.blocks) + (uintptr_t)((int64_t)p.n * row_bytes);
   constexpr int kRows = NT * 8;
@@ -595,7 +609,7 @@ __global__ void __launch_bounds__(kQWThreads, 1) q6k_wide_kernel(const Q6WidePar
       __syncwarp();  // the weight stage and the activation slot are read
       if (lane == 0) umma::arrive(empty0 + 8u * slot);
       // end of a slice of the 8-row kernels: add it to the total and restart
-      if ((sb + 1) % nsbw == 0 || sb + 1 == nsb) {
+      if (q6_slice_ends(nsb, sb)) {
 #pragma unroll
         for (int ct = 0; ct < NT; ++ct)
 #pragma unroll
@@ -607,8 +621,8 @@ __global__ void __launch_bounds__(kQWThreads, 1) q6k_wide_kernel(const Q6WidePar
     }
     cp_async_wait<0>();
     __syncwarp();
-    // slices past K (empty warps of the 8-row kernels) add +0
-    for (int w = (nsb + nsbw - 1) / nsbw; w < kQ6Warps; ++w)
+    // empty slices (nsb < 16: idle warps of the 8-row kernels) add +0
+    for (int w = nsb < kQ6Warps ? nsb : kQ6Warps; w < kQ6Warps; ++w)
 #pragma unroll
       for (int ct = 0; ct < NT; ++ct)
 #pragma unroll
