@@ -455,6 +455,24 @@ def other_formats(dev, stream, peak):
     return res
 
 
+def profile_q6k(n):
+    """A Q6_K profiling case for ncu: n x 7168 super-blocks (n = 32768: 193 MB, above the
+    126 MB L2), 8 BF16 rows, four q6k_lm_head calls on cuda:0; prints one line and no bench
+    result.  Only for captures such as `ncu -k regex:q6k_stream -s 1 -c 2`."""
+    import decode_lm_head_b200 as dl
+    from decode_lm_head_b200 import synth
+
+    dev = torch.device("cuda", 0)
+    k = 7168
+    blocks = synth.q6k_blocks(n, k, 4, dev)
+    x = synth.bf16_rows(8, k, 4, dev)
+    out = torch.empty(8, n, dtype=torch.bfloat16, device=dev)
+    for _ in range(4):
+        dl.q6k_lm_head(blocks, x, out=out)
+    torch.cuda.synchronize()
+    print(f"q6k profile case: {n} x {k}, 8 rows, 4 calls, device fault {dl.device_fault(reset=True)}")
+
+
 def run_ours(args):
     world, rank, local = dist_setup(args)
     import decode_lm_head_b200 as dl
@@ -628,7 +646,12 @@ def main():
                     help="also time W8A8 (head, SiLU down), NVFP4 and Q6_K (extra 'formats' key)")
     ap.add_argument("--vocab", type=int, default=248320,
                     help="head rows; smaller values only for profiling captures (the workload is 248320)")
+    ap.add_argument("--profile-q6k", type=int, default=0, metavar="N",
+                    help="run only the Q6_K profiling case (N x 7168 blocks, 8 rows, 4 calls) and exit")
     args = ap.parse_args()
+    if args.profile_q6k > 0:
+        profile_q6k(args.profile_q6k)
+        return
     globals()["VOCAB"] = args.vocab
     if args.warmup < 3:
         args.warmup = 3
