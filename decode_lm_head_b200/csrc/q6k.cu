@@ -18,6 +18,7 @@
 // 16-bit read-only loads (each 32-byte sector still comes from DRAM once).
 #include "dlmh_common.cuh"
 #include "gemv_launch.h"
+#include "q6k_slices.h"
 #include "umma_common.cuh"
 
 namespace dlmh {
@@ -45,23 +46,8 @@ __device__ __forceinline__ float q6_block_step(float acc, int is, float d, float
   return __fmaf_rn(__fmul_rn((float)is, d), dx, acc);
 }
 
-// First super-block of K-slice w (w <= kQ6Warps): the nsb super-blocks of a row split into
-// kQ6Warps slices as evenly as possible, the longer slices first.  The 8-row kernels run
-// slice w on warp w; at nsb = 28 (K = 7168) slices 0..11 hold two super-blocks and 12..15
-// one, so each SM sub-partition (warps w, w+4, w+8, w+12) gets seven.  Every Q6_K kernel
-// accumulates each slice alone from 0 and adds the slices in order: the split is part of the
-// arithmetic they share.
-__device__ __forceinline__ int q6_slice_begin(int nsb, int w) {
-  const int q = nsb / kQ6Warps, r = nsb % kQ6Warps;
-  return w * q + (w < r ? w : r);
-}
-// Whether a slice of q6_slice_begin's split ends with super-block sb: the r slices of q + 1
-// end at multiples of q + 1, the rest every q super-blocks after them (q = 0: every sb).
-__device__ __forceinline__ bool q6_slice_ends(int nsb, int sb) {
-  const int q = nsb / kQ6Warps, r = nsb % kQ6Warps;
-  const int e = sb + 1, long_end = r * (q + 1);
-  return e <= long_end ? e % (q + 1) == 0 : (e - long_end) % q == 0;
-}
+// The K-slices (q6k_slices.h): warp w of the 8-row kernels runs slice w.
+static_assert(kQ6Warps == kQ6Slices, "one K-slice per warp of the 8-row kernels");
 
 // One super-block for rows g (a) and g+8 (b) of a 16-row tile against activation columns 2t
 // and 2t+1 (acc[0..1]: row a, acc[2..3]: row b).  Per q8_1 block (sub-blocks j0, j1) the two
