@@ -62,12 +62,6 @@ int pass_rows(int op, int k) {
   }
 }
 
-int op_row_cap(int op) {
-  switch (op) {
-    case DLMH_OP_W4A16: return DLMH_W4A16_MAX_ROWS;
-    default: return 0;  // any rows
-  }
-}
 
 }  // namespace
 
@@ -97,7 +91,7 @@ const char* dlmh_error_string(int code) {
 int dlmh_plan_chunks(int op, int rows, int k, int* offsets, int* counts, int* tiers, int cap) {
   if (op < DLMH_OP_W8A16 || op > DLMH_OP_W4A4) return DLMH_ERR_SHAPE;
   if (k <= 0) return DLMH_ERR_SHAPE;
-  DLMH_TRY(check_rows(rows, op_row_cap(op)));
+  DLMH_TRY(check_rows(rows, 0));
   const int width = pass_rows(op, k);
   if (width <= 0) return DLMH_ERR_UNSUPPORTED;
   int nchunks = 0;
@@ -282,7 +276,7 @@ int w8a8_gate_up_proj(const uint8_t* w_gate, const float* s_gate, const uint8_t*
 
 int w4a16_gemv(const uint8_t* w_packed, const uint8_t* w_block_scale, float global_scale, int n, int k,
                const dlmh_bf16* x, int64_t ldx, int rows, dlmh_bf16* out, int64_t ldc, void* stream) {
-  DLMH_TRY(check_rows(rows, DLMH_W4A16_MAX_ROWS));
+  DLMH_TRY(check_rows(rows, 0));
   DLMH_TRY(check_nk(n, k, 128));
   if (rows == 0) return DLMH_OK;
   if (!w_packed || !w_block_scale) return DLMH_ERR_NULL;

@@ -90,8 +90,8 @@ typedef enum dlmh_status {
 /* Rows per weight pass of the FP8 W8A16 head (16-row chunks above 16 rows,
  * lm_head_fp8_rows.rs module doc). */
 #define DLMH_W8A16_CHUNK_ROWS 16
-/* Largest row count of one NVFP4 W4A16 call (w4a16_gemv_tiers.rs, kernel_within:
- * more than 32 rows is refused). */
+/* Widest NVFP4 W4A16 weight pass (w4a16_gemv_tiers.rs, kernel_within: one kernel launch
+ * serves at most 32 rows).  w4a16_gemv runs more rows as several such passes. */
 #define DLMH_W4A16_MAX_ROWS 32
 /* Widest W4A4 pass (w4a4_proj::W4A4_MAX_M in w4a16_gemv_tiers.rs). */
 #define DLMH_W4A4_MAX_ROWS 32
@@ -236,7 +236,10 @@ DLMH_API int w8a8_proj_noalloc(const uint8_t* w, const float* w_scale, int n, in
  *   w_packed      [n, k/2] bytes, element 2i in the low nibble of byte i.
  *   w_block_scale [n, k/16] E4M3 bytes, one per 16 consecutive k of a row.
  *   global_scale  the folded float32 multiplier g.
- *   k % 128 == 0, k <= 8192.  rows <= 32 (else DLMH_ERR_ROWS); one weight pass per call.
+ *   k % 128 == 0, k <= 8192.  Any rows >= 0: weight passes of at most DLMH_W4A16_MAX_ROWS
+ *   (the pages' kernel_within limit of one launch; fewer when the activation tile of a wider
+ *   tier does not fit on chip, see dlmh_plan_chunks), each through the narrowest tier of
+ *   8 / 16 / 32 rows that covers it; a row's bits do not depend on `rows`.
  * ------------------------------------------------------------------------------------- */
 DLMH_API int w4a16_gemv(const uint8_t* w_packed, const uint8_t* w_block_scale, float global_scale, int n, int k,
                const dlmh_bf16* x, int64_t ldx, int rows, dlmh_bf16* out, int64_t ldc, void* stream);
@@ -358,7 +361,7 @@ typedef enum dlmh_op {
  * its width is counts[i] rounded up to 16 (the MMA's N, doubled inside for W8A16).
  * The pass width is a pure function of (op, k) (which kernel serves k, and which activation
  * tile fits on chip), so this needs no GPU.  Returns the number of passes (0 for rows == 0), DLMH_ERR_ROWS for
- * rows < 0 or above the op's cap, DLMH_ERR_SHAPE for an unknown op or k <= 0,
+ * rows < 0, DLMH_ERR_SHAPE for an unknown op or k <= 0,
  * DLMH_ERR_UNSUPPORTED when no tier fits k, DLMH_ERR_CAPACITY when more than `cap`
  * passes are needed.  Arrays may be NULL when cap == 0 (count only). */
 DLMH_API int dlmh_plan_chunks(int op, int rows, int k, int* offsets, int* counts, int* tiers, int cap);

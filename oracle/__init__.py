@@ -15,9 +15,10 @@ with the formats decoded from their definitions:
 * ``plan``      - the row-chunk and tier rules of the host dispatch.
 
 Pinning status (what each function is checked against, in ``tests/``):
-pinned by library routines, closed forms, printed tables and brute force --
-except the element order inside a Q6_K super-block, which the pages do not
-print: that part is "parity unpinned" (see ``gemv.q6k_unpack``).
+pinned by library routines, closed forms, printed tables and brute force.  The
+element order inside a Q6_K super-block, which the pages do not print, is pinned
+by hand-derived single-byte probes and by the gguf library's Q6_K dequantizer
+(see ``gemv.q6k_unpack``).
 """
 
 from . import numerics, gemv, plan  # noqa: F401

@@ -339,8 +339,10 @@ def q6k_unpack(blocks):
     low 4 bits from ``ql[64h + l]`` (t = 0: low nibble, t = 2: high nibble) or
     ``ql[64h + 32 + l]`` (t = 1: low nibble, t = 3: high nibble), and its top 2
     bits from bits 2t..2t+1 of ``qh[32h + l]``.  Element i uses ``scales[i // 16]``.
-    The element order inside a super-block has no pin on the pages:
-    parity unpinned for that order.
+    The pages print no element order; it is pinned by hand-derived single-byte
+    probes (tests/golden/q6k_single_byte_probes.txt) and by bit-exact agreement
+    with the gguf library's independent Q6_K dequantizer on blocks covering every
+    byte value of ql, qh and the scales (tests/test_oracle_pins.py).
     """
     b = np.asarray(blocks, dtype=np.uint8)
     ql = b[..., 0:128].astype(np.int64)

@@ -38,8 +38,7 @@ def test_error_strings_and_version():
                                            (dl.OP_Q6K, 7168, 64),
                                            (dl.OP_W4A4, 4096, 32), (dl.OP_W4A4, 14336, 8), (dl.OP_W4A4, 6144, 16)])
 def test_plan_matches_oracle_rules(opid, k, width):
-    cap = 32 if opid == dl.OP_W4A16 else 300
-    for rows in range(0, cap + 1):
+    for rows in range(0, 301):
         plan = dl.plan_chunks(opid, rows, k)
         ref = op.chunk_plan(rows, width)
         assert [(o, c) for o, c, _ in plan] == ref
@@ -57,7 +56,7 @@ def test_plan_matches_oracle_rules(opid, k, width):
 
 
 def test_plan_rejects():
-    assert L.dlmh_plan_chunks(dl.OP_W4A16, 33, 4096, None, None, None, 0) == -4
+    assert L.dlmh_plan_chunks(dl.OP_W4A16, 33, 4096, None, None, None, 0) == 3  # 16 + 16 + 1
     assert L.dlmh_plan_chunks(dl.OP_W8A16, -1, 5120, None, None, None, 0) == -4
     assert L.dlmh_plan_chunks(9, 1, 5120, None, None, None, 0) == -2
     # k % 128 != 0 keeps the register-fragment tiers, whose activation tile must fit on chip
@@ -107,7 +106,7 @@ def test_w8a8_argument_errors():
 
 def test_w4a16_argument_errors():
     f = L.w4a16_gemv
-    assert f(A, A, ctypes.c_float(1.0), 16, 128, A, 128, 33, A, 16, None) == -4
+    assert f(A, A, ctypes.c_float(1.0), 16, 128, A, 128, -1, A, 16, None) == -4
     assert f(A, A, ctypes.c_float(1.0), 16, 64, A, 128, 1, A, 16, None) == -2
     assert f(A, U, ctypes.c_float(1.0), 16, 128, A, 128, 1, A, 16, None) == -3
     assert f(A, None, ctypes.c_float(1.0), 16, 128, A, 128, 1, A, 16, None) == -1

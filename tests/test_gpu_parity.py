@@ -143,11 +143,26 @@ def test_w8a16_extreme_codes_and_row_magnitudes():
     x[5, 5] = 3.0e38                               # one huge value beside ordinary ones
     out = bits(dl.lm_head_fp8_w8a16(w, s, x))
     ref = og.w8a16_gemv(bits(w), bits(s), bits(x))
-    for m in range(6):
-        if m == 5:
-            continue  # |x| < 2^-31 amax for the ordinary values: outside the exactness range
+    for m in range(5):
         assert_bf16_close(out[m:m + 1], ref[m:m + 1], f"w8a16 extreme row {m}")
     assert not nx.bf16_decode(out[4]).any()
+    # Row 5: one 3e38 value among N(0,1) values.  k = 1024 takes the tensor-core path, whose
+    # two-term E4M3 split of a row is exact for |x| >= 2^-13 max|x| (here x[5, 5] alone) and
+    # may drop the rest (|x| <= 5 < 2^-13 * 3e38).  So, per output,
+    #   |got - ref| <= 2^-7 |ref| + s[n] * sum over the other k of |e4m3(w[n, k]) x[5, k]|,
+    # and where s[n] e4m3(w[n, 5]) 3e38 passes the BF16 range both sides round to the same
+    # infinity.
+    got5, ref5 = nx.bf16_decode(out[5]), nx.bf16_decode(ref[5])
+    wv = nx.e4m3_decode(bits(w)).astype(np.float64)
+    xv = nx.bf16_decode(bits(x)[5]).astype(np.float64)
+    small = np.abs(xv) < 2.0 ** -13 * np.abs(xv).max()
+    assert small.sum() == k - 1
+    dropped = bits(s).view(np.float32).astype(np.float64) * (np.abs(wv[:, small]) @ np.abs(xv[small]))
+    inf = np.isinf(ref5)
+    assert inf.any() and np.array_equal(got5[inf], ref5[inf])
+    fin = ~inf
+    assert np.all(np.isfinite(got5[fin]))
+    assert np.all(np.abs(got5[fin] - ref5[fin]) <= 2.0 ** -7 * np.abs(ref5[fin]) + dropped[fin])
 
 
 # ---------------------------------------------------------------------------
@@ -406,6 +421,68 @@ def test_q6k_wide_tiers_one_pass(n, k):
     fb[2:2 + blocks.numel()] = blocks.reshape(-1)
     bshift = fb[2:2 + blocks.numel()].view(blocks.shape)
     assert np.array_equal(bits(dl.q6k_mmvq(bshift, q8)), full[:40])
+    assert dl.device_fault(reset=True) == 0
+
+
+def test_q6k_kernel_element_map_hand_probes():
+    # The 15 hand-derived probe blocks of tests/golden/q6k_single_byte_probes.txt as the 15
+    # weight rows of a K = 256 matrix, against 256 one-hot q8_1 rows (row m: d = 1, code 1 at
+    # value m): out[m, n] is then value m of probe block n, exactly (every expected value is a
+    # BF16 integer).  Run through the wide kernel (64-row passes), the streamed 8-row kernel
+    # (q8 rows only 4-byte aligned) and the register kernel (blocks only 2-byte aligned).
+    from q6k_probes import load
+
+    probes = load()
+    n = len(probes)
+    blocks = torch.from_numpy(np.stack([b for _, b, _ in probes])[:, None, :].copy()).to(DEV)
+    want = np.stack([e for _, _, e in probes]).T                 # [256 values, n]
+    q8 = np.zeros((256, 8, 36), np.uint8)
+    for m in range(256):
+        q8[m, m // 32, 0:4] = (0x00, 0x3C, 0x00, 0x3C)         # d = 1.0, s = 1.0
+        q8[m, m // 32, 4 + m % 32] = 1
+    q8d = torch.from_numpy(q8).to(DEV)
+    got = {"wide": bits(dl.q6k_mmvq(blocks, q8d))}
+    flat = torch.zeros(q8d.numel() + 16, dtype=torch.uint8, device=DEV)
+    flat[4:4 + q8d.numel()] = q8d.reshape(-1)
+    got["streamed 8-row"] = bits(dl.q6k_mmvq(blocks, flat[4:4 + q8d.numel()].view(q8d.shape)))
+    fb = torch.zeros(blocks.numel() + 16, dtype=torch.uint8, device=DEV)
+    fb[2:2 + blocks.numel()] = blocks.reshape(-1)
+    got["register 8-row"] = bits(dl.q6k_mmvq(fb[2:2 + blocks.numel()].view(blocks.shape), q8d))
+    for kind, g in got.items():
+        v = nx.bf16_decode(g)
+        bad = np.argwhere(v != want)
+        assert bad.size == 0, (f"{kind}: (value, probe) {bad[:6].tolist()} got {v[tuple(bad[:6].T)].tolist()} "
+                               f"want {want[tuple(bad[:6].T)].tolist()} ({probes[bad[0][1]][0]})")
+    assert dl.device_fault(reset=True) == 0
+
+
+def test_q6k_two_passes_128_rows():
+    # 128 rows: two 64-row weight passes; the oracle on every output, and row invariance
+    # against one 64-row pass of each half
+    n, k = 1000, 7168
+    blocks = synth.q6k_blocks(n, k, 8, DEV)
+    x = synth.bf16_rows(128, k, 8, DEV)
+    full = bits(dl.q6k_lm_head(blocks, x))
+    ref = og.q6k_mmvq(bits(blocks), og.q8_1_quantize_rows(bits(x)))
+    assert_bf16_close(full, ref, "q6k M=128")
+    assert np.array_equal(bits(dl.q6k_lm_head(blocks, x[:64])), full[:64])
+    assert np.array_equal(bits(dl.q6k_lm_head(blocks, x[64:])), full[64:])
+    for m in (65, 100):
+        assert np.array_equal(bits(dl.q6k_lm_head(blocks, x[:m])), full[:m]), f"row invariance M={m}"
+    assert dl.device_fault(reset=True) == 0
+
+
+@pytest.mark.parametrize("n,k", [(14336, 4096), (300, 1024)])
+def test_w4a16_above_32_rows(n, k):
+    # every M in 1..128: passes of at most 32 rows (one w4a16_gemv_tiers kernel_within-sized
+    # launch each); the oracle on every output at M = 128, row invariance at 33 and 64
+    wp, ws, gl = synth.nvfp4_weight(n, k, 21, DEV)
+    x = synth.bf16_rows(128, k, 21, DEV)
+    full = bits(dl.w4a16_gemv(wp, ws, gl, x))
+    ref = og.w4a16_gemv(bits(wp), bits(ws), np.float32(gl), bits(x))
+    assert_bf16_close(full, ref, f"w4a16 {n}x{k} M=128")
+    for m in (1, 32, 33, 64):
+        assert np.array_equal(bits(dl.w4a16_gemv(wp, ws, gl, x[:m])), full[:m]), f"row invariance M={m}"
     assert dl.device_fault(reset=True) == 0
 
 

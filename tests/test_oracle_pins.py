@@ -526,6 +526,79 @@ def test_q6k_mmvq_brute_force_exact():
             _assert_correctly_rounded_bf16(r, out[m, n])
 
 
+def _q6k_values(blocks, unpack=og.q6k_unpack):
+    q, sc, d = unpack(blocks)
+    return d[..., None] * np.repeat(sc, 16, axis=-1) * (q - 32)
+
+
+def test_q6k_element_map_hand_probes():
+    # tests/golden/q6k_single_byte_probes.txt: one byte (or a few) set at a time, the 256
+    # expected values derived by hand from the public GGUF Q6_K layout; every nibble, qh bit
+    # pair, half, scale index and the position of d is probed
+    from q6k_probes import load
+
+    probes = load()
+    assert len(probes) == 15
+    for name, blk, exp in probes:
+        got = _q6k_values(blk[None])[0]
+        bad = np.flatnonzero(got != exp)
+        assert bad.size == 0, f"{name}: elements {bad[:8].tolist()} got {got[bad[:8]].tolist()}"
+
+
+def _gguf_q6k():
+    gq = pytest.importorskip("gguf.quants")
+    from gguf import GGMLQuantizationType
+
+    return lambda b: gq.dequantize(np.ascontiguousarray(b, np.uint8), GGMLQuantizationType.Q6_K)
+
+
+def test_q6k_element_map_matches_gguf_library():
+    # gguf.quants is an independent implementation of the public Q6_K block format (a library
+    # routine).  Its float32 result is d * sc * (q - 32) rounded once (d*sc is exact in f32),
+    # so the oracle's float64 value rounded to f32 must equal it bit for bit.  Blocks: every
+    # byte value in ql and qh, every int8 scale, several d.
+    deq = _gguf_q6k()
+    rng = np.random.default_rng(16)
+    b = rng.integers(0, 256, (256, 210)).astype(np.uint8)
+    b[:, 0] = np.arange(256)                       # every ql byte value (low/high nibble pairs)
+    b[:, 128] = np.arange(256)[::-1]               # every qh byte value (all bit pairs)
+    b[:, 192] = np.arange(256)                     # every int8 scale
+    d = np.concatenate([rng.uniform(1e-4, 1e-3, 200), rng.uniform(0.5, 4.0, 56)])
+    b[:, 208:210] = np.frombuffer(np.float16(d).tobytes(), np.uint8).reshape(256, 2)
+    ref = deq(b)
+    got = _q6k_values(b).astype(np.float32)
+    assert ref.shape == got.shape == (256, 256)
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+    # the hand probes agree with the library too
+    from q6k_probes import load
+
+    for name, blk, exp in load():
+        assert np.array_equal(deq(blk[None])[0].astype(np.float64), exp), name
+
+
+def test_q6k_element_map_pins_catch_a_nibble_swap():
+    # a plausible slip: values 32..63 of each half from the high nibble of ql[64h + l] and
+    # values 64..95 from the low nibble of ql[64h + 32 + l] (t = 1 and t = 2 swapped).  Both
+    # pins above must reject it.
+    def swapped_unpack(blocks):
+        q, sc, d = og.q6k_unpack(blocks)
+        q2 = q.copy()
+        for h in range(2):
+            o = 128 * h
+            q2[..., o + 32:o + 64], q2[..., o + 64:o + 96] = q[..., o + 64:o + 96], q[..., o + 32:o + 64]
+        return q2, sc, d
+
+    from q6k_probes import load
+
+    probes = load()
+    assert any(not np.array_equal(_q6k_values(blk[None], swapped_unpack)[0], exp) for _, blk, exp in probes)
+    deq = _gguf_q6k()
+    rng = np.random.default_rng(17)
+    b = rng.integers(0, 256, (8, 210)).astype(np.uint8)
+    b[:, 208:210] = np.frombuffer(np.float16(np.full(8, 1e-3)).tobytes(), np.uint8).reshape(8, 2)
+    assert not np.array_equal(_q6k_values(b, swapped_unpack).astype(np.float32), deq(b))
+
+
 def test_row_invariance_all_formats():
     rng = np.random.default_rng(15)
     N, K, M = 8, 256, 5
