@@ -39,6 +39,9 @@ SPEC_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 
 
+ROWS_PER_PASS = 128  # one tensor-core weight pass serves up to 128 rows at k % 128 == 0
+
+
 def passes(m):
     """Weight passes of one lm_head_fp8_w8a16 call at m rows (the library's own plan)."""
     import decode_lm_head_b200 as dl
@@ -46,21 +49,32 @@ def passes(m):
     return len(dl.plan_chunks(dl.OP_W8A16, m, HIDDEN))
 
 
-def launches_per_call(m, sms):
-    """Kernels one call launches: per pass the activation split, the GEMV and, when the
-    stream-K schedule has a remainder (tiles not a multiple of the SM count), the fixup."""
-    ntiles = -(-VOCAB // 128)
+def oracle_passes(m):
+    """The same count for the CPU legs, from the oracle's chunk rule (no product library)."""
+    from oracle import plan as op
+
+    return len(op.chunk_plan(m, ROWS_PER_PASS))
+
+
+def launches_per_call(m, sms, n):
+    """Kernels one call launches on an n-row head: per pass the activation split, the GEMV
+    and, when the stream-K schedule has a remainder (tiles not a multiple of the SM count),
+    the fixup."""
+    ntiles = -(-n // 128)
     rem = ntiles % sms if ntiles >= sms else ntiles
     return passes(m) * (2 + (1 if rem else 0))
 
 
-def weight_bytes():
-    return VOCAB * HIDDEN + VOCAB * 4
+def weight_bytes(n=None):
+    n = VOCAB if n is None else n
+    return n * HIDDEN + n * 4
 
 
-def algo_bytes(m):
-    """Algorithmic bytes of one call at m rows: weight+scales per pass, x once, logits once."""
-    return passes(m) * weight_bytes() + m * HIDDEN * 2 + m * VOCAB * 2
+def algo_bytes(m, n=None):
+    """Algorithmic bytes of one call at m rows on an n-row head: weight+scales per pass, x
+    once, logits once."""
+    n = VOCAB if n is None else n
+    return passes(m) * weight_bytes(n) + m * HIDDEN * 2 + m * n * 2
 
 
 def measured_peaks():
@@ -119,14 +133,19 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index):
+    def __init__(self, gpu_index, path=None):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+        self.keep = path is not None
+        if path is None:
+            import tempfile
+
+            fd, path = tempfile.mkstemp(prefix=f"dlmh_clocks_rank{gpu_index}_", suffix=".csv")
+            os.close(fd)
+        self.path = path
 
     def __enter__(self):
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
                                           "--format=csv,noheader,nounits", "-lms", "100"],
@@ -163,6 +182,11 @@ class ClockSampler:
                 for name, v in zip(names, parts[5:9]):
                     if v.lower() == "active":
                         reasons.add(name)
+        if not self.keep:
+            try:
+                os.remove(self.path)
+            except OSError:
+                pass
         if not sms:
             return None
         return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxs), "samples": len(sms),
@@ -233,7 +257,7 @@ def oracle_sample(rows_sample=32768, seed=1):
     nbytes = 0
     for m in ROWS:
         og.w8a16_gemv(w, s, x[:m])
-        nbytes += passes(m) * rows_sample * (HIDDEN + 4)
+        nbytes += oracle_passes(m) * rows_sample * (HIDDEN + 4)
     dt = time.perf_counter() - t0
     desc = f"{rows_sample} of {VOCAB} vocab rows x {HIDDEN}, M in {list(ROWS)}, float64 numpy oracle"
     return nbytes / dt / 1e9, dt, desc
@@ -266,7 +290,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(1e3 * statistics.median(d for _, d in times), 3),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": f"FP8 E4M3 LM head W8A16 {VOCAB}x{HIDDEN}, M in {list(ROWS)}",
                    "rows_per_step": list(ROWS), "sample_vocab_rows": sample_rows},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cpu_threads(), "kind": "oracle",
@@ -282,8 +306,8 @@ def run_reference(args):
 
 
 def time_calls(fns, reps, stream):
-    """Median device time (us) of each callable, by CUDA events on `stream`; each callable is
-    replayed `reps` times back to back (its inputs rotate inside the callable)."""
+    """Mean device time (us) per call of each callable, by CUDA events on `stream` around
+    `reps` back-to-back calls after 3 warm-ups (its inputs rotate inside the callable)."""
     out = []
     for fn in fns:
         for _ in range(3):
@@ -299,9 +323,23 @@ def time_calls(fns, reps, stream):
     return out
 
 
+def bind_workspace(dl, stream, device, shapes):
+    """One caller workspace for every tensor-core call the bench makes on `stream` (the
+    largest dlmh_workspace_bytes over `shapes` = [(op, n, k, rows)]), bound to the stream:
+    no call in the timed regions allocates."""
+    need = max([dl.workspace_bytes(op, n, k, rows) for op, n, k, rows in shapes] + [256])
+    buf = torch.empty(need + 256, dtype=torch.uint8, device=device)
+    off = (-buf.data_ptr()) % 256
+    ws = buf[off:off + need]
+    dl.set_workspace(ws, stream=stream)
+    return buf
+
+
 def other_formats(dev, stream, peak):
-    """Weight GB/s of the other hot-path formats (secondary measurements, same protocol:
-    inputs resident, weights rotated through enough copies to exceed the 126 MB L2)."""
+    """Every other hot-path format (same protocol: inputs resident, weights rotated through
+    enough copies to exceed the 126 MB L2).  Per row count: device time per call, weight
+    GB/s, algorithmic GB/s (weight + scales + activations read + outputs written, one count
+    per weight pass) and its fraction of the measured copy peak."""
     import decode_lm_head_b200 as dl
     from decode_lm_head_b200 import synth
 
@@ -311,13 +349,17 @@ def other_formats(dev, stream, peak):
         copies = max(1, -(-400_000_000 // nbytes))  # >= 400 MB of distinct weights
         return [make(i) for i in range(copies)]
 
-    def entry(name, shape, wbytes, calls, rows_list):
+    def entry(name, shape, wbytes, calls, rows_list, algo, passes_of=lambda m: 1, note=None):
         per = {}
         for m, fn in zip(rows_list, calls):
             us = time_calls([fn], 20, stream)[0]
-            gbs = wbytes / (us * 1e-6) / 1e9
-            per[str(m)] = {"us": round(us, 2), "weight_gbs": round(gbs, 1), "frac_of_copy_peak": round(gbs / peak, 3)}
+            gbs = passes_of(m) * wbytes / (us * 1e-6) / 1e9
+            agbs = algo(m) / (us * 1e-6) / 1e9
+            per[str(m)] = {"us": round(us, 2), "weight_gbs": round(gbs, 1), "algo_gbs": round(agbs, 1),
+                           "frac": round(agbs / peak, 3), "passes": passes_of(m)}
         res[name] = {"shape": shape, "weight_bytes": wbytes, "per_m": per}
+        if note:
+            res[name]["note"] = note
 
     # W8A8 on the FP8 head (one tensor-core pass for up to 128 rows)
     n, k = VOCAB, HIDDEN
@@ -327,12 +369,13 @@ def other_formats(dev, stream, peak):
     xq = torch.empty(128 * k, dtype=torch.uint8, device=dev)
     xs = torch.empty(128, dtype=torch.float32, device=dev)
     outs = torch.empty(128, n, dtype=torch.bfloat16, device=dev)
-    rows_list = [1, 8, 16, 32, 64, 128]
+    rows_list = [1, 2, 4, 8, 16, 32, 64, 128]
     # views are cut once, outside the timed calls (slicing costs host time per call)
     calls = [(lambda xm=x[:m], om=outs[:m]: dl.w8a8_proj(w, s_, xm, out=om, xq_scratch=xq, xscale_scratch=xs,
                                                          stream=stream))
              for m in rows_list]
-    entry("w8a8_head", f"{n}x{k}", n * k + 4 * n, calls, rows_list)
+    entry("w8a8_head", f"{n}x{k}", n * k + 4 * n, calls, rows_list,
+          lambda m: n * k + 4 * n + 2 * m * k + 2 * m * n)
     del w
 
     # W8A8 FFN down projection from bf16(silu(gate)*up)
@@ -343,7 +386,8 @@ def other_formats(dev, stream, peak):
     xq = torch.empty(128 * k, dtype=torch.uint8, device=dev)
     outd = torch.empty(128, n, dtype=torch.bfloat16, device=dev)
     ctr = [0]
-    views = {m: (gate[:m], up[:m], outd[:m]) for m in (1, 16, 128)}
+    rows_list = [1, 4, 16, 64, 128]
+    views = {m: (gate[:m], up[:m], outd[:m]) for m in rows_list}
 
     def down(m):
         w_, s2 = ws[ctr[0] % len(ws)]
@@ -351,12 +395,11 @@ def other_formats(dev, stream, peak):
         g, u, o = views[m]
         dl.w8a8_silu_proj(w_, s2, g, u, out=o, xq_scratch=xq, xscale_scratch=xs, stream=stream)
 
-    rows_list = [1, 16, 128]
-    entry("w8a8_silu_down", f"{n}x{k}", n * k + 4 * n, [(lambda m=m: down(m)) for m in rows_list], rows_list)
+    entry("w8a8_silu_down", f"{n}x{k}", n * k + 4 * n, [(lambda m=m: down(m)) for m in rows_list], rows_list,
+          lambda m: n * k + 4 * n + 4 * m * k + 2 * m * n)
     del ws
 
-    # W8A8 FFN gate + up on one quantized x (one launch over both weights), against the same
-    # two projections as two w8a8_proj calls
+    # W8A8 FFN gate + up on one quantized x (one launch over both weights)
     n, k = 14336, 4096
     pairs = rotating(lambda i: (synth.fp8_weight(n, k, 50 + i, dev, tensor_id=1), synth.row_scales(n, 50 + i, dev),
                                 synth.fp8_weight(n, k, 50 + i, dev, tensor_id=6),
@@ -368,30 +411,25 @@ def other_formats(dev, stream, peak):
     rows_list = [1, 16, 128]
     gviews = {m: (xg[:m], og_[:m], ou_[:m]) for m in rows_list}
 
-    def gate_up(m, paired):
+    def gate_up(m):
         wg, sg, wu, su = pairs[ctr[0] % len(pairs)]
         ctr[0] += 1
         xm, gm, um = gviews[m]
-        if paired:
-            dl.w8a8_gate_up_proj(wg, sg, wu, su, xm, gate_out=gm, up_out=um, xq_scratch=xq, xscale_scratch=xs,
-                                 stream=stream)
-        else:
-            dl.w8a8_proj(wg, sg, xm, out=gm, xq_scratch=xq, xscale_scratch=xs, stream=stream)
-            dl.w8a8_proj(wu, su, xm, out=um, xq_scratch=xq, xscale_scratch=xs, stream=stream)
+        dl.w8a8_gate_up_proj(wg, sg, wu, su, xm, gate_out=gm, up_out=um, xq_scratch=xq, xscale_scratch=xs,
+                             stream=stream)
 
-    for name, paired in (("w8a8_gate_up_pair", True), ("w8a8_gate_up_two_calls", False)):
-        entry(name, f"2x{n}x{k}", 2 * (n * k + 4 * n), [(lambda m=m, p=paired: gate_up(m, p)) for m in rows_list],
-              rows_list)
+    entry("w8a8_gate_up_pair", f"2x{n}x{k}", 2 * (n * k + 4 * n), [(lambda m=m: gate_up(m)) for m in rows_list],
+          rows_list, lambda m: 2 * (n * k + 4 * n) + 2 * m * k + 4 * m * n)
     del pairs
 
-    # NVFP4 W4A16
+    # NVFP4 W4A16 (passes of at most 32 rows, narrower where the activation tile does not fit)
     n, k = 14336, 4096
     wf = rotating(lambda i: synth.nvfp4_weight(n, k, 20 + i, dev), n * k // 2)
-    xf = synth.bf16_rows(32, k, 4, dev)
-    outf = torch.empty(32, n, dtype=torch.bfloat16, device=dev)
-
-    rows_list = [1, 4, 8, 16, 32]
+    xf = synth.bf16_rows(128, k, 4, dev)
+    outf = torch.empty(128, n, dtype=torch.bfloat16, device=dev)
+    rows_list = [1, 4, 5, 6, 7, 8, 16, 32, 64, 128]
     fviews = {m: (xf[:m], outf[:m]) for m in rows_list}
+    wbytes4 = n * k // 2 + n * k // 16
 
     def fp4(m):
         wp, sc, gl = wf[ctr[0] % len(wf)]
@@ -399,10 +437,12 @@ def other_formats(dev, stream, peak):
         xm, om = fviews[m]
         dl.w4a16_gemv(wp, sc, gl, xm, out=om, stream=stream)
 
-    entry("nvfp4_w4a16", f"{n}x{k}", n * k // 2 + n * k // 16, [(lambda m=m: fp4(m)) for m in rows_list], rows_list)
+    p16 = {m: len(dl.plan_chunks(dl.OP_W4A16, m, k)) for m in rows_list}
+    entry("nvfp4_w4a16", f"{n}x{k}", wbytes4, [(lambda m=m: fp4(m)) for m in rows_list], rows_list,
+          lambda m: p16[m] * wbytes4 + 2 * m * k + 2 * m * n, passes_of=lambda m: p16[m])
 
     # NVFP4 W4A4: the same weights against per-row NVFP4-quantized activations (quantize + GEMV)
-    rows_list = [1, 8, 16, 32]
+    rows_list = [1, 8, 16, 32, 64]
     xq4 = torch.empty(32 * k // 2, dtype=torch.uint8, device=dev)
     xs4 = torch.empty(32 * k // 16, dtype=torch.uint8, device=dev)
     xg4 = torch.empty(32, dtype=torch.float32, device=dev)
@@ -413,7 +453,9 @@ def other_formats(dev, stream, peak):
         xm, om = fviews[m]
         dl.w4a4_proj(wp, sc, gl, xm, out=om, xq_scratch=xq4, xs_scratch=xs4, xg_scratch=xg4, stream=stream)
 
-    entry("nvfp4_w4a4", f"{n}x{k}", n * k // 2 + n * k // 16, [(lambda m=m: fp4a4(m)) for m in rows_list], rows_list)
+    p44 = {m: len(dl.plan_chunks(dl.OP_W4A4, m, k)) for m in rows_list}
+    entry("nvfp4_w4a4", f"{n}x{k}", wbytes4, [(lambda m=m: fp4a4(m)) for m in rows_list], rows_list,
+          lambda m: p44[m] * wbytes4 + 2 * m * k + 2 * m * n, passes_of=lambda m: p44[m])
     del wf
 
     # load-time NVFP4 / E8M0 dequant to BF16 (HBM stream: codes + scales in, BF16 out)
@@ -437,22 +479,60 @@ def other_formats(dev, stream, peak):
         nbytes = n * k // 2 + sbytes + 2 * n * k
         gbs = nbytes / (us * 1e-6) / 1e9
         res[name] = {"shape": f"{n}x{k}", "bytes_per_call": nbytes,
-                     "per_call": {"us": round(us, 2), "gbs": round(gbs, 1), "frac_of_copy_peak": round(gbs / peak, 3)}}
+                     "per_call": {"us": round(us, 2), "algo_gbs": round(gbs, 1), "frac": round(gbs / peak, 3)}}
     del wq, e8
 
-    # Q6_K head
+    # Q6_K head (q8_1 quantize + one weight pass per 64 rows)
     n, k = 129280, 7168
     blocks = synth.q6k_blocks(n, k, 4, dev)
-    xk = synth.bf16_rows(64, k, 4, dev)
+    xk = synth.bf16_rows(128, k, 4, dev)
     q8s = torch.empty(64 * (k // 32) * 36, dtype=torch.uint8, device=dev)  # one pass per 64 rows
-    outk = torch.empty(64, n, dtype=torch.bfloat16, device=dev)
-    rows_list = [1, 8, 16, 32, 64]
+    outk = torch.empty(128, n, dtype=torch.bfloat16, device=dev)
+    rows_list = [1, 2, 4, 8, 16, 32, 64, 128]
+    wq6 = n * (k // 256) * 210
     calls = [(lambda xm=xk[:m], om=outk[:m]: dl.q6k_lm_head(blocks, xm, out=om, q8_scratch=q8s, stream=stream))
              for m in rows_list]
-    entry("q6k_head", f"{n}x{k}", n * (k // 256) * 210, calls, rows_list)
+    pq = {m: len(dl.plan_chunks(dl.OP_Q6K, m, k)) for m in rows_list}
+    entry("q6k_head", f"{n}x{k}", wq6, calls, rows_list, lambda m: pq[m] * wq6 + 2 * m * k + 2 * m * n,
+          passes_of=lambda m: pq[m])
     del blocks
     torch.cuda.synchronize()
     return res
+
+
+def oracle_single_thread():
+    """The oracle on ONE host thread (BLAS limited to 1), on the tiny FP8 config (all of it)
+    and on a 2048-row sample of the NVFP4 W4A16 config; weight GB/s per call."""
+    from threadpoolctl import threadpool_limits
+
+    from decode_lm_head_b200 import synth
+    from oracle import gemv as og
+
+    out = {}
+    with threadpool_limits(limits=1):
+        n, k = 8192, 1024
+        w = synth.to_numpy_bits(synth.fp8_weight(n, k, 0))
+        s = synth.to_numpy_bits(synth.row_scales(n, 0))
+        x = synth.to_numpy_bits(synth.bf16_rows(4, k, 0))
+        t0 = time.perf_counter()
+        for m in (1, 2, 3, 4):
+            og.w8a16_gemv(w, s, x[:m])
+        dt = time.perf_counter() - t0
+        out["tiny_fp8_w8a16"] = {"value": round(4 * n * (k + 4) / dt / 1e9, 5), "unit": "GB/s", "cores": 1,
+                                 "seconds": round(dt, 2), "sample": f"all of {n}x{k}, M in 1..4"}
+        n, k, rows = 14336, 4096, 2048
+        wp, sc, gl = synth.nvfp4_weight(n, k, 20)
+        wp, sc = synth.to_numpy_bits(wp[:rows]), synth.to_numpy_bits(sc[:rows])
+        xf = synth.to_numpy_bits(synth.bf16_rows(32, k, 4))
+        ms = (1, 4, 5, 6, 7, 8, 16, 32)
+        t0 = time.perf_counter()
+        for m in ms:
+            og.w4a16_gemv(wp, sc, np.float32(gl), xf[:m])
+        dt = time.perf_counter() - t0
+        out["nvfp4_w4a16"] = {"value": round(len(ms) * rows * (k // 2 + k // 16) / dt / 1e9, 5), "unit": "GB/s",
+                              "cores": 1, "seconds": round(dt, 2),
+                              "sample": f"{rows} of {n} rows x {k}, M in {list(ms)}"}
+    return out
 
 
 def profile_q6k(n):
@@ -476,23 +556,46 @@ def profile_q6k(n):
 def run_ours(args):
     world, rank, local = dist_setup(args)
     import decode_lm_head_b200 as dl
-    from decode_lm_head_b200 import synth
+    from decode_lm_head_b200 import shard, synth
 
     dl.lib()
     dev = torch.device("cuda", local)
-    seed = 1 + rank
-    w = synth.fp8_weight(VOCAB, HIDDEN, seed, dev)
-    s = synth.row_scales(VOCAB, seed, dev)
-    x = synth.bf16_rows(max(ROWS), HIDDEN, seed, dev, std=0.5)
-    outs = {m: torch.empty(m, VOCAB, dtype=torch.bfloat16, device=dev) for m in ROWS}
+    # This rank's stripe of the head: the whole head on one GPU, a vocab stripe on several
+    a, b = shard.stripe(VOCAB, world, rank)
+    ns, S = b - a, shard.stripe_width(VOCAB, world)
+    w = synth.fp8_weight(ns, HIDDEN, 1 + rank, dev)
+    s = synth.row_scales(ns, 1 + rank, dev)
+    x = synth.bf16_rows(max(ROWS), HIDDEN, 1, dev, std=0.5)  # the activation rows, the same on every rank
     stream = torch.cuda.current_stream(dev)
+    ws_keep = bind_workspace(dl, stream, dev, [(dl.OP_W8A16, ns, HIDDEN, max(ROWS))] + (
+        [(dl.OP_W8A8, VOCAB, HIDDEN, 128), (dl.OP_W8A8, 4096, 14336, 128), (dl.OP_W8A8_PAIR, 14336, 4096, 128)]
+        if world == 1 and not args.no_formats else []))
+    # logits of each call, [m, S] (a short last stripe keeps zero padding), double-buffered so
+    # that a step's GEMV never writes a buffer the previous step's all-gather still reads
+    outs = {m: [torch.zeros(m, S, dtype=torch.bfloat16, device=dev) for _ in range(2)] for m in ROWS}
+    views = {m: [o[:, :ns] for o in outs[m]] for m in ROWS}
+    xs = {m: x[:m] for m in ROWS}
+    comm = torch.cuda.Stream(dev) if world > 1 else None
+    gathered = {m: shard.gather_buffer(m, VOCAB, world, dev) for m in ROWS} if world > 1 else None
+    released = {m: [None, None] for m in ROWS}
 
-    def step():
+    def step(parity):
         for m in ROWS:
-            dl.lm_head_fp8_w8a16(w, s, x[:m], out=outs[m], stream=stream)
+            if released[m][parity] is not None:
+                stream.wait_event(released[m][parity])
+            dl.lm_head_fp8_w8a16(w, s, xs[m], out=views[m][parity], stream=stream)
+            if world > 1:  # the exchange: every rank's stripe of these logits to every rank
+                done = torch.cuda.Event()
+                done.record(stream)
+                comm.wait_event(done)
+                with torch.cuda.stream(comm):
+                    shard.all_gather_stripes(outs[m][parity], gathered[m])
+                ev = torch.cuda.Event()
+                ev.record(comm)
+                released[m][parity] = ev
 
-    for _ in range(args.warmup):
-        step()
+    for i in range(args.warmup):
+        step(i & 1)
     torch.cuda.synchronize()
 
     # ---- device-timed region (inputs resident)
@@ -500,12 +603,14 @@ def run_ours(args):
     # each call's pre-pass may launch behind the previous call's last kernel); the per-call
     # breakdown comes from a separate pass with events around every call.
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clk:
+    with ClockSampler(local, args.clock_log) as clk:
         barrier(world)
         torch.cuda.synchronize()
         ev0.record(stream)
-        for _ in range(args.steps):
-            step()
+        for i in range(args.steps):
+            step(i & 1)
+        if comm is not None:
+            stream.wait_stream(comm)
         ev1.record(stream)
         torch.cuda.synchronize()
         barrier(world)
@@ -515,51 +620,54 @@ def run_ours(args):
     per_m_events = {m: [] for m in ROWS}
     for _ in range(args.steps):
         for m in ROWS:
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            dl.lm_head_fp8_w8a16(w, s, x[:m], out=outs[m], stream=stream)
-            b.record(stream)
-            per_m_events[m].append((a, b))
+            e_a, e_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e_a.record(stream)
+            dl.lm_head_fp8_w8a16(w, s, xs[m], out=views[m][0], stream=stream)
+            e_b.record(stream)
+            per_m_events[m].append((e_a, e_b))
     torch.cuda.synchronize()
 
-    step_bytes = sum(passes(m) * weight_bytes() for m in ROWS)
-    value = job_value(world, args.steps, step_bytes, elapsed_ms)
+    # whole-job bytes: every rank streams its stripe once per pass, i.e. the whole head
+    step_bytes = sum(passes(m) * weight_bytes(VOCAB) for m in ROWS)
+    value = args.steps * step_bytes / (elapsed_ms * 1e-3) / 1e9
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     passes_per_step = sum(passes(m) for m in ROWS)
-    launches_per_step = sum(launches_per_call(m, sms) for m in ROWS)
-    rows_nk = world * args.steps * sum(ROWS) * VOCAB * HIDDEN / (elapsed_ms * 1e-3)
+    launches_per_step = sum(launches_per_call(m, sms, ns) for m in ROWS)
+    rows_nk = args.steps * sum(ROWS) * VOCAB * HIDDEN / (elapsed_ms * 1e-3)
     per_m = {}
     for m in ROWS:
-        us = statistics.median(a.elapsed_time(b) for a, b in per_m_events[m]) * 1e3
-        per_m[str(m)] = {"us": round(us, 2), "weight_gbs": round(passes(m) * weight_bytes() / (us * 1e-6) / 1e9, 1),
+        us = statistics.median(e_a.elapsed_time(e_b) for e_a, e_b in per_m_events[m]) * 1e3
+        per_m[str(m)] = {"us": round(us, 2), "weight_gbs": round(passes(m) * weight_bytes(ns) / (us * 1e-6) / 1e9, 1),
                          "passes": passes(m)}
 
     peak, peak_kind = measured_peaks()
-    algo = sum(algo_bytes(m) for m in ROWS)
+    algo = sum(algo_bytes(m, ns) for m in ROWS)
     achieved = args.steps * algo / (elapsed_ms * 1e-3) / 1e9  # per rank: this rank's kernels only
-    traffic = ncu_traffic()
+    traffic = ncu_traffic() if world == 1 else None
 
     # ---- end to end through the public API, host buffers, copies inside the region.  Each
-    # call's logits go back to pinned host memory on a copy stream while the next call
-    # computes (the way a serving loop overlaps them); outputs are double-buffered per M, a
-    # call waits for the copy that last read its buffer, and the region ends after the last
-    # copy has landed.  The step's calls are the same as in the device-timed loop.
+    # call's logits (this rank's stripe) go back to pinned host memory on a copy stream while
+    # the next call computes (the way a serving loop overlaps them); outputs are
+    # double-buffered per M, a call waits for the copy that last read its buffer, and the
+    # region ends after the last copy has landed.  The step's calls are the same as in the
+    # device-timed loop.
     xh = x.cpu().pin_memory()
-    outh = {m: torch.empty(m, VOCAB, dtype=torch.bfloat16).pin_memory() for m in ROWS}
-    outd = {m: [outs[m], torch.empty_like(outs[m])] for m in ROWS}
+    outh = {m: torch.empty(m, ns, dtype=torch.bfloat16).pin_memory() for m in ROWS}
+    outd = {m: [torch.empty(m, ns, dtype=torch.bfloat16, device=dev) for _ in range(2)] for m in ROWS}
     xd = torch.empty_like(x)
+    xdv = {m: xd[:m] for m in ROWS}
     copy_stream = torch.cuda.Stream(dev)
     copied = {m: [None, None] for m in ROWS}
 
     def e2e_step(parity):
-        # the widest call first: its 64 MB of logits cross the host link while the other
-        # calls compute, and the step ends on the smallest copy
+        # the widest call first: its logits cross the host link while the other calls
+        # compute, and the step ends on the smallest copy
         for m in sorted(ROWS, reverse=True):
             buf = outd[m][parity]
             if copied[m][parity] is not None:
                 stream.wait_event(copied[m][parity])
-            xd[:m].copy_(xh[:m], non_blocking=True)
-            dl.lm_head_fp8_w8a16(w, s, xd[:m], out=buf, stream=stream)
+            xdv[m].copy_(xh[:m], non_blocking=True)
+            dl.lm_head_fp8_w8a16(w, s, xdv[m], out=buf, stream=stream)
             done = torch.cuda.Event()
             done.record(stream)
             copy_stream.wait_event(done)
@@ -582,30 +690,34 @@ def run_ours(args):
     torch.cuda.synchronize()
     barrier(world)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-    e2e_value = job_value(world, args.steps, step_bytes, e2e_ms)
+    e2e_value = args.steps * step_bytes / (e2e_ms * 1e-3) / 1e9
 
     formats = None
-    if args.all_formats:
-        formats = other_formats(dev, stream, measured_peaks()[0])
+    if world == 1 and not args.no_formats:
+        formats = other_formats(dev, stream, peak)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         gbs, dt, desc = oracle_sample()
         cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": cpu_threads(), "kind": "oracle",
-               "sample": f"{desc}; {dt:.1f} s"}
+               "sample": f"{desc}; {dt:.1f} s", "single_thread": oracle_single_thread()}
 
     if rank == 0:
+        parallelism = ("one GPU, the whole head" if world == 1 else
+                       f"vocab-sharded head: {world} stripes of {S} rows, NCCL all-gather of the BF16 logits"
+                       " overlapped with the next call")
         line = {
             "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(elapsed_ms / args.steps, 4), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None,
+            "scaling": "strong", "vs_baseline": None,
             "dtype": "e4m3 x e4m3 tcgen05 MMA, f32 accumulation (bf16 rows split exactly into two e4m3 terms)",
             "data": "synthetic (seeded; E4M3 of clamp(N(0,1)*64), scales U[1e-3,4e-3], x bf16 N(0,1)*0.5)",
             "config": {"workload": f"FP8 E4M3 LM head W8A16 {VOCAB}x{HIDDEN} ({VOCAB * HIDDEN / 1e9:.2f} GB),"
                                    " one call per M",
                        "rows_per_step": list(ROWS), "weight_passes_per_step": passes_per_step,
-                       "rows_per_pass": 128, "l2": "weight 1.27 GB > 126 MB L2: no flush needed",
-                       "parallelism": f"replica per GPU (vocab-shard layout), {world} rank(s)"},
+                       "rows_per_pass": ROWS_PER_PASS, "l2": "weight 1.27 GB > 126 MB L2: no flush needed",
+                       "workspace": "caller workspace bound to the stream (no allocation in the timed region)",
+                       "parallelism": parallelism},
             "hbm_fraction": {"of_measured_copy": round(value / world / peak, 4),
                              "of_spec_8tbs": round(value / world / SPEC_HBM_GBS, 4),
                              "of_measured_read": round(value / world / read_peak, 4),
@@ -621,7 +733,7 @@ def run_ours(args):
                          "algorithmic_bytes_per_step": algo},
             "e2e": {"value": round(e2e_value, 1), "unit": "GB/s",
                     "h2d_bytes_per_step": sum(m * HIDDEN * 2 for m in ROWS),
-                    "d2h_bytes_per_step": sum(m * VOCAB * 2 for m in ROWS)},
+                    "d2h_bytes_per_step": sum(m * ns * 2 for m in ROWS)},
             "gpu_launches": args.steps * launches_per_step,
             "clocks": clocks,
             "cpu_baseline": cpu,
@@ -629,6 +741,8 @@ def run_ours(args):
         if formats is not None:
             line["formats"] = formats
         print(json.dumps(line), flush=True)
+    dl.set_workspace(None, stream=stream)
+    del ws_keep
     if world > 1:
         import torch.distributed as dist
 
@@ -642,8 +756,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--all-formats", action="store_true",
-                    help="also time W8A8 (head, SiLU down), NVFP4 and Q6_K (extra 'formats' key)")
+    ap.add_argument("--no-formats", action="store_true",
+                    help="skip the other formats (W8A8, NVFP4 W4A16/W4A4, Q6_K, dequant) in the 'formats' key")
+    ap.add_argument("--clock-log", default=None,
+                    help="keep the nvidia-smi clock samples of the timed region in this file")
     ap.add_argument("--vocab", type=int, default=248320,
                     help="head rows; smaller values only for profiling captures (the workload is 248320)")
     ap.add_argument("--profile-q6k", type=int, default=0, metavar="N",

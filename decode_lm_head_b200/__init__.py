@@ -11,6 +11,7 @@ from ._lib import (  # noqa: F401
     OP_W4A4,
     OP_W4A16,
     OP_W8A8,
+    OP_W8A8_PAIR,
     OP_W8A16,
     check_bounded_wait,
     device_fault,
@@ -21,9 +22,11 @@ from ._lib import (  # noqa: F401
     nvfp4_dequant_bf16,
     nvfp4_quantize_rows,
     plan_chunks,
+    pool_stats,
     q6k_lm_head,
     q6k_mmvq,
     q8_1_quantize_rows,
+    set_workspace,
     version,
     w4a16_gemv,
     w4a4_gemv,
@@ -35,4 +38,5 @@ from ._lib import (  # noqa: F401
     w8a8_quantize_rows,
     w8a8_silu_proj,
     w8a8_silu_quantize_rows,
+    workspace_bytes,
 )

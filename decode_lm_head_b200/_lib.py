@@ -18,7 +18,7 @@ LIB_PATH = os.environ.get("DLMH_LIBRARY") or os.path.join(_HERE, "libdlmh.so")
 HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "dlmh.h")
 
 # op ids of dlmh_plan_chunks (dlmh_op in dlmh.h)
-OP_W8A16, OP_W8A8, OP_W4A16, OP_Q6K, OP_W4A4 = 0, 1, 2, 3, 4
+OP_W8A16, OP_W8A8, OP_W4A16, OP_Q6K, OP_W4A4, OP_W8A8_PAIR = 0, 1, 2, 3, 4, 5
 W4A4_MAX_ROWS = 32
 
 W8A8_MAX_ROWS = 128
@@ -62,6 +62,8 @@ _SIGNATURES = {
     "nvfp4_dequant_bf16": [_P, _P, _F, _I, _I, _I, _P, _L, _P],
     "e8m0_fp4_dequant_bf16": [_P, _P, _L, _I, _I, _P, _L, _P],
     "dlmh_plan_chunks": [_I, _I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I), _I],
+    "dlmh_set_workspace": [_P, ctypes.c_size_t, _P],
+    "dlmh_pool_stats": [ctypes.POINTER(_L), ctypes.POINTER(_L), _I],
     "dlmh_device_fault": [_I],
     "dlmh_check_bounded_wait": [_P],
     "dlmh_version": [],
@@ -81,6 +83,8 @@ def lib():
             fn.restype = _I
         h.dlmh_error_string.argtypes = [_I]
         h.dlmh_error_string.restype = ctypes.c_char_p
+        h.dlmh_workspace_bytes.argtypes = [_I, _I, _I, _I, _I]
+        h.dlmh_workspace_bytes.restype = _L
         _lib = h
     return _lib
 
@@ -112,6 +116,32 @@ def device_fault(reset=False):
 def check_bounded_wait(stream=None):
     """Run the library's bounded-wait check on the current device (see dlmh.h)."""
     _check(lib().dlmh_check_bounded_wait(_stream(stream)), "dlmh_check_bounded_wait")
+
+
+def workspace_bytes(op, n, k, rows, sm_count=0):
+    """Bytes of caller workspace a call of `op` (n weight rows, reduction k, up to `rows` rows)
+    needs; sm_count 0 sizes for the current device (see dlmh.h)."""
+    rc = lib().dlmh_workspace_bytes(op, n, k, rows, sm_count)
+    if rc < 0:
+        raise DlmhError(rc, "dlmh_workspace_bytes")
+    return rc
+
+
+def set_workspace(ws, stream=None):
+    """Bind the CUDA uint8 tensor `ws` (256-byte aligned) as the workspace of `stream` (the
+    current stream if None); ws=None unbinds.  The caller keeps `ws` alive while bound."""
+    if ws is None:
+        _check(lib().dlmh_set_workspace(None, 0, _stream(stream)), "dlmh_set_workspace")
+        return
+    _cuda(ws, torch.uint8, "ws", 1)
+    _check(lib().dlmh_set_workspace(_ptr(ws), ws.numel(), _stream(stream, ws.device)), "dlmh_set_workspace")
+
+
+def pool_stats(reset_high=False):
+    """(bytes in use, peak bytes) of the library pool on the current device."""
+    cur, high = _L(0), _L(0)
+    _check(lib().dlmh_pool_stats(ctypes.byref(cur), ctypes.byref(high), 1 if reset_high else 0), "dlmh_pool_stats")
+    return cur.value, high.value
 
 
 def _check(rc, what):

@@ -83,15 +83,17 @@ const char* dlmh_error_string(int code) {
     case DLMH_ERR_LD: return "a leading dimension is smaller than the row it holds";
     case DLMH_ERR_CUDA: return "a CUDA runtime call or kernel launch failed";
     case DLMH_ERR_UNSUPPORTED: return "shape beyond this build's on-chip limits";
-    case DLMH_ERR_CAPACITY: return "output array too small";
+    case DLMH_ERR_CAPACITY: return "output array or table too small";
+    case DLMH_ERR_WORKSPACE: return "the stream's workspace is smaller than the call needs (dlmh_workspace_bytes)";
     default: return "unknown status";
   }
 }
 
 int dlmh_plan_chunks(int op, int rows, int k, int* offsets, int* counts, int* tiers, int cap) {
-  if (op < DLMH_OP_W8A16 || op > DLMH_OP_W4A4) return DLMH_ERR_SHAPE;
+  if (op < DLMH_OP_W8A16 || op > DLMH_OP_W8A8_PAIR) return DLMH_ERR_SHAPE;
   if (k <= 0) return DLMH_ERR_SHAPE;
   DLMH_TRY(check_rows(rows, 0));
+  if (op == DLMH_OP_W8A8_PAIR) op = DLMH_OP_W8A8;  // the pair runs w8a8_proj's passes
   const int width = pass_rows(op, k);
   if (width <= 0) return DLMH_ERR_UNSUPPORTED;
   int nchunks = 0;
@@ -125,8 +127,11 @@ int lm_head_fp8_w8a16(const uint8_t* w, const float* w_scale, int n, int k, cons
   if (!aligned16(w)) return DLMH_ERR_ALIGN;
   DLMH_TRY(check_bf16_in(x, ldx, k));
   DLMH_TRY(check_out(out, ldc, n));
-  if (dlmh::w8a16_umma_supported(k))
-    return dlmh::w8a16_umma_run(w, w_scale, n, k, x, ldx, rows, out, ldc, as_stream(stream));
+  if (dlmh::w8a16_umma_supported(k)) {
+    dlmh::UmmaScratch sc;
+    DLMH_TRY(dlmh::call_scratch(DLMH_OP_W8A16, n, k, rows, as_stream(stream), &sc));
+    return dlmh::w8a16_umma_run(w, w_scale, n, k, x, ldx, rows, out, ldc, as_stream(stream), sc);
+  }
   const int width = pass_rows(DLMH_OP_W8A16, k);
   if (width <= 0) return DLMH_ERR_UNSUPPORTED;
   for (int done = 0; done < rows;) {
@@ -166,9 +171,11 @@ int w8a8_silu_quantize_rows(const dlmh_bf16* gate, const dlmh_bf16* up, int64_t 
   return dlmh::w8a8_silu_quantize_launch(gate, up, ld, rows, k, xq, ldq, x_scale, as_stream(stream));
 }
 
+// `fixed`: the tensor-core scratch chosen by the caller of this helper (null: the stream's
+// workspace or the pool, resolved after the argument checks).
 static int w8a8_gemv_impl(const uint8_t* w, const float* w_scale, int n, int k, const uint8_t* xq, int64_t ldq,
                           const float* x_scale, int rows, dlmh_bf16* out, int64_t ldc, void* stream,
-                          float* partial_ws, size_t partial_cap, bool after_prepass = false) {
+                          const dlmh::UmmaScratch* fixed, bool after_prepass = false) {
   DLMH_TRY(check_rows(rows, DLMH_W8A8_MAX_ROWS));
   DLMH_TRY(check_nk(n, k, 16));
   if (rows == 0) return DLMH_OK;
@@ -180,11 +187,16 @@ static int w8a8_gemv_impl(const uint8_t* w, const float* w_scale, int n, int k, 
   DLMH_TRY(check_out(out, ldc, n));
   const int width = pass_rows(DLMH_OP_W8A8, k);
   if (width <= 0) return DLMH_ERR_UNSUPPORTED;
+  dlmh::UmmaScratch sc;
+  if (fixed)
+    sc = *fixed;
+  else if (dlmh::w8a8_umma_supported(k))
+    DLMH_TRY(dlmh::call_scratch(DLMH_OP_W8A8, n, k, rows, as_stream(stream), &sc));
   for (int done = 0; done < rows;) {
     const int m = rows - done < width ? rows - done : width;
     if (dlmh::w8a8_umma_supported(k))
       DLMH_TRY(dlmh::w8a8_umma_pass(w, w_scale, n, k, xq + (int64_t)done * ldq, ldq, x_scale + done, m,
-                                    out + (int64_t)done * ldc, ldc, as_stream(stream), partial_ws, partial_cap,
+                                    out + (int64_t)done * ldc, ldc, as_stream(stream), sc,
                                     after_prepass && done == 0));
     else
       DLMH_TRY(dlmh::w8a8_gemv_pass(w, w_scale, n, k, xq + (int64_t)done * ldq, ldq, x_scale + done, m,
@@ -196,12 +208,12 @@ static int w8a8_gemv_impl(const uint8_t* w, const float* w_scale, int n, int k, 
 
 int w8a8_gemv(const uint8_t* w, const float* w_scale, int n, int k, const uint8_t* xq, int64_t ldq,
               const float* x_scale, int rows, dlmh_bf16* out, int64_t ldc, void* stream) {
-  return w8a8_gemv_impl(w, w_scale, n, k, xq, ldq, x_scale, rows, out, ldc, stream, nullptr, 0);
+  return w8a8_gemv_impl(w, w_scale, n, k, xq, ldq, x_scale, rows, out, ldc, stream, nullptr);
 }
 
 static int w8a8_proj_impl(const uint8_t* w, const float* w_scale, int n, int k, const dlmh_bf16* x,
                           const dlmh_bf16* up, int64_t ldx, int rows, dlmh_bf16* out, int64_t ldc, uint8_t* xq,
-                          float* xs, void* stream, float* partial_ws = nullptr, size_t partial_cap = 0) {
+                          float* xs, void* stream, const dlmh::UmmaScratch* fixed = nullptr) {
   DLMH_TRY(check_rows(rows, 0));
   DLMH_TRY(check_nk(n, k, 16));
   if (rows == 0) return DLMH_OK;
@@ -214,6 +226,11 @@ static int w8a8_proj_impl(const uint8_t* w, const float* w_scale, int n, int k, 
   if (!aligned16(xq) || k % 16 != 0) return DLMH_ERR_ALIGN;
   if (pass_rows(DLMH_OP_W8A8, k) <= 0) return DLMH_ERR_UNSUPPORTED;
   cudaStream_t s = as_stream(stream);
+  dlmh::UmmaScratch sc;  // resolved before the first launch
+  if (fixed)
+    sc = *fixed;
+  else if (dlmh::w8a8_umma_supported(k))
+    DLMH_TRY(dlmh::call_scratch(DLMH_OP_W8A8, n, k, rows, s, &sc));
   for (int done = 0; done < rows;) {
     const int m = rows - done < DLMH_W8A8_MAX_ROWS ? rows - done : DLMH_W8A8_MAX_ROWS;
     const dlmh_bf16* xc = x + (int64_t)done * ldx;
@@ -221,8 +238,7 @@ static int w8a8_proj_impl(const uint8_t* w, const float* w_scale, int n, int k, 
       DLMH_TRY(dlmh::w8a8_silu_quantize_launch(xc, up + (int64_t)done * ldx, ldx, m, k, xq, k, xs, s));
     else
       DLMH_TRY(dlmh::w8a8_quantize_launch(xc, ldx, m, k, xq, k, xs, s));
-    DLMH_TRY(w8a8_gemv_impl(w, w_scale, n, k, xq, k, xs, m, out + (int64_t)done * ldc, ldc, stream, partial_ws,
-                            partial_cap, true));
+    DLMH_TRY(w8a8_gemv_impl(w, w_scale, n, k, xq, k, xs, m, out + (int64_t)done * ldc, ldc, stream, &sc, true));
     done += m;
   }
   return DLMH_OK;
@@ -257,6 +273,8 @@ int w8a8_gate_up_proj(const uint8_t* w_gate, const float* s_gate, const uint8_t*
   if (!aligned16(xq_scratch) || k % 16 != 0) return DLMH_ERR_ALIGN;
   if (pass_rows(DLMH_OP_W8A8, k) <= 0) return DLMH_ERR_UNSUPPORTED;
   cudaStream_t s = as_stream(stream);
+  dlmh::UmmaScratch sc;  // resolved before the first launch
+  if (dlmh::w8a8_umma_supported(k)) DLMH_TRY(dlmh::call_scratch(DLMH_OP_W8A8_PAIR, n, k, rows, s, &sc));
   for (int done = 0; done < rows;) {
     const int m = rows - done < DLMH_W8A8_MAX_ROWS ? rows - done : DLMH_W8A8_MAX_ROWS;
     DLMH_TRY(dlmh::w8a8_quantize_launch(x + (int64_t)done * ldx, ldx, m, k, xq_scratch, k, xscale_scratch, s));
@@ -264,10 +282,10 @@ int w8a8_gate_up_proj(const uint8_t* w_gate, const float* s_gate, const uint8_t*
     dlmh_bf16* u = up_out + (int64_t)done * ldc;
     if (dlmh::w8a8_umma_supported(k)) {
       DLMH_TRY(dlmh::w8a8_umma_pair_pass(w_gate, s_gate, n, g, ldc, w_up, s_up, n, u, ldc, k, xq_scratch, k,
-                                         xscale_scratch, m, s, true));
+                                         xscale_scratch, m, s, sc, true));
     } else {
-      DLMH_TRY(w8a8_gemv_impl(w_gate, s_gate, n, k, xq_scratch, k, xscale_scratch, m, g, ldc, stream, nullptr, 0));
-      DLMH_TRY(w8a8_gemv_impl(w_up, s_up, n, k, xq_scratch, k, xscale_scratch, m, u, ldc, stream, nullptr, 0));
+      DLMH_TRY(w8a8_gemv_impl(w_gate, s_gate, n, k, xq_scratch, k, xscale_scratch, m, g, ldc, stream, &sc));
+      DLMH_TRY(w8a8_gemv_impl(w_up, s_up, n, k, xq_scratch, k, xscale_scratch, m, u, ldc, stream, &sc));
     }
     done += m;
   }
@@ -448,10 +466,9 @@ int e8m0_fp4_dequant_bf16(const uint8_t* w_packed, const uint8_t* scales, int64_
 namespace dlmh {
 
 int w8a8_proj_fixed_scratch(const uint8_t* w, const float* w_scale, int n, int k, const uint16_t* x, int64_t ldx,
-                            int rows, uint16_t* out, int64_t ldc, uint8_t* xq, float* xs, float* partial_ws,
-                            size_t partial_cap, cudaStream_t stream) {
-  return w8a8_proj_impl(w, w_scale, n, k, x, nullptr, ldx, rows, out, ldc, xq, xs, stream, partial_ws,
-                        partial_cap);
+                            int rows, uint16_t* out, int64_t ldc, uint8_t* xq, float* xs, const UmmaScratch& scratch,
+                            cudaStream_t stream) {
+  return w8a8_proj_impl(w, w_scale, n, k, x, nullptr, ldx, rows, out, ldc, xq, xs, stream, &scratch);
 }
 
 }  // namespace dlmh

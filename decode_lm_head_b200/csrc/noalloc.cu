@@ -18,6 +18,7 @@
 
 #include "dlmh_common.cuh"
 #include "gemv_launch.h"
+#include "workspace_plan.h"
 
 namespace {
 
@@ -62,15 +63,26 @@ extern "C" int w8a8_proj_noalloc(const uint8_t* w, const float* w_scale, int n, 
   if (n <= 0 || k <= 0 || k % 16 != 0) return DLMH_ERR_SHAPE;
   if (k > DLMH_NOALLOC_MAX_K) return DLMH_ERR_UNSUPPORTED;
   if (rows == 0) return DLMH_OK;
+  // The partial sums the tensor-core schedule of this shape needs on this device must fit the
+  // fixed area; checked before any launch, so a refused call touches nothing.
+  if (dlmh::w8a8_umma_supported(k)) {
+    const int sms = dlmh::device_info().sms;
+    if (sms <= 0) return DLMH_ERR_CUDA;
+    const int ntiles = (n + dlmh::kUmmaTileRows - 1) / dlmh::kUmmaTileRows;
+    const int widest = rows < DLMH_W8A8_MAX_ROWS ? rows : DLMH_W8A8_MAX_ROWS;
+    if ((size_t)dlmh::umma_partial_bytes(false, ntiles, k, widest, sms) > kPartialBytes) return DLMH_ERR_UNSUPPORTED;
+  }
   uint8_t* base = nullptr;
   const int rc = scratch_on_current_device(&base);
   if (rc != DLMH_OK) return rc;
   // Each chunk's quantize writes every code and scale the following GEMV reads, and every
   // partial sum is written before the fixup reads it, so nothing in the shared array has to
-  // start at zero.  A device with more SMs than the partial area serves gets
-  // DLMH_ERR_UNSUPPORTED.
+  // start at zero.  Whole tiles go in the static order (no queue to keep at zero).
+  dlmh::UmmaScratch sc;
+  sc.caller = true;
+  sc.partial = reinterpret_cast<float*>(base + kPartialOffset);
+  sc.partial_cap = kPartialBytes;
   return dlmh::w8a8_proj_fixed_scratch(w, w_scale, n, k, x, ldx, rows, out, ldc, base,
-                                       reinterpret_cast<float*>(base + kScaleOffset),
-                                       reinterpret_cast<float*>(base + kPartialOffset), kPartialBytes,
+                                       reinterpret_cast<float*>(base + kScaleOffset), sc,
                                        static_cast<cudaStream_t>(stream));
 }

@@ -38,6 +38,7 @@
 #include "gemv_launch.h"
 #include "umma_common.cuh"
 #include "umma_sched.h"
+#include "workspace_plan.h"
 
 namespace dlmh {
 namespace {
@@ -45,7 +46,8 @@ namespace {
 using namespace umma;
 
 constexpr int kUmmaThreads = 192;
-constexpr int kKC = 2;  // 128-byte K-chunks per stage
+constexpr int kKC = kUmmaStageChunks;  // 128-byte K-chunks per stage
+static_assert(kBM == kUmmaTileRows, "the workspace layout assumes 128-row tiles");
 constexpr int kChunkBytesA = kBM * 128;
 constexpr int kMaxUStages = 6;
 constexpr int kJobRing = 4;  // job descriptors in flight from the producer to the MMA and epilogue warps
@@ -77,10 +79,11 @@ struct UmmaParams {
   // the SM count, never of the row count; partial sums are laid out [slot][col][128 rows].
   int spt, wt, rem;
   float* partial;
-  // Dynamic hand-out of the whole tiles (null: the static order of the schedule).  queue[0]
-  // counts tiles claimed beyond each CTA's first, queue[1] the CTAs that have finished; the
-  // last CTA to finish puts both back to 0 for the next launch on the stream.  A whole tile's
-  // bits do not depend on which CTA ran it, so both orders give the same outputs.
+  // Dynamic hand-out of the whole tiles from the caller workspace's queue (null: the static
+  // order of the schedule).  queue[0] counts tiles claimed beyond each CTA's first, queue[1]
+  // the CTAs that have finished; the last CTA to finish puts both back to 0 for the next
+  // launch on the stream.  A whole tile's bits do not depend on which CTA ran it, so both
+  // orders give the same outputs.
   int* queue;
   int early_w;  // 1: the preceding kernel is this library's activation pre-pass (it writes
                 // neither W nor the outputs), so weight loads may start before it completes
@@ -436,13 +439,15 @@ __global__ void __launch_bounds__(kBM) umma_f8_fixup_kernel(const UmmaParams p, 
 constexpr size_t kUmmaSmemLimit = 232448 - 2048;
 
 // Library-owned stream-ordered pool for the W8A16 activation codes and the stream-K partial
-// sums (one per device; memory is kept between calls so that steady-state calls map nothing).
+// sums of calls without a caller workspace (one per device; memory is kept between calls so
+// that steady-state calls map nothing).
+std::mutex g_pool_mu;
+cudaMemPool_t g_pools[64] = {};
+
 cudaMemPool_t scratch_pool(int dev) {
-  static std::mutex mu;
-  static cudaMemPool_t pools[64] = {};
   if (dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> lock(mu);
-  if (!pools[dev]) {
+  std::lock_guard<std::mutex> lock(g_pool_mu);
+  if (!g_pools[dev]) {
     cudaMemPoolProps props{};
     props.allocType = cudaMemAllocationTypePinned;
     props.location.type = cudaMemLocationTypeDevice;
@@ -451,9 +456,9 @@ cudaMemPool_t scratch_pool(int dev) {
     if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) return nullptr;
     uint64_t keep = ~uint64_t(0);
     cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
-    pools[dev] = pool;
+    g_pools[dev] = pool;
   }
-  return pools[dev];
+  return g_pools[dev];
 }
 
 // The optional second weight matrix of a paired launch (same k, same activations).
@@ -465,59 +470,9 @@ struct SecondWeight {
   int64_t ldc;
 };
 
-// Whole-tile queue of a stream (two ints, zero between launches): one per stream, keyed by
-// the device and the stream's id (cudaStreamGetId: unique within the context, never reused
-// after the stream is destroyed), so that launches on different streams never share one.
-// Allocated on the stream's first eager call (cudaMalloc, then zeroed in stream order).  A
-// launch being captured into a graph gets nullptr, i.e. the static order (same outputs), so
-// no graph holds a counter that its replays on other streams could share; so does a stream
-// past the table's capacity.
-int* tile_queue(cudaStream_t s) {
-  struct Entry {
-    int dev;
-    unsigned long long id;
-    int* q;
-  };
-  constexpr int kMaxQueues = 1024;
-  static std::mutex mu;
-  static Entry entries[kMaxQueues];
-  static int count = 0;
-  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
-  if (cudaStreamIsCapturing(s, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) {
-    (void)cudaGetLastError();
-    return nullptr;
-  }
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
-  unsigned long long id = 0;
-  if (cudaStreamGetId(s, &id) != cudaSuccess) {
-    (void)cudaGetLastError();
-    // the legacy default stream (this library is built with it as stream 0) is never
-    // destroyed: its handle is a key of its own.  Anything else takes the static order.
-    if (s != nullptr && s != cudaStreamLegacy) return nullptr;
-    id = ~0ull;
-  }
-  std::lock_guard<std::mutex> lock(mu);
-  for (int i = 0; i < count; ++i)
-    if (entries[i].dev == dev && entries[i].id == id) return entries[i].q;
-  if (count == kMaxQueues) return nullptr;
-  void* q = nullptr;
-  if (cudaMalloc(&q, 256) != cudaSuccess) {
-    (void)cudaGetLastError();
-    return nullptr;
-  }
-  if (cudaMemsetAsync(q, 0, 256, s) != cudaSuccess) {
-    (void)cudaGetLastError();
-    cudaFree(q);
-    return nullptr;
-  }
-  entries[count++] = Entry{dev, id, static_cast<int*>(q)};
-  return static_cast<int*>(q);
-}
-
 int launch_umma_f8(const uint8_t* w, const float* w_scale, int n, int k, const uint8_t* b_codes, int64_t ldb,
                    int b_rows, const float* x_scale, int rows, int split, uint16_t* out, int64_t ldc, cudaStream_t s,
-                   float* partial_ws, size_t partial_cap, int early_w, const SecondWeight* second = nullptr) {
+                   const UmmaScratch& scratch, int early_w, const SecondWeight* second = nullptr) {
   const DeviceInfo di = device_info();
   if (di.sms <= 0) return DLMH_ERR_CUDA;
   UmmaParams p{};
@@ -526,7 +481,7 @@ int launch_umma_f8(const uint8_t* w, const float* w_scale, int n, int k, const u
   p.rows = rows;
   p.npad = (rows + 15) / 16 * 16;
   p.lo_off = (rows + 7) / 8 * 8;
-  p.nb = split ? 2 * p.lo_off : p.npad;
+  p.nb = umma_mma_n(split != 0, rows);
   // the epilogue reads 16 columns from lo_off + c0 (c0 < npad): keep that inside the
   // accumulator when lo_off is not a multiple of 16
   p.accw = tmem_cols_for(split && (p.lo_off % 16) ? p.nb + 16 : p.nb);
@@ -565,14 +520,14 @@ int launch_umma_f8(const uint8_t* w, const float* w_scale, int n, int k, const u
   if (G > kMaxParts) return DLMH_ERR_UNSUPPORTED;
   p.wt = sched.wt;
   p.rem = sched.rem;
-  // whole tiles from a per-stream queue, except for callers with fixed scratch (they must not
-  // allocate); both orders give the same outputs
-  p.queue = (p.wt > 0 && partial_ws == nullptr) ? tile_queue(s) : nullptr;
+  // whole tiles from the caller workspace's queue when there is one (both orders give the
+  // same outputs); the static order otherwise
+  p.queue = p.wt > 0 ? scratch.queue : nullptr;
   void* ws = nullptr;
-  const size_t need = (size_t)2 * G * p.nb * kBM * sizeof(float);
-  if (p.rem > 0 && partial_ws) {
-    if (partial_cap < need) return DLMH_ERR_UNSUPPORTED;
-    p.partial = partial_ws;
+  const size_t need = (size_t)umma_partial_bytes(split != 0, ntiles, k, rows, di.sms);
+  if (p.rem > 0 && scratch.caller) {
+    if (!scratch.partial || scratch.partial_cap < need) return DLMH_ERR_WORKSPACE;
+    p.partial = scratch.partial;
   } else if (p.rem > 0) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return DLMH_ERR_CUDA;
@@ -601,47 +556,52 @@ bool w8a8_umma_supported(int k) {
 bool w8a16_umma_supported(int k) { return k > 0 && k % 128 == 0; }
 
 int w8a8_umma_pass(const uint8_t* w, const float* w_scale, int n, int k, const uint8_t* xq, int64_t ldq,
-                   const float* x_scale, int rows, uint16_t* out, int64_t ldc, cudaStream_t s, float* partial_ws,
-                   size_t partial_cap, bool after_prepass) {
+                   const float* x_scale, int rows, uint16_t* out, int64_t ldc, cudaStream_t s,
+                   const UmmaScratch& scratch, bool after_prepass) {
   if (rows < 1 || rows > 128) return DLMH_ERR_ROWS;
   if (!w8a8_umma_supported(k)) return DLMH_ERR_SHAPE;
   if ((reinterpret_cast<uintptr_t>(w) & 15u) || (reinterpret_cast<uintptr_t>(xq) & 15u) || ldq % 16 != 0)
     return DLMH_ERR_ALIGN;
-  return launch_umma_f8(w, w_scale, n, k, xq, ldq, rows, x_scale, rows, 0, out, ldc, s, partial_ws, partial_cap,
+  return launch_umma_f8(w, w_scale, n, k, xq, ldq, rows, x_scale, rows, 0, out, ldc, s, scratch,
                         after_prepass ? 1 : 0);
 }
 
 int w8a8_umma_pair_pass(const uint8_t* w1, const float* s1, int n1, uint16_t* out1, int64_t ldc1,
                         const uint8_t* w2, const float* s2, int n2, uint16_t* out2, int64_t ldc2, int k,
                         const uint8_t* xq, int64_t ldq, const float* x_scale, int rows, cudaStream_t s,
-                        bool after_prepass) {
+                        const UmmaScratch& scratch, bool after_prepass) {
   if (rows < 1 || rows > 128) return DLMH_ERR_ROWS;
   if (!w8a8_umma_supported(k)) return DLMH_ERR_SHAPE;
   if ((reinterpret_cast<uintptr_t>(w1) & 15u) || (reinterpret_cast<uintptr_t>(w2) & 15u) ||
       (reinterpret_cast<uintptr_t>(xq) & 15u) || ldq % 16 != 0)
     return DLMH_ERR_ALIGN;
   const SecondWeight second{w2, s2, n2, out2, ldc2};
-  return launch_umma_f8(w1, s1, n1, k, xq, ldq, rows, x_scale, rows, 0, out1, ldc1, s, nullptr, 0,
+  return launch_umma_f8(w1, s1, n1, k, xq, ldq, rows, x_scale, rows, 0, out1, ldc1, s, scratch,
                         after_prepass ? 1 : 0, &second);
 }
 
 int w8a16_umma_run(const uint8_t* w, const float* w_scale, int n, int k, const uint16_t* x, int64_t ldx, int rows,
-                   uint16_t* out, int64_t ldc, cudaStream_t s) {
+                   uint16_t* out, int64_t ldc, cudaStream_t s, const UmmaScratch& scratch) {
   if (!w8a16_umma_supported(k)) return DLMH_ERR_SHAPE;
   if (rows <= 0) return DLMH_OK;
   if ((reinterpret_cast<uintptr_t>(w) & 15u) || (reinterpret_cast<uintptr_t>(x) & 15u) || ldx % 8 != 0)
     return DLMH_ERR_ALIGN;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return DLMH_ERR_CUDA;
-  cudaMemPool_t pool = scratch_pool(dev);
-  if (!pool) return DLMH_ERR_CUDA;
   const int first = rows < 128 ? rows : 128;
-  const int half_max = (first + 7) / 8 * 8;
-  const size_t code_bytes = (size_t)2 * half_max * k;  // a multiple of 256 (k % 128 == 0)
-  void* scratch = nullptr;
-  if (cudaMallocFromPoolAsync(&scratch, code_bytes + 128 * sizeof(float), pool, s) != cudaSuccess)
-    return DLMH_ERR_CUDA;
-  uint8_t* codes = static_cast<uint8_t*>(scratch);
+  const size_t code_bytes = (size_t)2 * ((first + 7) / 8 * 8) * k;  // a multiple of 256 (k % 128 == 0)
+  void* pooled = nullptr;
+  uint8_t* codes = nullptr;
+  if (scratch.caller) {
+    if (!scratch.codes || scratch.codes_cap < (size_t)w8a16_code_bytes(first, k)) return DLMH_ERR_WORKSPACE;
+    codes = scratch.codes;
+  } else {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return DLMH_ERR_CUDA;
+    cudaMemPool_t pool = scratch_pool(dev);
+    if (!pool) return DLMH_ERR_CUDA;
+    if (cudaMallocFromPoolAsync(&pooled, code_bytes + 128 * sizeof(float), pool, s) != cudaSuccess)
+      return DLMH_ERR_CUDA;
+    codes = static_cast<uint8_t*>(pooled);
+  }
   float* x_mul = reinterpret_cast<float*>(codes + code_bytes);
   int rc = DLMH_OK;
   for (int done = 0; done < rows && rc == DLMH_OK;) {
@@ -650,11 +610,34 @@ int w8a16_umma_run(const uint8_t* w, const float* w_scale, int n, int k, const u
     rc = w8a16_split_launch(x + (int64_t)done * ldx, ldx, m, k, half, codes, x_mul, s);
     if (rc == DLMH_OK)
       rc = launch_umma_f8(w, w_scale, n, k, codes, k, 2 * half, x_mul, m, 1, out + (int64_t)done * ldc, ldc, s,
-                          nullptr, 0, 1);
+                          scratch, 1);
     done += m;
   }
-  if (cudaFreeAsync(scratch, s) != cudaSuccess && rc == DLMH_OK) rc = DLMH_ERR_CUDA;
+  if (pooled && cudaFreeAsync(pooled, s) != cudaSuccess && rc == DLMH_OK) rc = DLMH_ERR_CUDA;
   return rc;
+}
+
+int pool_stats(int64_t* used_current, int64_t* used_high, int reset_high) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DLMH_ERR_CUDA;
+  cudaMemPool_t pool = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_pool_mu);
+    pool = g_pools[dev];
+  }
+  uint64_t cur = 0, high = 0;
+  if (pool) {
+    if (cudaMemPoolGetAttribute(pool, cudaMemPoolAttrUsedMemCurrent, &cur) != cudaSuccess ||
+        cudaMemPoolGetAttribute(pool, cudaMemPoolAttrUsedMemHigh, &high) != cudaSuccess)
+      return DLMH_ERR_CUDA;
+    if (reset_high) {
+      uint64_t zero = 0;
+      if (cudaMemPoolSetAttribute(pool, cudaMemPoolAttrUsedMemHigh, &zero) != cudaSuccess) return DLMH_ERR_CUDA;
+    }
+  }
+  if (used_current) *used_current = (int64_t)cur;
+  if (used_high) *used_high = (int64_t)high;
+  return DLMH_OK;
 }
 
 namespace {

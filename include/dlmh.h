@@ -20,19 +20,18 @@
  *   - Every pointer argument named w*, x*, gate, up, out*, xq*, *scale*, q8*, blocks or
  *     *scratch is a DEVICE pointer on the current CUDA device.  The caller owns all of
  *     them; the library keeps no pointer after return.
- *   - Internal scratch: the tensor-core passes (k % 128 == 0) of lm_head_fp8_w8a16 and of
- *     the W8A8 GEMV take stream-ordered scratch (W8A16 activation codes; stream-K partial
- *     sums) from a library-owned memory pool of the current device, with
- *     cudaMallocFromPoolAsync / cudaFreeAsync on `stream`.  The pool keeps its memory between
- *     calls, so steady-state calls map nothing and never synchronize; concurrent calls on
- *     different streams get distinct scratch.  w8a8_proj_noalloc never uses the pool.
- *   - Tile queue: when a tensor-core pass has more weight tiles than SMs, its CTAs take the
- *     whole tiles from an atomic counter, one per stream (keyed by the device and
- *     cudaStreamGetId, which is never reused within a context), allocated on the stream's
- *     first eager such call (cudaMalloc, so that first call synchronizes the device) and
- *     left at zero by every launch.  Launches captured into a CUDA graph, and
- *     w8a8_proj_noalloc, use the static tile order instead, so a graph holds no counter
- *     and its replays may run on any streams at once; both orders give the same outputs.
+ *   - Internal scratch of the tensor-core passes (k % 128 == 0) of lm_head_fp8_w8a16 and of
+ *     the W8A8 GEMVs (W8A16 activation codes, stream-K partial sums, a whole-tile queue):
+ *       * with a caller workspace bound to the stream (dlmh_set_workspace, sized with
+ *         dlmh_workspace_bytes) it comes from that workspace and NO call allocates anything;
+ *         the CTAs then take the whole weight tiles from the workspace's atomic queue;
+ *       * without one, the codes and partial sums come from a library-owned memory pool of
+ *         the current device (cudaMallocFromPoolAsync / cudaFreeAsync on `stream`; the pool
+ *         keeps its memory, so steady-state calls map nothing and never synchronize) and the
+ *         whole tiles go in a static order.
+ *     Both tile orders give the same outputs.  A launch being captured into a CUDA graph
+ *     takes the static order (a graph holds no counter).  w8a8_proj_noalloc uses neither the
+ *     pool nor a workspace.
  *   - BF16 values are passed as raw 16-bit patterns (dlmh_bf16).
  *   - Matrices are row-major.  Leading dimensions (ld*) count ELEMENTS of the pointed-to
  *     type, so row r of x starts at x + r * ldx.
@@ -81,7 +80,8 @@ typedef enum dlmh_status {
   DLMH_ERR_LD = -5,          /* a leading dimension is smaller than the row it holds */
   DLMH_ERR_CUDA = -6,        /* a CUDA runtime call or launch failed */
   DLMH_ERR_UNSUPPORTED = -7, /* the shape is valid but beyond this build's limits (k too large) */
-  DLMH_ERR_CAPACITY = -8     /* an output array passed to a host helper is too small */
+  DLMH_ERR_CAPACITY = -8,    /* an output array passed to a host helper (or a table) is too small */
+  DLMH_ERR_WORKSPACE = -9    /* the stream's bound workspace is smaller than the call needs */
 } dlmh_status;
 
 /* Largest row count of one W8A8 quantize / GEMV call (ops::W8A8_MAX_ROWS in
@@ -119,7 +119,8 @@ typedef enum dlmh_status {
  *   x' exactly for every element with |x| >= 2^-13 max|x| of its row (every BF16 value has
  *   8 significant bits, E4M3 4); smaller elements keep an error below 2^-21 max|x|.
  *   Scratch: 2 * roundup8(min(rows, 128)) * k bytes + 512 B, plus the stream-K partial
- *   sums (at most 2 * #SMs * 128 * 256 * 4 bytes), from the library pool (see above).
+ *   sums (at most 2 * #SMs * 128 * 256 * 4 bytes), from the stream's workspace or the
+ *   library pool (see above; dlmh_workspace_bytes(DLMH_OP_W8A16, ...)).
  *   Other k: one weight pass per 16 rows; E4M3 weights decoded exactly to f16 and each x row
  *   scaled by a power of two into f16 (exact for every |x| >= 2^-31 max|x|), products
  *   summed in f32.  k above the shared-memory limit of a 16-row chunk (k > 6144) returns
@@ -156,7 +157,7 @@ DLMH_API int w8a8_silu_quantize_rows(const dlmh_bf16* gate, const dlmh_bf16* up,
  *   out[m, n] = bf16( s[n] * sx[m] * sum_k e4m3(w[n, k]) * e4m3(xq[m, k]) )
  * lm_head_fp8_rows.rs (W8A8 branch), w8a8_layer.rs (ops::w8a8_gemv).
  *   rows <= 128; one weight pass per call when k % 128 == 0 (tensor cores; stream-K partial
- *   sums in pool scratch, see above), else passes of up to 32 rows (k bounded by the
+ *   sums in the stream's workspace or pool scratch, see above), else passes of up to 32 rows (k bounded by the
  *   shared-memory activation tile, DLMH_ERR_UNSUPPORTED beyond).  xq [rows, ldq] as written
  *   by the quantize entry points; x_scale [rows].  k % 16 == 0.
  * ------------------------------------------------------------------------------------- */
@@ -209,13 +210,15 @@ DLMH_API int w8a8_gate_up_proj(const uint8_t* w_gate, const float* s_gate, const
  *
  *   Limits: k <= DLMH_NOALLOC_MAX_K (16384), else DLMH_ERR_UNSUPPORTED; a device with more
  *   than DLMH_NOALLOC_MAX_SMS (160) SMs gets DLMH_ERR_UNSUPPORTED for shapes whose
- *   tensor-core pass needs stream-K partial sums.  Every GPU that loads the library holds
+ *   tensor-core pass needs stream-K partial sums.  Both are checked before any launch.  Every GPU that loads the library holds
  *   the array until the process exits: 2 MiB of codes, 512 B of scales and 20 MiB of
  *   partial sums (22 MiB + 512 B).
  *
  *   Set-up: a device's first call looks the array's device address up
- *   (cudaGetSymbolAddress, with that device current).  Make that first call before any
- *   stream capture.
+ *   (cudaGetSymbolAddress, with that device current) and keeps it for the life of the
+ *   process.  Make that first call before any stream capture.  The kept address does not
+ *   survive cudaDeviceReset (the module, and the array with it, is loaded again): do not
+ *   call this entry point after resetting a device it was used on.
  *
  *   Sharing: all calls on a device share the one array, and it keeps the last call's codes
  *   and scales.  Each call overwrites, before reading, every byte it uses, so nothing needs
@@ -351,7 +354,8 @@ typedef enum dlmh_op {
   DLMH_OP_W8A8 = 1,  /* w8a8_proj / w8a8_silu_proj */
   DLMH_OP_W4A16 = 2, /* w4a16_gemv */
   DLMH_OP_Q6K = 3,   /* q6k_mmvq / q6k_lm_head */
-  DLMH_OP_W4A4 = 4   /* w4a4_gemv / w4a4_proj */
+  DLMH_OP_W4A4 = 4,  /* w4a4_gemv / w4a4_proj */
+  DLMH_OP_W8A8_PAIR = 5 /* w8a8_gate_up_proj (n = rows of EACH weight) */
 } dlmh_op;
 
 /* The weight passes an entry point runs for `rows` at reduction length k: pass i covers rows
@@ -365,6 +369,42 @@ typedef enum dlmh_op {
  * DLMH_ERR_UNSUPPORTED when no tier fits k, DLMH_ERR_CAPACITY when more than `cap`
  * passes are needed.  Arrays may be NULL when cap == 0 (count only). */
 DLMH_API int dlmh_plan_chunks(int op, int rows, int k, int* offsets, int* counts, int* tiers, int cap);
+
+/* ---------------------------------------------------------------------------------------
+ * Caller-owned workspace (w8a8_layer.rs, W8a8Ctx::new: the scratch is allocated once per
+ * model, outside the launch path, and shared by every projection of a stream)
+ *
+ * dlmh_workspace_bytes: bytes of workspace a call of `op` (a dlmh_op) with weight rows n,
+ *   reduction length k and `rows` activation rows needs; a workspace of that size serves
+ *   every call of that op and shape with at most `rows` rows.  0 when the call runs no
+ *   tensor-core pass (k % 128 != 0, W4A16, W4A4, Q6_K) or rows == 0.  The stream-K schedule
+ *   depends on the SM count: sm_count > 0 sizes for that many SMs (host-only, no GPU
+ *   needed), 0 for the current device.  Errors: DLMH_ERR_SHAPE (unknown op, n <= 0,
+ *   k <= 0, sm_count < 0), DLMH_ERR_ROWS (rows < 0), DLMH_ERR_CUDA (no current device).
+ *   Layout (256-byte aligned regions): a 256-byte tile queue, the W8A16 two-term codes
+ *   2 * roundup8(min(rows, 128)) * k bytes + 512, the stream-K partial sums
+ *   2 * G * N_mma * 128 * 4 bytes when the schedule has a remainder.
+ *
+ * dlmh_set_workspace: binds the device buffer ws (256-byte aligned, `bytes` long, owned by the
+ *   caller, kept bound until replaced) to `stream` on the current device.  From then on every
+ *   FP8 call on that stream takes its internal scratch from ws and allocates nothing; a call
+ *   whose shape needs more than `bytes` returns DLMH_ERR_WORKSPACE before launching anything.
+ *   The call zeroes the first 256 bytes (the tile queue) with cudaMemsetAsync on `stream`;
+ *   every launch leaves them at zero.  ws == NULL unbinds (calls go back to the pool).  Calls
+ *   that use one workspace must not overlap on the GPU: bind one per stream.  The library
+ *   never frees ws; unbind before freeing it.  Bind outside stream capture
+ *   (DLMH_ERR_UNSUPPORTED while the stream is capturing).  Errors: DLMH_ERR_ALIGN,
+ *   DLMH_ERR_WORKSPACE (bytes < 256), DLMH_ERR_CAPACITY (1024 streams bound),
+ *   DLMH_ERR_CUDA.  (No counterpart in the pages' argument lists: their scratch is a field
+ *   of the context; here the stream carries it, so the entry points keep the pages' lists.)
+ *
+ * dlmh_pool_stats: bytes of the library pool of the current device in use now and at the
+ *   peak since the last reset (both 0 before the pool's first use); reset_high != 0 sets the
+ *   peak back to the current use.  A diagnostic: a stream with a workspace never raises them.
+ * ------------------------------------------------------------------------------------- */
+DLMH_API int64_t dlmh_workspace_bytes(int op, int n, int k, int rows, int sm_count);
+DLMH_API int dlmh_set_workspace(void* ws, size_t bytes, void* stream);
+DLMH_API int dlmh_pool_stats(int64_t* used_current, int64_t* used_high, int reset_high);
 
 /* Fault bits recorded on the current device by the kernels' bounded waits (a wait for a
  * shared-memory stage that did not complete in time; the kernel then finishes without

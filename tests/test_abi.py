@@ -28,7 +28,7 @@ def test_library_exports_every_declared_function():
 
 def test_error_strings_and_version():
     assert dl.version() >= 100
-    for code in range(-8, 1):
+    for code in range(-9, 1):
         assert dl.error_string(code)
     assert dl.error_string(-99) == "unknown status"
 
@@ -160,3 +160,44 @@ def test_dequant_argument_errors():
     assert e(A, A, 7, 16, 64, A, 64, None) == -2           # 1024 elements not a multiple of 7 groups
     assert e(A, A, 0, 16, 64, A, 64, None) == -2
     assert e(U, A, 4, 16, 64, A, 64, None) == -3
+
+
+def test_workspace_bytes_sizes_and_errors():
+    # Sizes of the caller workspace (dlmh.h): a 256-byte tile queue, the W8A16 two-term codes
+    # of the widest pass (2 roundup8(min(rows,128)) k + 512 bytes, rounded to 256), then the
+    # stream-K partial sums 2 G N_mma 128 4 bytes when tiles % G != 0 (G = the SM count once
+    # there are more tiles than SMs).  Worked by hand for 148 SMs:
+    ws = dl.workspace_bytes
+    # FP8 head 248320 x 5120: 1940 tiles, 13 whole waves + 16 remainder tiles
+    assert ws(dl.OP_W8A16, 248320, 5120, 128, 148) == 256 + (2 * 128 * 5120 + 512) + 2 * 148 * 256 * 128 * 4
+    assert ws(dl.OP_W8A8, 248320, 5120, 128, 148) == 256 + 2 * 148 * 128 * 128 * 4
+    assert ws(dl.OP_W8A8, 248320, 5120, 1000, 148) == ws(dl.OP_W8A8, 248320, 5120, 128, 148)  # 128-row passes
+    assert ws(dl.OP_W8A16, 248320, 5120, 3, 148) == 256 + (2 * 8 * 5120 + 512) + 2 * 148 * 16 * 128 * 4
+    # 148 x 128 rows: whole waves only, no partial sums
+    assert ws(dl.OP_W8A8, 148 * 128, 5120, 64, 148) == 256
+    # down projection 4096 x 14336: 32 tiles < 148 SMs, all of them remainder tiles
+    assert ws(dl.OP_W8A8, 4096, 14336, 1, 148) == 256 + 2 * 148 * 16 * 128 * 4
+    # gate + up pair: the tiles of both weights
+    assert ws(dl.OP_W8A8_PAIR, 14336, 4096, 16, 148) == 256 + 2 * 148 * 16 * 128 * 4
+    # no tensor-core pass: nothing
+    for op_, k in ((dl.OP_W8A16, 1040), (dl.OP_W8A8, 1040), (dl.OP_W4A16, 4096), (dl.OP_Q6K, 7168),
+                   (dl.OP_W4A4, 4096)):
+        assert ws(op_, 1000, k, 16, 148) == 0
+    assert ws(dl.OP_W8A16, 1000, 5120, 0, 148) == 0
+    # errors (no GPU is touched with an explicit SM count)
+    f = L.dlmh_workspace_bytes
+    assert f(6, 16, 128, 1, 148) == -2
+    assert f(dl.OP_W8A8, 0, 128, 1, 148) == -2
+    assert f(dl.OP_W8A8, 16, 128, 1, -1) == -2
+    assert f(dl.OP_W8A8, 16, 128, -1, 148) == -4
+
+
+def test_set_workspace_argument_errors():
+    assert L.dlmh_set_workspace(A + 16, 1 << 20, None) == -3      # not 256-byte aligned
+    assert L.dlmh_set_workspace(A, 255, None) == -9               # smaller than the tile queue
+    assert dl.error_string(-9).startswith("the stream's workspace")
+
+
+def test_plan_pair_op_runs_w8a8_passes():
+    for rows in (1, 128, 129, 300):
+        assert dl.plan_chunks(dl.OP_W8A8_PAIR, rows, 4096) == dl.plan_chunks(dl.OP_W8A8, rows, 4096)

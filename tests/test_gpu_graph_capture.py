@@ -1,9 +1,9 @@
 """Tensor-core calls captured into a CUDA graph on a stream that already ran them eagerly.
 
-An eager call with more weight tiles than SMs hands its whole tiles out from the stream's
-counter; a captured call takes the static tile order, so no graph holds a counter that two
-replays on different streams could share.  A whole tile's bits do not depend on which CTA
-ran it, so every replay must give the eager call's bits.
+Without a caller workspace the captured call's scratch comes from the library pool (a graph
+memory node) and its whole tiles go in the static order; every replay must give the eager
+call's bits.  (With a workspace the eager calls take the queue order: see
+test_gpu_workspace.py.)
 """
 
 import numpy as np
