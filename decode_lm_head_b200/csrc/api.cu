@@ -425,7 +425,7 @@ int q6k_lm_head(const void* blocks, int n, int k, const dlmh_bf16* x, int64_t ld
     const int m = rows - done < width ? rows - done : width;
     DLMH_TRY(dlmh::q8_1_quantize_launch(x + (int64_t)done * ldx, ldx, m, k, static_cast<uint8_t*>(q8_scratch), s));
     DLMH_TRY(dlmh::q6k_mmvq_launch(static_cast<const uint8_t*>(blocks), n, k,
-                                   static_cast<const uint8_t*>(q8_scratch), m, out + (int64_t)done * ldc, ldc, s));
+                                   static_cast<const uint8_t*>(q8_scratch), m, out + (int64_t)done * ldc, ldc, s, true));
     done += m;
   }
   return DLMH_OK;

@@ -108,7 +108,9 @@ int q6k_fault(int reset);
 // Q6_K GEMV of 1..64 q8_1 rows in one weight pass: the 8-row kernels up to 8 rows, the wide
 // kernel (tiers 16 / 32 / 64, q8 16-byte aligned, else DLMH_ERR_ALIGN) above; same bits.
 int q6k_wide_rows(int rows);
+// after_prepass: the preceding kernel on `s` is q8_1_quantize_launch (weight copies may start
+// before it completes).
 int q6k_mmvq_launch(const uint8_t* blocks, int n, int k, const uint8_t* q8, int rows, uint16_t* out, int64_t ldc,
-                    cudaStream_t s);
+                    cudaStream_t s, bool after_prepass = false);
 
 }  // namespace dlmh

@@ -1,21 +1,23 @@
 // Q6_K super-blocks x block_q8_1 rows on int8 warp MMAs.
 //
-// Same decomposition as the row-tile GEMV: one persistent 512-thread CTA per SM over
-// 16-row weight tiles, the super-blocks of a tile split across 16 warps as evenly as
-// possible (q6_slice_begin), a fixed-order
-// cross-warp reduction at the end of each tile.  Per 16-value sub-block j a warp runs one
-// s8 m16n8k16 MMA: the weight codes (q - 32) times the q8_1 codes, an exact int32 dot;
-// the dot is then scaled in f32 by d(super-block) * scales[j] of the weight row, and
-// every 32 values (one q8_1 block) by the row's q8_1 d.
+// Per 16-value sub-block j one m16n8k16 integer MMA gives the exact int32 dot
+//   D_j = sum_{i in j} (q_i - 32) * qs_i
+// for 16 weight rows x 8 activation columns.  Per q8_1 block (sub-blocks 2b, 2b+1) the two
+// dots are weighted by their int8 sub-scales in int32 (exact: |sum| < 2^24, so its float
+// conversion is exact too) and accumulated in float over the super-block's 8 blocks with the
+// block's q8_1 d:  t = fma(float(D_2b sc_2b + D_2b+1 sc_2b+1), d8(b), t)  from t = 0; the
+// super-block then adds  acc = fma(t, d(super-block), acc).  The super-blocks of a row are cut
+// into 16 K-slices (q6k_slices.h); each slice is accumulated alone from 0 and the slices are
+// added in order.  Every kernel below takes exactly these steps for every output, so a row's
+// bits do not depend on which kernel, or how many rows, served it.
 //
-// Super-block byte map (210 bytes): ql[128] @0, qh[64] @128, int8 scales[16] @192,
-// f16 d @208.  Value i = 128h + 32u + l (h < 2, u < 4, l < 32): low 4 bits from
-// ql[64h + 32(u&1) + l] (low nibble for u < 2, high nibble for u >= 2), top 2 bits from
-// bits 2u..2u+1 of qh[32h + l]; sub-block j = i / 16 uses scales[j].
-// Lane (g, t) of a warp feeds the MMA with values 4t..4t+3 of every sub-block, i.e. the
-// 4 consecutive ql / qh bytes at l = 16(j&1) + 4t, for rows g and g+8.
-// Super-blocks are only 2-byte aligned in the raw layout, so bytes are fetched with
-// 16-bit read-only loads (each 32-byte sector still comes from DRAM once).
+// The weight codes enter the MMA as (q - 32) in signed bytes (bit tricks, no table).
+//
+// Super-block byte map (210 bytes): ql[128] @0, qh[64] @128, int8 scales[16] @192, f16 d @208.
+// Value i = 128h + 32u + l (h < 2, u < 4, l < 32): low 4 bits from ql[64h + 32(u&1) + l] (low
+// nibble for u < 2, high for u >= 2), top 2 bits from bits 2u..2u+1 of qh[32h + l]; sub-block
+// j = i / 16 uses scales[j].  Lane (g, t) feeds the MMA with values 4t..4t+3 of every sub-block,
+// i.e. the 4 consecutive ql / qh bytes at l = 16(j&1) + 4t, for weight rows g and g+8.
 #include "dlmh_common.cuh"
 #include "gemv_launch.h"
 #include "q6k_slices.h"
@@ -27,69 +29,157 @@ namespace {
 constexpr int kQ6Warps = 16;
 constexpr int kQ6Threads = kQ6Warps * 32;
 constexpr int kQ6TileRows = 16;
-constexpr int kQ6MaxRows = 8;  // q8_1 rows per launch (one 8-column MMA tile)
+constexpr int kQ6MaxRows = 8;  // q8_1 rows of the 8-row kernels (one 8-column MMA tile)
+
+static_assert(kQ6Warps == kQ6Slices, "one K-slice per warp of the 8-row kernels");
+
+// ---------------------------------------------------------------------------------------
+// The shared arithmetic
+// ---------------------------------------------------------------------------------------
+
+// One weight row's super-block as lane (g, t) needs it: ql bytes 16i + 4t (i < 8), qh bytes
+// 128 + 16i + 4t (i < 4), the 16 scale bytes, and d.
+struct Q6W {
+  uint32_t ql[8], qh[4], sc[4];
+  float d;
+};
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
+}
+
+// The four 6-bit codes q (one per byte, 0..63) of sub-block j, values 4t..4t+3.
+__device__ __forceinline__ uint32_t q6_codes_u8(const Q6W& w, int j) {
+  const int h = j >> 3, u = (j & 7) >> 1, e = j & 1;
+  const uint32_t qlw = w.ql[4 * h + 2 * (u & 1) + e];
+  const uint32_t qhw = w.qh[2 * h + e];
+  const uint32_t lo = u >= 2 ? qlw >> 4 : qlw;
+  const uint32_t hi = u == 0 ? qhw << 4 : u == 1 ? qhw << 2 : u == 2 ? qhw : qhw >> 2;
+  return (lo & 0x0f0f0f0fu) | (hi & 0x30303030u);
+}
+
+// The same codes as (q - 32) in signed bytes: flipping bit 5 gives the 6-bit two's complement,
+// then bit 5 is copied into bits 6 and 7 (adding 6 * 0x20 sets them; they are 0, so no carry).
+__device__ __forceinline__ uint32_t q6_codes_s8(const Q6W& w, int j) {
+  const uint32_t a = q6_codes_u8(w, j) ^ 0x20202020u;
+  return a + (a & 0x20202020u) * 6u;
+}
+
+// Sub-scale j of the row, sign-extended (prmt: byte j&3, its sign replicated into the others).
+__device__ __forceinline__ int q6_scale(const Q6W& w, int j) {
+  const uint32_t q = (uint32_t)(j & 3);
+  return (int)prmt(w.sc[j >> 2], 0u, q | ((8u | q) << 4) | ((8u | q) << 8) | ((8u | q) << 12));
+}
+
+// One q8_1 block of one 8-column group: t[i] += float(D0[i] sc0 + D1[i] sc1) * d8(column).
+// Outputs i: 0 = (row g, column 2t), 1 = (g, 2t+1), 2 = (g+8, 2t), 3 = (g+8, 2t+1).
+__device__ __forceinline__ void q6_block_step(float (&tsb)[4], const int (&d0)[4], const int (&d1)[4], int ra0, int ra1,
+                                              int rb0, int rb1, float dx0, float dx1) {
+  tsb[0] = __fmaf_rn((float)(d0[0] * ra0 + d1[0] * ra1), dx0, tsb[0]);
+  tsb[1] = __fmaf_rn((float)(d0[1] * ra0 + d1[1] * ra1), dx1, tsb[1]);
+  tsb[2] = __fmaf_rn((float)(d0[2] * rb0 + d1[2] * rb1), dx0, tsb[2]);
+  tsb[3] = __fmaf_rn((float)(d0[3] * rb0 + d1[3] * rb1), dx1, tsb[3]);
+}
+
+// End of a super-block: acc += t * d(row).
+__device__ __forceinline__ void q6_superblock_end(float (&acc)[4], const float (&tsb)[4], float da, float db) {
+  acc[0] = __fmaf_rn(tsb[0], da, acc[0]);
+  acc[1] = __fmaf_rn(tsb[1], da, acc[1]);
+  acc[2] = __fmaf_rn(tsb[2], db, acc[2]);
+  acc[3] = __fmaf_rn(tsb[3], db, acc[3]);
+}
+
+// ---- weight fragment loads
+
+__device__ __forceinline__ uint32_t lds_u32(uint32_t saddr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(saddr));
+  return v;
+}
+__device__ __forceinline__ uint2 lds_u64(uint32_t saddr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(saddr));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds_u16(uint32_t saddr) {
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(saddr));
+  return v;
+}
+// 32-bit load from a 2-byte aligned shared address: two aligned words joined.
+__device__ __forceinline__ uint32_t lds_u32_a2(uint32_t saddr) {
+  const uint32_t a = saddr & ~3u;
+  return __funnelshift_r(lds_u32(a), lds_u32(a + 4), (saddr & 3u) * 8u);
+}
+
+// Super-block at shared address `ba` (4-byte aligned when kAligned, else 2-byte aligned).
+template <bool kAligned>
+__device__ __forceinline__ void q6_load_smem(Q6W& w, bool valid, uint32_t ba, int t) {
+  if (!valid) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w.ql[i] = 0u;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w.qh[i] = w.sc[i] = 0u;
+    w.d = 0.f;
+    return;
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) w.ql[i] = kAligned ? lds_u32(ba + 16 * i + 4 * t) : lds_u32_a2(ba + 16 * i + 4 * t);
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    w.qh[i] = kAligned ? lds_u32(ba + 128 + 16 * i + 4 * t) : lds_u32_a2(ba + 128 + 16 * i + 4 * t);
+  if (kAligned) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w.sc[i] = lds_u32(ba + 192 + 4 * i);
+  } else {  // 16 bytes at 2 mod 4: five aligned words, four byte-permutes
+    uint32_t v[5];
+#pragma unroll
+    for (int i = 0; i < 5; ++i) v[i] = lds_u32(ba + 190 + 4 * i);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w.sc[i] = prmt(v[i], v[i + 1], 0x5432u);
+  }
+  w.d = f16_bits_to_f32(lds_u16(ba + 208));
+}
 
 __device__ __forceinline__ uint32_t ldg_u32_a2(const uint8_t* p) {  // 2-byte aligned 32-bit load
   return ldg_u16(p) | (ldg_u16(p + 2) << 16);
 }
 
-// (q - 32) as int8 for four 6-bit codes packed one per byte.
-__device__ __forceinline__ uint32_t q6_to_s8x4(uint32_t q) {
-  const uint32_t x = q ^ 0x20202020u;          // bit 5 set <=> q < 32
-  const uint32_t s = x & 0x20202020u;
-  return x | (s * 6u);                          // sign-extend bit 5 into bits 6, 7
-}
-
-// acc + (is * d) * dx with one rounding per step (a product, then a fused multiply-add), the
-// same in every Q6_K kernel whatever the compiler would contract.
-__device__ __forceinline__ float q6_block_step(float acc, int is, float d, float dx) {
-  return __fmaf_rn(__fmul_rn((float)is, d), dx, acc);
-}
-
-// The K-slices (q6k_slices.h): warp w of the 8-row kernels runs slice w.
-static_assert(kQ6Warps == kQ6Slices, "one K-slice per warp of the 8-row kernels");
-
-// One super-block for rows g (a) and g+8 (b) of a 16-row tile against activation columns 2t
-// and 2t+1 (acc[0..1]: row a, acc[2..3]: row b).  Per q8_1 block (sub-blocks j0, j1) the two
-// exact int32 sub-block dots are scaled by their int8 sub-scales and summed in int32 -- exact,
-// |sum| < 2^24 so its f32 conversion is exact too -- then multiplied by the super-block d and
-// the q8_1 d in f32.  Shared by both Q6_K kernels so that they give the same bits.
-__device__ __forceinline__ void q6_superblock(float (&acc)[4], const uint32_t (&qla)[8], const uint32_t (&qlb)[8],
-                                              const uint32_t (&qha)[4], const uint32_t (&qhb)[4],
-                                              const uint32_t (&sca)[4], const uint32_t (&scb)[4], float da, float db,
-                                              const int8_t* xsb, const float* dx, int nb32, int sb, int t) {
+__device__ __forceinline__ void q6_load_global(Q6W& w, bool valid, const uint8_t* b, int t) {
 #pragma unroll
-  for (int blk = 0; blk < 8; ++blk) {  // q8_1 block = sub-blocks 2blk, 2blk+1
-    int is0 = 0, is1 = 0, is2 = 0, is3 = 0;
+  for (int i = 0; i < 8; ++i) w.ql[i] = valid ? ldg_u32_a2(b + 16 * i + 4 * t) : 0u;
 #pragma unroll
-    for (int hj = 0; hj < 2; ++hj) {
-      const int j = 2 * blk + hj;
-      const int h = j >> 3, u = (j & 7) >> 1;
-      // ql word index: 64h + 32(u&1) + 16(j&1) -> q = 4h + 2(u&1) + (j&1); qh: 32h + 16(j&1)
-      const int qi = 4 * h + 2 * (u & 1) + (j & 1);
-      const int hi = 2 * h + (j & 1);
-      const int nsh = (u >> 1) * 4, hsh = 2 * u;
-      const uint32_t qa = ((qla[qi] >> nsh) & 0x0f0f0f0fu) | (((qha[hi] >> hsh) & 0x03030303u) << 4);
-      const uint32_t qb = ((qlb[qi] >> nsh) & 0x0f0f0f0fu) | (((qhb[hi] >> hsh) & 0x03030303u) << 4);
-      const uint32_t bx = *reinterpret_cast<const uint32_t*>(xsb + 16 * j + 4 * t);
-      int d4[4] = {0, 0, 0, 0};
-      mma_s8_16816(d4, q6_to_s8x4(qa), q6_to_s8x4(qb), bx);
-      const int sha = 24 - 8 * (j & 3);  // sign-extend byte j&3 of the scale word
-      const int ra = (int)(sca[j >> 2] << sha) >> 24;
-      const int rb = (int)(scb[j >> 2] << sha) >> 24;
-      is0 += d4[0] * ra;
-      is1 += d4[1] * ra;
-      is2 += d4[2] * rb;
-      is3 += d4[3] * rb;
-    }
-    const int b32 = sb * 8 + blk;
-    const float dx0 = dx[(2 * t) * nb32 + b32], dx1 = dx[(2 * t + 1) * nb32 + b32];
-    acc[0] = q6_block_step(acc[0], is0, da, dx0);
-    acc[1] = q6_block_step(acc[1], is1, da, dx1);
-    acc[2] = q6_block_step(acc[2], is2, db, dx0);
-    acc[3] = q6_block_step(acc[3], is3, db, dx1);
+  for (int i = 0; i < 4; ++i) {
+    w.qh[i] = valid ? ldg_u32_a2(b + 128 + 16 * i + 4 * t) : 0u;
+    w.sc[i] = valid ? ldg_u32_a2(b + 192 + 4 * i) : 0u;
   }
+  w.d = valid ? f16_bits_to_f32(ldg_u16(b + 208)) : 0.f;
 }
+
+// ---------------------------------------------------------------------------------------
+// 8-row kernels (1..8 q8_1 rows, one 8-column MMA group)
+// ---------------------------------------------------------------------------------------
+//
+// One persistent 512-thread CTA per SM over 16-row weight tiles; warp w runs K-slice w of every
+// tile (q6_slice_begin), and the 16 slices of a tile are summed in warp order through shared
+// memory.  Activations:
+//   - dxs [K/32][8] float32 q8_1 d, staged once per CTA;
+//   - the B fragments (4 codes of column g, values 4t..4t+3 of each sub-block): for K <= 8192
+//     (at most 2 super-blocks per slice) each warp keeps the 32 words of its own slice in
+//     registers, loaded once; beyond that the codes are staged whole, xs [8][rs] with
+//     rs % 128 == 64, value k of super-block sb of column c at
+//     c rs + 256 sb + 64 (k >> 6) + 16 ((k >> 2) & 3) + 4 ((k >> 4) & 3) + (k & 3),
+//     so that lane (g, t) reads the fragments of sub-blocks 4q..4q+3 as one 16-byte word
+//     (the 8 lanes of each phase on 8 distinct 16-byte bank groups).
+// Padding columns (rows <= c < 8) are zero.
+// Weights: either 1-D bulk copies (TMA) of stages of SR = 8 or 4 consecutive rows into a ring
+// of shared memory (blocks 16-byte aligned; SR rows are 210 SR (k / 256) bytes, a multiple of
+// 16 for SR = 8 always and for SR = 4 when k / 256 is even; a ragged last stage copies its
+// 16-byte-multiple prefix in bulk and its last bytes with plain loads), or 16-bit global loads
+// (blocks only 2-byte aligned).  A tile's stages are released at the tile's reduction barrier,
+// so the ring holds two tiles when it can: one computed, the next one landing.
 
 struct Q6Params {
   const uint8_t* blocks;
@@ -100,158 +190,119 @@ struct Q6Params {
   int64_t ldc;
 };
 
-__device__ __forceinline__ int q6_row_stride(int k) {  // qs bytes per staged row, % 128 == 16
-  int s = k;
-  int r = s % 128;
-  return s + ((16 - r) + 128) % 128;
-}
-
-__global__ void __launch_bounds__(kQ6Threads, 1) q6k_mmvq_kernel(const Q6Params p) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  grid_dependents_launch();
-  grid_dependency_wait();  // launched early (programmatic): q8, blocks and out follow the preceding kernel
-  const int nsb = p.k / 256;
-  const int nb32 = p.k / 32;
-  const int rs = q6_row_stride(p.k);
-  int8_t* xs = reinterpret_cast<int8_t*>(smem);                              // [8][rs]
-  float* dx = reinterpret_cast<float*>(smem + kQ6MaxRows * rs);              // [8][nb32]
-  float* red = dx + kQ6MaxRows * nb32;                                       // [2][16 warps][32 lanes][4]
-
-  // ---- stage the q8_1 rows: codes in natural order, d as f32
-  for (int it = threadIdx.x; it < kQ6MaxRows * nb32; it += kQ6Threads) {
-    const int m = it / nb32, b = it % nb32;
-    uint32_t w[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    float d = 0.f;
-    if (m < p.rows) {
-      const uint8_t* blk = p.q8 + ((int64_t)m * nb32 + b) * 36;
-      const uint32_t* bw = reinterpret_cast<const uint32_t*>(blk);
-      d = f16_bits_to_f32(bw[0] & 0xffff);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) w[i] = bw[1 + i];
-    }
-    dx[m * nb32 + b] = d;
-    uint4* dst = reinterpret_cast<uint4*>(xs + m * rs + b * 32);
-    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-    dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-  }
-  __syncthreads();
-
-  const int ntiles = (p.n + kQ6TileRows - 1) / kQ6TileRows;
-  const int T0 = (int)((int64_t)blockIdx.x * ntiles / gridDim.x);
-  const int T1 = (int)((int64_t)(blockIdx.x + 1) * ntiles / gridDim.x);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, t = lane & 3;
-  const int sb_begin = q6_slice_begin(nsb, warp), sb_end = q6_slice_begin(nsb, warp + 1);
-  const int64_t row_bytes = (int64_t)nsb * 210;
-  const int8_t* xrow = xs + g * rs;  // B column g
-  int parity = 0;
-
-  for (int tile = T0; tile < T1; ++tile) {
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    const int r0 = tile * kQ6TileRows + g;
-    const bool va = r0 < p.n, vb = r0 + 8 < p.n;
-    for (int sb = sb_begin; sb < sb_end; ++sb) {
-      const uint8_t* ba = p.blocks + (int64_t)r0 * row_bytes + (int64_t)sb * 210;
-      const uint8_t* bb = ba + 8 * row_bytes;
-      uint32_t qla[8], qlb[8], qha[4], qhb[4], sca[4], scb[4];
-      float da = 0.f, db = 0.f;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {  // ql bytes 16i + 4t (i = 4h + c: 64h + 16c)
-        qla[i] = va ? ldg_u32_a2(ba + 16 * i + 4 * t) : 0u;
-        qlb[i] = vb ? ldg_u32_a2(bb + 16 * i + 4 * t) : 0u;
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {  // qh bytes 128 + 16i + 4t
-        qha[i] = va ? ldg_u32_a2(ba + 128 + 16 * i + 4 * t) : 0u;
-        qhb[i] = vb ? ldg_u32_a2(bb + 128 + 16 * i + 4 * t) : 0u;
-        sca[i] = va ? ldg_u32_a2(ba + 192 + 4 * i) : 0u;
-        scb[i] = vb ? ldg_u32_a2(bb + 192 + 4 * i) : 0u;
-      }
-      if (va) da = f16_bits_to_f32(ldg_u16(ba + 208));
-      if (vb) db = f16_bits_to_f32(ldg_u16(bb + 208));
-
-      q6_superblock(acc, qla, qlb, qha, qhb, sca, scb, da, db, xrow + sb * 256, dx, nb32, sb, t);
-    }
-    // ---- fixed-order reduction over warps
-    float* rb_ = red + parity * (kQ6Warps * 32 * 4);
-    reinterpret_cast<float4*>(rb_)[warp * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-    __syncthreads();
-    if (threadIdx.x < kQ6TileRows * kQ6MaxRows) {
-      const int rr = threadIdx.x % kQ6TileRows, cc = threadIdx.x / kQ6TileRows;
-      const int row = tile * kQ6TileRows + rr;
-      if (cc < p.rows && row < p.n) {
-        const int gg = rr & 7, up = rr >> 3;
-        const int ln = gg * 4 + (cc >> 1), comp = up * 2 + (cc & 1);
-        float sum = 0.f;
-#pragma unroll
-        for (int ww = 0; ww < kQ6Warps; ++ww) sum = __fadd_rn(sum, rb_[(ww * 32 + ln) * 4 + comp]);
-        p.out[(int64_t)cc * p.ldc + row] = f32_to_bf16_bits(sum);
-      }
-    }
-    parity ^= 1;
-  }
-}
-
-// ---------------------------------------------------------------------------------------
-// Streamed variant: the weight reaches shared memory through 1-D bulk copies (TMA) of 8-row
-// stages.  8 rows of Q6_K are 8 * 210 * (k / 256) = 1680 * (k / 256) bytes, a multiple of 16,
-// so every full stage starts and ends 16-byte aligned for any k; a ragged last stage copies
-// its 16-byte-multiple prefix in bulk and its last few bytes with plain loads.  A 16-row MMA
-// tile is two consecutive stages; the ring holds NS >= 3 stages, so the next tile is in
-// flight while this one is computed.  Each lane reads its bytes from shared memory as aligned
-// 32-bit pairs joined by a funnel shift (super-blocks are only 2-byte aligned).  The
-// arithmetic, its order and the warp split are those of q6k_mmvq_kernel, so the two give the
-// same bits.
-constexpr int kQ6StageRows = 8;
-constexpr int kQ6MaxStages = 6;
+constexpr int kQ6RegSlice = 2;    // super-blocks per slice whose B fragments stay in registers
+constexpr int kQ6MaxStages = 16;
 static __device__ int q6_fault_word = 0;
 
-__device__ __forceinline__ uint32_t lds_u32_a2(uint32_t saddr) {  // 2-byte aligned 32-bit load
-  const uint32_t a = saddr & ~3u;
-  uint32_t w0, w1;
-  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w0) : "r"(a));
-  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w1) : "r"(a + 4));
-  return __funnelshift_r(w0, w1, (saddr & 3u) * 8u);
-}
-__device__ __forceinline__ uint32_t lds_u16(uint32_t saddr) {
-  unsigned short v;
-  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(saddr));
-  return v;
-}
-
-struct Q6StreamParams {
+struct Q6RowsParams {
   Q6Params q;
-  int ns;             // ring stages
-  int stage_stride;   // bytes per stage slot (>= 8 rows, multiple of 128)
-  int ring_offset;    // byte offset of the ring in dynamic shared memory
+  int ns;            // ring stages (streamed)
+  int stage_rows;    // SR: 4 or 8
+  int stage_stride;  // bytes per stage slot (>= SR rows, multiple of 128)
+  int ring_offset;   // byte offset of the ring in dynamic shared memory
+  int early_w;       // the preceding kernel is this library's q8_1 quantize: weight copies may start before it ends
 };
 
-__global__ void __launch_bounds__(kQ6Threads, 1) q6k_stream_kernel(const Q6StreamParams sp) {
+__host__ __device__ __forceinline__ int q6_act_stride(int k) { return k + ((64 - k % 128) + 128) % 128; }
+__host__ __device__ __forceinline__ bool q6_reg_acts(int k) { return (k / 256 + kQ6Slices - 1) / kQ6Slices <= kQ6RegSlice; }
+constexpr size_t kQ6RedBytes = 2ull * kQ6Warps * 32 * 4 * 4;  // [2][warps][32 lanes][4 floats]
+// dxs, then (smem activations) xs, then the reduction buffer.
+__host__ __device__ __forceinline__ size_t q6_dx_bytes(int k) { return (size_t)(k / 32) * kQ6MaxRows * 4; }
+__host__ __device__ __forceinline__ size_t q6_base_bytes(int k, bool reg_acts) {
+  return q6_dx_bytes(k) + (reg_acts ? 0 : (size_t)kQ6MaxRows * q6_act_stride(k)) + kQ6RedBytes;
+}
+
+// Stage dxs (and, without register fragments, xs).
+__device__ void q6_stage_acts(const Q6Params& p, uint8_t* smem, bool stage_codes) {
+  const int nb32 = p.k / 32;
+  const int rs = q6_act_stride(p.k);
+  float* dxs = reinterpret_cast<float*>(smem);
+  uint8_t* xs = smem + q6_dx_bytes(p.k);
+  for (int it = threadIdx.x; it < kQ6MaxRows * nb32; it += blockDim.x) {
+    const int m = it / nb32, b = it % nb32;
+    const uint32_t* bw = reinterpret_cast<const uint32_t*>(p.q8 + ((int64_t)m * nb32 + b) * 36);
+    dxs[b * kQ6MaxRows + m] = m < p.rows ? f16_bits_to_f32(bw[0] & 0xffffu) : 0.f;
+    if (!stage_codes) continue;
+    uint8_t* dst = xs + m * rs + (b >> 3) * 256;
+    const int kb = (b & 7) * 32;  // first value of this block inside its super-block
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int k = kb + 4 * i;
+      *reinterpret_cast<uint32_t*>(dst + 64 * (k >> 6) + 16 * ((k >> 2) & 3) + 4 * ((k >> 4) & 3)) =
+          m < p.rows ? bw[1 + i] : 0u;
+    }
+  }
+}
+
+// B fragment of lane (g, t) for sub-block j of super-block sb, straight from the q8_1 rows.
+__device__ __forceinline__ uint32_t q6_bfrag(const Q6Params& p, int col, int sb, int j, int t) {
+  if (col >= p.rows) return 0u;
+  const int nb32 = p.k / 32;
+  return *reinterpret_cast<const uint32_t*>(p.q8 + ((int64_t)col * nb32 + 8 * sb + (j >> 1)) * 36 + 4 +
+                                            16 * (j & 1) + 4 * t);
+}
+
+// One super-block of the 16-row tile (rows g: wa, g+8: wb) against the 8 columns: bw[j] is the
+// lane's B fragment of sub-block j; dxs = dxs + (8 sb) 32 + 8 t.
+__device__ __forceinline__ void q6_superblock_8(float (&acc)[4], const Q6W& wa, const Q6W& wb, const uint32_t (&bw)[16],
+                                                uint32_t dxs) {
+  float tsb[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int blk = 0; blk < 8; ++blk) {
+    const int j0 = 2 * blk, j1 = j0 + 1;
+    int d0[4] = {0, 0, 0, 0}, d1[4] = {0, 0, 0, 0};
+    mma_s8_16816(d0, q6_codes_s8(wa, j0), q6_codes_s8(wb, j0), bw[j0]);
+    mma_s8_16816(d1, q6_codes_s8(wa, j1), q6_codes_s8(wb, j1), bw[j1]);
+    const uint2 dx = lds_u64(dxs + 32 * blk);
+    q6_block_step(tsb, d0, d1, q6_scale(wa, j0), q6_scale(wa, j1), q6_scale(wb, j0), q6_scale(wb, j1),
+                  __uint_as_float(dx.x), __uint_as_float(dx.y));
+  }
+  q6_superblock_end(acc, tsb, wa.d, wb.d);
+}
+
+// Fixed-order sum over the 16 warps' partials of a tile, one BF16 store per output.
+__device__ __forceinline__ void q6_reduce_store(const Q6Params& p, float* red, int tile, const float (&acc)[4]) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  reinterpret_cast<float4*>(red)[warp * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+  __syncthreads();
+  if (threadIdx.x < kQ6TileRows * kQ6MaxRows) {
+    const int rr = threadIdx.x % kQ6TileRows, cc = threadIdx.x / kQ6TileRows;
+    const int row = tile * kQ6TileRows + rr;
+    if (cc < p.rows && row < p.n) {
+      const int gg = rr & 7, up = rr >> 3;
+      const int ln = gg * 4 + (cc >> 1), comp = up * 2 + (cc & 1);
+      float sum = 0.f;
+#pragma unroll
+      for (int ww = 0; ww < kQ6Warps; ++ww) sum = __fadd_rn(sum, red[(ww * 32 + ln) * 4 + comp]);
+      p.out[(int64_t)cc * p.ldc + row] = f32_to_bf16_bits(sum);
+    }
+  }
+}
+
+template <bool kStream, bool kRegActs>
+__global__ void __launch_bounds__(kQ6Threads, 1) q6k_rows8_kernel(const Q6RowsParams sp) {
   extern __shared__ __align__(128) uint8_t smem[];
-  grid_dependents_launch();
-  grid_dependency_wait();  // launched early (programmatic): q8, blocks and out follow the preceding kernel
   __shared__ __align__(8) uint64_t full[kQ6MaxStages];
+  grid_dependents_launch();
   const Q6Params& p = sp.q;
   const int nsb = p.k / 256;
-  const int nb32 = p.k / 32;
-  const int rs = q6_row_stride(p.k);
+  const int rs = q6_act_stride(p.k);
   const int64_t row_bytes = (int64_t)nsb * 210;
-  int8_t* xs = reinterpret_cast<int8_t*>(smem);                              // [8][rs]
-  float* dx = reinterpret_cast<float*>(smem + kQ6MaxRows * rs);              // [8][nb32]
-  float* red = dx + kQ6MaxRows * nb32;                                       // [2][16 warps][32 lanes][4]
+  float* red = reinterpret_cast<float*>(smem + q6_base_bytes(p.k, kRegActs) - kQ6RedBytes);
   const uint32_t ring = smem_u32(smem + sp.ring_offset);
   const uint32_t full0 = smem_u32(full);
+  const int SR = kStream ? sp.stage_rows : 8, spt = kQ6TileRows / SR;
 
   const int ntiles = (p.n + kQ6TileRows - 1) / kQ6TileRows;
   const int T0 = (int)((int64_t)blockIdx.x * ntiles / gridDim.x);
   const int T1 = (int)((int64_t)(blockIdx.x + 1) * ntiles / gridDim.x);
-  const int nstages = 2 * (T1 - T0);
+  const int nstages = spt * (T1 - T0);
 
-  // Stage s of this CTA: rows [16 (T0 + s/2) + 8 (s%2), +8) clipped to n, into slot s % NS.
+  // Stage s of this CTA: rows [16 (T0 + s / spt) + SR (s % spt), +SR) clipped to n, slot s % NS.
   auto produce = [&](int s) {
     const int slot = s % sp.ns;
-    const int64_t r0 = (int64_t)(T0 + s / 2) * kQ6TileRows + (s % 2) * kQ6StageRows;
-    const int64_t nr = r0 >= p.n ? 0 : (p.n - r0 < kQ6StageRows ? p.n - r0 : kQ6StageRows);
+    const int64_t r0 = (int64_t)(T0 + s / spt) * kQ6TileRows + (s % spt) * SR;
+    const int64_t nr = r0 >= p.n ? 0 : (p.n - r0 < SR ? p.n - r0 : SR);
     const uint32_t bytes = (uint32_t)(nr * row_bytes);
     const uint32_t bulk = bytes & ~15u;
     const uint32_t dst = ring + (uint32_t)slot * sp.stage_stride;
@@ -264,90 +315,90 @@ __global__ void __launch_bounds__(kQ6Threads, 1) q6k_stream_kernel(const Q6Strea
     if (bulk) umma::bulk_load(dst, src, bulk, full0 + 8u * slot, umma::l2_policy_evict_first());
   };
 
-  if (threadIdx.x == 0) {
+  if (kStream && threadIdx.x == 0) {
     for (int i = 0; i < sp.ns; ++i) umma::bar_init(full0 + 8u * i, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    // Weight copies before the dependency wait only when the preceding kernel is this library's
+    // q8_1 quantize (it writes neither the weights nor the ragged tail's source).
+    if (sp.early_w)
+      for (int s = 0; s < sp.ns && s < nstages; ++s) produce(s);
+  }
+  grid_dependency_wait();  // q8, and the blocks unless early_w, follow the preceding kernel
+  if (kStream && threadIdx.x == 0 && !sp.early_w)
     for (int s = 0; s < sp.ns && s < nstages; ++s) produce(s);
-  }
-
-  // ---- stage the q8_1 rows (while the first weight stages are in flight)
-  for (int it = threadIdx.x; it < kQ6MaxRows * nb32; it += kQ6Threads) {
-    const int m = it / nb32, b = it % nb32;
-    uint32_t w[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    float d = 0.f;
-    if (m < p.rows) {
-      const uint8_t* blk = p.q8 + ((int64_t)m * nb32 + b) * 36;
-      const uint32_t* bw = reinterpret_cast<const uint32_t*>(blk);
-      d = f16_bits_to_f32(bw[0] & 0xffff);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) w[i] = bw[1 + i];
-    }
-    dx[m * nb32 + b] = d;
-    uint4* dst = reinterpret_cast<uint4*>(xs + m * rs + b * 32);
-    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-    dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-  }
-  __syncthreads();
+  q6_stage_acts(p, smem, !kRegActs);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int sb_begin = q6_slice_begin(nsb, warp), sb_end = q6_slice_begin(nsb, warp + 1);
-  const int8_t* xrow = xs + g * rs;  // B column g
-  int parity = 0;
+  const uint32_t dx0 = smem_u32(smem) + (uint32_t)(8 * t);
+  const uint32_t xs0 = smem_u32(smem) + (uint32_t)(q6_dx_bytes(p.k) + g * rs + 16 * t);
+  uint32_t bfr[kQ6RegSlice][16];
+  if (kRegActs) {
+#pragma unroll
+    for (int s = 0; s < kQ6RegSlice; ++s)
+#pragma unroll
+      for (int j = 0; j < 16; ++j) bfr[s][j] = sb_begin + s < sb_end ? q6_bfrag(p, g, sb_begin + s, j, t) : 0u;
+  }
+  __syncthreads();
 
+  const int sa_off = g / SR, sb_off = (g + 8) / SR;  // stages of rows g and g+8 within a tile
+  int parity = 0;
   for (int i = 0; T0 + i < T1; ++i) {
     const int tile = T0 + i;
-    const int sa = 2 * i, sb2 = 2 * i + 1;
-    const bool oka = umma::wait(full0 + 8u * (sa % sp.ns), (sa / sp.ns) & 1);
-    const bool okb = umma::wait(full0 + 8u * (sb2 % sp.ns), (sb2 / sp.ns) & 1);
-    if (!(oka && okb)) atomicOr(&q6_fault_word, 1);
-    const uint32_t base_a = ring + (uint32_t)(sa % sp.ns) * sp.stage_stride + (uint32_t)(g * row_bytes);
-    const uint32_t base_b = ring + (uint32_t)(sb2 % sp.ns) * sp.stage_stride + (uint32_t)(g * row_bytes);
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
     const int r0 = tile * kQ6TileRows + g;
     const bool va = r0 < p.n, vb = r0 + 8 < p.n;
-    for (int sb = sb_begin; sb < sb_end; ++sb) {
-      const uint32_t ba = base_a + (uint32_t)sb * 210u;
-      const uint32_t bb = base_b + (uint32_t)sb * 210u;
-      uint32_t qla[8], qlb[8], qha[4], qhb[4], sca[4], scb[4];
-      float da = 0.f, db = 0.f;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {  // ql bytes 16q + 4t
-        qla[q] = va ? lds_u32_a2(ba + 16 * q + 4 * t) : 0u;
-        qlb[q] = vb ? lds_u32_a2(bb + 16 * q + 4 * t) : 0u;
+    uint32_t base_a = 0, base_b = 0;
+    if (kStream) {
+      bool ok = true;
+      for (int q = 0; q < spt; ++q) {
+        const int s = spt * i + q;
+        ok &= umma::wait(full0 + 8u * (s % sp.ns), (s / sp.ns) & 1);
       }
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {  // qh bytes 128 + 16q + 4t, scales 192 + 4q
-        qha[q] = va ? lds_u32_a2(ba + 128 + 16 * q + 4 * t) : 0u;
-        qhb[q] = vb ? lds_u32_a2(bb + 128 + 16 * q + 4 * t) : 0u;
-        sca[q] = va ? lds_u32_a2(ba + 192 + 4 * q) : 0u;
-        scb[q] = vb ? lds_u32_a2(bb + 192 + 4 * q) : 0u;
+      if (!ok) atomicOr(&q6_fault_word, 1);
+      const int s_a = spt * i + sa_off, s_b = spt * i + sb_off;
+      base_a = ring + (uint32_t)(s_a % sp.ns) * sp.stage_stride + (uint32_t)((g % SR) * row_bytes);
+      base_b = ring + (uint32_t)(s_b % sp.ns) * sp.stage_stride + (uint32_t)(((g + 8) % SR) * row_bytes);
+    }
+    const uint8_t* ga = p.blocks + (int64_t)r0 * row_bytes;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    auto one = [&](int sb, const uint32_t (&bw)[16]) {
+      Q6W wa, wb;
+      if (kStream) {
+        const uint32_t ba = base_a + (uint32_t)sb * 210u, bb = base_b + (uint32_t)sb * 210u;
+        if (__all_sync(0xffffffffu, ((ba | bb) & 3u) == 0)) {
+          q6_load_smem<true>(wa, va, ba, t);
+          q6_load_smem<true>(wb, vb, bb, t);
+        } else {
+          q6_load_smem<false>(wa, va, ba, t);
+          q6_load_smem<false>(wb, vb, bb, t);
+        }
+      } else {
+        q6_load_global(wa, va, ga + (int64_t)sb * 210, t);
+        q6_load_global(wb, vb, ga + 8 * row_bytes + (int64_t)sb * 210, t);
       }
-      if (va) da = f16_bits_to_f32(lds_u16(ba + 208));
-      if (vb) db = f16_bits_to_f32(lds_u16(bb + 208));
-
-      q6_superblock(acc, qla, qlb, qha, qhb, sca, scb, da, db, xrow + sb * 256, dx, nb32, sb, t);
-    }
-    // ---- fixed-order reduction over warps; after its barrier the tile's stages are free
-    float* rb_ = red + parity * (kQ6Warps * 32 * 4);
-    reinterpret_cast<float4*>(rb_)[warp * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      if (sa + sp.ns < nstages) produce(sa + sp.ns);
-      if (sb2 + sp.ns < nstages) produce(sb2 + sp.ns);
-    }
-    if (threadIdx.x < kQ6TileRows * kQ6MaxRows) {
-      const int rr = threadIdx.x % kQ6TileRows, cc = threadIdx.x / kQ6TileRows;
-      const int row = tile * kQ6TileRows + rr;
-      if (cc < p.rows && row < p.n) {
-        const int gg = rr & 7, up = rr >> 3;
-        const int ln = gg * 4 + (cc >> 1), comp = up * 2 + (cc & 1);
-        float sum = 0.f;
+      q6_superblock_8(acc, wa, wb, bw, dx0 + 256u * sb);
+    };
+    if (kRegActs) {
 #pragma unroll
-        for (int ww = 0; ww < kQ6Warps; ++ww) sum = __fadd_rn(sum, rb_[(ww * 32 + ln) * 4 + comp]);
-        p.out[(int64_t)cc * p.ldc + row] = f32_to_bf16_bits(sum);
+      for (int s = 0; s < kQ6RegSlice; ++s)
+        if (sb_begin + s < sb_end) one(sb_begin + s, bfr[s]);
+    } else {
+      for (int sb = sb_begin; sb < sb_end; ++sb) {
+        uint32_t bw[16];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint4 v = lds128(xs0 + 256u * sb + 64 * q);
+          bw[4 * q] = v.x, bw[4 * q + 1] = v.y, bw[4 * q + 2] = v.z, bw[4 * q + 3] = v.w;
+        }
+        one(sb, bw);
       }
     }
+    // fixed-order reduction over warps; after its barrier the tile's stages are free
+    q6_reduce_store(p, red + parity * (kQ6Warps * 32 * 4), tile, acc);
+    if (kStream && threadIdx.x == 0)
+      for (int q = 0; q < spt; ++q)
+        if (spt * i + q + sp.ns < nstages) produce(spt * i + q + sp.ns);
     parity ^= 1;
   }
 }
@@ -355,43 +406,40 @@ __global__ void __launch_bounds__(kQ6Threads, 1) q6k_stream_kernel(const Q6Strea
 // ---------------------------------------------------------------------------------------
 // Wide variant: 9..64 q8_1 rows in one weight pass.  Whole activation rows no longer fit in
 // shared memory (64 rows of codes at K = 7168 take 458 KB), so the loop order is turned
-// around: a CTA takes its 16-row weight tiles in row-blocks of up to kQWWarps tiles, one tile
-// per consumer warp, and the row-block walks K one super-block at a time.
+// around: a CTA takes its 16-row weight tiles in row-blocks of up to W tiles, one tile per
+// consumer warp, and the row-block walks K one super-block at a time.
 //   - Activations: a producer warp copies each super-block's q8_1 blocks of every activation
 //     row (288 contiguous bytes per row) into a ring shared by the row-block's warps, with
 //     16-byte cp.async and one mbarrier arrival per lane; the activations are re-read (from
 //     L2) once per row-block, not once per tile.
-//   - Weights: every consumer warp streams its own tile through a private ring of kQWDepth
-//     stages with 16-byte cp.async (Ampere-style multistage pipeline, no registers held):
-//     per row the 16-byte aligned span that covers the super-block's 210 bytes (at most 224;
-//     super-blocks are only 2-byte aligned), read back at the span's offset with
-//     funnel-shifted 32-bit shared loads.  The buffer's last bytes past its last 16-byte
-//     boundary are stored with plain loads, so no copy reads past the weight buffer.
-// Each consumer warp runs NT 8-column MMAs per sub-block on one decoded A fragment.
-// The per-output arithmetic and its order are those of the 8-row kernels: K is cut into the
-// same 16 slices (q6_slice_begin), each slice is accumulated alone from 0 with the same
-// per-block step, and the slices are added to 0 in order -- so a row's bits do not depend on
-// which kernel, or how many rows, served it.
-// 15 consumer warps + 1 producer: 16 warps, 4 per SM sub-partition, so 128 registers a thread
-constexpr int kQWWarps = 15;
-constexpr int kQWThreads = (kQWWarps + 1) * 32;
+//   - Weights: every consumer warp streams its own tile through a private ring of `depth`
+//     stages with 16-byte cp.async: per row the 16-byte aligned span that covers the
+//     super-block's 210 bytes (at most 224; super-blocks are only 2-byte aligned), read back
+//     at the span's offset.  The buffer's last bytes past its last 16-byte boundary are stored
+//     with plain loads, so no copy reads past the weight buffer.
+// Each consumer warp decodes a weight fragment once per sub-block ((q - 32) as signed bytes)
+// and runs NT 8-column MMAs on it.  The K-slices of the 8-row kernels are kept: each slice is
+// accumulated alone from 0 and added to the total at the slice's end (q6_slice_ends).
+// NT <= 4: 15 consumer warps + 1 producer (128 registers a thread); NT = 8: 7 + 1 (255).
 constexpr int kQWRowBytes = 288;   // one super-block of one q8_1 row: 8 blocks
 constexpr int kQWRowStride = 304;  // 76 words: the 8 B-fragment rows hit 32 banks
 constexpr int kQWSpan = 240;       // staged bytes per weight row and super-block (>= 224)
 constexpr int kQWTileBytes = kQ6TileRows * kQWSpan;
 constexpr int kQWMaxActStages = 4;
 
+template <int NT>
+struct QW {
+  static constexpr int kWarps = NT >= 8 ? 7 : 15;  // consumer warps
+  static constexpr int kThreads = (kWarps + 1) * 32;
+};
+
 struct Q6WideParams {
   Q6Params q;
   int act_stages;  // activation ring stages of NT * 8 * kQWRowStride bytes
   int depth;       // weight stages per consumer warp (>= 2)
+  int early_w;     // the preceding kernel is this library's q8_1 quantize (see Q6RowsParams)
 };
 
-__device__ __forceinline__ uint32_t lds_u32(uint32_t saddr) {
-  uint32_t v;
-  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(saddr));
-  return v;
-}
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
@@ -407,49 +455,34 @@ __device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
 
 // One super-block of one warp's 16-row tile against NT 8-column groups of the staged chunk at
 // `xs` (row stride kQWRowStride, block b of row m at m * stride + 36 b: f16 d, f16 s, 32 codes).
-// Per (row, column) the same integer and float steps, in the same order, as q6_superblock.
 template <int NT>
-__device__ __forceinline__ void q6_superblock_wide(float (&acc)[NT][4], const uint32_t (&qla)[8],
-                                                   const uint32_t (&qlb)[8], const uint32_t (&qha)[4],
-                                                   const uint32_t (&qhb)[4], const uint32_t (&sca)[4],
-                                                   const uint32_t (&scb)[4], float da, float db, uint32_t xs, int g,
-                                                   int t) {
+__device__ __forceinline__ void q6_superblock_wide(float (&acc)[NT][4], const Q6W& wa, const Q6W& wb, uint32_t xs,
+                                                   int g, int t) {
+  float tsb[NT][4];
 #pragma unroll
-  for (int blk = 0; blk < 8; ++blk) {  // unrolled: the fragment arrays stay in registers
-    uint32_t a0[2], a1[2];
-    int ra[2], rb[2];
+  for (int ct = 0; ct < NT; ++ct)
 #pragma unroll
-    for (int hj = 0; hj < 2; ++hj) {
-      const int j = 2 * blk + hj;
-      const int h = j >> 3, u = (j & 7) >> 1;
-      const int qi = 4 * h + 2 * (u & 1) + (j & 1);
-      const int hi = 2 * h + (j & 1);
-      const int nsh = (u >> 1) * 4, hsh = 2 * u;
-      a0[hj] = q6_to_s8x4(((qla[qi] >> nsh) & 0x0f0f0f0fu) | (((qha[hi] >> hsh) & 0x03030303u) << 4));
-      a1[hj] = q6_to_s8x4(((qlb[qi] >> nsh) & 0x0f0f0f0fu) | (((qhb[hi] >> hsh) & 0x03030303u) << 4));
-      const int sha = 24 - 8 * (j & 3);
-      ra[hj] = (int)(sca[j >> 2] << sha) >> 24;
-      rb[hj] = (int)(scb[j >> 2] << sha) >> 24;
-    }
+    for (int i = 0; i < 4; ++i) tsb[ct][i] = 0.f;
+#pragma unroll
+  for (int blk = 0; blk < 8; ++blk) {
+    const int j0 = 2 * blk, j1 = j0 + 1;
+    const uint32_t a00 = q6_codes_s8(wa, j0), a01 = q6_codes_s8(wb, j0);
+    const uint32_t a10 = q6_codes_s8(wa, j1), a11 = q6_codes_s8(wb, j1);
+    const int ra0 = q6_scale(wa, j0), ra1 = q6_scale(wa, j1), rb0 = q6_scale(wb, j0), rb1 = q6_scale(wb, j1);
 #pragma unroll
     for (int ct = 0; ct < NT; ++ct) {
       const uint32_t brow = xs + (uint32_t)((8 * ct + g) * kQWRowStride + 36 * blk + 4 + 4 * t);
       int d0[4] = {0, 0, 0, 0}, d1[4] = {0, 0, 0, 0};
-      mma_s8_16816(d0, a0[0], a1[0], lds_u32(brow));
-      mma_s8_16816(d1, a0[1], a1[1], lds_u32(brow + 16));
-      const int is0 = d0[0] * ra[0] + d1[0] * ra[1];
-      const int is1 = d0[1] * ra[0] + d1[1] * ra[1];
-      const int is2 = d0[2] * rb[0] + d1[2] * rb[1];
-      const int is3 = d0[3] * rb[0] + d1[3] * rb[1];
+      mma_s8_16816(d0, a00, a01, lds_u32(brow));
+      mma_s8_16816(d1, a10, a11, lds_u32(brow + 16));
       const uint32_t drow = xs + (uint32_t)((8 * ct + 2 * t) * kQWRowStride + 36 * blk);
       const float dx0 = f16_bits_to_f32(lds_u16(drow));
       const float dx1 = f16_bits_to_f32(lds_u16(drow + kQWRowStride));
-      acc[ct][0] = q6_block_step(acc[ct][0], is0, da, dx0);
-      acc[ct][1] = q6_block_step(acc[ct][1], is1, da, dx1);
-      acc[ct][2] = q6_block_step(acc[ct][2], is2, db, dx0);
-      acc[ct][3] = q6_block_step(acc[ct][3], is3, db, dx1);
+      q6_block_step(tsb[ct], d0, d1, ra0, ra1, rb0, rb1, dx0, dx1);
     }
   }
+#pragma unroll
+  for (int ct = 0; ct < NT; ++ct) q6_superblock_end(acc[ct], tsb[ct], wa.d, wb.d);
 }
 
 // Stage super-block sb of the 16 rows of tile `tile` into `dst` (row i at i * kQWSpan) with
@@ -477,10 +510,13 @@ __device__ __forceinline__ void q6_stage_tile(const Q6Params& p, int64_t row_byt
 }
 
 template <int NT>
-__global__ void __launch_bounds__(kQWThreads, 1) q6k_wide_kernel(const Q6WideParams wp) {
+__global__ void __launch_bounds__(QW<NT>::kThreads, 1) q6k_wide_kernel(const Q6WideParams wp) {
+  constexpr int kWarps = QW<NT>::kWarps;
   extern __shared__ __align__(128) uint8_t smem[];
   grid_dependents_launch();
-  grid_dependency_wait();  // launched early (programmatic): q8, blocks and out follow the preceding kernel
+  // launched early (programmatic): q8, blocks and out follow the preceding kernel; with early_w
+  // only the consumers' first weight stages are requested before the wait
+  if (!wp.early_w) grid_dependency_wait();
   __shared__ __align__(8) uint64_t full[kQWMaxActStages], empty[kQWMaxActStages];
   const Q6Params& p = wp.q;
   const int nsb = p.k / 256;
@@ -498,7 +534,7 @@ __global__ void __launch_bounds__(kQWThreads, 1) q6k_wide_kernel(const Q6WidePar
   const int T0 = (int)((int64_t)blockIdx.x * ntiles / gridDim.x);
   const int T1 = (int)((int64_t)(blockIdx.x + 1) * ntiles / gridDim.x);
   const int nt = T1 - T0;
-  const int nrb = (nt + kQWWarps - 1) / kQWWarps;  // row-blocks, as even as possible
+  const int nrb = (nt + kWarps - 1) / kWarps;  // row-blocks, as even as possible
   const int nchunks = nrb * nsb;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -510,14 +546,15 @@ __global__ void __launch_bounds__(kQWThreads, 1) q6k_wide_kernel(const Q6WidePar
   if (threadIdx.x == 0) {
     for (int i = 0; i < ns; ++i) {
       umma::bar_init(full0 + 8u * i, 32);  // one arrival per producer lane, when its copies land
-      umma::bar_init(empty0 + 8u * i, kQWWarps);
+      umma::bar_init(empty0 + 8u * i, kWarps);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
 
-  if (warp == kQWWarps) {
+  if (warp == kWarps) {
     // ---------------- producer: chunk c = (row-block c / nsb, super-block c % nsb)
+    if (wp.early_w) grid_dependency_wait();
     constexpr int kPieces = kQWRowBytes / 16;
     for (int c = 0; c < nchunks; ++c) {
       const int slot = c % ns, sb = c % nsb;
@@ -550,6 +587,7 @@ __global__ void __launch_bounds__(kQWThreads, 1) q6k_wide_kernel(const Q6WidePar
       if (active && s < nsb) q6_stage_tile(p, row_bytes, buf_end, tile, s, my_ring + (uint32_t)(s * kQWTileBytes), lane);
       cp_async_commit();
     }
+    if (wp.early_w && r == 0) grid_dependency_wait();
     float tot[NT][4], sl[NT][4];
 #pragma unroll
     for (int ct = 0; ct < NT; ++ct)
@@ -574,23 +612,15 @@ __global__ void __launch_bounds__(kQWThreads, 1) q6k_wide_kernel(const Q6WidePar
                             (uint32_t)((reinterpret_cast<uintptr_t>(p.blocks) + (uintptr_t)((int64_t)r0 * row_bytes + 210 * sb)) & 15u);
         const uint32_t bb = wbase + (uint32_t)((g + 8) * kQWSpan) +
                             (uint32_t)((reinterpret_cast<uintptr_t>(p.blocks) + (uintptr_t)((int64_t)(r0 + 8) * row_bytes + 210 * sb)) & 15u);
-        uint32_t qla[8], qlb[8], qha[4], qhb[4], sca[4], scb[4];
-        float da = 0.f, db = 0.f;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          qla[q] = va ? lds_u32_a2(ba + 16 * q + 4 * t) : 0u;
-          qlb[q] = vb ? lds_u32_a2(bb + 16 * q + 4 * t) : 0u;
+        Q6W wa, wb;
+        if (__all_sync(0xffffffffu, ((ba | bb) & 3u) == 0)) {
+          q6_load_smem<true>(wa, va, ba, t);
+          q6_load_smem<true>(wb, vb, bb, t);
+        } else {
+          q6_load_smem<false>(wa, va, ba, t);
+          q6_load_smem<false>(wb, vb, bb, t);
         }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          qha[q] = va ? lds_u32_a2(ba + 128 + 16 * q + 4 * t) : 0u;
-          qhb[q] = vb ? lds_u32_a2(bb + 128 + 16 * q + 4 * t) : 0u;
-          sca[q] = va ? lds_u32_a2(ba + 192 + 4 * q) : 0u;
-          scb[q] = vb ? lds_u32_a2(bb + 192 + 4 * q) : 0u;
-        }
-        if (va) da = f16_bits_to_f32(lds_u16(ba + 208));
-        if (vb) db = f16_bits_to_f32(lds_u16(bb + 208));
-        q6_superblock_wide<NT>(sl, qla, qlb, qha, qhb, sca, scb, da, db, st, g, t);
+        q6_superblock_wide<NT>(sl, wa, wb, st, g, t);
       }
       __syncwarp();  // the weight stage and the activation slot are read
       if (lane == 0) umma::arrive(empty0 + 8u * slot);
@@ -627,23 +657,19 @@ __global__ void __launch_bounds__(kQWThreads, 1) q6k_wide_kernel(const Q6WidePar
   }
 }
 
-size_t q6k_smem_bytes(int k) {
-  int rs = k + ((16 - k % 128) + 128) % 128;
-  return (size_t)kQ6MaxRows * rs + (size_t)kQ6MaxRows * (k / 32) * 4 + 2ull * kQ6Warps * 32 * 4 * 4;
-}
-
 }  // namespace
 
 namespace {
 
 template <int NT>
-int launch_wide(const Q6Params& p, int sms, int smem_optin, cudaStream_t s) {
+int launch_wide(const Q6Params& p, int sms, int smem_optin, cudaStream_t s, bool early_w) {
+  constexpr int kWarps = QW<NT>::kWarps;
   const size_t act = (size_t)NT * 8 * kQWRowStride;
   const size_t limit = (size_t)smem_optin > 1024 ? (size_t)smem_optin - 1024 : 0;  // static smem < 1 KB
   // three weight stages per warp when they fit beside at least two activation stages
   int depth = 3;
-  if ((size_t)kQWWarps * depth * kQWTileBytes + 2 * act > limit) depth = 2;
-  const size_t wbytes = (size_t)kQWWarps * depth * kQWTileBytes;
+  if ((size_t)kWarps * depth * kQWTileBytes + 2 * act > limit) depth = 2;
+  const size_t wbytes = (size_t)kWarps * depth * kQWTileBytes;
   if (wbytes + 2 * act > limit) return DLMH_ERR_UNSUPPORTED;
   int ns = (int)((limit - wbytes) / act);
   if (ns > kQWMaxActStages) ns = kQWMaxActStages;
@@ -652,7 +678,15 @@ int launch_wide(const Q6Params& p, int sms, int smem_optin, cudaStream_t s) {
     return DLMH_ERR_CUDA;
   const int ntiles = (p.n + kQ6TileRows - 1) / kQ6TileRows;
   const int grid = ntiles < sms ? ntiles : sms;
-  return umma::launch_pdl(q6k_wide_kernel<NT>, dim3(grid), dim3(kQWThreads), smem, s, Q6WideParams{p, ns, depth});
+  return umma::launch_pdl(q6k_wide_kernel<NT>, dim3(grid), dim3(QW<NT>::kThreads), smem, s,
+                          Q6WideParams{p, ns, depth, early_w ? 1 : 0});
+}
+
+template <bool kStream, bool kRegActs>
+int launch_rows8(const Q6RowsParams& sp, int grid, size_t smem, cudaStream_t s) {
+  if (ensure_dynamic_smem(reinterpret_cast<const void*>(q6k_rows8_kernel<kStream, kRegActs>), (int)smem) != DLMH_OK)
+    return DLMH_ERR_CUDA;
+  return umma::launch_pdl(q6k_rows8_kernel<kStream, kRegActs>, dim3(grid), dim3(kQ6Threads), smem, s, sp);
 }
 
 }  // namespace
@@ -660,41 +694,52 @@ int launch_wide(const Q6Params& p, int sms, int smem_optin, cudaStream_t s) {
 int q6k_wide_rows(int rows) { return rows <= 8 ? 8 : rows <= 16 ? 16 : rows <= 32 ? 32 : 64; }
 
 int q6k_mmvq_launch(const uint8_t* blocks, int n, int k, const uint8_t* q8, int rows, uint16_t* out, int64_t ldc,
-                    cudaStream_t s) {
+                    cudaStream_t s, bool after_prepass) {
   const DeviceInfo di = device_info();
   if (di.sms <= 0) return DLMH_ERR_CUDA;
+  const Q6Params p{blocks, n, k, q8, rows, out, ldc};
   if (rows > kQ6MaxRows) {  // 9..64 rows: one pass of the wide kernel (16-byte aligned blocks, q8_1 rows)
     if (rows > 64) return DLMH_ERR_ROWS;
     if ((reinterpret_cast<uintptr_t>(q8) & 15u) || (reinterpret_cast<uintptr_t>(blocks) & 15u)) return DLMH_ERR_ALIGN;
-    const Q6Params p{blocks, n, k, q8, rows, out, ldc};
     switch (q6k_wide_rows(rows)) {
-      case 16: return launch_wide<2>(p, di.sms, di.smem_optin, s);
-      case 32: return launch_wide<4>(p, di.sms, di.smem_optin, s);
-      default: return launch_wide<8>(p, di.sms, di.smem_optin, s);
+      case 16: return launch_wide<2>(p, di.sms, di.smem_optin, s, after_prepass);
+      case 32: return launch_wide<4>(p, di.sms, di.smem_optin, s, after_prepass);
+      default: return launch_wide<8>(p, di.sms, di.smem_optin, s, after_prepass);
     }
   }
-  const size_t base_smem = q6k_smem_bytes(k);
-  Q6Params p{blocks, n, k, q8, rows, out, ldc};
+  const bool reg = q6_reg_acts(k);
+  const size_t base_smem = q6_base_bytes(k, reg);
   const int ntiles = (n + kQ6TileRows - 1) / kQ6TileRows;
   const int grid = ntiles < di.sms ? ntiles : di.sms;
-  // streamed variant when the ring holds at least three 8-row stages and the blocks start
-  // 16-byte aligned (then every 8-row stage does); both variants give the same bits
+  // Streamed when the B fragments stay in registers (K <= 8192: then the ring has room), the
+  // blocks start 16-byte aligned (then every stage does) and the ring holds more than one tile:
+  // the stage size (8 or 4 rows) that gives the most tiles in the ring, up to two (the next
+  // tile lands while this one is computed).  Otherwise 16-bit global weight loads.
   const size_t ring_offset = (base_smem + 127) / 128 * 128;
-  const size_t stage_stride = ((size_t)kQ6StageRows * (k / 256) * 210 + 127) / 128 * 128;
   const size_t limit = (size_t)di.smem_optin > 2048 ? (size_t)di.smem_optin - 2048 : 0;
-  int ns = limit > ring_offset ? (int)((limit - ring_offset) / stage_stride) : 0;
-  if (ns > kQ6MaxStages) ns = kQ6MaxStages;
-  if (ns >= 3 && (reinterpret_cast<uintptr_t>(blocks) & 15u) == 0) {
-    const size_t smem = ring_offset + (size_t)ns * stage_stride;
-    if (ensure_dynamic_smem(reinterpret_cast<const void*>(q6k_stream_kernel), (int)smem) != DLMH_OK)
-      return DLMH_ERR_CUDA;
-    Q6StreamParams sp{p, ns, (int)stage_stride, (int)ring_offset};
-    return umma::launch_pdl(q6k_stream_kernel, dim3(grid), dim3(kQ6Threads), smem, s, sp);
+  const int nsb = k / 256;
+  Q6RowsParams best{p, 0, 0, 0, (int)ring_offset, after_prepass ? 1 : 0};
+  double best_tiles = 1.0;
+  for (int sr = 8; sr >= 4 && reg && (reinterpret_cast<uintptr_t>(blocks) & 15u) == 0; sr -= 4) {
+    if (((size_t)sr * nsb * 210) % 16 != 0) continue;
+    const size_t stage_stride = ((size_t)sr * nsb * 210 + 127) / 128 * 128;
+    int ns = limit > ring_offset ? (int)((limit - ring_offset) / stage_stride) : 0;
+    const int spt = kQ6TileRows / sr;
+    if (ns > 2 * spt) ns = 2 * spt;
+    if (ns > kQ6MaxStages) ns = kQ6MaxStages;
+    const double tiles = (double)ns / spt;
+    if (tiles > best_tiles + 1e-9) {
+      best.ns = ns, best.stage_rows = sr, best.stage_stride = (int)stage_stride;
+      best_tiles = tiles;
+    }
+  }
+  if (best.ns > 0) {
+    const size_t smem = ring_offset + (size_t)best.ns * best.stage_stride;
+    return launch_rows8<true, true>(best, grid, smem, s);
   }
   if (base_smem + 1024 > (size_t)di.smem_optin) return DLMH_ERR_UNSUPPORTED;
-  if (ensure_dynamic_smem(reinterpret_cast<const void*>(q6k_mmvq_kernel), (int)base_smem) != DLMH_OK)
-    return DLMH_ERR_CUDA;
-  return umma::launch_pdl(q6k_mmvq_kernel, dim3(grid), dim3(kQ6Threads), base_smem, s, p);
+  const Q6RowsParams sp{p, 1, 8, 0, 0, 0};
+  return reg ? launch_rows8<false, true>(sp, grid, base_smem, s) : launch_rows8<false, false>(sp, grid, base_smem, s);
 }
 
 int q6k_fault(int reset) {

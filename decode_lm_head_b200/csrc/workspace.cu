@@ -17,6 +17,7 @@ namespace {
 struct Binding {
   int dev;
   unsigned long long stream_id;
+  cudaStream_t handle;
   uint8_t* ws;
   size_t bytes;
 };
@@ -27,7 +28,8 @@ Binding g_bind[kMaxBindings];
 int g_nbind = 0;
 
 // A stream's key: cudaStreamGetId (unique within the context, never reused after the stream
-// is destroyed); the legacy default stream, which has no id, keys as ~0.
+// is destroyed); the legacy default stream, which has no id, keys as ~0.  Not called while
+// the stream is being captured (the query would invalidate the capture).
 int stream_key(cudaStream_t s, int* dev, unsigned long long* id) {
   if (cudaGetDevice(dev) != cudaSuccess) return DLMH_ERR_CUDA;
   if (cudaStreamGetId(s, id) != cudaSuccess) {
@@ -41,6 +43,13 @@ int stream_key(cudaStream_t s, int* dev, unsigned long long* id) {
 int find(int dev, unsigned long long id) {
   for (int i = 0; i < g_nbind; ++i)
     if (g_bind[i].dev == dev && g_bind[i].stream_id == id) return i;
+  return -1;
+}
+
+// During capture the stream's id cannot be queried: the binding is found by its handle.
+int find_handle(int dev, cudaStream_t s) {
+  for (int i = 0; i < g_nbind; ++i)
+    if (g_bind[i].dev == dev && g_bind[i].handle == s) return i;
   return -1;
 }
 
@@ -59,13 +68,20 @@ int tiles_of(int op, int n) {
 
 int call_scratch(int op, int n, int k, int rows, cudaStream_t s, UmmaScratch* out) {
   *out = UmmaScratch{};
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) return DLMH_ERR_CUDA;
+  const bool capturing = cs != cudaStreamCaptureStatusNone;
   int dev = 0;
   unsigned long long id = 0;
-  if (stream_key(s, &dev, &id) != DLMH_OK) return DLMH_OK;  // no binding can exist: the pool
+  if (capturing) {
+    if (cudaGetDevice(&dev) != cudaSuccess) return DLMH_ERR_CUDA;
+  } else if (stream_key(s, &dev, &id) != DLMH_OK) {
+    return DLMH_OK;  // no binding can exist: the pool
+  }
   Binding b{};
   {
     std::lock_guard<std::mutex> lock(g_mu);
-    const int i = find(dev, id);
+    const int i = capturing ? find_handle(dev, s) : find(dev, id);
     if (i < 0) return DLMH_OK;
     b = g_bind[i];
   }
@@ -73,15 +89,10 @@ int call_scratch(int op, int n, int k, int rows, cudaStream_t s, UmmaScratch* ou
   if (di.sms <= 0) return DLMH_ERR_CUDA;
   const WsLayout L = ws_layout(op == DLMH_OP_W8A16, tiles_of(op, n), k, rows, di.sms);
   if ((int64_t)b.bytes < L.total) return DLMH_ERR_WORKSPACE;
-  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
-  if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) {
-    (void)cudaGetLastError();
-    cs = cudaStreamCaptureStatusActive;  // unknown: keep the static order
-  }
   out->caller = true;
   // a captured launch takes the static tile order: a graph holds no counter, so replays of it
   // may run anywhere; both orders give the same outputs
-  out->queue = cs == cudaStreamCaptureStatusNone ? reinterpret_cast<int*>(b.ws) : nullptr;
+  out->queue = capturing ? nullptr : reinterpret_cast<int*>(b.ws);
   out->codes = b.ws + L.codes_off;
   out->codes_cap = (size_t)L.codes_bytes;
   out->partial = reinterpret_cast<float*>(b.ws + L.partial_off);
@@ -112,13 +123,13 @@ int dlmh_set_workspace(void* ws, size_t bytes, void* stream) {
   unsigned long long id = 0;
   if (ws && (reinterpret_cast<uintptr_t>(ws) & 255u)) return DLMH_ERR_ALIGN;
   if (ws && bytes < (size_t)dlmh::kWsQueueBytes) return DLMH_ERR_WORKSPACE;
-  if (dlmh::stream_key(s, &dev, &id) != DLMH_OK) return DLMH_ERR_CUDA;
   cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
   if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) {
     (void)cudaGetLastError();
     return DLMH_ERR_CUDA;
   }
   if (cs != cudaStreamCaptureStatusNone) return DLMH_ERR_UNSUPPORTED;
+  if (dlmh::stream_key(s, &dev, &id) != DLMH_OK) return DLMH_ERR_CUDA;
   std::lock_guard<std::mutex> lock(dlmh::g_mu);
   const int i = dlmh::find(dev, id);
   if (!ws) {  // unbind: the stream's calls go back to the pool
@@ -131,7 +142,7 @@ int dlmh_set_workspace(void* ws, size_t bytes, void* stream) {
     (void)cudaGetLastError();
     return DLMH_ERR_CUDA;
   }
-  const dlmh::Binding b{dev, id, static_cast<uint8_t*>(ws), bytes};
+  const dlmh::Binding b{dev, id, s, static_cast<uint8_t*>(ws), bytes};
   if (i >= 0)
     dlmh::g_bind[i] = b;
   else

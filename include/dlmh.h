@@ -392,7 +392,9 @@ DLMH_API int dlmh_plan_chunks(int op, int rows, int k, int* offsets, int* counts
  *   The call zeroes the first 256 bytes (the tile queue) with cudaMemsetAsync on `stream`;
  *   every launch leaves them at zero.  ws == NULL unbinds (calls go back to the pool).  Calls
  *   that use one workspace must not overlap on the GPU: bind one per stream.  The library
- *   never frees ws; unbind before freeing it.  Bind outside stream capture
+ *   never frees ws; unbind before freeing it, and before destroying the stream (a call being
+ *   captured into a CUDA graph finds its stream's workspace by the stream handle, which a
+ *   new stream may reuse; eager calls use the stream's id).  Bind outside stream capture
  *   (DLMH_ERR_UNSUPPORTED while the stream is capturing).  Errors: DLMH_ERR_ALIGN,
  *   DLMH_ERR_WORKSPACE (bytes < 256), DLMH_ERR_CAPACITY (1024 streams bound),
  *   DLMH_ERR_CUDA.  (No counterpart in the pages' argument lists: their scratch is a field

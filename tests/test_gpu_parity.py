@@ -309,8 +309,6 @@ def test_w4a16_tiers(n, k):
     for m in (1, 4, 5, 6, 7, 8, 16, 17):
         part = bits(dl.w4a16_gemv(wp, ws, gl, x[:m]))
         assert np.array_equal(part, full[:m]), f"row invariance M={m}"
-    with pytest.raises(dl.DlmhError):
-        dl.w4a16_gemv(wp, ws, gl, synth.bf16_rows(33, k, 10, DEV))
 
 
 # ---------------------------------------------------------------------------
@@ -377,10 +375,12 @@ def test_q6k_mmvq_and_head(n, k):
         assert np.array_equal(part, full[:m]), f"row invariance M={m}"
 
 
-@pytest.mark.parametrize("n,k", [(1000, 7168), (37, 512), (45, 1280)])
+@pytest.mark.parametrize("n,k", [(1000, 7168), (37, 512), (45, 1280), (1000, 8192), (300, 8448)])
 def test_q6k_streamed_and_register_kernels_agree(n, k):
-    # 16-byte-aligned blocks take the TMA-streamed kernel, 2-byte-aligned ones the
-    # register-load kernel; both use the same arithmetic in the same order
+    # 16-byte-aligned blocks take the TMA-streamed kernel (8-row stages; 4-row ones at k = 8192),
+    # 2-byte-aligned ones the register-load kernel; k = 8448 (33 super-blocks: slices of 3)
+    # stages the activation codes in shared memory instead of registers.  All use the same
+    # arithmetic in the same order
     blocks = synth.q6k_blocks(n, k, 6, DEV)
     flat = torch.zeros(blocks.numel() + 16, dtype=torch.uint8, device=DEV)
     flat[2:2 + blocks.numel()] = blocks.reshape(-1)
