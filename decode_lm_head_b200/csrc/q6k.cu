@@ -114,7 +114,10 @@ __device__ __forceinline__ uint32_t lds_u32_a2(uint32_t saddr) {
   return __funnelshift_r(lds_u32(a), lds_u32(a + 4), (saddr & 3u) * 8u);
 }
 
-// Super-block at shared address `ba` (4-byte aligned when kAligned, else 2-byte aligned).
+// Super-block at shared address `ba`: kAligned only when ba is 4-byte aligned; the other path
+// takes any even ba (the lanes of one warp may mix both alignments when a row holds an odd
+// number of super-blocks).  It reads the aligned words that cover each field, all inside
+// [ba - 2, ba + 210).
 template <bool kAligned>
 __device__ __forceinline__ void q6_load_smem(Q6W& w, bool valid, uint32_t ba, int t) {
   if (!valid) {
@@ -133,12 +136,13 @@ __device__ __forceinline__ void q6_load_smem(Q6W& w, bool valid, uint32_t ba, in
   if (kAligned) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) w.sc[i] = lds_u32(ba + 192 + 4 * i);
-  } else {  // 16 bytes at 2 mod 4: five aligned words, four byte-permutes
+  } else {  // 16 bytes at any even offset: five aligned words, four funnel shifts
+    const uint32_t a0 = (ba + 192) & ~3u, sh = ((ba + 192) & 3u) * 8u;
     uint32_t v[5];
 #pragma unroll
-    for (int i = 0; i < 5; ++i) v[i] = lds_u32(ba + 190 + 4 * i);
+    for (int i = 0; i < 5; ++i) v[i] = lds_u32(a0 + 4 * i);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) w.sc[i] = prmt(v[i], v[i + 1], 0x5432u);
+    for (int i = 0; i < 4; ++i) w.sc[i] = __funnelshift_r(v[i], v[i + 1], sh);
   }
   w.d = f16_bits_to_f32(lds_u16(ba + 208));
 }
