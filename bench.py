@@ -553,6 +553,44 @@ def profile_q6k(n):
     print(f"q6k profile case: {n} x {k}, 8 rows, 4 calls, device fault {dl.device_fault(reset=True)}")
 
 
+def profile_case(name):
+    """Small single-GPU cases for ncu captures (one kernel of interest, few launches, inputs well
+    above the 126 MB L2 or, for the small weights, rotated copies); prints one line and no bench
+    result.  down: the W8A8 SiLU down projection 4096 x 14336 at M = 1, 6 calls over 3 weight
+    copies; nvfp4: NVFP4 W4A16 14336 x 4096 at M = 1, 6 calls over 6 weight copies."""
+    import decode_lm_head_b200 as dl
+    from decode_lm_head_b200 import synth
+
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev)
+    if name == "down":
+        n, k = 4096, 14336
+        ws = [(synth.fp8_weight(n, k, 10 + i, dev), synth.row_scales(n, 10 + i, dev)) for i in range(3)]
+        gate = synth.bf16_rows(1, k, 3, dev, tensor_id=4)
+        up = synth.bf16_rows(1, k, 3, dev, tensor_id=5)
+        keep = bind_workspace(dl, stream, dev, [(dl.OP_W8A8, n, k, 1)])
+        xq = torch.empty(128 * k, dtype=torch.uint8, device=dev)
+        xs = torch.empty(128, dtype=torch.float32, device=dev)
+        out = torch.empty(1, n, dtype=torch.bfloat16, device=dev)
+        for i in range(6):
+            w, s = ws[i % 3]
+            dl.w8a8_silu_proj(w, s, gate, up, out=out, xq_scratch=xq, xscale_scratch=xs, stream=stream)
+        torch.cuda.synchronize()
+        dl.set_workspace(None, stream=stream)
+        del keep
+    elif name == "nvfp4":
+        n, k = 14336, 4096
+        wf = [synth.nvfp4_weight(n, k, 20 + i, dev) for i in range(6)]
+        x = synth.bf16_rows(1, k, 4, dev)
+        out = torch.empty(1, n, dtype=torch.bfloat16, device=dev)
+        for wp, sc, gl in wf:
+            dl.w4a16_gemv(wp, sc, gl, x, out=out, stream=stream)
+        torch.cuda.synchronize()
+    else:
+        raise SystemExit(f"unknown profile case {name}")
+    print(f"profile case {name}: done, device fault {dl.device_fault(reset=True)}")
+
+
 def run_ours(args):
     world, rank, local = dist_setup(args)
     import decode_lm_head_b200 as dl
@@ -764,9 +802,14 @@ def main():
                     help="head rows; smaller values only for profiling captures (the workload is 248320)")
     ap.add_argument("--profile-q6k", type=int, default=0, metavar="N",
                     help="run only the Q6_K profiling case (N x 7168 blocks, 8 rows, 4 calls) and exit")
+    ap.add_argument("--profile", choices=["down", "nvfp4"], default=None,
+                    help="run only a small profiling case for ncu (see profile_case) and exit")
     args = ap.parse_args()
     if args.profile_q6k > 0:
         profile_q6k(args.profile_q6k)
+        return
+    if args.profile:
+        profile_case(args.profile)
         return
     globals()["VOCAB"] = args.vocab
     if args.warmup < 3:

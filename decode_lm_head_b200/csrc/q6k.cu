@@ -11,7 +11,11 @@
 // added in order.  Every kernel below takes exactly these steps for every output, so a row's
 // bits do not depend on which kernel, or how many rows, served it.
 //
-// The weight codes enter the MMA as (q - 32) in signed bytes (bit tricks, no table).
+// Two exact ways to the same D_j:
+//   - 8-row kernels: the MMA multiplies the unsigned codes q (u8 x s8) and its accumulator
+//     starts at -32 * sum_{i in j} qs_i, from a table built once per CTA;
+//   - wide kernel (several 8-column groups share one weight fragment): the codes are turned
+//     into (q - 32) as signed bytes once (bit tricks, no table) and every MMA starts from 0.
 //
 // Super-block byte map (210 bytes): ql[128] @0, qh[64] @128, int8 scales[16] @192, f16 d @208.
 // Value i = 128h + 32u + l (h < 2, u < 4, l < 32): low 4 bits from ql[64h + 32(u&1) + l] (low
@@ -73,6 +77,19 @@ __device__ __forceinline__ int q6_scale(const Q6W& w, int j) {
   return (int)prmt(w.sc[j >> 2], 0u, q | ((8u | q) << 4) | ((8u | q) << 8) | ((8u | q) << 12));
 }
 
+// D = A (u8) x B (s8) + C, C given as two values per row pair (columns 2t, 2t+1).
+__device__ __forceinline__ void mma_u8s8_c(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t b0, int c0, int c1) {
+  asm volatile("mma.sync.aligned.m16n8k16.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5}, {%6}, {%7,%8,%7,%8};"
+               : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+               : "r"(a0), "r"(a1), "r"(b0), "r"(c0), "r"(c1));
+}
+// D = A (s8) x B (s8), accumulator from zero (one zero register for all of C).
+__device__ __forceinline__ void mma_s8s8_z(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
+  asm volatile("mma.sync.aligned.m16n8k16.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5}, {%6}, {%7,%7,%7,%7};"
+               : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+               : "r"(a0), "r"(a1), "r"(b0), "r"(0));
+}
+
 // One q8_1 block of one 8-column group: t[i] += float(D0[i] sc0 + D1[i] sc1) * d8(column).
 // Outputs i: 0 = (row g, column 2t), 1 = (g, 2t+1), 2 = (g+8, 2t), 3 = (g+8, 2t+1).
 __device__ __forceinline__ void q6_block_step(float (&tsb)[4], const int (&d0)[4], const int (&d1)[4], int ra0, int ra1,
@@ -108,11 +125,6 @@ __device__ __forceinline__ uint32_t lds_u16(uint32_t saddr) {
   asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(saddr));
   return v;
 }
-// 32-bit load from a 2-byte aligned shared address: two aligned words joined.
-__device__ __forceinline__ uint32_t lds_u32_a2(uint32_t saddr) {
-  const uint32_t a = saddr & ~3u;
-  return __funnelshift_r(lds_u32(a), lds_u32(a + 4), (saddr & 3u) * 8u);
-}
 
 // Super-block at shared address `ba`: kAligned only when ba is 4-byte aligned; the other path
 // takes any even ba (the lanes of one warp may mix both alignments when a row holds an odd
@@ -128,19 +140,27 @@ __device__ __forceinline__ void q6_load_smem(Q6W& w, bool valid, uint32_t ba, in
     w.d = 0.f;
     return;
   }
-#pragma unroll
-  for (int i = 0; i < 8; ++i) w.ql[i] = kAligned ? lds_u32(ba + 16 * i + 4 * t) : lds_u32_a2(ba + 16 * i + 4 * t);
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-    w.qh[i] = kAligned ? lds_u32(ba + 128 + 16 * i + 4 * t) : lds_u32_a2(ba + 128 + 16 * i + 4 * t);
   if (kAligned) {
+    const uint32_t a = ba + 4 * t;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w.ql[i] = lds_u32(a + 16 * i);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w.qh[i] = lds_u32(a + 128 + 16 * i);
 #pragma unroll
     for (int i = 0; i < 4; ++i) w.sc[i] = lds_u32(ba + 192 + 4 * i);
-  } else {  // 16 bytes at any even offset: five aligned words, four funnel shifts
-    const uint32_t a0 = (ba + 192) & ~3u, sh = ((ba + 192) & 3u) * 8u;
-    uint32_t v[5];
+  } else {
+    // every field starts at ba plus a multiple of 4: one aligned base, one shift for all
+    const uint32_t b = ba & ~3u, sh = (ba & 3u) * 8u;
+    const uint32_t a = b + 4 * t;
 #pragma unroll
-    for (int i = 0; i < 5; ++i) v[i] = lds_u32(a0 + 4 * i);
+    for (int i = 0; i < 8; ++i) w.ql[i] = __funnelshift_r(lds_u32(a + 16 * i), lds_u32(a + 16 * i + 4), sh);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      w.qh[i] = __funnelshift_r(lds_u32(a + 128 + 16 * i), lds_u32(a + 128 + 16 * i + 4), sh);
+    uint32_t v[5];  // the 16 scale bytes: five aligned words (the fifth only matters when sh != 0)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = lds_u32(b + 192 + 4 * i);
+    v[4] = lds_u32(b + (sh ? 208u : 204u));  // never past the super-block's last byte
 #pragma unroll
     for (int i = 0; i < 4; ++i) w.sc[i] = __funnelshift_r(v[i], v[i + 1], sh);
   }
@@ -169,7 +189,8 @@ __device__ __forceinline__ void q6_load_global(Q6W& w, bool valid, const uint8_t
 // One persistent 512-thread CTA per SM over 16-row weight tiles; warp w runs K-slice w of every
 // tile (q6_slice_begin), and the 16 slices of a tile are summed in warp order through shared
 // memory.  Activations:
-//   - dxs [K/32][8] float32 q8_1 d, staged once per CTA;
+//   - dxs [K/32][8] float32 q8_1 d, and cor [K/16][8] int32 -32 * (sum of the 16 codes of
+//     the sub-block), staged once per CTA;
 //   - the B fragments (4 codes of column g, values 4t..4t+3 of each sub-block): for K <= 8192
 //     (at most 2 super-blocks per slice) each warp keeps the 32 words of its own slice in
 //     registers, loaded once; beyond that the codes are staged whole, xs [8][rs] with
@@ -210,22 +231,34 @@ struct Q6RowsParams {
 __host__ __device__ __forceinline__ int q6_act_stride(int k) { return k + ((64 - k % 128) + 128) % 128; }
 __host__ __device__ __forceinline__ bool q6_reg_acts(int k) { return (k / 256 + kQ6Slices - 1) / kQ6Slices <= kQ6RegSlice; }
 constexpr size_t kQ6RedBytes = 2ull * kQ6Warps * 32 * 4 * 4;  // [2][warps][32 lanes][4 floats]
-// dxs, then (smem activations) xs, then the reduction buffer.
+// dxs, cor, then (smem activations) xs, then the reduction buffer.
 __host__ __device__ __forceinline__ size_t q6_dx_bytes(int k) { return (size_t)(k / 32) * kQ6MaxRows * 4; }
+__host__ __device__ __forceinline__ size_t q6_cor_bytes(int k) { return (size_t)(k / 16) * kQ6MaxRows * 4; }
 __host__ __device__ __forceinline__ size_t q6_base_bytes(int k, bool reg_acts) {
-  return q6_dx_bytes(k) + (reg_acts ? 0 : (size_t)kQ6MaxRows * q6_act_stride(k)) + kQ6RedBytes;
+  return q6_dx_bytes(k) + q6_cor_bytes(k) + (reg_acts ? 0 : (size_t)kQ6MaxRows * q6_act_stride(k)) + kQ6RedBytes;
 }
 
-// Stage dxs (and, without register fragments, xs).
+// Stage dxs and cor (and, without register fragments, xs).
 __device__ void q6_stage_acts(const Q6Params& p, uint8_t* smem, bool stage_codes) {
   const int nb32 = p.k / 32;
   const int rs = q6_act_stride(p.k);
   float* dxs = reinterpret_cast<float*>(smem);
-  uint8_t* xs = smem + q6_dx_bytes(p.k);
+  int* cor = reinterpret_cast<int*>(smem + q6_dx_bytes(p.k));
+  uint8_t* xs = smem + q6_dx_bytes(p.k) + q6_cor_bytes(p.k);
   for (int it = threadIdx.x; it < kQ6MaxRows * nb32; it += blockDim.x) {
     const int m = it / nb32, b = it % nb32;
     const uint32_t* bw = reinterpret_cast<const uint32_t*>(p.q8 + ((int64_t)m * nb32 + b) * 36);
     dxs[b * kQ6MaxRows + m] = m < p.rows ? f16_bits_to_f32(bw[0] & 0xffffu) : 0.f;
+    int s0 = 0, s1 = 0;
+    if (m < p.rows) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        s0 = __dp4a((int)bw[1 + i], 0x01010101, s0);
+        s1 = __dp4a((int)bw[5 + i], 0x01010101, s1);
+      }
+    }
+    cor[(2 * b) * kQ6MaxRows + m] = -32 * s0;
+    cor[(2 * b + 1) * kQ6MaxRows + m] = -32 * s1;
     if (!stage_codes) continue;
     uint8_t* dst = xs + m * rs + (b >> 3) * 256;
     const int kb = (b & 7) * 32;  // first value of this block inside its super-block
@@ -247,16 +280,17 @@ __device__ __forceinline__ uint32_t q6_bfrag(const Q6Params& p, int col, int sb,
 }
 
 // One super-block of the 16-row tile (rows g: wa, g+8: wb) against the 8 columns: bw[j] is the
-// lane's B fragment of sub-block j; dxs = dxs + (8 sb) 32 + 8 t.
+// lane's B fragment of sub-block j; dxs = dxs + (8 sb) 32 + 8 t; cor = cor + (16 sb) 32 + 8 t.
 __device__ __forceinline__ void q6_superblock_8(float (&acc)[4], const Q6W& wa, const Q6W& wb, const uint32_t (&bw)[16],
-                                                uint32_t dxs) {
+                                                uint32_t dxs, uint32_t cor) {
   float tsb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int blk = 0; blk < 8; ++blk) {
     const int j0 = 2 * blk, j1 = j0 + 1;
-    int d0[4] = {0, 0, 0, 0}, d1[4] = {0, 0, 0, 0};
-    mma_s8_16816(d0, q6_codes_s8(wa, j0), q6_codes_s8(wb, j0), bw[j0]);
-    mma_s8_16816(d1, q6_codes_s8(wa, j1), q6_codes_s8(wb, j1), bw[j1]);
+    const uint2 c0 = lds_u64(cor + 32 * j0), c1 = lds_u64(cor + 32 * j1);
+    int d0[4], d1[4];
+    mma_u8s8_c(d0, q6_codes_u8(wa, j0), q6_codes_u8(wb, j0), bw[j0], (int)c0.x, (int)c0.y);
+    mma_u8s8_c(d1, q6_codes_u8(wa, j1), q6_codes_u8(wb, j1), bw[j1], (int)c1.x, (int)c1.y);
     const uint2 dx = lds_u64(dxs + 32 * blk);
     q6_block_step(tsb, d0, d1, q6_scale(wa, j0), q6_scale(wa, j1), q6_scale(wb, j0), q6_scale(wb, j1),
                   __uint_as_float(dx.x), __uint_as_float(dx.y));
@@ -336,7 +370,8 @@ __global__ void __launch_bounds__(kQ6Threads, 1) q6k_rows8_kernel(const Q6RowsPa
   const int g = lane >> 2, t = lane & 3;
   const int sb_begin = q6_slice_begin(nsb, warp), sb_end = q6_slice_begin(nsb, warp + 1);
   const uint32_t dx0 = smem_u32(smem) + (uint32_t)(8 * t);
-  const uint32_t xs0 = smem_u32(smem) + (uint32_t)(q6_dx_bytes(p.k) + g * rs + 16 * t);
+  const uint32_t co0 = smem_u32(smem) + (uint32_t)(q6_dx_bytes(p.k) + 8 * t);
+  const uint32_t xs0 = smem_u32(smem) + (uint32_t)(q6_dx_bytes(p.k) + q6_cor_bytes(p.k) + g * rs + 16 * t);
   uint32_t bfr[kQ6RegSlice][16];
   if (kRegActs) {
 #pragma unroll
@@ -381,7 +416,7 @@ __global__ void __launch_bounds__(kQ6Threads, 1) q6k_rows8_kernel(const Q6RowsPa
         q6_load_global(wa, va, ga + (int64_t)sb * 210, t);
         q6_load_global(wb, vb, ga + 8 * row_bytes + (int64_t)sb * 210, t);
       }
-      q6_superblock_8(acc, wa, wb, bw, dx0 + 256u * sb);
+      q6_superblock_8(acc, wa, wb, bw, dx0 + 256u * sb, co0 + 512u * sb);
     };
     if (kRegActs) {
 #pragma unroll
@@ -476,9 +511,9 @@ __device__ __forceinline__ void q6_superblock_wide(float (&acc)[NT][4], const Q6
 #pragma unroll
     for (int ct = 0; ct < NT; ++ct) {
       const uint32_t brow = xs + (uint32_t)((8 * ct + g) * kQWRowStride + 36 * blk + 4 + 4 * t);
-      int d0[4] = {0, 0, 0, 0}, d1[4] = {0, 0, 0, 0};
-      mma_s8_16816(d0, a00, a01, lds_u32(brow));
-      mma_s8_16816(d1, a10, a11, lds_u32(brow + 16));
+      int d0[4], d1[4];
+      mma_s8s8_z(d0, a00, a01, lds_u32(brow));
+      mma_s8s8_z(d1, a10, a11, lds_u32(brow + 16));
       const uint32_t drow = xs + (uint32_t)((8 * ct + 2 * t) * kQWRowStride + 36 * blk);
       const float dx0 = f16_bits_to_f32(lds_u16(drow));
       const float dx1 = f16_bits_to_f32(lds_u16(drow + kQWRowStride));
