@@ -298,22 +298,21 @@ __device__ __forceinline__ void q6_superblock_8(float (&acc)[4], const Q6W& wa, 
   q6_superblock_end(acc, tsb, wa.d, wb.d);
 }
 
-// Fixed-order sum over the 16 warps' partials of a tile, one BF16 store per output.
-__device__ __forceinline__ void q6_reduce_store(const Q6Params& p, float* red, int tile, const float (&acc)[4]) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  reinterpret_cast<float4*>(red)[warp * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-  __syncthreads();
-  if (threadIdx.x < kQ6TileRows * kQ6MaxRows) {
-    const int rr = threadIdx.x % kQ6TileRows, cc = threadIdx.x / kQ6TileRows;
-    const int row = tile * kQ6TileRows + rr;
-    if (cc < p.rows && row < p.n) {
-      const int gg = rr & 7, up = rr >> 3;
-      const int ln = gg * 4 + (cc >> 1), comp = up * 2 + (cc & 1);
-      float sum = 0.f;
+// Fixed-order sum over the 16 warps' partials of a tile, one BF16 store per output; run by the
+// 128 threads of warps 12..15 (the K-slices are split with the longer ones first, so these
+// warps never have more super-blocks than the others), thread r of them output r.
+constexpr int kQ6RedWarp0 = kQ6Warps - 4;
+__device__ __forceinline__ void q6_reduce_tile(const Q6Params& p, const float* red, int tile) {
+  const int o = threadIdx.x - kQ6RedWarp0 * 32;
+  const int rr = o % kQ6TileRows, cc = o / kQ6TileRows;
+  const int row = tile * kQ6TileRows + rr;
+  if (cc < p.rows && row < p.n) {
+    const int gg = rr & 7, up = rr >> 3;
+    const int ln = gg * 4 + (cc >> 1), comp = up * 2 + (cc & 1);
+    float sum = 0.f;
 #pragma unroll
-      for (int ww = 0; ww < kQ6Warps; ++ww) sum = __fadd_rn(sum, red[(ww * 32 + ln) * 4 + comp]);
-      p.out[(int64_t)cc * p.ldc + row] = f32_to_bf16_bits(sum);
-    }
+    for (int ww = 0; ww < kQ6Warps; ++ww) sum = __fadd_rn(sum, red[(ww * 32 + ln) * 4 + comp]);
+    p.out[(int64_t)cc * p.ldc + row] = f32_to_bf16_bits(sum);
   }
 }
 
@@ -382,7 +381,6 @@ __global__ void __launch_bounds__(kQ6Threads, 1) q6k_rows8_kernel(const Q6RowsPa
   __syncthreads();
 
   const int sa_off = g / SR, sb_off = (g + 8) / SR;  // stages of rows g and g+8 within a tile
-  int parity = 0;
   for (int i = 0; T0 + i < T1; ++i) {
     const int tile = T0 + i;
     const int r0 = tile * kQ6TileRows + g;
@@ -399,6 +397,9 @@ __global__ void __launch_bounds__(kQ6Threads, 1) q6k_rows8_kernel(const Q6RowsPa
       base_a = ring + (uint32_t)(s_a % sp.ns) * sp.stage_stride + (uint32_t)((g % SR) * row_bytes);
       base_b = ring + (uint32_t)(s_b % sp.ns) * sp.stage_stride + (uint32_t)(((g + 8) % SR) * row_bytes);
     }
+    // the previous tile's reduction, on the warps with the shortest slices, while the others
+    // start this tile
+    if (warp >= kQ6RedWarp0 && i > 0) q6_reduce_tile(p, red + ((i - 1) & 1) * (kQ6Warps * 32 * 4), tile - 1);
     const uint8_t* ga = p.blocks + (int64_t)r0 * row_bytes;
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     auto one = [&](int sb, const uint32_t (&bw)[16]) {
@@ -433,13 +434,17 @@ __global__ void __launch_bounds__(kQ6Threads, 1) q6k_rows8_kernel(const Q6RowsPa
         one(sb, bw);
       }
     }
-    // fixed-order reduction over warps; after its barrier the tile's stages are free
-    q6_reduce_store(p, red + parity * (kQ6Warps * 32 * 4), tile, acc);
+    // publish the partial sums; after the barrier the tile's stages are free, and its sums are
+    // reduced during the next tile (the buffer of parity i & 1 is written again two tiles on,
+    // after the next barrier, by when that reduction has read it)
+    reinterpret_cast<float4*>(red + (i & 1) * (kQ6Warps * 32 * 4))[warp * 32 + lane] =
+        make_float4(acc[0], acc[1], acc[2], acc[3]);
+    __syncthreads();
     if (kStream && threadIdx.x == 0)
       for (int q = 0; q < spt; ++q)
         if (spt * i + q + sp.ns < nstages) produce(spt * i + q + sp.ns);
-    parity ^= 1;
   }
+  if (warp >= kQ6RedWarp0 && T1 > T0) q6_reduce_tile(p, red + ((T1 - T0 - 1) & 1) * (kQ6Warps * 32 * 4), T1 - 1);
 }
 
 // ---------------------------------------------------------------------------------------
