@@ -146,17 +146,20 @@ __device__ __forceinline__ void kb_w4a16_reg(float (&acc)[NT][4], const uint4& r
   const uint32_t sa0 = __byte_perm(sa, 0, 0x1010), sa1 = __byte_perm(sa, 0, 0x3232);
   const uint32_t sb0 = __byte_perm(sb, 0, 0x1010), sb1 = __byte_perm(sb, 0, 0x3232);
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {  // MMA step j: bytes 2j, 2j+1 of the lane's 16 (values 4j..4j+3)
-    const uint32_t word_a = wa[j >> 1], word_b = wb[j >> 1];
-    const int sh = (j & 1) * 16;
-    const uint32_t ssa = (j < 4) ? sa0 : sa1;
-    const uint32_t ssb = (j < 4) ? sb0 : sb1;
-    const uint32_t a0 = hmul2(e2m1x2_to_f16x2((word_a >> sh) & 0xff), ssa);
-    const uint32_t a2 = hmul2(e2m1x2_to_f16x2((word_a >> (sh + 8)) & 0xff), ssa);
-    const uint32_t a1 = hmul2(e2m1x2_to_f16x2((word_b >> sh) & 0xff), ssb);
-    const uint32_t a3 = hmul2(e2m1x2_to_f16x2((word_b >> (sh + 8)) & 0xff), ssb);
+  for (int q = 0; q < 4; ++q) {  // word q: bytes 4q..4q+3 feed MMA steps 2q (bytes 4q, 4q+1) and 2q+1
+    uint32_t fa[4], fb[4];
+    e2m1x8_to_f16x2x4(wa[q], fa);
+    e2m1x8_to_f16x2x4(wb[q], fb);
+    const uint32_t ssa = (q < 2) ? sa0 : sa1;
+    const uint32_t ssb = (q < 2) ? sb0 : sb1;
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) mma_f16_16816(acc[nt], a0, a1, a2, a3, xr[nt][2 * j], xr[nt][2 * j + 1]);
+    for (int h = 0; h < 2; ++h) {  // MMA step j = 2q + h: bytes 2j, 2j+1 of the lane's 16 (values 4j..4j+3)
+      const int j = 2 * q + h;
+      const uint32_t a0 = hmul2(fa[2 * h], ssa), a2 = hmul2(fa[2 * h + 1], ssa);
+      const uint32_t a1 = hmul2(fb[2 * h], ssb), a3 = hmul2(fb[2 * h + 1], ssb);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) mma_f16_16816(acc[nt], a0, a1, a2, a3, xr[nt][2 * j], xr[nt][2 * j + 1]);
+    }
   }
 }
 
@@ -173,22 +176,25 @@ __device__ __forceinline__ void kb_w4a4_reg(float (&acc)[NT][4], const uint4& ra
   const uint32_t sa0 = __byte_perm(sa, 0, 0x1010), sa1 = __byte_perm(sa, 0, 0x3232);
   const uint32_t sb0 = __byte_perm(sb, 0, 0x1010), sb1 = __byte_perm(sb, 0, 0x3232);
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const uint32_t word_a = wa[j >> 1], word_b = wb[j >> 1];
-    const int sh = (j & 1) * 16;
-    const uint32_t ssa = (j < 4) ? sa0 : sa1;
-    const uint32_t ssb = (j < 4) ? sb0 : sb1;
-    const uint32_t a0 = hmul2(e2m1x2_to_f16x2((word_a >> sh) & 0xff), ssa);
-    const uint32_t a2 = hmul2(e2m1x2_to_f16x2((word_a >> (sh + 8)) & 0xff), ssa);
-    const uint32_t a1 = hmul2(e2m1x2_to_f16x2((word_b >> sh) & 0xff), ssb);
-    const uint32_t a3 = hmul2(e2m1x2_to_f16x2((word_b >> (sh + 8)) & 0xff), ssb);
+  for (int q = 0; q < 4; ++q) {  // word q feeds MMA steps 2q, 2q+1 (as in kb_w4a16_reg)
+    uint32_t fa[4], fb[4];
+    e2m1x8_to_f16x2x4(wa[q], fa);
+    e2m1x8_to_f16x2x4(wb[q], fb);
+    const uint32_t ssa = (q < 2) ? sa0 : sa1;
+    const uint32_t ssb = (q < 2) ? sb0 : sb1;
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const uint32_t cw = xr[nt][j >> 1];
-      const uint32_t sx = (j < 4) ? __byte_perm(xr[nt][4], 0, 0x1010) : __byte_perm(xr[nt][4], 0, 0x3232);
-      const uint32_t b0 = hmul2(e2m1x2_to_f16x2((cw >> sh) & 0xff), sx);
-      const uint32_t b1 = hmul2(e2m1x2_to_f16x2((cw >> (sh + 8)) & 0xff), sx);
-      mma_f16_16816(acc[nt], a0, a1, a2, a3, b0, b1);
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t a0 = hmul2(fa[2 * h], ssa), a2 = hmul2(fa[2 * h + 1], ssa);
+      const uint32_t a1 = hmul2(fb[2 * h], ssb), a3 = hmul2(fb[2 * h + 1], ssb);
+      const int sh = 16 * h;  // the activation side: bytes 4q + 2h, 4q + 2h + 1 of its codes
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const uint32_t cw = xr[nt][q];
+        const uint32_t sx = (q < 2) ? __byte_perm(xr[nt][4], 0, 0x1010) : __byte_perm(xr[nt][4], 0, 0x3232);
+        const uint32_t b0 = hmul2(e2m1x2_to_f16x2((cw >> sh) & 0xff), sx);
+        const uint32_t b1 = hmul2(e2m1x2_to_f16x2((cw >> (sh + 8)) & 0xff), sx);
+        mma_f16_16816(acc[nt], a0, a1, a2, a3, b0, b1);
+      }
     }
   }
 }
