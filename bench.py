@@ -58,10 +58,10 @@ def oracle_passes(m):
 
 def launches_per_call(m, sms, n):
     """Kernels one call launches on an n-row head: per pass the activation split, the GEMV
-    and, when the stream-K schedule has a remainder (tiles not a multiple of the SM count),
-    the fixup."""
-    ntiles = -(-n // 128)
-    rem = ntiles % sms if ntiles >= sms else ntiles
+    and, when the stream-K schedule has a remainder (tile pairs not a multiple of the party
+    count, sms // 2 CTA pairs), the fixup."""
+    pairs, parties = -(-n // 256), max(1, sms // 2)
+    rem = pairs % parties if pairs >= parties else pairs
     return passes(m) * (2 + (1 if rem else 0))
 
 

@@ -56,6 +56,65 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// ---- CTA pairs (a cluster of two CTAs on one TPC sharing each MMA, cta_group::2)
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// The shared::cluster address of the object at this CTA's shared address `addr` in CTA `rank`
+// of the cluster (the same offset there).
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+
+// Arrive on an mbarrier given by its shared::cluster address (this CTA's or the peer's), with
+// release semantics at cluster scope.
+__device__ __forceinline__ void arrive_cluster(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
+
+// Every thread of both CTAs: all shared-memory writes and arrivals before it are visible
+// cluster-wide after it.
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// 3-D tiled TMA load into this CTA's shared memory (no multicast) whose completion is counted
+// on an mbarrier of either CTA of the pair (`bar_cluster`, a shared::cluster address).
+__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* map, int c0, int c1, int c2,
+                                                 uint32_t bar_cluster, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
+      "[%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(dst),
+      "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(bar_cluster), "l"(policy)
+      : "memory");
+}
+
+// Arrive (once each) on the mbarrier at shared offset `bar` of every CTA in `cta_mask` when the
+// pair MMAs issued so far by this thread have completed.
+__device__ __forceinline__ void commit_pair(uint32_t bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+      "h"(cta_mask)
+      : "memory");
+}
+
+// Warp-wide in both CTAs of the pair (the same warp of each): allocate `cols` TMEM columns in
+// both, at the same address, written to the same shared offset of each CTA.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t cols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(cols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t cols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols) : "memory");
+}
+
 // 1-D bulk copy global -> this CTA's shared memory, completing on `bar` (both addresses
 // 16-byte aligned, bytes a multiple of 16).
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar,
@@ -96,6 +155,10 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
 // code 0 (E4M3 under kind::f8f6f4, F16 under kind::f16).
 __device__ __forceinline__ uint32_t idesc_m128(int n) {
   return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
+}
+// The same for a pair MMA: M = 256 (128 rows in each CTA of the pair).
+__device__ __forceinline__ uint32_t idesc_m256(int n) {
+  return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)((2 * kBM) >> 4) << 24);
 }
 
 __device__ __forceinline__ void commit(uint32_t bar) {
@@ -198,27 +261,39 @@ inline bool cached_map_k128(CUtensorMap* m, const void* base, int elem_bytes, in
   return true;
 }
 
-// Launch with programmatic stream serialization: the kernel may start while the preceding
+// Launch with programmatic stream serialization (the kernel may start while the preceding
 // kernel of the stream finishes; it must call grid_dependency_wait() before touching
-// anything that kernel writes.
+// anything that kernel writes), in clusters of `cluster_x` CTAs along x (grid.x a multiple
+// of it; 1: no cluster).
 template <typename... KArgs, typename... Args>
-inline int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
-                      Args&&... args) {
+inline int launch_pdl_cluster(int cluster_x, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t s, Args&&... args) {
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = (unsigned)cluster_x;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = cluster_x > 1 ? 2 : 1;
   if (cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) != cudaSuccess) {
     (void)cudaGetLastError();
     return DLMH_ERR_CUDA;
   }
   return DLMH_OK;
+}
+
+// The same without clusters.
+template <typename... KArgs, typename... Args>
+inline int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                      Args&&... args) {
+  return launch_pdl_cluster(1, kernel, grid, block, smem, s, std::forward<Args>(args)...);
 }
 
 // Smallest power of two >= max(v, 32) (TMEM allocation granularity).

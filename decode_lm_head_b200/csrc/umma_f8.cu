@@ -63,6 +63,18 @@ __device__ __forceinline__ void umma_f8(uint32_t tmem_d, uint64_t adesc, uint64_
       : "memory");
 }
 
+// The pair form: M = 256, A rows [0, 128) and B rows [0, N/2) from the issuing CTA's shared
+// memory, A rows [128, 256) and B rows [N/2, N) from its peer's (same offsets); D rows
+// [0, 128) into the issuer's TMEM, [128, 256) into the peer's (same address).
+__device__ __forceinline__ void umma_f8_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                             int accum) {
+  asm volatile(
+      "{ .reg .pred p; setp.ne.b32 p, %4, 0; "
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p; }" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
+      : "memory");
+}
+
 struct UmmaParams {
   int n, k, rows, npad;  // npad: rows rounded up to 16 (the epilogue's column loop)
   int nb;                // MMA N = B rows: npad (W8A8) or 2 * roundup8(rows) (W8A16 hi | lo)
@@ -75,8 +87,9 @@ struct UmmaParams {
   int64_t ldc;
   int ns;                // ring stages
   int stage_bytes;       // A + B bytes of one stage
-  // Stream-K schedule (umma_sched.h) over G = gridDim.x CTAs, a pure function of n, k and
-  // the SM count, never of the row count; partial sums are laid out [slot][col][128 rows].
+  // Stream-K schedule (umma_schedule) over P = gridDim.x / 2 parties (CTA pairs) and tile
+  // pairs, a pure function of n, k and the SM count, never of the row count; partial sums are
+  // laid out [slot][col][128 rows], two slots per CTA.
   int spt, wt, rem;
   float* partial;
   // Dynamic hand-out of the whole tiles from the caller workspace's queue (null: the static
@@ -110,6 +123,18 @@ __device__ __forceinline__ TileDst tile_dst(const UmmaParams& p, int tile) {
 }
 
 
+// The schedule's parties are CTA pairs and its tiles tile pairs (umma_schedule): CTAs 2j and
+// 2j + 1 both run party j's jobs, CTA 2j + h on single tile 2T + h of tile pair T, so the two
+// tiles of a pair always get the same K split (whichever kernel runs them, and whatever the row
+// count).  Whole tiles may also be claimed one by one from the workspace queue.
+//
+// kPair: each pair is a cluster on one TPC and the two CTAs share every MMA (cta_group::2,
+// M = 256): CTA rank h loads its tile's weight rows and rows [h N/2, (h + 1) N/2) of the
+// activation box into its own ring.  Rank 0 issues the MMAs; the copies of both CTAs count on
+// rank 0's full barriers, and each commit arrives on the empty (or accumulator-full) barrier of
+// both CTAs.  Per SM the activation box and its shared memory are halved, so the ring holds
+// more stages when N is large.  Static tile order.
+template <bool kPair>
 __global__ void __launch_bounds__(kUmmaThreads, 1)
     umma_f8_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_w2,
                    const __grid_constant__ CUtensorMap map_x, const UmmaParams p) {
@@ -120,14 +145,19 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
   __shared__ int4 s_job[kJobRing];  // (tile, first unit, end unit, partial slot); tile < 0 ends
   __shared__ uint32_t s_tmem;
 
-  const Sched sc{p.spt, p.wt, p.rem, (int)gridDim.x};
-  const int b = blockIdx.x;
-  const int G = (int)gridDim.x;
+  // party b = CTAs 2b and 2b + 1; this CTA is half h of it (in a pair, its cluster rank)
+  const int h = kPair ? (int)cluster_ctarank() : (int)(blockIdx.x & 1);
+  const bool leader = !kPair || h == 0;  // issues the MMAs (a pair's rank 0 for both CTAs)
+  const int nctas = (int)gridDim.x;
+  const int P = nctas / 2;
+  const int b = (int)blockIdx.x / 2;
+  const Sched sc{p.spt, p.wt, p.rem, P};
   {
     int tile, u0, u1, slot;
-    if (!sc.job(b, 0, tile, u0, u1, slot)) return;  // no work at all (uniform over the CTA)
+    if (!sc.job(b, 0, tile, u0, u1, slot)) return;  // no work at all (uniform over the party)
   }
-  const bool dyn = p.queue != nullptr && p.wt > 0;
+  const bool dyn = !kPair && p.queue != nullptr && p.wt > 0;
+  const int nwhole = 2 * p.wt * P;  // single tiles [0, nwhole) are whole
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kchunks = p.k / 128;
@@ -135,7 +165,8 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
   const uint32_t full0 = smem_u32(bar_full), empty0 = smem_u32(bar_empty);
   const uint32_t tfull0 = smem_u32(bar_tfull), tempty0 = smem_u32(bar_tempty);
   const int a_bytes = kKC * kChunkBytesA;
-  const int b_chunk = p.nb * 128;
+  const int bn = kPair ? p.nb / 2 : p.nb;  // activation rows in this CTA's stages
+  const int b_chunk = bn * 128;
   const uint32_t tmem_cols = 2u * (uint32_t)p.accw;
 
   if (threadIdx.x == 0) {
@@ -145,17 +176,27 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       bar_init(tfull0 + 8u * i, 1);
-      bar_init(tempty0 + 8u * i, 4);  // the four epilogue warps
+      bar_init(tempty0 + 8u * i, kPair ? 8 : 4);  // the four epilogue warps (of both CTAs)
     }
     for (int i = 0; i < kJobRing; ++i) {
       bar_init(smem_u32(&bar_jfull[i]), 1);
-      bar_init(smem_u32(&bar_jempty[i]), 5);  // the MMA thread and the four epilogue warps
+      // the MMA thread (rank 0 only) and the four epilogue warps
+      bar_init(smem_u32(&bar_jempty[i]), leader ? 5 : 4);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 1) tmem_alloc(smem_u32(&s_tmem), tmem_cols);
+  if (warp == 1) {
+    if constexpr (kPair)
+      tmem_alloc_pair(smem_u32(&s_tmem), tmem_cols);
+    else
+      tmem_alloc(smem_u32(&s_tmem), tmem_cols);
+  }
   fence_before();
-  __syncthreads();
+  __syncwarp();
+  if constexpr (kPair)
+    cluster_sync();  // both CTAs' barriers exist before either signals the other's
+  else
+    __syncthreads();
   fence_after();
   const uint32_t tmem_base = s_tmem;
   grid_dependents_launch();  // the fixup may be scheduled; it waits for this grid to finish
@@ -164,9 +205,10 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
     // ---------------- producer: hands out the jobs and streams their stages
     if (lane == 0) {
       const uint64_t pol_w = l2_policy_evict_first(), pol_x = l2_policy_evict_last();
-      // Job sequence: the whole tiles (the first static -- tile b, or b*wt in the static
-      // order -- the rest claimed from the queue or taken in order), then the CTA's remainder
-      // segments, then an end marker.
+      // Job sequence (single tile, first unit, end unit, partial slot): the whole tiles (the
+      // first static -- tile 2b + h, or the party's tile pairs in the static order -- the rest
+      // claimed from the queue or taken in order), then the party's remainder segments on this
+      // CTA's half of their tile pairs, then an end marker.
       bool whole = p.wt > 0;  // still handing out whole tiles
       int wj = 0;             // whole tiles taken so far
       int rj = p.wt;          // schedule index of the next remainder segment
@@ -174,20 +216,21 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
         if (whole) {
           int tile;
           if (dyn)
-            tile = wj == 0 ? b : G + atomicAdd(p.queue, 1);
+            tile = wj == 0 ? (int)blockIdx.x : nctas + atomicAdd(p.queue, 1);
           else
-            tile = wj < p.wt ? b * p.wt + wj : -1;
-          if (tile >= 0 && tile < p.wt * G) {
+            tile = wj < p.wt ? 2 * (b * p.wt + wj) + h : -1;
+          if (tile >= 0 && tile < nwhole) {
             ++wj;
             jb = make_int4(tile, 0, p.spt, -1);
             return true;
           }
           whole = false;
         }
-        int tile, u0, u1, ps;
-        if (sc.job(b, rj, tile, u0, u1, ps)) {
+        int tp, u0, u1, ps;
+        if (sc.job(b, rj, tp, u0, u1, ps)) {
           ++rj;
-          jb = make_int4(tile, u0, u1, ps);
+          // the party's slot 2b + s is this CTA's 2 (2b + h) + s
+          jb = make_int4(2 * tp + h, u0, u1, 2 * (int)blockIdx.x + (ps - 2 * b));
           return true;
         }
         return false;
@@ -206,13 +249,27 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
       int4 jb;
       next_job(jb);
       publish(jb);
+      // Copies count on this CTA's full barrier, or in a pair on rank 0's, whose producer
+      // expects both CTAs' bytes.
+      const uint32_t fullc0 = kPair ? mapa_shared(full0, 0) : full0;
+      const uint32_t expect = kPair ? 2u * (uint32_t)p.stage_bytes : (uint32_t)p.stage_bytes;
+      auto load = [&](uint32_t dst, const CUtensorMap* map, int c1, int c2, int slot_, uint64_t pol) {
+        if constexpr (kPair)
+          tma_load_3d_pair(dst, map, 0, c1, c2, fullc0 + 8u * slot_, pol);
+        else
+          tma_load_3d(dst, map, 0, c1, c2, full0 + 8u * slot_, pol);
+      };
+      // A: weight rows [tile*128, +128) x chunks [u*KC, u*KC + KC) of the tile's matrix
+      // (the tile after the last of an odd tile count is read past the end: zero fill, no traffic)
+      auto load_w = [&](uint32_t dst, int tt, int u, int slot_) {
+        const bool first = tt < p.t1;
+        const int row0 = first ? tt * kBM : (p.n2 > 0 ? (tt - p.t1) * kBM : p.t1 * kBM);
+        load(dst, first ? &map_w : &map_w2, row0, u * kKC, slot_, pol_w);
+      };
       const int npre = p.early_w ? min(p.ns, jb.z - jb.y) : 0;
       for (int s = 0; s < npre; ++s) {
-        const int u = jb.y + s;
-        expect_tx(full0 + 8u * s, (uint32_t)p.stage_bytes);
-        const bool first = jb.x < p.t1;
-        tma_load_3d(ring_u32 + s * p.stage_bytes, first ? &map_w : &map_w2, 0, (first ? jb.x : jb.x - p.t1) * kBM,
-                    u * kKC, full0 + 8u * s, pol_w);
+        if (leader) expect_tx(full0 + 8u * s, expect);
+        load_w(ring_u32 + s * p.stage_bytes, jb.x, jb.y + s, s);
       }
       grid_dependency_wait();
       int slot = 0, phase = 0, s = 0;
@@ -224,14 +281,11 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
           // the full boxes always land (rows past n, rows past `rows` and a chunk past K are
           // zero-filled), so every stage completes exactly stage_bytes
           if (s >= npre) {
-            expect_tx(full0 + 8u * slot, (uint32_t)p.stage_bytes);
-            // A: weight rows [tile*128, +128) x chunks [u*KC, u*KC + KC) of the tile's matrix
-            const bool first = tile < p.t1;
-            tma_load_3d(st, first ? &map_w : &map_w2, 0, (first ? tile : tile - p.t1) * kBM, u * kKC,
-                        full0 + 8u * slot, pol_w);
+            if (leader) expect_tx(full0 + 8u * slot, expect);
+            load_w(st, tile, u, slot);
           }
-          // B: all activation rows, the same chunks
-          tma_load_3d(st + a_bytes, &map_x, 0, 0, u * kKC, full0 + 8u * slot, pol_x);
+          // B: the activation rows (this CTA's half of them in a pair), the same chunks
+          load(st + a_bytes, &map_x, kPair ? h * bn : 0, u * kKC, slot, pol_x);
           if (++slot == p.ns) {
             slot = 0;
             phase ^= 1;
@@ -242,14 +296,17 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
       }
       const int nunits = s;
       // no copy may still be landing when the CTA exits: wait (bounded) for the last
-      // phase of every slot (already complete in a healthy run, where the MMAs consumed it)
-      for (int t = nunits - 1; t >= 0 && t >= nunits - p.ns; --t)
-        if (!wait(full0 + 8u * (t % p.ns), (t / p.ns) & 1)) atomicOr(&umma_fault_word, 1);
+      // phase of every slot (already complete in a healthy run, where the MMAs consumed it).
+      // In a pair, rank 0's barriers count both CTAs' copies and the closing cluster barrier
+      // holds rank 1 until rank 0 has seen them land.
+      if (leader)
+        for (int t = nunits - 1; t >= 0 && t >= nunits - p.ns; --t)
+          if (!wait(full0 + 8u * (t % p.ns), (t / p.ns) & 1)) atomicOr(&umma_fault_word, 1);
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc = idesc_m128(p.nb);
+    // ---------------- MMA issuer (rank 0 of a pair issues for both CTAs)
+    if (lane == 0 && leader) {
+      const uint32_t idesc = kPair ? idesc_m256(p.nb) : idesc_m128(p.nb);
       int slot = 0, phase = 0;
       for (int i = 0;; ++i) {
         const int r = i % kJobRing;
@@ -274,17 +331,30 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
             const uint32_t a0 = st + c * kChunkBytesA;
             const uint32_t b0 = st + a_bytes + c * b_chunk;
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)  // K = 32 bytes per MMA
-              umma_f8(tmem_d, desc_sw128(a0 + kk * 32), desc_sw128(b0 + kk * 32), idesc,
-                      ((u - u0) | c | kk) != 0);
+            for (int kk = 0; kk < 4; ++kk) {  // K = 32 bytes per MMA
+              if constexpr (kPair)
+                umma_f8_pair(tmem_d, desc_sw128(a0 + kk * 32), desc_sw128(b0 + kk * 32), idesc,
+                             ((u - u0) | c | kk) != 0);
+              else
+                umma_f8(tmem_d, desc_sw128(a0 + kk * 32), desc_sw128(b0 + kk * 32), idesc,
+                        ((u - u0) | c | kk) != 0);
+            }
           }
-          commit(empty0 + 8u * slot);  // the stage is free once these MMAs have read it
+          // the stage (of both CTAs) is free once these MMAs have read it
+          if constexpr (kPair)
+            commit_pair(empty0 + 8u * slot, 3);
+          else
+            commit(empty0 + 8u * slot);
           if (++slot == p.ns) {
             slot = 0;
             phase ^= 1;
           }
         }
-        commit(tfull0 + 8u * acc);  // the accumulator is complete
+        // the accumulator (of both CTAs) is complete
+        if constexpr (kPair)
+          commit_pair(tfull0 + 8u * acc, 3);
+        else
+          commit(tfull0 + 8u * acc);
       }
     }
   } else {
@@ -348,20 +418,32 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
       }
       fence_before();
       __syncwarp();
-      if (lane == 0) arrive(tempty0 + 8u * acc);
+      if (lane == 0) {
+        if constexpr (kPair)
+          arrive_cluster(mapa_shared(tempty0 + 8u * acc, 0));  // rank 0's MMA thread waits on it
+        else
+          arrive(tempty0 + 8u * acc);
+      }
     }
   }
 
   fence_before();
-  __syncthreads();
+  __syncwarp();
+  if constexpr (kPair)
+    cluster_sync();  // neither CTA frees TMEM or exits while the pair's MMAs or arrivals may reach it
+  else
+    __syncthreads();
   fence_after();
   if (warp == 1) {
     __syncwarp();
-    tmem_dealloc(tmem_base, tmem_cols);
+    if constexpr (kPair)
+      tmem_dealloc_pair(tmem_base, tmem_cols);
+    else
+      tmem_dealloc(tmem_base, tmem_cols);
   }
   if (dyn && threadIdx.x == 0) {  // this CTA claims no more tiles; the last one resets the queue
     __threadfence();
-    if (atomicAdd(p.queue + 1, 1) == G - 1) {
+    if (atomicAdd(p.queue + 1, 1) == nctas - 1) {
       p.queue[0] = 0;
       p.queue[1] = 0;
     }
@@ -372,15 +454,19 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
 // weight row r.  All partial sums of (r, m) are loaded first, then added in K order (the
 // CTAs that ran the tile's units, lowest first), so the result does not depend on which CTA
 // finished first, and the loads take one round trip.
-constexpr int kMaxParts = 512;  // >= G (the host checks)
+constexpr int kMaxParts = 512;  // >= the party count (the host checks)
 constexpr int kFixupBatch = 16;
 
-__global__ void __launch_bounds__(kBM) umma_f8_fixup_kernel(const UmmaParams p, int G) {
+// With the schedule over CTA pairs and tile pairs (P parties): CTA (2 t + h, m) finishes half h
+// (single tile 2 T + h) of remainder tile pair t, whose sums are in the slots of CTA 2 j + h of
+// each contributing party j.
+__global__ void __launch_bounds__(kBM) umma_f8_fixup_kernel(const UmmaParams p, int P) {
   __shared__ int s_slot[kMaxParts];
   __shared__ int s_nparts;
   grid_dependents_launch();  // the next call's pre-pass may launch; it waits for this grid
-  const Sched sc{p.spt, p.wt, p.rem, G};
-  const int t_rem = blockIdx.x, m = blockIdx.y;
+  const Sched sc{p.spt, p.wt, p.rem, P};
+  const int h = (int)(blockIdx.x & 1);
+  const int t_rem = (int)(blockIdx.x >> 1), m = blockIdx.y;
   // Contributors of this tile (independent of the main kernel's data, so computed before the
   // dependency wait): consecutive CTAs from the owner of its first unit; thread i checks
   // candidate owner + i, i.e. the list is built in parallel, in K order.
@@ -389,11 +475,11 @@ __global__ void __launch_bounds__(kBM) umma_f8_fixup_kernel(const UmmaParams p, 
   {
     const int64_t tu0 = (int64_t)t_rem * p.spt, tu1 = tu0 + p.spt;
     const int b0 = sc.owner(tu0);
-    for (int i = threadIdx.x; i < kMaxParts && b0 + i < G; i += kBM) {
+    for (int i = threadIdx.x; i < kMaxParts && b0 + i < P; i += kBM) {
       const int bb = b0 + i;
       const int64_t a = sc.r0(bb), e = sc.r0(bb + 1);
       if (a < tu1 && e > a) {  // non-empty range starting before the tile's end (it ends after tu0)
-        s_slot[i] = 2 * bb + (a / p.spt == t_rem ? 0 : 1);
+        s_slot[i] = 2 * (2 * bb + h) + (a / p.spt == t_rem ? 0 : 1);
         atomicMax(&s_nparts, i + 1);
       } else if (a < tu1) {
         s_slot[i] = -1;  // empty range inside the run: skipped
@@ -403,7 +489,7 @@ __global__ void __launch_bounds__(kBM) umma_f8_fixup_kernel(const UmmaParams p, 
   }
   __syncthreads();
   grid_dependency_wait();  // the partial sums and scales of the preceding kernels
-  const TileDst d = tile_dst(p, p.wt * G + t_rem);
+  const TileDst d = tile_dst(p, 2 * (p.wt * P + t_rem) + h);
   const int row = d.row0 + threadIdx.x;
   if (row >= d.n) return;
   const int np = s_nparts;
@@ -488,17 +574,19 @@ int launch_umma_f8(const uint8_t* w, const float* w_scale, int n, int k, const u
   if (2 * p.accw > 512) return DLMH_ERR_UNSUPPORTED;
   p.split = split;
   p.early_w = early_w;
+  const bool pair = umma_pair_mode(p.nb, di.sms);
+  const int bn = pair ? p.nb / 2 : p.nb;  // activation rows in each CTA's stages
   p.w_scale = w_scale;
   p.x_scale = x_scale;
   p.out = out;
   p.ldc = ldc;
-  p.stage_bytes = kKC * (kChunkBytesA + p.nb * 128);
+  p.stage_bytes = kKC * (kChunkBytesA + bn * 128);
   int ns = (int)(kUmmaSmemLimit / (size_t)p.stage_bytes);
   if (ns > kMaxUStages) ns = kMaxUStages;
   if (ns < 2) return DLMH_ERR_UNSUPPORTED;
   p.ns = ns;
   CUtensorMap mw, mw2, mx;
-  if (!cached_map_k128(&mw, w, 1, n, k, k, kBM, kKC) || !cached_map_k128(&mx, b_codes, 1, b_rows, k, ldb, p.nb, kKC))
+  if (!cached_map_k128(&mw, w, 1, n, k, k, kBM, kKC) || !cached_map_k128(&mx, b_codes, 1, b_rows, k, ldb, bn, kKC))
     return DLMH_ERR_CUDA;
   p.t1 = (n + kBM - 1) / kBM;
   if (second) {
@@ -511,18 +599,21 @@ int launch_umma_f8(const uint8_t* w, const float* w_scale, int n, int k, const u
     mw2 = mw;
   }
   const size_t smem = (size_t)ns * p.stage_bytes + 1024;
-  if (ensure_dynamic_smem(reinterpret_cast<const void*>(umma_f8_kernel), (int)smem) != DLMH_OK) return DLMH_ERR_CUDA;
-  // schedule: whole tiles in full waves over the SMs, the rest split into units
+  const void* kfn = pair ? reinterpret_cast<const void*>(umma_f8_kernel<true>)
+                        : reinterpret_cast<const void*>(umma_f8_kernel<false>);
+  if (ensure_dynamic_smem(kfn, (int)smem) != DLMH_OK) return DLMH_ERR_CUDA;
+  // schedule: whole tiles in full waves over the SMs (or SM pairs, over tile pairs), the rest
+  // split into units
   const int ntiles = p.t1 + (second ? (second->n + kBM - 1) / kBM : 0);
   p.spt = (k / 128 + kKC - 1) / kKC;
-  const Sched sched = make_sched(ntiles, p.spt, di.sms);
-  const int G = sched.G;
-  if (G > kMaxParts) return DLMH_ERR_UNSUPPORTED;
+  const Sched sched = umma_schedule(ntiles, k, di.sms);
+  const int P = sched.G;  // parties: CTA pairs
+  if (P > kMaxParts) return DLMH_ERR_UNSUPPORTED;
   p.wt = sched.wt;
   p.rem = sched.rem;
   // whole tiles from the caller workspace's queue when there is one (both orders give the
-  // same outputs); the static order otherwise
-  p.queue = p.wt > 0 ? scratch.queue : nullptr;
+  // same outputs); the static order otherwise, and always for pairs
+  p.queue = !pair && p.wt > 0 ? scratch.queue : nullptr;
   void* ws = nullptr;
   const size_t need = (size_t)umma_partial_bytes(split != 0, ntiles, k, rows, di.sms);
   if (p.rem > 0 && scratch.caller) {
@@ -537,9 +628,10 @@ int launch_umma_f8(const uint8_t* w, const float* w_scale, int n, int k, const u
       return DLMH_ERR_CUDA;
     p.partial = static_cast<float*>(ws);
   }
-  int rc = launch_pdl(umma_f8_kernel, dim3(G), dim3(kUmmaThreads), smem, s, mw, mw2, mx, p);
+  int rc = pair ? launch_pdl_cluster(2, umma_f8_kernel<true>, dim3(2 * P), dim3(kUmmaThreads), smem, s, mw, mw2, mx, p)
+                : launch_pdl(umma_f8_kernel<false>, dim3(2 * P), dim3(kUmmaThreads), smem, s, mw, mw2, mx, p);
   if (rc == DLMH_OK && p.rem > 0) {
-    rc = launch_pdl(umma_f8_fixup_kernel, dim3(p.rem, rows), dim3(kBM), 0, s, p, G);
+    rc = launch_pdl(umma_f8_fixup_kernel, dim3(2 * p.rem, rows), dim3(kBM), 0, s, p, P);
   }
   if (ws && cudaFreeAsync(ws, s) != cudaSuccess && rc == DLMH_OK) rc = DLMH_ERR_CUDA;
   return rc;

@@ -29,12 +29,25 @@ inline int64_t ws_round256(int64_t v) { return (v + 255) / 256 * 256; }
 // W8A16 the hi and lo terms, each rows rounded up to 8.
 inline int umma_mma_n(bool split, int rows) { return split ? 2 * ((rows + 7) / 8 * 8) : (rows + 15) / 16 * 16; }
 
-// Bytes of the stream-K partial sums of one pass (0 when every tile is whole).
-inline int64_t umma_partial_bytes(bool split, int ntiles, int k, int rows, int sms) {
+// From this MMA N up, the two CTAs of a party share each MMA on one TPC (M = 256, each CTA
+// holding half of the activation box): the per-SM activation stream and its shared memory halve.
+constexpr int kUmmaPairMinN = 128;
+inline bool umma_pair_mode(int nb, int sms) { return nb >= kUmmaPairMinN && sms >= 2; }
+
+// The schedule of every pass: parties of two CTAs (sms / 2 of them, at least one) over tile
+// pairs, a pure function of the tile count, k and the SM count (never of the row count, so
+// that both kernels give a tile the same K split at every row count).
+inline Sched umma_schedule(int ntiles, int k, int sms) {
   const int spt = (k / 128 + kUmmaStageChunks - 1) / kUmmaStageChunks;
-  const Sched s = make_sched(ntiles, spt, sms);
+  return make_sched((ntiles + 1) / 2, spt, sms >= 2 ? sms / 2 : 1);
+}
+
+// Bytes of the stream-K partial sums of one pass (0 when every tile is whole): two slots per
+// CTA of MMA-N columns of 128 float32 weight rows.
+inline int64_t umma_partial_bytes(bool split, int ntiles, int k, int rows, int sms) {
+  const Sched s = umma_schedule(ntiles, k, sms);
   if (s.rem <= 0) return 0;
-  return (int64_t)2 * s.G * umma_mma_n(split, rows) * kUmmaTileRows * (int64_t)sizeof(float);
+  return (int64_t)2 * (2 * s.G) * umma_mma_n(split, rows) * kUmmaTileRows * (int64_t)sizeof(float);
 }
 
 // Bytes of the W8A16 code area of a pass over `rows` rows (codes + 128 row multipliers).

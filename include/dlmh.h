@@ -383,7 +383,9 @@ DLMH_API int dlmh_plan_chunks(int op, int rows, int k, int* offsets, int* counts
  *   k <= 0, sm_count < 0), DLMH_ERR_ROWS (rows < 0), DLMH_ERR_CUDA (no current device).
  *   Layout (256-byte aligned regions): a 256-byte tile queue, the W8A16 two-term codes
  *   2 * roundup8(min(rows, 128)) * k bytes + 512, the stream-K partial sums
- *   2 * G * N_mma * 128 * 4 bytes when the schedule has a remainder.
+ *   2 * (2 P) * N_mma * 128 * 4 bytes when the schedule has a remainder (P = sm_count / 2
+ *   parties of two CTAs over pairs of 128-row tiles; a remainder when the tile pairs are
+ *   fewer than P or not a multiple of it).
  *
  * dlmh_set_workspace: binds the device buffer ws (256-byte aligned, `bytes` long, owned by the
  *   caller, kept bound until replaced) to `stream` on the current device.  From then on every

@@ -165,16 +165,22 @@ def test_dequant_argument_errors():
 def test_workspace_bytes_sizes_and_errors():
     # Sizes of the caller workspace (dlmh.h): a 256-byte tile queue, the W8A16 two-term codes
     # of the widest pass (2 roundup8(min(rows,128)) k + 512 bytes, rounded to 256), then the
-    # stream-K partial sums 2 G N_mma 128 4 bytes when tiles % G != 0 (G = the SM count once
-    # there are more tiles than SMs).  Worked by hand for 148 SMs:
+    # stream-K partial sums, two slots of N_mma x 128 float32 per CTA (2 P CTAs, P = 74
+    # parties), when the tile pairs do not make whole waves over the parties.  Worked by hand
+    # for 148 SMs:
     ws = dl.workspace_bytes
-    # FP8 head 248320 x 5120: 1940 tiles, 13 whole waves + 16 remainder tiles
+    # FP8 head 248320 x 5120: 1940 tiles = 970 pairs, 13 whole waves + 8 remainder pairs
     assert ws(dl.OP_W8A16, 248320, 5120, 128, 148) == 256 + (2 * 128 * 5120 + 512) + 2 * 148 * 256 * 128 * 4
     assert ws(dl.OP_W8A8, 248320, 5120, 128, 148) == 256 + 2 * 148 * 128 * 128 * 4
     assert ws(dl.OP_W8A8, 248320, 5120, 1000, 148) == ws(dl.OP_W8A8, 248320, 5120, 128, 148)  # 128-row passes
     assert ws(dl.OP_W8A16, 248320, 5120, 3, 148) == 256 + (2 * 8 * 5120 + 512) + 2 * 148 * 16 * 128 * 4
     # 148 x 128 rows: whole waves only, no partial sums
     assert ws(dl.OP_W8A8, 148 * 128, 5120, 64, 148) == 256
+    # 147 tiles are 74 tile pairs: one whole wave over the 74 parties (CTA pairs), at any N
+    assert ws(dl.OP_W8A8, 147 * 128, 5120, 64, 148) == 256
+    assert ws(dl.OP_W8A8, 147 * 128, 5120, 128, 148) == 256
+    # 150 tiles are 75 tile pairs: one whole wave and one remainder pair
+    assert ws(dl.OP_W8A8, 150 * 128, 5120, 128, 148) == 256 + 2 * 148 * 128 * 128 * 4
     # down projection 4096 x 14336: 32 tiles < 148 SMs, all of them remainder tiles
     assert ws(dl.OP_W8A8, 4096, 14336, 1, 148) == 256 + 2 * 148 * 16 * 128 * 4
     # gate + up pair: the tiles of both weights
