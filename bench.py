@@ -557,7 +557,8 @@ def profile_case(name):
     """Small single-GPU cases for ncu captures (one kernel of interest, few launches, inputs well
     above the 126 MB L2 or, for the small weights, rotated copies); prints one line and no bench
     result.  down: the W8A8 SiLU down projection 4096 x 14336 at M = 1, 6 calls over 3 weight
-    copies; nvfp4: NVFP4 W4A16 14336 x 4096 at M = 1, 6 calls over 6 weight copies."""
+    copies; nvfp4: NVFP4 W4A16 14336 x 4096 at M = 1, 6 calls over 6 weight copies; head: FP8
+    W8A16 on a 38188 x 5120 head (196 MB), three calls at M = 32 then three at M = 128."""
     import decode_lm_head_b200 as dl
     from decode_lm_head_b200 import synth
 
@@ -586,6 +587,17 @@ def profile_case(name):
         for wp, sc, gl in wf:
             dl.w4a16_gemv(wp, sc, gl, x, out=out, stream=stream)
         torch.cuda.synchronize()
+    elif name == "head":
+        n, k = 38188, 5120
+        w, s = synth.fp8_weight(n, k, 1, dev), synth.row_scales(n, 1, dev)
+        x = synth.bf16_rows(128, k, 1, dev, std=0.5)
+        keep = bind_workspace(dl, stream, dev, [(dl.OP_W8A16, n, k, 128)])
+        out = torch.empty(128, n, dtype=torch.bfloat16, device=dev)
+        for m in (32, 32, 32, 128, 128, 128):
+            dl.lm_head_fp8_w8a16(w, s, x[:m], out=out[:m], stream=stream)
+        torch.cuda.synchronize()
+        dl.set_workspace(None, stream=stream)
+        del keep
     else:
         raise SystemExit(f"unknown profile case {name}")
     print(f"profile case {name}: done, device fault {dl.device_fault(reset=True)}")
@@ -802,7 +814,7 @@ def main():
                     help="head rows; smaller values only for profiling captures (the workload is 248320)")
     ap.add_argument("--profile-q6k", type=int, default=0, metavar="N",
                     help="run only the Q6_K profiling case (N x 7168 blocks, 8 rows, 4 calls) and exit")
-    ap.add_argument("--profile", choices=["down", "nvfp4"], default=None,
+    ap.add_argument("--profile", choices=["down", "nvfp4", "head"], default=None,
                     help="run only a small profiling case for ncu (see profile_case) and exit")
     args = ap.parse_args()
     if args.profile_q6k > 0:

@@ -46,10 +46,11 @@ namespace {
 using namespace umma;
 
 constexpr int kUmmaThreads = 192;
-constexpr int kKC = kUmmaStageChunks;  // 128-byte K-chunks per stage
+constexpr int kKC = kUmmaStageChunks;  // 128-byte K-chunks per schedule unit
 static_assert(kBM == kUmmaTileRows, "the workspace layout assumes 128-row tiles");
 constexpr int kChunkBytesA = kBM * 128;
-constexpr int kMaxUStages = 6;
+constexpr int kMaxUStages = 8;
+static_assert(kKC % 2 == 0, "a unit is one stage or two");
 constexpr int kJobRing = 4;  // job descriptors in flight from the producer to the MMA and epilogue warps
 
 static __device__ int umma_fault_word = 0;  // 1: producer, 2: MMA (stage), 4: MMA (tmem), 8: epilogue
@@ -86,6 +87,7 @@ struct UmmaParams {
   uint16_t* out;
   int64_t ldc;
   int ns;                // ring stages
+  int cps;               // 128-byte chunks per stage: kKC, or kKC / 2 (each unit as two stages)
   int stage_bytes;       // A + B bytes of one stage
   // Stream-K schedule (umma_schedule) over P = gridDim.x / 2 parties (CTA pairs) and tile
   // pairs, a pure function of n, k and the SM count, never of the row count; partial sums are
@@ -164,7 +166,8 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
   const uint32_t ring_u32 = smem_u32(ring);
   const uint32_t full0 = smem_u32(bar_full), empty0 = smem_u32(bar_empty);
   const uint32_t tfull0 = smem_u32(bar_tfull), tempty0 = smem_u32(bar_tempty);
-  const int a_bytes = kKC * kChunkBytesA;
+  const int a_bytes = p.cps * kChunkBytesA;
+  const int sub = kKC / p.cps;  // stages per schedule unit
   const int bn = kPair ? p.nb / 2 : p.nb;  // activation rows in this CTA's stages
   const int b_chunk = bn * 128;
   const uint32_t tmem_cols = 2u * (uint32_t)p.accw;
@@ -264,18 +267,19 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
       auto load_w = [&](uint32_t dst, int tt, int u, int slot_) {
         const bool first = tt < p.t1;
         const int row0 = first ? tt * kBM : (p.n2 > 0 ? (tt - p.t1) * kBM : p.t1 * kBM);
-        load(dst, first ? &map_w : &map_w2, row0, u * kKC, slot_, pol_w);
+        load(dst, first ? &map_w : &map_w2, row0, u * p.cps, slot_, pol_w);
       };
-      const int npre = p.early_w ? min(p.ns, jb.z - jb.y) : 0;
+      // stages v = unit * sub + i, covering chunks [v cps, (v + 1) cps)
+      const int npre = p.early_w ? min(p.ns, (jb.z - jb.y) * sub) : 0;
       for (int s = 0; s < npre; ++s) {
         if (leader) expect_tx(full0 + 8u * s, expect);
-        load_w(ring_u32 + s * p.stage_bytes, jb.x, jb.y + s, s);
+        load_w(ring_u32 + s * p.stage_bytes, jb.x, jb.y * sub + s, s);
       }
       grid_dependency_wait();
       int slot = 0, phase = 0, s = 0;
       for (bool have = true; have;) {
         const int tile = jb.x;
-        for (int u = jb.y; u < jb.z; ++u, ++s) {
+        for (int u = jb.y * sub; u < jb.z * sub; ++u, ++s) {
           if (s >= p.ns && !wait(empty0 + 8u * slot, phase ^ 1)) atomicOr(&umma_fault_word, 1);
           const uint32_t st = ring_u32 + slot * p.stage_bytes;
           // the full boxes always land (rows past n, rows past `rows` and a chunk past K are
@@ -285,7 +289,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
             load_w(st, tile, u, slot);
           }
           // B: the activation rows (this CTA's half of them in a pair), the same chunks
-          load(st + a_bytes, &map_x, kPair ? h * bn : 0, u * kKC, slot, pol_x);
+          load(st + a_bytes, &map_x, kPair ? h * bn : 0, u * p.cps, slot, pol_x);
           if (++slot == p.ns) {
             slot = 0;
             phase ^= 1;
@@ -322,10 +326,10 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
         if (i >= 2 && !wait(tempty0 + 8u * acc, ((i - 2) >> 1) & 1)) atomicOr(&umma_fault_word, 4);
         fence_after();
         const uint32_t tmem_d = tmem_base + (uint32_t)(acc * p.accw);
-        for (int u = u0; u < u1; ++u) {
+        for (int u = u0 * sub; u < u1 * sub; ++u) {  // stages
           if (!wait(full0 + 8u * slot, phase)) atomicOr(&umma_fault_word, 2);
           fence_after();
-          const int nch = min(kKC, kchunks - u * kKC);
+          const int nch = min(p.cps, kchunks - u * p.cps);  // <= 0: a stage wholly past K
           const uint32_t st = ring_u32 + slot * p.stage_bytes;
           for (int c = 0; c < nch; ++c) {
             const uint32_t a0 = st + c * kChunkBytesA;
@@ -334,10 +338,10 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
             for (int kk = 0; kk < 4; ++kk) {  // K = 32 bytes per MMA
               if constexpr (kPair)
                 umma_f8_pair(tmem_d, desc_sw128(a0 + kk * 32), desc_sw128(b0 + kk * 32), idesc,
-                             ((u - u0) | c | kk) != 0);
+                             ((u - u0 * sub) | c | kk) != 0);
               else
                 umma_f8(tmem_d, desc_sw128(a0 + kk * 32), desc_sw128(b0 + kk * 32), idesc,
-                        ((u - u0) | c | kk) != 0);
+                        ((u - u0 * sub) | c | kk) != 0);
             }
           }
           // the stage (of both CTAs) is free once these MMAs have read it
@@ -580,17 +584,20 @@ int launch_umma_f8(const uint8_t* w, const float* w_scale, int n, int k, const u
   p.x_scale = x_scale;
   p.out = out;
   p.ldc = ldc;
-  p.stage_bytes = kKC * (kChunkBytesA + bn * 128);
+  // a stage is a whole unit (the longest run of each weight row per copy) when the ring holds
+  // two of them, else half a unit
+  p.cps = kUmmaSmemLimit / ((size_t)kKC * (kChunkBytesA + bn * 128)) >= 2 ? kKC : kKC / 2;
+  p.stage_bytes = p.cps * (kChunkBytesA + bn * 128);
   int ns = (int)(kUmmaSmemLimit / (size_t)p.stage_bytes);
   if (ns > kMaxUStages) ns = kMaxUStages;
   if (ns < 2) return DLMH_ERR_UNSUPPORTED;
   p.ns = ns;
   CUtensorMap mw, mw2, mx;
-  if (!cached_map_k128(&mw, w, 1, n, k, k, kBM, kKC) || !cached_map_k128(&mx, b_codes, 1, b_rows, k, ldb, bn, kKC))
+  if (!cached_map_k128(&mw, w, 1, n, k, k, kBM, p.cps) || !cached_map_k128(&mx, b_codes, 1, b_rows, k, ldb, bn, p.cps))
     return DLMH_ERR_CUDA;
   p.t1 = (n + kBM - 1) / kBM;
   if (second) {
-    if (!cached_map_k128(&mw2, second->w, 1, second->n, k, k, kBM, kKC)) return DLMH_ERR_CUDA;
+    if (!cached_map_k128(&mw2, second->w, 1, second->n, k, k, kBM, p.cps)) return DLMH_ERR_CUDA;
     p.n2 = second->n;
     p.w_scale2 = second->w_scale;
     p.out2 = second->out;

@@ -20,7 +20,7 @@
 namespace dlmh {
 
 constexpr int kUmmaTileRows = 128;     // weight rows per tile (the MMA's M)
-constexpr int kUmmaStageChunks = 2;    // 128-byte K chunks per pipeline stage
+constexpr int kUmmaStageChunks = 4;    // 128-byte K chunks per schedule unit
 constexpr int64_t kWsQueueBytes = 256;
 
 inline int64_t ws_round256(int64_t v) { return (v + 255) / 256 * 256; }
