@@ -558,7 +558,8 @@ def profile_case(name):
     above the 126 MB L2 or, for the small weights, rotated copies); prints one line and no bench
     result.  down: the W8A8 SiLU down projection 4096 x 14336 at M = 1, 6 calls over 3 weight
     copies; nvfp4: NVFP4 W4A16 14336 x 4096 at M = 1, 6 calls over 6 weight copies; head: FP8
-    W8A16 on a 38188 x 5120 head (196 MB), three calls at M = 32 then three at M = 128."""
+    W8A16 on a 38188 x 5120 head (196 MB), three calls at M = 32 then three at M = 128;
+    q6k_wide: Q6_K 32768 x 7168 (193 MB), two calls at M = 16 then two at M = 64."""
     import decode_lm_head_b200 as dl
     from decode_lm_head_b200 import synth
 
@@ -598,6 +599,14 @@ def profile_case(name):
         torch.cuda.synchronize()
         dl.set_workspace(None, stream=stream)
         del keep
+    elif name == "q6k_wide":
+        n, k = 32768, 7168
+        blocks = synth.q6k_blocks(n, k, 4, dev)
+        x = synth.bf16_rows(64, k, 4, dev)
+        out = torch.empty(64, n, dtype=torch.bfloat16, device=dev)
+        for m in (16, 16, 64, 64):
+            dl.q6k_lm_head(blocks, x[:m], out=out[:m], stream=stream)
+        torch.cuda.synchronize()
     else:
         raise SystemExit(f"unknown profile case {name}")
     print(f"profile case {name}: done, device fault {dl.device_fault(reset=True)}")
@@ -814,7 +823,7 @@ def main():
                     help="head rows; smaller values only for profiling captures (the workload is 248320)")
     ap.add_argument("--profile-q6k", type=int, default=0, metavar="N",
                     help="run only the Q6_K profiling case (N x 7168 blocks, 8 rows, 4 calls) and exit")
-    ap.add_argument("--profile", choices=["down", "nvfp4", "head"], default=None,
+    ap.add_argument("--profile", choices=["down", "nvfp4", "head", "q6k_wide"], default=None,
                     help="run only a small profiling case for ncu (see profile_case) and exit")
     args = ap.parse_args()
     if args.profile_q6k > 0:
