@@ -9,10 +9,10 @@
 // rounding it to E4M3's 4 leaves a residual of at most 4 bits, so hi + lo/16 == x' exactly
 // whenever |x'| >= 2^-6 (every element within 2^-13 of the row maximum); below that the
 // error is at most 2^-14 in x' units.  The two terms are the B operand's first and second
-// roundup8(rows) columns, so the weights stay E4M3 in the A operand: the tensor core takes an M=128,
-// K=32-byte instruction in the same ~142 clocks whatever N <= 256, i.e. it consumes A at
-// ~29 bytes/clock/SM, above the HBM share of an SM (~24); a 16-bit A operand would halve
-// the weight rate and make the kernel MMA-bound.
+// roundup8(rows) columns, so the weights stay E4M3 in the A operand.  The tensor pipe's time per
+// M=128, K=32-byte instruction grows with N (about 41 clocks at N = 64, 184 at N = 256): small
+// row counts stay far from it, while at 128 W8A16 rows (N = 256) the MMA time per weight byte
+// matches the HBM share of an SM and the two co-bound the call.
 //
 // Swap-AB: the weight is the MMA's A operand (M = 128 weight rows per tile) and the
 // activation codes are its B operand (N = rows rounded up to 16; for W8A16 twice the rows
