@@ -10,9 +10,9 @@
 // whenever |x'| >= 2^-6 (every element within 2^-13 of the row maximum); below that the
 // error is at most 2^-14 in x' units.  The two terms are the B operand's first and second
 // roundup8(rows) columns, so the weights stay E4M3 in the A operand.  The tensor pipe's time per
-// M=128, K=32-byte instruction grows with N (about 41 clocks at N = 64, 184 at N = 256): small
-// row counts stay far from it, while at 128 W8A16 rows (N = 256) the MMA time per weight byte
-// matches the HBM share of an SM and the two co-bound the call.
+// M=128, K=32-byte instruction grows with N (about 32 clocks at N = 64, 129 at N = 256: the
+// dense FP8 rate): small row counts stay far from it, while at 128 W8A16 rows (N = 256) the MMA
+// is busy for about 70 % of the weight stream's time.
 //
 // Swap-AB: the weight is the MMA's A operand (M = 128 weight rows per tile) and the
 // activation codes are its B operand (N = rows rounded up to 16; for W8A16 twice the rows
