@@ -3,9 +3,11 @@
 //   - E8M0:   out[f]    = bf16( e2m1(W[f]) * 2^(e[f / block] - 127) )          (flat index f)
 // Float32 arithmetic: the E2M1 x E4M3 product is exact (at most 6 significant bits), the
 // product with g is one float32 rounding, the cast to BF16 rounds to nearest-even; the E8M0
-// product is exact unless it leaves the float32 range.  Each thread converts 16 consecutive
-// elements of a row: one 8-byte load of codes, one scale, two 16-byte stores, so loads and
-// stores are coalesced across the warp and the kernel is a plain HBM stream.
+// product is exact unless it leaves the float32 range.  NVFP4: a lane converts 8-element
+// groups, one 4-byte load of codes and one 16-byte store each, laid out so that every load and
+// store instruction of a warp covers one contiguous run.  E8M0: each thread converts 16
+// consecutive elements of a row (one 8-byte load, two 16-byte stores), which measured faster
+// for it than the warp-span layout (33 against 39 us on 14336 x 4096).
 #include "dlmh_common.cuh"
 #include "gemv_launch.h"
 
@@ -31,43 +33,45 @@ __device__ __forceinline__ void fp4x8_to_bf16(uint32_t word, float scale, float 
   }
 }
 
-// Index type: 32-bit when every chunk index fits (the usual case), 64-bit otherwise.
+// Work split: a flat sequence of 8-element groups (rows are k/8 groups long, k % 16 == 0, so a
+// group never crosses a row).  A warp takes kDqSpan consecutive groups per step, lane l the
+// groups l, l + 32, ...: every code load (4 bytes a lane) and every 16-byte output store of
+// the warp covers one contiguous run, and all of a lane's loads are issued before its first
+// conversion.  Index type: 32-bit when every index fits, 64-bit otherwise.
+constexpr int kDqPerLane = 4;
+constexpr int kDqSpan = 32 * kDqPerLane;
+
 template <typename I>
 __global__ void __launch_bounds__(kDqThreads) nvfp4_dequant_kernel(const uint8_t* __restrict__ packed,
                                                                    const uint8_t* __restrict__ bscale, float g,
                                                                    int n, int k, uint16_t* __restrict__ out,
                                                                    int64_t ldo) {
-  const I per_row = k / 16;
-  const I chunks = (I)n * per_row;
-  const I stride = (I)gridDim.x * blockDim.x;
-  // two chunks per iteration, both loads issued before either is converted
-  for (I c = (I)blockIdx.x * blockDim.x + threadIdx.x; c < chunks; c += 2 * stride) {
-    const I c1 = c + stride;
-    const bool has1 = c1 < chunks;
-    const I row0 = c / per_row, cb0 = c - row0 * per_row;
-    const I row1 = has1 ? c1 / per_row : 0, cb1 = has1 ? c1 - row1 * per_row : 0;
-    const uint2 pk0 = *reinterpret_cast<const uint2*>(packed + (int64_t)c * 8);
-    const uint8_t s0 = bscale[c];
-    uint2 pk1 = make_uint2(0, 0);
-    uint8_t s1 = 0;
-    if (has1) {
-      pk1 = *reinterpret_cast<const uint2*>(packed + (int64_t)c1 * 8);
-      s1 = bscale[c1];
+  const I per_row = k / 8;
+  const I groups = (I)n * per_row;
+  const int lane = threadIdx.x & 31;
+  const I warp0 = ((I)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const I nwarps = ((I)gridDim.x * blockDim.x) >> 5;
+  for (I base = warp0 * kDqSpan; base < groups; base += nwarps * kDqSpan) {
+    uint32_t w[kDqPerLane];
+    uint32_t sb[kDqPerLane];
+#pragma unroll
+    for (int j = 0; j < kDqPerLane; ++j) {
+      const I g8 = base + lane + 32 * j;
+      const bool ok = g8 < groups;
+      w[j] = ok ? __ldg(reinterpret_cast<const unsigned int*>(packed) + g8) : 0u;
+      sb[j] = ok ? (uint32_t)__ldg(bscale + (g8 >> 1)) : 0u;  // one scale per 16 values
     }
-    uint32_t lo[4], hi[4];
-    const float sc0 = f16_bits_to_f32(e4m3x2_to_f16x2((uint16_t)s0) & 0xffffu);
-    fp4x8_to_bf16<true>(pk0.x, sc0, g, lo);
-    fp4x8_to_bf16<true>(pk0.y, sc0, g, hi);
-    uint4* dst = reinterpret_cast<uint4*>(out + (int64_t)row0 * ldo + (int64_t)cb0 * 16);
-    dst[0] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-    dst[1] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-    if (has1) {
-      const float sc1 = f16_bits_to_f32(e4m3x2_to_f16x2((uint16_t)s1) & 0xffffu);
-      fp4x8_to_bf16<true>(pk1.x, sc1, g, lo);
-      fp4x8_to_bf16<true>(pk1.y, sc1, g, hi);
-      dst = reinterpret_cast<uint4*>(out + (int64_t)row1 * ldo + (int64_t)cb1 * 16);
-      dst[0] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-      dst[1] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+#pragma unroll
+    for (int j = 0; j < kDqPerLane; ++j) {
+      const I g8 = base + lane + 32 * j;
+      if (g8 < groups) {
+        uint32_t o[4];
+        const float sc = f16_bits_to_f32(e4m3x2_to_f16x2((uint16_t)sb[j]) & 0xffffu);
+        fp4x8_to_bf16<true>(w[j], sc, g, o);
+        const I row = g8 / per_row;
+        *reinterpret_cast<uint4*>(out + (int64_t)row * ldo + (int64_t)(g8 - row * per_row) * 8) =
+            make_uint4(o[0], o[1], o[2], o[3]);
+      }
     }
   }
 }
@@ -136,10 +140,22 @@ __global__ void __launch_bounds__(kDqThreads) e8m0_dequant_kernel(const uint8_t*
   }
 }
 
-int grid_for(int64_t chunks) {
+// Blocks for the E8M0 kernel's `chunks` 16-element chunks: one per thread, capped at 16 blocks
+// per SM.
+int grid_for_chunks(int64_t chunks) {
   const DeviceInfo di = device_info();
   const int64_t want = (chunks + kDqThreads - 1) / kDqThreads;
   const int64_t cap = (int64_t)(di.sms > 0 ? di.sms : 148) * 16;
+  return (int)(want < cap ? want : cap);
+}
+
+// Blocks for `groups` 8-element groups: enough warps for one span each, at most 8 resident
+// blocks per SM (2048 threads).
+int grid_for(int64_t groups) {
+  const DeviceInfo di = device_info();
+  const int64_t warps = (groups + kDqSpan - 1) / kDqSpan;
+  const int64_t want = (warps + kDqThreads / 32 - 1) / (kDqThreads / 32);
+  const int64_t cap = (int64_t)(di.sms > 0 ? di.sms : 148) * 8;
   return (int)(want < cap ? want : cap);
 }
 
@@ -147,12 +163,12 @@ int grid_for(int64_t chunks) {
 
 int nvfp4_dequant_launch(const uint8_t* packed, const uint8_t* bscale, float g, int n, int k, uint16_t* out,
                          int64_t ldo, cudaStream_t s) {
-  const int64_t chunks = (int64_t)n * (k / 16);
-  if (chunks == 0) return DLMH_OK;
-  if (chunks * 16 < ((int64_t)1 << 31))
-    nvfp4_dequant_kernel<int32_t><<<grid_for(chunks), kDqThreads, 0, s>>>(packed, bscale, g, n, k, out, ldo);
+  const int64_t groups = (int64_t)n * (k / 8);
+  if (groups == 0) return DLMH_OK;
+  if (groups * 8 + (int64_t)kDqSpan * 8 * 148 * 8 < ((int64_t)1 << 31))
+    nvfp4_dequant_kernel<int32_t><<<grid_for(groups), kDqThreads, 0, s>>>(packed, bscale, g, n, k, out, ldo);
   else
-    nvfp4_dequant_kernel<int64_t><<<grid_for(chunks), kDqThreads, 0, s>>>(packed, bscale, g, n, k, out, ldo);
+    nvfp4_dequant_kernel<int64_t><<<grid_for(groups), kDqThreads, 0, s>>>(packed, bscale, g, n, k, out, ldo);
   return launch_status();
 }
 
@@ -161,9 +177,9 @@ int e8m0_dequant_launch(const uint8_t* packed, const uint8_t* scales, int64_t bl
   const int64_t chunks = (int64_t)n * k / 16;
   if (chunks == 0) return DLMH_OK;
   if (chunks * 16 < ((int64_t)1 << 31))
-    e8m0_dequant_kernel<int32_t><<<grid_for(chunks), kDqThreads, 0, s>>>(packed, scales, block, n, k, out, ldo);
+    e8m0_dequant_kernel<int32_t><<<grid_for_chunks(chunks), kDqThreads, 0, s>>>(packed, scales, block, n, k, out, ldo);
   else
-    e8m0_dequant_kernel<int64_t><<<grid_for(chunks), kDqThreads, 0, s>>>(packed, scales, block, n, k, out, ldo);
+    e8m0_dequant_kernel<int64_t><<<grid_for_chunks(chunks), kDqThreads, 0, s>>>(packed, scales, block, n, k, out, ldo);
   return launch_status();
 }
 

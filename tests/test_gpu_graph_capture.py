@@ -2,7 +2,7 @@
 
 Without a caller workspace the captured call's scratch comes from the library pool (a graph
 memory node) and its whole tiles go in the static order; every replay must give the eager
-call's bits.  (With a workspace the eager calls take the queue order: see
+call's bits.  At 100 rows (MMA N = 208) the GEMV runs as clusters of CTA pairs.  (With a workspace the eager calls take the queue order: see
 test_gpu_workspace.py.)
 """
 
@@ -16,7 +16,7 @@ from decode_lm_head_b200 import synth
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("rows", [5, 40])
+@pytest.mark.parametrize("rows", [5, 40, 100])
 def test_lm_head_graph_replays_match_eager(rows):
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
