@@ -464,7 +464,9 @@ __global__ void __launch_bounds__(kQ6Threads, 1) q6k_rows8_kernel(const Q6RowsPa
 // Each consumer warp decodes a weight fragment once per sub-block ((q - 32) as signed bytes)
 // and runs NT 8-column MMAs on it.  The K-slices of the 8-row kernels are kept: each slice is
 // accumulated alone from 0 and added to the total at the slice's end (q6_slice_ends).
-// NT <= 4: 15 consumer warps + 1 producer (128 registers a thread); NT = 8: 7 + 1 (255).
+// NT <= 4: 15 consumer warps + 1 producer (128 registers a thread); NT = 8: 11 + 1 (168, a
+// small spill; 7 warps of 228 registers left the schedulers short of warps: 1040 against
+// 881 us for 64 rows on a 129280 x 7168 head).
 constexpr int kQWRowBytes = 288;   // one super-block of one q8_1 row: 8 blocks
 constexpr int kQWRowStride = 304;  // 76 words: the 8 B-fragment rows hit 32 banks
 constexpr int kQWSpan = 240;       // staged bytes per weight row and super-block (>= 224)
@@ -473,7 +475,7 @@ constexpr int kQWMaxActStages = 4;
 
 template <int NT>
 struct QW {
-  static constexpr int kWarps = NT >= 8 ? 7 : 15;  // consumer warps
+  static constexpr int kWarps = NT >= 8 ? 11 : 15;  // consumer warps
   static constexpr int kThreads = (kWarps + 1) * 32;
 };
 
