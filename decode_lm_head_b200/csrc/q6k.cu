@@ -189,8 +189,10 @@ __device__ __forceinline__ void q6_load_global(Q6W& w, bool valid, const uint8_t
 // One persistent 512-thread CTA per SM over 16-row weight tiles; warp w runs K-slice w of every
 // tile (q6_slice_begin), and the 16 slices of a tile are summed in warp order through shared
 // memory.  Activations:
-//   - dxs [K/32][8] float32 q8_1 d, and cor [K/16][8] int32 -32 * (sum of the 16 codes of
-//     the sub-block), staged once per CTA;
+//   - the q8_1 d of block b and column c (float32, dxs) and -32 * (sum of the 16 codes of
+//     sub-block 2b + e of column c) (int32, cor), staged once per CTA in the order lane (g, t)
+//     reads them, 16 bytes at a time: dxs [b / 2][c / 2][b % 2][c % 2] (two blocks per load),
+//     cor [b][c / 2][e][c % 2] (one block per load);
 //   - the B fragments (4 codes of column g, values 4t..4t+3 of each sub-block): for K <= 8192
 //     (at most 2 super-blocks per slice) each warp keeps the 32 words of its own slice in
 //     registers, loaded once; beyond that the codes are staged whole, xs [8][rs] with
@@ -205,6 +207,10 @@ __device__ __forceinline__ void q6_load_global(Q6W& w, bool valid, const uint8_t
 // 16-byte-multiple prefix in bulk and its last bytes with plain loads), or 16-bit global loads
 // (blocks only 2-byte aligned).  A tile's stages are released at the tile's reduction barrier,
 // so the ring holds two tiles when it can: one computed, the next one landing.
+// MMA rows g and g + 8 of lane (g, t) are tile rows (g, g + 8) or (2g, 2g + 1), and the stage
+// slots are padded, as the host finds fewest shared-memory bank conflicts for the weight
+// fragment loads: rows 5880 bytes apart (K = 7168) put rows g and g + 1 on overlapping banks,
+// rows 2g with 64 bytes of slot padding spread the 8 rows of one load over all 32 banks.
 
 struct Q6Params {
   const uint8_t* blocks;
@@ -225,6 +231,7 @@ struct Q6RowsParams {
   int stage_rows;    // SR: 4 or 8
   int stage_stride;  // bytes per stage slot (>= SR rows, multiple of 128)
   int ring_offset;   // byte offset of the ring in dynamic shared memory
+  int row_pair;      // 1: MMA rows g, g + 8 are tile rows 2g, 2g + 1; 0: tile rows g, g + 8
   int early_w;       // the preceding kernel is this library's q8_1 quantize: weight copies may start before it ends
 };
 
@@ -248,7 +255,7 @@ __device__ void q6_stage_acts(const Q6Params& p, uint8_t* smem, bool stage_codes
   for (int it = threadIdx.x; it < kQ6MaxRows * nb32; it += blockDim.x) {
     const int m = it / nb32, b = it % nb32;
     const uint32_t* bw = reinterpret_cast<const uint32_t*>(p.q8 + ((int64_t)m * nb32 + b) * 36);
-    dxs[b * kQ6MaxRows + m] = m < p.rows ? f16_bits_to_f32(bw[0] & 0xffffu) : 0.f;
+    dxs[(b >> 1) * 16 + (m >> 1) * 4 + (b & 1) * 2 + (m & 1)] = m < p.rows ? f16_bits_to_f32(bw[0] & 0xffffu) : 0.f;
     int s0 = 0, s1 = 0;
     if (m < p.rows) {
 #pragma unroll
@@ -257,8 +264,8 @@ __device__ void q6_stage_acts(const Q6Params& p, uint8_t* smem, bool stage_codes
         s1 = __dp4a((int)bw[5 + i], 0x01010101, s1);
       }
     }
-    cor[(2 * b) * kQ6MaxRows + m] = -32 * s0;
-    cor[(2 * b + 1) * kQ6MaxRows + m] = -32 * s1;
+    cor[b * 16 + (m >> 1) * 4 + (m & 1)] = -32 * s0;
+    cor[b * 16 + (m >> 1) * 4 + 2 + (m & 1)] = -32 * s1;
     if (!stage_codes) continue;
     uint8_t* dst = xs + m * rs + (b >> 3) * 256;
     const int kb = (b & 7) * 32;  // first value of this block inside its super-block
@@ -279,21 +286,23 @@ __device__ __forceinline__ uint32_t q6_bfrag(const Q6Params& p, int col, int sb,
                                             16 * (j & 1) + 4 * t);
 }
 
-// One super-block of the 16-row tile (rows g: wa, g+8: wb) against the 8 columns: bw[j] is the
-// lane's B fragment of sub-block j; dxs = dxs + (8 sb) 32 + 8 t; cor = cor + (16 sb) 32 + 8 t.
+// One super-block of the 16-row tile (MMA rows g: wa, g+8: wb) against the 8 columns: bw[j] is
+// the lane's B fragment of sub-block j; dxs and cor point at the super-block's staged values
+// (256 and 512 bytes a super-block) plus 16 t.
 __device__ __forceinline__ void q6_superblock_8(float (&acc)[4], const Q6W& wa, const Q6W& wb, const uint32_t (&bw)[16],
                                                 uint32_t dxs, uint32_t cor) {
   float tsb[4] = {0.f, 0.f, 0.f, 0.f};
+  uint4 dx;
 #pragma unroll
   for (int blk = 0; blk < 8; ++blk) {
     const int j0 = 2 * blk, j1 = j0 + 1;
-    const uint2 c0 = lds_u64(cor + 32 * j0), c1 = lds_u64(cor + 32 * j1);
+    const uint4 c = lds128(cor + 64 * blk);  // columns 2t, 2t + 1 of sub-blocks j0, j1
     int d0[4], d1[4];
-    mma_u8s8_c(d0, q6_codes_u8(wa, j0), q6_codes_u8(wb, j0), bw[j0], (int)c0.x, (int)c0.y);
-    mma_u8s8_c(d1, q6_codes_u8(wa, j1), q6_codes_u8(wb, j1), bw[j1], (int)c1.x, (int)c1.y);
-    const uint2 dx = lds_u64(dxs + 32 * blk);
+    mma_u8s8_c(d0, q6_codes_u8(wa, j0), q6_codes_u8(wb, j0), bw[j0], (int)c.x, (int)c.y);
+    mma_u8s8_c(d1, q6_codes_u8(wa, j1), q6_codes_u8(wb, j1), bw[j1], (int)c.z, (int)c.w);
+    if ((blk & 1) == 0) dx = lds128(dxs + 64 * (blk >> 1));  // blocks blk, blk + 1
     q6_block_step(tsb, d0, d1, q6_scale(wa, j0), q6_scale(wa, j1), q6_scale(wb, j0), q6_scale(wb, j1),
-                  __uint_as_float(dx.x), __uint_as_float(dx.y));
+                  __uint_as_float((blk & 1) ? dx.z : dx.x), __uint_as_float((blk & 1) ? dx.w : dx.y));
   }
   q6_superblock_end(acc, tsb, wa.d, wb.d);
 }
@@ -302,12 +311,12 @@ __device__ __forceinline__ void q6_superblock_8(float (&acc)[4], const Q6W& wa, 
 // 128 threads of warps 12..15 (the K-slices are split with the longer ones first, so these
 // warps never have more super-blocks than the others), thread r of them output r.
 constexpr int kQ6RedWarp0 = kQ6Warps - 4;
-__device__ __forceinline__ void q6_reduce_tile(const Q6Params& p, const float* red, int tile) {
+__device__ __forceinline__ void q6_reduce_tile(const Q6Params& p, const float* red, int tile, int row_pair) {
   const int o = threadIdx.x - kQ6RedWarp0 * 32;
   const int rr = o % kQ6TileRows, cc = o / kQ6TileRows;
   const int row = tile * kQ6TileRows + rr;
   if (cc < p.rows && row < p.n) {
-    const int gg = rr & 7, up = rr >> 3;
+    const int gg = row_pair ? rr >> 1 : rr & 7, up = row_pair ? rr & 1 : rr >> 3;  // lane row, MMA half
     const int ln = gg * 4 + (cc >> 1), comp = up * 2 + (cc & 1);
     float sum = 0.f;
 #pragma unroll
@@ -368,8 +377,8 @@ __global__ void __launch_bounds__(kQ6Threads, 1) q6k_rows8_kernel(const Q6RowsPa
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int sb_begin = q6_slice_begin(nsb, warp), sb_end = q6_slice_begin(nsb, warp + 1);
-  const uint32_t dx0 = smem_u32(smem) + (uint32_t)(8 * t);
-  const uint32_t co0 = smem_u32(smem) + (uint32_t)(q6_dx_bytes(p.k) + 8 * t);
+  const uint32_t dx0 = smem_u32(smem) + (uint32_t)(16 * t);
+  const uint32_t co0 = smem_u32(smem) + (uint32_t)(q6_dx_bytes(p.k) + 16 * t);
   const uint32_t xs0 = smem_u32(smem) + (uint32_t)(q6_dx_bytes(p.k) + q6_cor_bytes(p.k) + g * rs + 16 * t);
   uint32_t bfr[kQ6RegSlice][16];
   if (kRegActs) {
@@ -380,11 +389,12 @@ __global__ void __launch_bounds__(kQ6Threads, 1) q6k_rows8_kernel(const Q6RowsPa
   }
   __syncthreads();
 
-  const int sa_off = g / SR, sb_off = (g + 8) / SR;  // stages of rows g and g+8 within a tile
+  const int lra = sp.row_pair ? 2 * g : g, lrb = sp.row_pair ? 2 * g + 1 : g + 8;  // tile rows of MMA rows g, g+8
+  const int sa_off = lra / SR, sb_off = lrb / SR;  // their stages within a tile
   for (int i = 0; T0 + i < T1; ++i) {
     const int tile = T0 + i;
-    const int r0 = tile * kQ6TileRows + g;
-    const bool va = r0 < p.n, vb = r0 + 8 < p.n;
+    const int ra = tile * kQ6TileRows + lra, rb = tile * kQ6TileRows + lrb;
+    const bool va = ra < p.n, vb = rb < p.n;
     uint32_t base_a = 0, base_b = 0;
     if (kStream) {
       bool ok = true;
@@ -394,13 +404,14 @@ __global__ void __launch_bounds__(kQ6Threads, 1) q6k_rows8_kernel(const Q6RowsPa
       }
       if (!ok) atomicOr(&q6_fault_word, 1);
       const int s_a = spt * i + sa_off, s_b = spt * i + sb_off;
-      base_a = ring + (uint32_t)(s_a % sp.ns) * sp.stage_stride + (uint32_t)((g % SR) * row_bytes);
-      base_b = ring + (uint32_t)(s_b % sp.ns) * sp.stage_stride + (uint32_t)(((g + 8) % SR) * row_bytes);
+      base_a = ring + (uint32_t)(s_a % sp.ns) * sp.stage_stride + (uint32_t)((lra % SR) * row_bytes);
+      base_b = ring + (uint32_t)(s_b % sp.ns) * sp.stage_stride + (uint32_t)((lrb % SR) * row_bytes);
     }
     // the previous tile's reduction, on the warps with the shortest slices, while the others
     // start this tile
-    if (warp >= kQ6RedWarp0 && i > 0) q6_reduce_tile(p, red + ((i - 1) & 1) * (kQ6Warps * 32 * 4), tile - 1);
-    const uint8_t* ga = p.blocks + (int64_t)r0 * row_bytes;
+    if (warp >= kQ6RedWarp0 && i > 0) q6_reduce_tile(p, red + ((i - 1) & 1) * (kQ6Warps * 32 * 4), tile - 1, sp.row_pair);
+    const uint8_t* ga = p.blocks + (int64_t)ra * row_bytes;
+    const uint8_t* gb = p.blocks + (int64_t)rb * row_bytes;
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     auto one = [&](int sb, const uint32_t (&bw)[16]) {
       Q6W wa, wb;
@@ -415,7 +426,7 @@ __global__ void __launch_bounds__(kQ6Threads, 1) q6k_rows8_kernel(const Q6RowsPa
         }
       } else {
         q6_load_global(wa, va, ga + (int64_t)sb * 210, t);
-        q6_load_global(wb, vb, ga + 8 * row_bytes + (int64_t)sb * 210, t);
+        q6_load_global(wb, vb, gb + (int64_t)sb * 210, t);
       }
       q6_superblock_8(acc, wa, wb, bw, dx0 + 256u * sb, co0 + 512u * sb);
     };
@@ -444,7 +455,7 @@ __global__ void __launch_bounds__(kQ6Threads, 1) q6k_rows8_kernel(const Q6RowsPa
       for (int q = 0; q < spt; ++q)
         if (spt * i + q + sp.ns < nstages) produce(spt * i + q + sp.ns);
   }
-  if (warp >= kQ6RedWarp0 && T1 > T0) q6_reduce_tile(p, red + ((T1 - T0 - 1) & 1) * (kQ6Warps * 32 * 4), T1 - 1);
+  if (warp >= kQ6RedWarp0 && T1 > T0) q6_reduce_tile(p, red + ((T1 - T0 - 1) & 1) * (kQ6Warps * 32 * 4), T1 - 1, sp.row_pair);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -737,6 +748,45 @@ int launch_rows8(const Q6RowsParams& sp, int grid, size_t smem, cudaStream_t s) 
 
 }  // namespace
 
+// Bank conflicts of the weight-fragment loads of the streamed 8-row kernel: for each of the
+// two loads (MMA rows g and g + 8) of an even and an odd super-block, the largest number of
+// distinct 4-byte words that the 32 lanes ask of one bank, summed.  Stage slot s starts at
+// s * stride (the ring is 128-byte aligned); the tile's first slot stands for all.
+static int q6_bank_cost(int64_t row_bytes, int sr, size_t stride, int row_pair) {
+  int cost = 0;
+  for (int odd = 0; odd < 2; ++odd)
+    for (int half = 0; half < 2; ++half) {
+      int64_t words[32][32];
+      int nw[32] = {0}, ways = 0;
+      for (int g = 0; g < 8; ++g) {
+        const int lr = row_pair ? 2 * g + half : g + 8 * half;
+        const int64_t off = (int64_t)(lr / sr) * (int64_t)stride + (lr % sr) * row_bytes + 210 * odd;
+        for (int t = 0; t < 4; ++t) {
+          const int64_t w = (off >> 2) + t;
+          const int bank = (int)(w & 31);
+          bool seen = false;
+          for (int i = 0; i < nw[bank]; ++i) seen |= words[bank][i] == w;
+          if (!seen) words[bank][nw[bank]++] = w;
+          ways = nw[bank] > ways ? nw[bank] : ways;
+        }
+      }
+      cost += ways;
+    }
+  return cost;
+}
+
+// The lane row map and the stage-slot padding (0, 16, ..., 112 bytes) with the fewest conflicts
+// (ties: the plain map, then the least padding).
+static void q6_bank_layout(int64_t row_bytes, int sr, int* row_pair, size_t* pad) {
+  const size_t base = ((size_t)sr * (size_t)row_bytes + 127) / 128 * 128;
+  int best = -1;
+  for (int rp = 0; rp < 2; ++rp)
+    for (size_t pd = 0; pd < 128; pd += 16) {
+      const int c = q6_bank_cost(row_bytes, sr, base + pd, rp);
+      if (best < 0 || c < best) best = c, *row_pair = rp, *pad = pd;
+    }
+}
+
 int q6k_wide_rows(int rows) { return rows <= 8 ? 8 : rows <= 16 ? 16 : rows <= 32 ? 32 : 64; }
 
 int q6k_mmvq_launch(const uint8_t* blocks, int n, int k, const uint8_t* q8, int rows, uint16_t* out, int64_t ldc,
@@ -764,18 +814,21 @@ int q6k_mmvq_launch(const uint8_t* blocks, int n, int k, const uint8_t* q8, int 
   const size_t ring_offset = (base_smem + 127) / 128 * 128;
   const size_t limit = (size_t)di.smem_optin > 2048 ? (size_t)di.smem_optin - 2048 : 0;
   const int nsb = k / 256;
-  Q6RowsParams best{p, 0, 0, 0, (int)ring_offset, after_prepass ? 1 : 0};
+  Q6RowsParams best{p, 0, 0, 0, (int)ring_offset, 0, after_prepass ? 1 : 0};
   double best_tiles = 1.0;
   for (int sr = 8; sr >= 4 && reg && (reinterpret_cast<uintptr_t>(blocks) & 15u) == 0; sr -= 4) {
     if (((size_t)sr * nsb * 210) % 16 != 0) continue;
-    const size_t stage_stride = ((size_t)sr * nsb * 210 + 127) / 128 * 128;
-    int ns = limit > ring_offset ? (int)((limit - ring_offset) / stage_stride) : 0;
     const int spt = kQ6TileRows / sr;
+    int row_pair = 0;
+    size_t pad = 0;
+    q6_bank_layout((int64_t)nsb * 210, sr, &row_pair, &pad);
+    const size_t stage_stride = ((size_t)sr * nsb * 210 + 127) / 128 * 128 + pad;
+    int ns = limit > ring_offset ? (int)((limit - ring_offset) / stage_stride) : 0;
     if (ns > 2 * spt) ns = 2 * spt;
     if (ns > kQ6MaxStages) ns = kQ6MaxStages;
     const double tiles = (double)ns / spt;
     if (tiles > best_tiles + 1e-9) {
-      best.ns = ns, best.stage_rows = sr, best.stage_stride = (int)stage_stride;
+      best.ns = ns, best.stage_rows = sr, best.stage_stride = (int)stage_stride, best.row_pair = row_pair;
       best_tiles = tiles;
     }
   }
@@ -784,7 +837,7 @@ int q6k_mmvq_launch(const uint8_t* blocks, int n, int k, const uint8_t* q8, int 
     return launch_rows8<true, true>(best, grid, smem, s);
   }
   if (base_smem + 1024 > (size_t)di.smem_optin) return DLMH_ERR_UNSUPPORTED;
-  const Q6RowsParams sp{p, 1, 8, 0, 0, 0};
+  const Q6RowsParams sp{p, 1, 8, 0, 0, 0, 0};
   return reg ? launch_rows8<false, true>(sp, grid, base_smem, s) : launch_rows8<false, false>(sp, grid, base_smem, s);
 }
 
