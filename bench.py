@@ -544,7 +544,7 @@ def oracle_single_thread():
 def profile_q6k(n):
     """A Q6_K profiling case for ncu: n x 7168 super-blocks (n = 32768: 193 MB, above the
     126 MB L2), 8 BF16 rows, four q6k_lm_head calls on cuda:0; prints one line and no bench
-    result.  Only for captures such as `ncu -k regex:q6k_stream -s 1 -c 2`."""
+    result.  Only for captures such as `ncu -k regex:q6k_rows8 -s 1 -c 1`."""
     import decode_lm_head_b200 as dl
     from decode_lm_head_b200 import synth
 

@@ -92,20 +92,23 @@ __device__ __forceinline__ void mma_s8s8_z(int (&d)[4], uint32_t a0, uint32_t a1
 
 // One q8_1 block of one 8-column group: t[i] += float(D0[i] sc0 + D1[i] sc1) * d8(column).
 // Outputs i: 0 = (row g, column 2t), 1 = (g, 2t+1), 2 = (g+8, 2t), 3 = (g+8, 2t+1).
+// kCol0: only column 0 is live (one activation row), the odd columns are left alone.
+template <bool kCol0 = false>
 __device__ __forceinline__ void q6_block_step(float (&tsb)[4], const int (&d0)[4], const int (&d1)[4], int ra0, int ra1,
                                               int rb0, int rb1, float dx0, float dx1) {
   tsb[0] = __fmaf_rn((float)(d0[0] * ra0 + d1[0] * ra1), dx0, tsb[0]);
-  tsb[1] = __fmaf_rn((float)(d0[1] * ra0 + d1[1] * ra1), dx1, tsb[1]);
+  if (!kCol0) tsb[1] = __fmaf_rn((float)(d0[1] * ra0 + d1[1] * ra1), dx1, tsb[1]);
   tsb[2] = __fmaf_rn((float)(d0[2] * rb0 + d1[2] * rb1), dx0, tsb[2]);
-  tsb[3] = __fmaf_rn((float)(d0[3] * rb0 + d1[3] * rb1), dx1, tsb[3]);
+  if (!kCol0) tsb[3] = __fmaf_rn((float)(d0[3] * rb0 + d1[3] * rb1), dx1, tsb[3]);
 }
 
 // End of a super-block: acc += t * d(row).
+template <bool kCol0 = false>
 __device__ __forceinline__ void q6_superblock_end(float (&acc)[4], const float (&tsb)[4], float da, float db) {
   acc[0] = __fmaf_rn(tsb[0], da, acc[0]);
-  acc[1] = __fmaf_rn(tsb[1], da, acc[1]);
+  if (!kCol0) acc[1] = __fmaf_rn(tsb[1], da, acc[1]);
   acc[2] = __fmaf_rn(tsb[2], db, acc[2]);
-  acc[3] = __fmaf_rn(tsb[3], db, acc[3]);
+  if (!kCol0) acc[3] = __fmaf_rn(tsb[3], db, acc[3]);
 }
 
 // ---- weight fragment loads
@@ -289,6 +292,7 @@ __device__ __forceinline__ uint32_t q6_bfrag(const Q6Params& p, int col, int sb,
 // One super-block of the 16-row tile (MMA rows g: wa, g+8: wb) against the 8 columns: bw[j] is
 // the lane's B fragment of sub-block j; dxs and cor point at the super-block's staged values
 // (256 and 512 bytes a super-block) plus 16 t.
+template <bool kCol0>
 __device__ __forceinline__ void q6_superblock_8(float (&acc)[4], const Q6W& wa, const Q6W& wb, const uint32_t (&bw)[16],
                                                 uint32_t dxs, uint32_t cor) {
   float tsb[4] = {0.f, 0.f, 0.f, 0.f};
@@ -301,10 +305,10 @@ __device__ __forceinline__ void q6_superblock_8(float (&acc)[4], const Q6W& wa, 
     mma_u8s8_c(d0, q6_codes_u8(wa, j0), q6_codes_u8(wb, j0), bw[j0], (int)c.x, (int)c.y);
     mma_u8s8_c(d1, q6_codes_u8(wa, j1), q6_codes_u8(wb, j1), bw[j1], (int)c.z, (int)c.w);
     if ((blk & 1) == 0) dx = lds128(dxs + 64 * (blk >> 1));  // blocks blk, blk + 1
-    q6_block_step(tsb, d0, d1, q6_scale(wa, j0), q6_scale(wa, j1), q6_scale(wb, j0), q6_scale(wb, j1),
-                  __uint_as_float((blk & 1) ? dx.z : dx.x), __uint_as_float((blk & 1) ? dx.w : dx.y));
+    q6_block_step<kCol0>(tsb, d0, d1, q6_scale(wa, j0), q6_scale(wa, j1), q6_scale(wb, j0), q6_scale(wb, j1),
+                         __uint_as_float((blk & 1) ? dx.z : dx.x), __uint_as_float((blk & 1) ? dx.w : dx.y));
   }
-  q6_superblock_end(acc, tsb, wa.d, wb.d);
+  q6_superblock_end<kCol0>(acc, tsb, wa.d, wb.d);
 }
 
 // Fixed-order sum over the 16 warps' partials of a tile, one BF16 store per output; run by the
@@ -325,7 +329,8 @@ __device__ __forceinline__ void q6_reduce_tile(const Q6Params& p, const float* r
   }
 }
 
-template <bool kStream, bool kRegActs>
+// kCol0: one activation row (column 0 only; the other columns' sums are never formed).
+template <bool kStream, bool kRegActs, bool kCol0>
 __global__ void __launch_bounds__(kQ6Threads, 1) q6k_rows8_kernel(const Q6RowsParams sp) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ __align__(8) uint64_t full[kQ6MaxStages];
@@ -428,7 +433,7 @@ __global__ void __launch_bounds__(kQ6Threads, 1) q6k_rows8_kernel(const Q6RowsPa
         q6_load_global(wa, va, ga + (int64_t)sb * 210, t);
         q6_load_global(wb, vb, gb + (int64_t)sb * 210, t);
       }
-      q6_superblock_8(acc, wa, wb, bw, dx0 + 256u * sb, co0 + 512u * sb);
+      q6_superblock_8<kCol0>(acc, wa, wb, bw, dx0 + 256u * sb, co0 + 512u * sb);
     };
     if (kRegActs) {
 #pragma unroll
@@ -739,11 +744,11 @@ int launch_wide(const Q6Params& p, int sms, int smem_optin, cudaStream_t s, bool
                           Q6WideParams{p, ns, depth, early_w ? 1 : 0});
 }
 
-template <bool kStream, bool kRegActs>
+template <bool kStream, bool kRegActs, bool kCol0 = false>
 int launch_rows8(const Q6RowsParams& sp, int grid, size_t smem, cudaStream_t s) {
-  if (ensure_dynamic_smem(reinterpret_cast<const void*>(q6k_rows8_kernel<kStream, kRegActs>), (int)smem) != DLMH_OK)
+  if (ensure_dynamic_smem(reinterpret_cast<const void*>(q6k_rows8_kernel<kStream, kRegActs, kCol0>), (int)smem) != DLMH_OK)
     return DLMH_ERR_CUDA;
-  return umma::launch_pdl(q6k_rows8_kernel<kStream, kRegActs>, dim3(grid), dim3(kQ6Threads), smem, s, sp);
+  return umma::launch_pdl(q6k_rows8_kernel<kStream, kRegActs, kCol0>, dim3(grid), dim3(kQ6Threads), smem, s, sp);
 }
 
 }  // namespace
@@ -834,7 +839,7 @@ int q6k_mmvq_launch(const uint8_t* blocks, int n, int k, const uint8_t* q8, int 
   }
   if (best.ns > 0) {
     const size_t smem = ring_offset + (size_t)best.ns * best.stage_stride;
-    return launch_rows8<true, true>(best, grid, smem, s);
+    return rows == 1 ? launch_rows8<true, true, true>(best, grid, smem, s) : launch_rows8<true, true>(best, grid, smem, s);
   }
   if (base_smem + 1024 > (size_t)di.smem_optin) return DLMH_ERR_UNSUPPORTED;
   const Q6RowsParams sp{p, 1, 8, 0, 0, 0, 0};

@@ -391,6 +391,9 @@ def test_q6k_streamed_and_register_kernels_agree(n, k):
     a = bits(dl.q6k_mmvq(blocks, q8))
     b = bits(dl.q6k_mmvq(shifted, q8))
     assert np.array_equal(a, b)
+    # one row: the streamed kernel's column-0 build against the register-load kernel
+    assert np.array_equal(bits(dl.q6k_mmvq(blocks, q8[:1])), a[:1])
+    assert np.array_equal(bits(dl.q6k_mmvq(shifted, q8[:1])), a[:1])
     assert_bf16_close(a, og.q6k_mmvq(bits(blocks), og.q8_1_quantize_rows(bits(x))), f"q6k streamed n={n} k={k}")
     assert dl.device_fault(reset=True) == 0
 
