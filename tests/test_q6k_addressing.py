@@ -1,14 +1,14 @@
 """Host restatement of the streamed 8-row Q6_K kernel's shared-memory addressing.
 
-The kernel (q6k_rows8_kernel<true, true>) reads each 210-byte super-block of a staged weight
+The kernel (q6k_rows8_kernel<true, true, *>) reads each 210-byte super-block of a staged weight
 row with 32-bit shared loads: single loads when every lane's super-block is 4-byte aligned,
 otherwise from one aligned base and a funnel shift (a row with an odd super-block count puts
-both alignments in one warp).  This test re-derives, for the shapes the tests and the bench
-use, the host's stage choice (rows per stage, ring depth) and every shared read the lanes make,
-and checks that each is aligned to its width and lies inside its super-block (two bytes before
-it at most, for the 2-mod-4 case), and that the ring fits the shared memory.  It also shows that
+both alignments in one warp).  This test re-derives, for the shapes the tests and the bench use, the host's stage choice (rows
+per stage, ring depth, lane row map, slot padding) and every shared read the lanes make, and
+checks that each is aligned to its width and lies inside its super-block (two bytes before it
+at most, for the 2-mod-4 case), and that the ring fits the shared memory.  It also shows that
 the scale load an earlier version used (five words from 2 bytes before the scales, whatever the
-lane's alignment) is misaligned at k = 1280.
+lane's alignment) is misaligned at k = 1280, and restates the activation tables' layout.
 """
 
 import pytest
@@ -26,6 +26,36 @@ def _slice_begin(nsb, w):
     return w * q + min(w, r)
 
 
+def _rows(row_pair, g):
+    """Tile rows of MMA rows g and g + 8 of lane (g, t)."""
+    return (2 * g, 2 * g + 1) if row_pair else (g, g + 8)
+
+
+def _bank_cost(row_bytes, sr, stride, row_pair):
+    cost = 0
+    for odd in (0, 1):
+        for half in (0, 1):
+            banks = {}
+            for g in range(8):
+                lr = _rows(row_pair, g)[half]
+                off = (lr // sr) * stride + (lr % sr) * row_bytes + 210 * odd
+                for t in range(4):
+                    w = (off >> 2) + t
+                    banks.setdefault(w & 31, set()).add(w)
+            cost += max(len(v) for v in banks.values())
+    return cost
+
+
+def _bank_layout(row_bytes, sr):
+    base, best = _rup(sr * row_bytes, 128), None
+    for rp in (0, 1):
+        for pad in range(0, 128, 16):
+            c = _bank_cost(row_bytes, sr, base + pad, rp)
+            if best is None or c < best[0]:
+                best = (c, rp, pad)
+    return best[1], best[2]
+
+
 def _config(k):
     nsb = k // 256
     reg = (nsb + 15) // 16 <= 2
@@ -37,18 +67,24 @@ def _config(k):
         for sr in (8, 4):
             if (sr * nsb * 210) % 16:
                 continue
-            stride = _rup(sr * nsb * 210, 128)
+            row_pair, pad = _bank_layout(nsb * 210, sr)
+            stride = _rup(sr * nsb * 210, 128) + pad
             spt = 16 // sr
             ns = min((limit - ring_off) // stride if limit > ring_off else 0, 2 * spt, 16)
             if ns / spt > best_t + 1e-9:
-                best, best_t = (ns, sr, stride), ns / spt
+                best, best_t = (ns, sr, stride, row_pair), ns / spt
     return ring_off, best
+
+
+def _scale_reads(a):
+    """The scales and d of a 4-byte aligned super-block at a."""
+    return [(a + 192 + 4 * q, 4) for q in range(4)] + [(a + 208, 2)]
 
 
 def _reads(a, t, aligned, old_scales=False):
     if aligned:
         r = [(a + 4 * t + 16 * q, 4) for q in range(8)] + [(a + 4 * t + 128 + 16 * q, 4) for q in range(4)]
-        r += [(a + 192 + 4 * q, 4) for q in range(4)]
+        return r + _scale_reads(a)
     else:
         b, sh = a & ~3, (a & 3) * 8
         r = []
@@ -57,17 +93,17 @@ def _reads(a, t, aligned, old_scales=False):
         for q in range(4):
             r += [(b + 4 * t + 128 + 16 * q, 4), (b + 4 * t + 128 + 16 * q + 4, 4)]
         if old_scales:
-            r += [(a + 190 + 4 * q, 4) for q in range(5)]
-        else:
-            r += [(b + 192 + 4 * q, 4) for q in range(4)] + [(b + (208 if sh else 204), 4)]
-    return r + [(a + 208, 2)]
+            return r + [(a + 190 + 4 * q, 4) for q in range(5)] + [(a + 208, 2)]
+        # the five words from b + 192 (the fifth only when sh != 0, else the fourth again)
+        r += [(b + 192 + 4 * q, 4) for q in range(4)] + [(b + (208 if sh else 204), 4)]
+        return r + [(a + 208, 2)]
 
 
 def _check(n, k, old_scales=False):
     nsb, row_bytes = k // 256, (k // 256) * 210
     ring_off, best = _config(k)
     assert best is not None, "streamed kernel expected"
-    ns, sr, stride = best
+    ns, sr, stride, row_pair = best
     spt = 16 // sr
     assert ring_off + ns * stride + 256 <= OPTIN
     ntiles = (n + 15) // 16
@@ -82,11 +118,12 @@ def _check(n, k, old_scales=False):
                     lanes = []
                     for lane in range(32):
                         g, t = lane >> 2, lane & 3
-                        sa, sbb = spt * i + g // sr, spt * i + (g + 8) // sr
-                        ba = ring_off + (sa % ns) * stride + (g % sr) * row_bytes + 210 * sb
-                        bb = ring_off + (sbb % ns) * stride + ((g + 8) % sr) * row_bytes + 210 * sb
-                        lanes.append((ba, tile * 16 + g < n, t))
-                        lanes.append((bb, tile * 16 + g + 8 < n, t))
+                        lra, lrb = _rows(row_pair, g)
+                        sa, sbb = spt * i + lra // sr, spt * i + lrb // sr
+                        ba = ring_off + (sa % ns) * stride + (lra % sr) * row_bytes + 210 * sb
+                        bb = ring_off + (sbb % ns) * stride + (lrb % sr) * row_bytes + 210 * sb
+                        lanes.append((ba, tile * 16 + lra < n, t))
+                        lanes.append((bb, tile * 16 + lrb < n, t))
                     aligned = all(a % 4 == 0 for a, _, _ in lanes)
                     for a, valid, t in lanes:
                         if not valid:
@@ -105,3 +142,41 @@ def test_streamed_q6k_reads_are_aligned_and_inside_their_super_block(n, k):
 def test_the_earlier_scale_load_is_caught():
     assert _check(45, 1280, old_scales=True) > 0
     assert _check(1000, 7168, old_scales=True) == 0  # even super-block counts never mix alignments
+
+
+def test_bank_layout_at_k7168_is_conflict_free():
+    # rows 5880 bytes apart: the plain map has 2-way conflicts on every fragment load, rows 2g
+    # and 2g + 1 with 64 bytes of slot padding none (one distinct word per bank per load)
+    assert _bank_cost(5880, 8, _rup(8 * 5880, 128), 0) == 8
+    assert _bank_layout(5880, 8) == (1, 64)
+    assert _bank_cost(5880, 8, _rup(8 * 5880, 128) + 64, 1) == 4
+
+
+@pytest.mark.parametrize("k", [512, 1280, 7168, 8192])
+def test_activation_tables_read_back_what_was_staged(k):
+    # staging: d of (block b, column m) at dxs[(b >> 1) * 16 + (m >> 1) * 4 + (b & 1) * 2 + (m & 1)],
+    # the correction of (sub-block 2b + e, column m) at cor[b * 16 + (m >> 1) * 4 + e * 2 + (m & 1)];
+    # lane t reads 16 bytes at dxs + 16 t + 256 sb + 64 (blk >> 1) and cor + 16 t + 512 sb + 64 blk
+    nb32 = k // 32
+    dxs, cor = {}, {}
+    for b in range(nb32):
+        for m in range(8):
+            o = (b >> 1) * 16 + (m >> 1) * 4 + (b & 1) * 2 + (m & 1)
+            assert o not in dxs and 0 <= o < nb32 * 8
+            dxs[o] = (b, m)
+            for e in range(2):
+                o = b * 16 + (m >> 1) * 4 + e * 2 + (m & 1)
+                assert o not in cor and 0 <= o < nb32 * 16
+                cor[o] = (2 * b + e, m)
+    for sb in range(k // 256):
+        for blk in range(8):
+            for t in range(4):
+                a = (16 * t + 256 * sb + 64 * (blk >> 1)) // 4
+                got = [dxs[a + c] for c in range(4)]
+                b = 8 * sb + blk
+                # components x, y: even block; z, w: odd block; columns 2t, 2t + 1
+                assert got[2 * (blk & 1)] == (b, 2 * t) and got[2 * (blk & 1) + 1] == (b, 2 * t + 1)
+                a = (16 * t + 512 * sb + 64 * blk) // 4
+                got = [cor[a + c] for c in range(4)]
+                j0 = 16 * sb + 2 * blk
+                assert got == [(j0, 2 * t), (j0, 2 * t + 1), (j0 + 1, 2 * t), (j0 + 1, 2 * t + 1)]
