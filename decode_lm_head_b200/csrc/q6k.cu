@@ -21,7 +21,8 @@
 // Value i = 128h + 32u + l (h < 2, u < 4, l < 32): low 4 bits from ql[64h + 32(u&1) + l] (low
 // nibble for u < 2, high for u >= 2), top 2 bits from bits 2u..2u+1 of qh[32h + l]; sub-block
 // j = i / 16 uses scales[j].  Lane (g, t) feeds the MMA with values 4t..4t+3 of every sub-block,
-// i.e. the 4 consecutive ql / qh bytes at l = 16(j&1) + 4t, for weight rows g and g+8.
+// i.e. the 4 consecutive ql / qh bytes at l = 16(j&1) + 4t, for the weight rows of MMA rows g
+// and g + 8 (tile rows g and g + 8, or 2g and 2g + 1: see the 8-row kernels).
 #include "dlmh_common.cuh"
 #include "gemv_launch.h"
 #include "q6k_slices.h"
