@@ -489,6 +489,13 @@ constexpr int kQWRowStride = 304;  // 76 words: the 8 B-fragment rows hit 32 ban
 constexpr int kQWSpan = 240;       // staged bytes per weight row and super-block (>= 224)
 constexpr int kQWTileBytes = kQ6TileRows * kQWSpan;
 constexpr int kQWMaxActStages = 4;
+// An activation stage: the NT * 8 rows' super-block (kQWRowStride apart), then the blocks' d
+// and s regrouped for the lanes: [block][8-column group][t][column 2t, 2t + 1] x (f16 d, f16 s),
+// so that lane (g, t) reads both of its columns' d with one 8-byte load.
+template <int NT>
+constexpr uint32_t qw_act_bytes() {
+  return (uint32_t)(NT * 8 * kQWRowStride + 256 * NT);
+}
 
 template <int NT>
 struct QW {
@@ -498,13 +505,16 @@ struct QW {
 
 struct Q6WideParams {
   Q6Params q;
-  int act_stages;  // activation ring stages of NT * 8 * kQWRowStride bytes
+  int act_stages;  // activation ring stages of qw_act_bytes<NT>() bytes
   int depth;       // weight stages per consumer warp (>= 2)
   int early_w;     // the preceding kernel is this library's q8_1 quantize (see Q6RowsParams)
 };
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
@@ -517,7 +527,8 @@ __device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
 }
 
 // One super-block of one warp's 16-row tile against NT 8-column groups of the staged chunk at
-// `xs` (row stride kQWRowStride, block b of row m at m * stride + 36 b: f16 d, f16 s, 32 codes).
+// `xs` (row stride kQWRowStride, block b of row m at m * stride + 36 b: f16 d, f16 s, 32 codes;
+// the regrouped d and s after the rows).
 template <int NT>
 __device__ __forceinline__ void q6_superblock_wide(float (&acc)[NT][4], const Q6W& wa, const Q6W& wb, uint32_t xs,
                                                    int g, int t) {
@@ -538,9 +549,8 @@ __device__ __forceinline__ void q6_superblock_wide(float (&acc)[NT][4], const Q6
       int d0[4], d1[4];
       mma_s8s8_z(d0, a00, a01, lds_u32(brow));
       mma_s8s8_z(d1, a10, a11, lds_u32(brow + 16));
-      const uint32_t drow = xs + (uint32_t)((8 * ct + 2 * t) * kQWRowStride + 36 * blk);
-      const float dx0 = f16_bits_to_f32(lds_u16(drow));
-      const float dx1 = f16_bits_to_f32(lds_u16(drow + kQWRowStride));
+      const uint2 dd = lds_u64(xs + (uint32_t)(NT * 8 * kQWRowStride + ((blk * NT + ct) * 4 + t) * 8));
+      const float dx0 = f16_bits_to_f32(dd.x & 0xffffu), dx1 = f16_bits_to_f32(dd.y & 0xffffu);
       q6_block_step(tsb[ct], d0, d1, ra0, ra1, rb0, rb1, dx0, dx1);
     }
   }
@@ -587,7 +597,7 @@ __global__ void __launch_bounds__(QW<NT>::kThreads, 1) q6k_wide_kernel(const Q6W
   const int64_t row_bytes = (int64_t)nsb * 210;
   const uintptr_t buf_end = reinterpret_cast<uintptr_t>(p.blocks) + (uintptr_t)((int64_t)p.n * row_bytes);
   constexpr int kRows = NT * 8;
-  constexpr uint32_t kActBytes = kRows * kQWRowStride;
+  constexpr uint32_t kActBytes = qw_act_bytes<NT>();
   const int ns = wp.act_stages, depth = wp.depth;
   const uint32_t act_ring = smem_u32(smem);
   const uint32_t w_rings = act_ring + (uint32_t)ns * kActBytes;
@@ -628,6 +638,11 @@ __global__ void __launch_bounds__(QW<NT>::kThreads, 1) q6k_wide_kernel(const Q6W
         const int m = q / kPieces, piece = q % kPieces;
         cp_async16(st + (uint32_t)(m * kQWRowStride + 16 * piece),
                    p.q8 + ((int64_t)m * nb32 + 8 * sb) * 36 + 16 * piece);
+      }
+      for (int q = lane; q < p.rows * 8; q += 32) {  // (d, s) of block b of row m, regrouped
+        const int m = q >> 3, b = q & 7;
+        cp_async4(st + (uint32_t)(kRows * kQWRowStride + ((((b * NT + (m >> 3)) * 4 + ((m & 7) >> 1)) * 2 + (m & 1)) * 4)),
+                  p.q8 + ((int64_t)m * nb32 + 8 * sb + b) * 36);
       }
       cp_async_arrive(full0 + 8u * slot);
     }
@@ -727,7 +742,7 @@ namespace {
 template <int NT>
 int launch_wide(const Q6Params& p, int sms, int smem_optin, cudaStream_t s, bool early_w) {
   constexpr int kWarps = QW<NT>::kWarps;
-  const size_t act = (size_t)NT * 8 * kQWRowStride;
+  const size_t act = qw_act_bytes<NT>();
   const size_t limit = (size_t)smem_optin > 1024 ? (size_t)smem_optin - 1024 : 0;  // static smem < 1 KB
   // three weight stages per warp when they fit beside at least two activation stages
   int depth = 3;
