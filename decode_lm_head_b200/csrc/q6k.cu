@@ -470,9 +470,9 @@ __global__ void __launch_bounds__(kQ6Threads, 1) q6k_rows8_kernel(const Q6RowsPa
 // around: a CTA takes its 16-row weight tiles in row-blocks of up to W tiles, one tile per
 // consumer warp, and the row-block walks K one super-block at a time.
 //   - Activations: a producer warp copies each super-block's q8_1 blocks of every activation
-//     row (288 contiguous bytes per row) into a ring shared by the row-block's warps, with
-//     16-byte cp.async and one mbarrier arrival per lane; the activations are re-read (from
-//     L2) once per row-block, not once per tile.
+//     row into a ring shared by the row-block's warps, with 4-byte cp.async into the order the
+//     lanes read them (below) and one mbarrier arrival per lane; the activations are re-read
+//     (from L2) once per row-block, not once per tile.
 //   - Weights: every consumer warp streams its own tile through a private ring of `depth`
 //     stages with 16-byte cp.async: per row the 16-byte aligned span that covers the
 //     super-block's 210 bytes (at most 224; super-blocks are only 2-byte aligned), read back
@@ -484,17 +484,22 @@ __global__ void __launch_bounds__(kQ6Threads, 1) q6k_rows8_kernel(const Q6RowsPa
 // NT <= 4: 15 consumer warps + 1 producer (128 registers a thread); NT = 8: 11 + 1 (168, a
 // small spill; 7 warps of 228 registers left the schedulers short of warps: 1040 against
 // 881 us for 64 rows on a 129280 x 7168 head).
-constexpr int kQWRowBytes = 288;   // one super-block of one q8_1 row: 8 blocks
-constexpr int kQWRowStride = 304;  // 76 words: the 8 B-fragment rows hit 32 banks
 constexpr int kQWSpan = 240;       // staged bytes per weight row and super-block (>= 224)
 constexpr int kQWTileBytes = kQ6TileRows * kQWSpan;
 constexpr int kQWMaxActStages = 4;
-// An activation stage: the NT * 8 rows' super-block (kQWRowStride apart), then the blocks' d
-// and s regrouped for the lanes: [block][8-column group][t][column 2t, 2t + 1] x (f16 d, f16 s),
-// so that lane (g, t) reads both of its columns' d with one 8-byte load.
+// An activation stage holds one super-block of the NT * 8 q8_1 rows, regrouped for the lanes:
+//   - codes: [block b][8-column group ct][g][t] x (codes 4t..4t+3, codes 16+4t..16+4t+3) of
+//     row 8 ct + g: lane (g, t)'s B words of sub-blocks 2b and 2b + 1 in one 8-byte load (the
+//     32 lanes read 256 contiguous bytes);
+//   - then (f16 d, f16 s): [block b][ct][t][column 2t, 2t + 1]: both of lane (g, t)'s columns'
+//     d in one 8-byte load.
+template <int NT>
+constexpr uint32_t qw_codes_bytes() {
+  return (uint32_t)(8 * NT * 32 * 8);
+}
 template <int NT>
 constexpr uint32_t qw_act_bytes() {
-  return (uint32_t)(NT * 8 * kQWRowStride + 256 * NT);
+  return qw_codes_bytes<NT>() + (uint32_t)(256 * NT);
 }
 
 template <int NT>
@@ -527,8 +532,7 @@ __device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
 }
 
 // One super-block of one warp's 16-row tile against NT 8-column groups of the staged chunk at
-// `xs` (row stride kQWRowStride, block b of row m at m * stride + 36 b: f16 d, f16 s, 32 codes;
-// the regrouped d and s after the rows).
+// `xs` (the regrouped codes, then d and s; see qw_act_bytes).
 template <int NT>
 __device__ __forceinline__ void q6_superblock_wide(float (&acc)[NT][4], const Q6W& wa, const Q6W& wb, uint32_t xs,
                                                    int g, int t) {
@@ -545,11 +549,11 @@ __device__ __forceinline__ void q6_superblock_wide(float (&acc)[NT][4], const Q6
     const int ra0 = q6_scale(wa, j0), ra1 = q6_scale(wa, j1), rb0 = q6_scale(wb, j0), rb1 = q6_scale(wb, j1);
 #pragma unroll
     for (int ct = 0; ct < NT; ++ct) {
-      const uint32_t brow = xs + (uint32_t)((8 * ct + g) * kQWRowStride + 36 * blk + 4 + 4 * t);
+      const uint2 bw = lds_u64(xs + (uint32_t)((((blk * NT + ct) * 8 + g) * 4 + t) * 8));
       int d0[4], d1[4];
-      mma_s8s8_z(d0, a00, a01, lds_u32(brow));
-      mma_s8s8_z(d1, a10, a11, lds_u32(brow + 16));
-      const uint2 dd = lds_u64(xs + (uint32_t)(NT * 8 * kQWRowStride + ((blk * NT + ct) * 4 + t) * 8));
+      mma_s8s8_z(d0, a00, a01, bw.x);
+      mma_s8s8_z(d1, a10, a11, bw.y);
+      const uint2 dd = lds_u64(xs + qw_codes_bytes<NT>() + (uint32_t)(((blk * NT + ct) * 4 + t) * 8));
       const float dx0 = f16_bits_to_f32(dd.x & 0xffffu), dx1 = f16_bits_to_f32(dd.y & 0xffffu);
       q6_block_step(tsb[ct], d0, d1, ra0, ra1, rb0, rb1, dx0, dx1);
     }
@@ -596,7 +600,6 @@ __global__ void __launch_bounds__(QW<NT>::kThreads, 1) q6k_wide_kernel(const Q6W
   const int nb32 = p.k / 32;
   const int64_t row_bytes = (int64_t)nsb * 210;
   const uintptr_t buf_end = reinterpret_cast<uintptr_t>(p.blocks) + (uintptr_t)((int64_t)p.n * row_bytes);
-  constexpr int kRows = NT * 8;
   constexpr uint32_t kActBytes = qw_act_bytes<NT>();
   const int ns = wp.act_stages, depth = wp.depth;
   const uint32_t act_ring = smem_u32(smem);
@@ -611,11 +614,8 @@ __global__ void __launch_bounds__(QW<NT>::kThreads, 1) q6k_wide_kernel(const Q6W
   const int nchunks = nrb * nsb;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // padding activation rows [rows, kRows) of every stage stay zero (never copied)
-  for (int i = threadIdx.x; i < ns * (int)(kActBytes / 4); i += blockDim.x) {
-    const int w = i % (int)(kActBytes / 4);
-    if (w / (kQWRowStride / 4) >= p.rows) reinterpret_cast<uint32_t*>(smem)[i] = 0u;
-  }
+  // the activation ring starts zero: the padding rows [rows, kRows) are never copied
+  for (int i = threadIdx.x; i < ns * (int)(kActBytes / 4); i += blockDim.x) reinterpret_cast<uint32_t*>(smem)[i] = 0u;
   if (threadIdx.x == 0) {
     for (int i = 0; i < ns; ++i) {
       umma::bar_init(full0 + 8u * i, 32);  // one arrival per producer lane, when its copies land
@@ -628,20 +628,19 @@ __global__ void __launch_bounds__(QW<NT>::kThreads, 1) q6k_wide_kernel(const Q6W
   if (warp == kWarps) {
     // ---------------- producer: chunk c = (row-block c / nsb, super-block c % nsb)
     if (wp.early_w) grid_dependency_wait();
-    constexpr int kPieces = kQWRowBytes / 16;
     for (int c = 0; c < nchunks; ++c) {
       const int slot = c % ns, sb = c % nsb;
       if (c >= ns && !umma::wait(empty0 + 8u * slot, ((c / ns) - 1) & 1)) atomicOr(&q6_fault_word, 4);
       __syncwarp();
       const uint32_t st = act_ring + (uint32_t)slot * kActBytes;
-      for (int q = lane; q < p.rows * kPieces; q += 32) {
-        const int m = q / kPieces, piece = q % kPieces;
-        cp_async16(st + (uint32_t)(m * kQWRowStride + 16 * piece),
-                   p.q8 + ((int64_t)m * nb32 + 8 * sb) * 36 + 16 * piece);
+      for (int q = lane; q < p.rows * 64; q += 32) {  // code word w of block b of row m
+        const int m = q >> 6, b = (q >> 3) & 7, w = q & 7;
+        cp_async4(st + (uint32_t)(((((b * NT + (m >> 3)) * 8 + (m & 7)) * 4 + (w & 3)) * 2 + (w >> 2)) * 4),
+                  p.q8 + ((int64_t)m * nb32 + 8 * sb + b) * 36 + 4 + 4 * w);
       }
-      for (int q = lane; q < p.rows * 8; q += 32) {  // (d, s) of block b of row m, regrouped
+      for (int q = lane; q < p.rows * 8; q += 32) {  // (d, s) of block b of row m
         const int m = q >> 3, b = q & 7;
-        cp_async4(st + (uint32_t)(kRows * kQWRowStride + ((((b * NT + (m >> 3)) * 4 + ((m & 7) >> 1)) * 2 + (m & 1)) * 4)),
+        cp_async4(st + qw_codes_bytes<NT>() + (uint32_t)((((b * NT + (m >> 3)) * 4 + ((m & 7) >> 1)) * 2 + (m & 1)) * 4),
                   p.q8 + ((int64_t)m * nb32 + 8 * sb + b) * 36);
       }
       cp_async_arrive(full0 + 8u * slot);
