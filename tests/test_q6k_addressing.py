@@ -8,7 +8,8 @@ per stage, ring depth, lane row map, slot padding) and every shared read the lan
 checks that each is aligned to its width and lies inside its super-block (two bytes before it
 at most, for the 2-mod-4 case), and that the ring fits the shared memory.  It also shows that
 the scale load an earlier version used (five words from 2 bytes before the scales, whatever the
-lane's alignment) is misaligned at k = 1280, and restates the activation tables' layout.
+lane's alignment) is misaligned at k = 1280, and restates the activation tables' layout of the
+8-row kernels and the wide kernel's regrouped activation stage.
 """
 
 import pytest
@@ -180,3 +181,35 @@ def test_activation_tables_read_back_what_was_staged(k):
                 got = [cor[a + c] for c in range(4)]
                 j0 = 16 * sb + 2 * blk
                 assert got == [(j0, 2 * t), (j0, 2 * t + 1), (j0 + 1, 2 * t), (j0 + 1, 2 * t + 1)]
+
+
+@pytest.mark.parametrize("nt,rows", [(2, 9), (2, 16), (4, 17), (4, 32), (8, 33), (8, 64)])
+def test_wide_activation_stage_reads_back_what_was_copied(nt, rows):
+    # the wide kernel's producer copies code word w (bytes 4w..4w+3 of a block's 32 codes) of
+    # block b of row m to word (((b NT + m / 8) 8 + m % 8) 4 + w % 4) 2 + w / 4 of the stage,
+    # and the (d, s) word of block b of row m to word ((b NT + m / 8) 4 + (m % 8) / 2) 2 + m % 2
+    # after 8 NT 32 8 bytes of codes; lane (g, t) of column group ct reads 8 bytes at
+    # (((blk NT + ct) 8 + g) 4 + t) 8 (its B words of sub-blocks 2 blk, 2 blk + 1) and at
+    # codes_bytes + ((blk NT + ct) 4 + t) 8 (the d of columns 2t, 2t + 1)
+    codes_words = 8 * nt * 32 * 8 // 4
+    stage = {}
+    for m in range(rows):
+        for b in range(8):
+            for w in range(8):
+                o = (((b * nt + (m >> 3)) * 8 + (m & 7)) * 4 + (w & 3)) * 2 + (w >> 2)
+                assert o not in stage and 0 <= o < codes_words
+                stage[o] = ("code", m, b, w)
+            o = codes_words + ((b * nt + (m >> 3)) * 4 + ((m & 7) >> 1)) * 2 + (m & 1)
+            assert o not in stage and o < codes_words + 256 * nt // 4
+            stage[o] = ("ds", m, b)
+    for blk in range(8):
+        for ct in range(nt):
+            for g in range(8):
+                for t in range(4):
+                    m = 8 * ct + g
+                    a = ((((blk * nt + ct) * 8 + g) * 4 + t) * 8) // 4
+                    want = [("code", m, blk, t), ("code", m, blk, 4 + t)] if m < rows else [None, None]
+                    assert [stage.get(a), stage.get(a + 1)] == want  # padding rows read the zeroed stage
+                    a = codes_words + (((blk * nt + ct) * 4 + t) * 8) // 4
+                    want = [("ds", c, blk) if c < rows else None for c in (8 * ct + 2 * t, 8 * ct + 2 * t + 1)]
+                    assert [stage.get(a), stage.get(a + 1)] == want
