@@ -585,8 +585,11 @@ int launch_umma_f8(const uint8_t* w, const float* w_scale, int n, int k, const u
   p.out = out;
   p.ldc = ldc;
   // a stage is a whole unit (the longest run of each weight row per copy) when the ring holds
-  // two of them, else half a unit
-  p.cps = kUmmaSmemLimit / ((size_t)kKC * (kChunkBytesA + bn * 128)) >= 2 ? kKC : kKC / 2;
+  // two of them and half units would not put more bytes in the ring, else half a unit (at
+  // 32 activation rows a CTA: two 80 KB units, or five 40 KB halves)
+  const size_t unit = (size_t)kKC * (kChunkBytesA + bn * 128);
+  const size_t whole = kUmmaSmemLimit / unit, halves = kUmmaSmemLimit / (unit / 2);
+  p.cps = whole >= 2 && halves <= 2 * whole ? kKC : kKC / 2;
   p.stage_bytes = p.cps * (kChunkBytesA + bn * 128);
   int ns = (int)(kUmmaSmemLimit / (size_t)p.stage_bytes);
   if (ns > kMaxUStages) ns = kMaxUStages;
