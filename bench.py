@@ -565,7 +565,7 @@ def profile_case(name):
     result.  down: the W8A8 SiLU down projection 4096 x 14336 at M = 1, 6 calls over 3 weight
     copies; nvfp4: NVFP4 W4A16 14336 x 4096 at M = 1, 6 calls over 6 weight copies; head: FP8
     W8A16 on a 38188 x 5120 head (196 MB), three calls at M = 32 then three at M = 128;
-    q6k_wide: Q6_K 32768 x 7168 (193 MB), two calls at M = 16 then two at M = 64."""
+    q6k_wide: Q6_K 32768 x 7168 (193 MB), two calls at M = 32 then two at M = 64."""
     import decode_lm_head_b200 as dl
     from decode_lm_head_b200 import synth
 
@@ -610,7 +610,7 @@ def profile_case(name):
         blocks = synth.q6k_blocks(n, k, 4, dev)
         x = synth.bf16_rows(64, k, 4, dev)
         out = torch.empty(64, n, dtype=torch.bfloat16, device=dev)
-        for m in (16, 16, 64, 64):
+        for m in (32, 32, 64, 64):
             dl.q6k_lm_head(blocks, x[:m], out=out[:m], stream=stream)
         torch.cuda.synchronize()
     else:

@@ -814,9 +814,19 @@ int q6k_mmvq_launch(const uint8_t* blocks, int n, int k, const uint8_t* q8, int 
   const DeviceInfo di = device_info();
   if (di.sms <= 0) return DLMH_ERR_CUDA;
   const Q6Params p{blocks, n, k, q8, rows, out, ldc};
-  if (rows > kQ6MaxRows) {  // 9..64 rows: one pass of the wide kernel (16-byte aligned blocks, q8_1 rows)
+  if (rows > kQ6MaxRows) {  // 9..64 rows (16-byte aligned blocks, q8_1 rows)
     if (rows > 64) return DLMH_ERR_ROWS;
     if ((reinterpret_cast<uintptr_t>(q8) & 15u) || (reinterpret_cast<uintptr_t>(blocks) & 15u)) return DLMH_ERR_ALIGN;
+    if (rows <= 2 * kQ6MaxRows && q6_reg_acts(k)) {
+      // 9..16 rows: two passes of the streamed 8-row kernel take less time than one of the
+      // 16-row wide kernel (on a 129280 x 7168 head, 2 x ~183 against 416 us); same bits.  The
+      // second pass follows the first, which writes neither the weights nor its q8_1 rows.
+      const int rc = q6k_mmvq_launch(blocks, n, k, q8, kQ6MaxRows, out, ldc, s, after_prepass);
+      if (rc != DLMH_OK) return rc;
+      const int64_t q8_row = (int64_t)(k / 32) * 36;
+      return q6k_mmvq_launch(blocks, n, k, q8 + kQ6MaxRows * q8_row, rows - kQ6MaxRows, out + kQ6MaxRows * ldc, ldc, s,
+                             true);
+    }
     switch (q6k_wide_rows(rows)) {
       case 16: return launch_wide<2>(p, di.sms, di.smem_optin, s, after_prepass);
       case 32: return launch_wide<4>(p, di.sms, di.smem_optin, s, after_prepass);

@@ -306,7 +306,8 @@ DLMH_API int q8_1_quantize_rows(const dlmh_bf16* x, int64_t ldx, int rows, int k
  *   q8     [rows][k/32] block_q8_1 as written by q8_1_quantize_rows.
  *   k % 256 == 0 (set_lm_head_q6k requires hidden % 256 == 0).  Any rows: one weight pass per
  *   64 rows, through the narrowest tier of 8 / 16 / 32 / 64 that covers them (above 8 rows the
- *   q8_1 rows must start 16-byte aligned, else the pass falls back to 8-row launches).  Every
+ *   q8_1 rows must start 16-byte aligned, else the pass falls back to 8-row launches); the
+ *   16-row tier runs as two 8-row passes when k <= 8192 (faster than one 16-row pass).  Every
  *   tier adds the same products in the same order, so a row's bits do not depend on `rows`.
  * ------------------------------------------------------------------------------------- */
 DLMH_API int q6k_mmvq(const void* blocks, int n, int k, const void* q8, int rows, dlmh_bf16* out, int64_t ldc,

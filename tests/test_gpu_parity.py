@@ -398,10 +398,11 @@ def test_q6k_streamed_and_register_kernels_agree(n, k):
     assert dl.device_fault(reset=True) == 0
 
 
-@pytest.mark.parametrize("n,k", [(1000, 7168), (45, 1280), (300, 512)])
+@pytest.mark.parametrize("n,k", [(1000, 7168), (45, 1280), (300, 512), (200, 8448)])
 def test_q6k_wide_tiers_one_pass(n, k):
     # (45 x 1280: the weight buffer ends off a 16-byte boundary, so its last bytes are staged
-    # with plain loads)
+    # with plain loads; at k <= 8192 the 16-row tier runs as two 8-row passes, at 8448 as one
+    # pass of the wide kernel)
     # 9..64 rows take one pass of the wide kernel (tiers 16 / 32 / 64); every row count must
     # give the 8-row kernels' bits (same slices, same order), and the oracle's values
     blocks = synth.q6k_blocks(n, k, 7, DEV)
